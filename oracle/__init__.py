@@ -1,0 +1,168 @@
+"""ctypes wrapper over the CPU oracle (``oracle.c``).
+
+TEST INFRASTRUCTURE: imported only by ``tests/``, ``__graft_entry__.smoke()``
+and ``bench.py``'s CPU-baseline / reference leg. The product package never
+imports it.
+
+``build()`` compiles ``oracle.c`` with gcc into ``liboracle.so`` next to it.
+Every function takes and returns numpy arrays; shapes follow ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle if the library is missing or older than its source."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            i64 = ctypes.c_int64
+            p = ctypes.c_void_p
+            lib.oracle_pack.argtypes = [p, p, i64, i64]
+            lib.oracle_unpack.argtypes = [p, p, i64, i64]
+            lib.oracle_quant.argtypes = [p, i64, i64, p, p, p]
+            lib.oracle_gemv.argtypes = [p, i64, i64, p, i64, i64, i64, p]
+            lib.oracle_epilogue.argtypes = [p, i64, i64, ctypes.c_float, p, p]
+            for f in (lib.oracle_pack, lib.oracle_unpack, lib.oracle_quant,
+                      lib.oracle_gemv, lib.oracle_epilogue):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+class OracleError(ValueError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc == 1:
+        raise OracleError(f"{what}: value outside the domain")
+    if rc == 2:
+        raise OracleError(f"{what}: bad shape")
+    if rc != 0:
+        raise OracleError(f"{what}: status {rc}")
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def pack(w: np.ndarray) -> np.ndarray:
+    """int8 [N,K] in {-1,0,1} -> uint8 [N/4,K]."""
+    w = np.ascontiguousarray(w, dtype=np.int8)
+    N, K = w.shape
+    if N % 4:
+        raise OracleError("pack: bad shape")
+    P = np.empty((N // 4, K), dtype=np.uint8)
+    _check(_load().oracle_pack(_ptr(w), _ptr(P), N, K), "pack")
+    return P
+
+
+def unpack(P: np.ndarray, N: int) -> np.ndarray:
+    """uint8 [N/4,K] -> int8 [N,K]."""
+    P = np.ascontiguousarray(P, dtype=np.uint8)
+    K = P.shape[1]
+    if P.shape[0] * 4 != N:
+        raise OracleError("unpack: bad shape")
+    w = np.empty((N, K), dtype=np.int8)
+    _check(_load().oracle_unpack(_ptr(P), _ptr(w), N, K), "unpack")
+    return w
+
+
+def quant(x_bf16: np.ndarray):
+    """uint16 bf16 bits [M,K] -> (q int8 [M,K], x_scale fp32 [M], x_sum int32 [M])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.int8)
+    s = np.empty(M, dtype=np.float32)
+    t = np.empty(M, dtype=np.int32)
+    _check(_load().oracle_quant(_ptr(x), M, K, _ptr(q), _ptr(s), _ptr(t)), "quant")
+    return q, s, t
+
+
+def gemv(P: np.ndarray, N: int, q: np.ndarray, n0: int = 0, n1: int | None = None) -> np.ndarray:
+    """int32 acc [M, n1-n0] for output rows n0..n1-1 of the packed projection P."""
+    P = np.ascontiguousarray(P, dtype=np.uint8)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    if q.ndim == 1:
+        q = q[None, :]
+    K = P.shape[1]
+    M = q.shape[0]
+    if q.shape[1] != K or P.shape[0] * 4 != N:
+        raise OracleError("gemv: bad shape")
+    if n1 is None:
+        n1 = N
+    acc = np.empty((M, n1 - n0), dtype=np.int32)
+    _check(_load().oracle_gemv(_ptr(P), N, K, _ptr(q), M, n0, n1, _ptr(acc)), "gemv")
+    return acc
+
+
+def gemv_threads(P: np.ndarray, N: int, q: np.ndarray, threads: int | None = None) -> np.ndarray:
+    """``gemv`` over all rows, run as disjoint row ranges on several host threads
+    (the C call releases the GIL). Same function, same result; for parity runs
+    on large shapes only."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    if q.ndim == 1:
+        q = q[None, :]
+    threads = threads or os.cpu_count() or 1
+    bounds = np.linspace(0, N, min(threads, max(1, N)) + 1).astype(np.int64)
+    out = np.empty((q.shape[0], N), dtype=np.int32)
+
+    def run(i):
+        a, b = int(bounds[i]), int(bounds[i + 1])
+        if b > a:
+            out[:, a:b] = gemv(P, N, q, a, b)
+
+    with ThreadPoolExecutor(len(bounds) - 1) as ex:
+        list(ex.map(run, range(len(bounds) - 1)))
+    return out
+
+
+def epilogue(acc: np.ndarray, w_scale: float, x_scale: np.ndarray) -> np.ndarray:
+    """fp64 y [M,N] = acc * w_scale * x_scale[m]."""
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    if acc.ndim == 1:
+        acc = acc[None, :]
+    x_scale = np.ascontiguousarray(x_scale, dtype=np.float32).reshape(-1)
+    M, N = acc.shape
+    y = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_epilogue(_ptr(acc), M, N, np.float32(w_scale), _ptr(x_scale), _ptr(y)),
+           "epilogue")
+    return y
+
+
+def forward(P: np.ndarray, N: int, w_scale: float, x_bf16: np.ndarray, threads: int = 1):
+    """The whole path for one projection: quant, accumulate, scale.
+    Returns (q, x_scale, x_sum, acc, y)."""
+    q, xs, xsum = quant(x_bf16)
+    acc = gemv(P, N, q) if threads == 1 else gemv_threads(P, N, q, threads)
+    y = epilogue(acc, w_scale, xs)
+    return q, xs, xsum, acc, y
