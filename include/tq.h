@@ -1,0 +1,178 @@
+/*
+ * tq.h -- C ABI of libtq, the B200 (sm_100a) ternary absmax-int8 GEMV library.
+ *
+ * The method: BitNet b1.58 style projections. Weights are ternary {-1, 0, +1}
+ * (1bit.systems post "the full arc ...", paper list item 1), stored four 2-bit
+ * codes per byte so that an [N, K] projection becomes uint8 [N/4, K]
+ * (lemon-mlx-engine issue "Feature request: BitNet 1.58-bit ternary inference
+ * on ROCm (gfx1151)", section "Weight mapping (bitnet-b1.58-2B-4T)"), with one
+ * fp32 scale per tensor (same issue, "What We Need" item 2, the .weight_scale
+ * keys). Activations are quantised per token to int8 by absmax, products are
+ * accumulated in int32 (adds and subtracts only: baguaai "BitNet" tag page,
+ * the C99 engine item) and a scale epilogue produces fp32. Decode is bound by
+ * the bytes of weights read per token (1bit engine blog, "Qwen3.8-27B at 45.7
+ * tok/s ..." and "Smaller files ..."); prompt processing by the matrix units
+ * (same blog, first of those two posts).
+ *
+ * Layout and value conventions (the pages leave these open; readings taken):
+ *   - packed[i, k] (row-major, K contiguous) holds, in bits 2p..2p+1
+ *     (p = 0..3), the code of weight w[i + p*N/4, k]; code = w + 1 in {0,1,2};
+ *     code 3 is not a weight and the output for a byte holding it is undefined
+ *     (the kernels neither fault nor detect it).
+ *   - per token m: amax = max_k |x[m,k]|; s = fl32(127 / amax);
+ *     xq = clamp(round_half_even(fl32(x * s)), -127, 127);
+ *     x_scale = fl32(amax / 127); x_sum = sum_k xq. An all-zero row gives
+ *     xq = 0, x_scale = 0, x_sum = 0. NaN or Inf input is outside the contract.
+ *   - acc[m, n] = sum_k w[n, k] * xq[m, k] (int32, exact);
+ *     y[m, n] = fl32(float(acc) * fl32(w_scale * x_scale[m])).
+ *
+ * Conventions for every call:
+ *   - The caller owns every buffer. "device" pointers are CUDA device memory
+ *     (any allocator); "host" pointers are ordinary host memory.
+ *   - Device work is enqueued on `stream` and returns without synchronising;
+ *     argument checks happen before anything is enqueued, and a failed check
+ *     enqueues nothing.
+ *   - Shapes: N % 4 == 0 and K % 16 == 0; M, N, K >= 0. M = 0 or N = 0 is a
+ *     no-op. Device pointers to byte tensors (packed, xq) and to x must be
+ *     16-byte aligned; fp32/int32 vectors 4-byte aligned.
+ *   - Errors are returned as tq_status; tq_last_error() gives a message for
+ *     the last failure on the calling thread. A kernel-launch failure is
+ *     TQ_ERR_CUDA. Kernel execution errors surface on the stream as usual.
+ *   - The library keeps no state between calls apart from per-device launch
+ *     settings and one device-side error word (tq_device_error).
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_NULL = 1,        /* a required pointer is NULL */
+    TQ_ERR_SHAPE = 2,       /* M, N or K outside the contract */
+    TQ_ERR_ALIGN = 3,       /* a pointer is not aligned as required */
+    TQ_ERR_VALUE = 4,       /* a value outside its domain (e.g. a weight not in {-1,0,1}) */
+    TQ_ERR_CUDA = 5,        /* a CUDA runtime call or a kernel launch failed */
+    TQ_ERR_UNSUPPORTED = 6  /* valid input this build does not handle (see each call) */
+} tq_status;
+
+/* Name of a status code (static string). */
+const char *tq_status_string(tq_status s);
+
+/* Message for the last failed call on this thread (static per thread; "" if none). */
+const char *tq_last_error(void);
+
+/*
+ * tq_pack_host -- pack ternary weights on the host.
+ *   w      host, int8 [N, K] row-major, every value in {-1, 0, 1}.
+ *   packed host, uint8 [N/4, K] row-major, written.
+ *   M, stream: unused (kept so that every call takes M, N, K and a stream).
+ * Synchronous. TQ_ERR_VALUE if any w is outside {-1, 0, 1} (packed is then
+ * partly written). Packing: lemon-mlx-engine issue, "Architecture" item 3 and
+ * "Weight mapping".
+ */
+tq_status tq_pack_host(const int8_t *w, uint8_t *packed, int M, int N, int K,
+                       cudaStream_t stream);
+
+/*
+ * tq_quantize_act -- per-token absmax int8 quantisation (BitNet b1.58
+ * activations; formula as in the header comment).
+ *   x       device, bf16 [M, K] row-major (raw bf16 bit patterns).
+ *   xq      device, int8 [M, K], written.
+ *   x_scale device, fp32 [M], written (amax / 127).
+ *   x_sum   device, int32 [M], written (sum of xq over k); may be NULL when the
+ *           caller will not pass it to a GEMV call.
+ *   N: unused. Any M >= 0; K % 16 == 0.
+ */
+tq_status tq_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
+                          int M, int N, int K, cudaStream_t stream);
+
+/*
+ * tq_gemv -- decode-shaped ternary GEMV, 1 <= M <= 24 tokens.
+ *   packed  device, uint8 [N/4, K] (layout above).
+ *   w_scale the projection's fp32 scale.
+ *   xq, x_scale, x_sum  device, as written by tq_quantize_act for [M, K].
+ *   y       device, fp32 [M, N], written.
+ *   acc_out device, int32 [M, N], written when not NULL (the exact
+ *           accumulator; for checking), else untouched.
+ * TQ_ERR_UNSUPPORTED for M > 24 (use tq_gemm_prefill) or K > 32768.
+ */
+tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq,
+                  const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
+                  int M, int N, int K, cudaStream_t stream);
+
+/*
+ * tq_gemm_prefill -- the same contract as tq_gemv for any M >= 1 (prompt
+ * processing). M >= 128 runs on the tensor cores (tcgen05, int8 in, int32
+ * accumulators in tensor memory, the 2-bit codes expanded in shared memory);
+ * smaller M runs tq_gemv's kernels. TQ_ERR_UNSUPPORTED for K > 32768.
+ */
+tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq,
+                          const float *x_scale, const int32_t *x_sum, float *y,
+                          int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
+
+/*
+ * One projection of a decode layer stack (M = 1), for the grouped calls below.
+ * All pointers are device pointers with the meanings they have in
+ * tq_quantize_act / tq_gemv for M = 1. tq_quantize_act_stack reads x and
+ * writes xq, x_scale, x_sum (packed, y, acc_out unused, may be NULL);
+ * tq_gemv_stack reads packed, xq, x_scale, x_sum and writes y and, when not
+ * NULL, acc_out (x unused, may be NULL).
+ */
+typedef struct tq_proj {
+    const uint8_t *packed;  /* [N/4, K] */
+    const uint16_t *x;      /* bf16 [K]   (read by tq_quantize_act_stack) */
+    int8_t *xq;             /* int8 [K]   (written by quantize, read by gemv) */
+    float *x_scale;         /* fp32 [1] */
+    int32_t *x_sum;         /* int32 [1] */
+    float *y;               /* fp32 [N]   (written by gemv) */
+    int32_t *acc_out;       /* int32 [N] or NULL */
+    float w_scale;
+    int N;
+    int K;
+} tq_proj;
+
+/* Flags for tq_gemv_stack. */
+#define TQ_STACK_OVERLAP_PREV 1u /* weights are not written by work still in flight on
+                                    the stream: the kernel may start streaming them
+                                    before the previous kernel on the stream ends
+                                    (programmatic dependent launch); activations,
+                                    scales and sums are read only after it ends. */
+
+/*
+ * tq_quantize_act_stack -- tq_quantize_act for each projection's single
+ * token, all in one launch. projs is a HOST array of n_proj entries (read
+ * during the call only). K % 16 == 0 for every entry.
+ */
+tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t stream);
+
+/*
+ * tq_gemv_stack -- tq_gemv (M = 1) for every projection, in one persistent
+ * launch per 384 projections that streams all their weights back to back, in
+ * projection order, with no drain between projections. projs is a HOST array
+ * (read during the call only; the table travels in the launch parameters).
+ * flags: 0 or TQ_STACK_OVERLAP_PREV. Projections are independent: y of one
+ * must not be another's input within the same call.
+ */
+tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream);
+
+/*
+ * tq_device_error -- read (and if reset != 0, clear) the library's device
+ * error word on the current device. Synchronises the device. 0 means no
+ * kernel has reported an error. A nonzero value means a kernel gave up a
+ * bounded wait (its outputs are then invalid); bits: 1 = pipeline wait timed
+ * out.
+ */
+tq_status tq_device_error(uint32_t *code, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

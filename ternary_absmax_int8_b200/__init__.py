@@ -1,0 +1,163 @@
+"""Python binding of libtq (include/tq.h): the same names, argument marshalling only.
+
+Every function forwards to the C ABI of the in-tree ``libtq.so``; all work runs
+in its CUDA kernels. Tensors are passed as raw pointers (``data_ptr()``), an
+``int`` is taken as a raw pointer, ``None`` as NULL. ``stream`` defaults to
+PyTorch's current CUDA stream. A non-OK status raises :class:`TQError`.
+
+There is no fallback: if ``libtq.so`` is missing, importing this package fails.
+Build it with ``python -m ternary_absmax_int8_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "TQError", "TQ_STACK_OVERLAP_PREV", "TqProj", "lib_path",
+    "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
+    "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error",
+    "tq_status_string", "tq_last_error", "make_proj",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libtq.so")
+
+if not os.path.exists(lib_path):
+    raise ImportError(
+        f"{lib_path} is missing: build it with `python -m ternary_absmax_int8_b200.build` "
+        "(there is no CPU fallback)")
+
+_lib = ctypes.CDLL(lib_path)
+
+TQ_STACK_OVERLAP_PREV = 1
+_STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN",
+           4: "TQ_ERR_VALUE", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_UNSUPPORTED"}
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        self.name = _STATUS.get(status, f"status {status}")
+        super().__init__(f"{self.name}: {message}")
+
+
+class TqProj(ctypes.Structure):
+    """Mirror of ``struct tq_proj``."""
+    _fields_ = [
+        ("packed", ctypes.c_void_p),
+        ("x", ctypes.c_void_p),
+        ("xq", ctypes.c_void_p),
+        ("x_scale", ctypes.c_void_p),
+        ("x_sum", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("acc_out", ctypes.c_void_p),
+        ("w_scale", ctypes.c_float),
+        ("N", ctypes.c_int),
+        ("K", ctypes.c_int),
+    ]
+
+
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_sigs = {
+    "tq_pack_host": [_vp, _vp, _i, _i, _i, _vp],
+    "tq_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_gemv": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_gemm_prefill": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_quantize_act_stack": [ctypes.POINTER(TqProj), _i, _vp],
+    "tq_gemv_stack": [ctypes.POINTER(TqProj), _i, ctypes.c_uint, _vp],
+    "tq_device_error": [ctypes.POINTER(ctypes.c_uint32), _i],
+}
+for _name, _args in _sigs.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int
+_lib.tq_status_string.argtypes = [ctypes.c_int]
+_lib.tq_status_string.restype = ctypes.c_char_p
+_lib.tq_last_error.argtypes = []
+_lib.tq_last_error.restype = ctypes.c_char_p
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return t.data_ptr()
+    if hasattr(t, "ctypes"):  # numpy array
+        return t.ctypes.data
+    raise TypeError(f"cannot pass {type(t).__name__} as a pointer")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        if not torch.cuda.is_available():
+            return None
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise TQError(rc, _lib.tq_last_error().decode())
+
+
+def tq_status_string(status: int) -> str:
+    return _lib.tq_status_string(status).decode()
+
+
+def tq_last_error() -> str:
+    return _lib.tq_last_error().decode()
+
+
+def tq_pack_host(w, packed, M: int, N: int, K: int, stream=0) -> None:
+    """Host packing: w int8 [N,K] (CPU tensor or numpy) -> packed uint8 [N/4,K]."""
+    _check(_lib.tq_pack_host(_ptr(w), _ptr(packed), M, N, K, None))
+
+
+def tq_quantize_act(x, xq, x_scale, x_sum, M: int, N: int, K: int, stream=None) -> None:
+    _check(_lib.tq_quantize_act(_ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, N, K,
+                                _stream(stream)))
+
+
+def tq_gemv(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int, K: int,
+            stream=None) -> None:
+    _check(_lib.tq_gemv(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale), _ptr(x_sum),
+                        _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
+
+
+def tq_gemm_prefill(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int,
+                    K: int, stream=None) -> None:
+    _check(_lib.tq_gemm_prefill(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
+                                _ptr(x_sum), _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
+
+
+def make_proj(packed=None, x=None, xq=None, x_scale=None, x_sum=None, y=None, acc_out=None,
+              w_scale: float = 0.0, N: int = 0, K: int = 0) -> TqProj:
+    return TqProj(_ptr(packed), _ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), _ptr(y),
+                  _ptr(acc_out), float(w_scale), int(N), int(K))
+
+
+def _proj_array(projs):
+    arr = (TqProj * len(projs))(*projs)
+    return arr, len(projs)
+
+
+def tq_quantize_act_stack(projs, stream=None) -> None:
+    arr, n = _proj_array(projs)
+    _check(_lib.tq_quantize_act_stack(arr, n, _stream(stream)))
+
+
+def tq_gemv_stack(projs, flags: int = 0, stream=None) -> None:
+    arr, n = _proj_array(projs)
+    _check(_lib.tq_gemv_stack(arr, n, int(flags), _stream(stream)))
+
+
+def tq_device_error(reset: bool = False) -> int:
+    code = ctypes.c_uint32(0)
+    _check(_lib.tq_device_error(ctypes.byref(code), 1 if reset else 0))
+    return int(code.value)

@@ -1,0 +1,361 @@
+// tq_api.cu -- the C ABI of libtq (declared in include/tq.h): argument
+// checks, then kernel launches. Nothing here allocates device memory.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "tq.h"
+#include "tq_internal.h"
+
+namespace tq {
+
+__device__ unsigned int g_device_error = 0;
+
+bool pack_ternary_host(const int8_t *w, uint8_t *packed, int N, int K);
+cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                              const float *x_scale, const int32_t *x_sum, float *y,
+                              int32_t *acc_out, int M, int N, int K, cudaStream_t stream,
+                              bool *handled);
+
+unsigned *device_error_word()
+{
+    static unsigned *cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    if (!cache[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess)
+            return nullptr;
+        cache[dev] = static_cast<unsigned *>(p);
+    }
+    return cache[dev];
+}
+
+int device_sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 1;
+    if (dev < 0 || dev >= 64)
+        dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 1;
+    }
+    return cache[dev];
+}
+
+}  // namespace tq
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+tq_status fail(tq_status s, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+tq_status ok()
+{
+    g_msg[0] = '\0';
+    return TQ_OK;
+}
+
+tq_status cuda_fail(cudaError_t e, const char *where)
+{
+    if (e == cudaErrorInvalidValue)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: launch plan rejected (shape beyond this build's limits)",
+                    where);
+    return fail(TQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
+
+constexpr int kGemvMaxM = 24;
+
+// Shared checks of the GEMV-shaped calls.
+tq_status check_gemv_args(const char *fn, const uint8_t *packed, const int8_t *xq,
+                          const float *x_scale, const int32_t *x_sum, const float *y,
+                          const int32_t *acc_out, int M, int N, int K)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return fail(TQ_ERR_SHAPE, "%s: negative size (M=%d N=%d K=%d)", fn, M, N, K);
+    if (N % 4 != 0)
+        return fail(TQ_ERR_SHAPE, "%s: N=%d is not a multiple of 4", fn, N);
+    if (K % 16 != 0)
+        return fail(TQ_ERR_SHAPE, "%s: K=%d is not a multiple of 16", fn, K);
+    if (M == 0 || N == 0)
+        return TQ_OK;
+    if (!packed || !xq || !x_scale || !x_sum || !y)
+        return fail(TQ_ERR_NULL, "%s: a required pointer is NULL", fn);
+    if (!aligned(packed, 16) || !aligned(xq, 16))
+        return fail(TQ_ERR_ALIGN, "%s: packed and xq must be 16-byte aligned", fn);
+    if (!aligned(x_scale, 4) || !aligned(x_sum, 4) || !aligned(y, 4) ||
+        (acc_out && !aligned(acc_out, 4)))
+        return fail(TQ_ERR_ALIGN, "%s: x_scale, x_sum, y, acc_out must be 4-byte aligned", fn);
+    if (K > tq::kStreamMaxK)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: K=%d exceeds %d", fn, K, tq::kStreamMaxK);
+    return TQ_OK;
+}
+
+// K == 0: every accumulator is 0 and so is every output.
+tq_status zero_outputs(float *y, int32_t *acc_out, size_t count, cudaStream_t s)
+{
+    cudaError_t e = cudaMemsetAsync(y, 0, count * sizeof(float), s);
+    if (e == cudaSuccess && acc_out)
+        e = cudaMemsetAsync(acc_out, 0, count * sizeof(int32_t), s);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "zero outputs");
+}
+
+// Tokens in groups of up to four, one streaming launch per group.
+tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
+                        const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
+                        int M, int N, int K, cudaStream_t stream, const char *fn)
+{
+    for (int m0 = 0; m0 < M; m0 += tq::kStreamMaxTokens) {
+        const int mg = M - m0 < tq::kStreamMaxTokens ? M - m0 : tq::kStreamMaxTokens;
+        tq::StreamEntry e = {};
+        e.packed = packed;
+        e.xq = xq + size_t(m0) * K;
+        e.x_scale = x_scale + m0;
+        e.x_sum = x_sum + m0;
+        e.y = y + size_t(m0) * N;
+        e.acc_out = acc_out ? acc_out + size_t(m0) * N : nullptr;
+        e.w_scale = w_scale;
+        e.N4 = N / 4;
+        e.K = K;
+        cudaError_t err = tq::launch_stream_gemv(&e, 1, mg, false, true, stream);
+        if (err != cudaSuccess)
+            return cuda_fail(err, fn);
+    }
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tq_status_string(tq_status s)
+{
+    switch (s) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_NULL: return "TQ_ERR_NULL";
+    case TQ_ERR_SHAPE: return "TQ_ERR_SHAPE";
+    case TQ_ERR_ALIGN: return "TQ_ERR_ALIGN";
+    case TQ_ERR_VALUE: return "TQ_ERR_VALUE";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    }
+    return "TQ_ERR_UNKNOWN";
+}
+
+const char *tq_last_error(void) { return g_msg; }
+
+tq_status tq_pack_host(const int8_t *w, uint8_t *packed, int M, int N, int K, cudaStream_t stream)
+{
+    (void)M;
+    (void)stream;
+    if (N < 0 || K < 0)
+        return fail(TQ_ERR_SHAPE, "tq_pack_host: negative size (N=%d K=%d)", N, K);
+    if (N % 4 != 0)
+        return fail(TQ_ERR_SHAPE, "tq_pack_host: N=%d is not a multiple of 4", N);
+    if (N == 0 || K == 0)
+        return ok();
+    if (!w || !packed)
+        return fail(TQ_ERR_NULL, "tq_pack_host: a required pointer is NULL");
+    if (!tq::pack_ternary_host(w, packed, N, K))
+        return fail(TQ_ERR_VALUE, "tq_pack_host: a weight is outside {-1, 0, 1}");
+    return ok();
+}
+
+tq_status tq_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum, int M,
+                          int N, int K, cudaStream_t stream)
+{
+    (void)N;
+    if (M < 0 || K < 0)
+        return fail(TQ_ERR_SHAPE, "tq_quantize_act: negative size (M=%d K=%d)", M, K);
+    if (K % 16 != 0)
+        return fail(TQ_ERR_SHAPE, "tq_quantize_act: K=%d is not a multiple of 16", K);
+    if (M == 0)
+        return ok();
+    if (!x_scale || (K > 0 && (!x || !xq)))
+        return fail(TQ_ERR_NULL, "tq_quantize_act: a required pointer is NULL");
+    if ((K > 0 && (!aligned(x, 16) || !aligned(xq, 16))) || !aligned(x_scale, 4) ||
+        (x_sum && !aligned(x_sum, 4)))
+        return fail(TQ_ERR_ALIGN, "tq_quantize_act: x, xq need 16-byte, x_scale, x_sum 4-byte alignment");
+    if (K == 0) {
+        cudaError_t e = cudaMemsetAsync(x_scale, 0, size_t(M) * sizeof(float), stream);
+        if (e == cudaSuccess && x_sum)
+            e = cudaMemsetAsync(x_sum, 0, size_t(M) * sizeof(int32_t), stream);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "tq_quantize_act");
+    }
+    cudaError_t e = tq::launch_quant_rows(x, xq, x_scale, x_sum, M, K, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "tq_quantize_act");
+}
+
+tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
+                  const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K,
+                  cudaStream_t stream)
+{
+    tq_status st = check_gemv_args("tq_gemv", packed, xq, x_scale, x_sum, y, acc_out, M, N, K);
+    if (st != TQ_OK)
+        return st;
+    if (M > kGemvMaxM)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_gemv: M=%d > %d (use tq_gemm_prefill)", M, kGemvMaxM);
+    if (M == 0 || N == 0)
+        return ok();
+    if (K == 0)
+        return zero_outputs(y, acc_out, size_t(M) * N, stream);
+    return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                         "tq_gemv");
+}
+
+tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq,
+                          const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
+                          int M, int N, int K, cudaStream_t stream)
+{
+    tq_status st =
+        check_gemv_args("tq_gemm_prefill", packed, xq, x_scale, x_sum, y, acc_out, M, N, K);
+    if (st != TQ_OK)
+        return st;
+    if (M == 0 || N == 0)
+        return ok();
+    if (K == 0)
+        return zero_outputs(y, acc_out, size_t(M) * N, stream);
+    bool handled = false;
+    cudaError_t e = tq::launch_prefill_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
+                                          stream, &handled);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "tq_gemm_prefill");
+    if (handled)
+        return ok();
+    return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                         "tq_gemm_prefill");
+}
+
+tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t stream)
+{
+    if (n_proj < 0)
+        return fail(TQ_ERR_SHAPE, "tq_quantize_act_stack: n_proj=%d", n_proj);
+    if (n_proj == 0)
+        return ok();
+    if (!projs)
+        return fail(TQ_ERR_NULL, "tq_quantize_act_stack: projs is NULL");
+    std::vector<tq::QuantStackEntry> list;
+    list.reserve(size_t(n_proj));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        if (p.K < 0 || p.K % 16 != 0)
+            return fail(TQ_ERR_SHAPE, "tq_quantize_act_stack: entry %d: K=%d", j, p.K);
+        if (!p.x_scale || (p.K > 0 && (!p.x || !p.xq)))
+            return fail(TQ_ERR_NULL, "tq_quantize_act_stack: entry %d: NULL pointer", j);
+        if ((p.K > 0 && (!aligned(p.x, 16) || !aligned(p.xq, 16))) || !aligned(p.x_scale, 4) ||
+            (p.x_sum && !aligned(p.x_sum, 4)))
+            return fail(TQ_ERR_ALIGN, "tq_quantize_act_stack: entry %d: misaligned pointer", j);
+        if (p.K == 0) {
+            cudaError_t e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
+            if (e == cudaSuccess && p.x_sum)
+                e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "tq_quantize_act_stack");
+            continue;
+        }
+        tq::QuantStackEntry q = {};
+        q.x = p.x;
+        q.xq = p.xq;
+        q.x_scale = p.x_scale;
+        q.x_sum = p.x_sum;
+        q.K = p.K;
+        list.push_back(q);
+    }
+    static thread_local tq::QuantStackParams params;
+    for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
+        const size_t n = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
+        params.n = int(n);
+        std::memcpy(params.e, list.data() + base, n * sizeof(tq::QuantStackEntry));
+        cudaError_t e = tq::launch_quant_stack(params, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "tq_quantize_act_stack");
+    }
+    return ok();
+}
+
+tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream)
+{
+    if (n_proj < 0)
+        return fail(TQ_ERR_SHAPE, "tq_gemv_stack: n_proj=%d", n_proj);
+    if (flags & ~unsigned(TQ_STACK_OVERLAP_PREV))
+        return fail(TQ_ERR_VALUE, "tq_gemv_stack: unknown flags 0x%x", flags);
+    if (n_proj == 0)
+        return ok();
+    if (!projs)
+        return fail(TQ_ERR_NULL, "tq_gemv_stack: projs is NULL");
+    std::vector<tq::StreamEntry> list;
+    list.reserve(size_t(n_proj));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        char fn[64];
+        snprintf(fn, sizeof fn, "tq_gemv_stack[%d]", j);
+        tq_status st =
+            check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, 1, p.N, p.K);
+        if (st != TQ_OK)
+            return st;
+        if (p.N == 0)
+            continue;
+        if (p.K == 0) {
+            st = zero_outputs(p.y, p.acc_out, size_t(p.N), stream);
+            if (st != TQ_OK)
+                return st;
+            continue;
+        }
+        tq::StreamEntry e = {};
+        e.packed = p.packed;
+        e.xq = p.xq;
+        e.x_scale = p.x_scale;
+        e.x_sum = p.x_sum;
+        e.y = p.y;
+        e.acc_out = p.acc_out;
+        e.w_scale = p.w_scale;
+        e.N4 = p.N / 4;
+        e.K = p.K;
+        list.push_back(e);
+    }
+    const bool overlap = (flags & TQ_STACK_OVERLAP_PREV) != 0;
+    for (size_t base = 0; base < list.size(); base += tq::kStreamStackMax) {
+        const int n = int(std::min(list.size() - base, size_t(tq::kStreamStackMax)));
+        cudaError_t e = tq::launch_stream_gemv(list.data() + base, n, 1, overlap && base == 0,
+                                               false, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "tq_gemv_stack");
+    }
+    return ok();
+}
+
+tq_status tq_device_error(uint32_t *code, int reset)
+{
+    if (!code)
+        return fail(TQ_ERR_NULL, "tq_device_error: code is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    unsigned v = 0;
+    if (e == cudaSuccess)
+        e = cudaMemcpyFromSymbol(&v, tq::g_device_error, sizeof v);
+    if (e == cudaSuccess && reset) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(tq::g_device_error, &zero, sizeof zero);
+    }
+    if (e != cudaSuccess)
+        return cuda_fail(e, "tq_device_error");
+    *code = v;
+    return ok();
+}
+
+}  // extern "C"

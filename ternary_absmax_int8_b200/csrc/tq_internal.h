@@ -1,0 +1,92 @@
+// tq_internal.h -- launch-parameter structs and launchers shared between the
+// C ABI (tq_api.cu) and the kernel files. Not installed; not part of the ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tq_device.cuh"
+
+namespace tq {
+
+// ---------------------------------------------------------------- quantise
+constexpr int kMaxQuantStack = 512;
+
+struct QuantStackEntry {
+    const uint16_t *x;
+    int8_t *xq;
+    float *x_scale;
+    int32_t *x_sum;
+    int K;
+    int pad_;
+};
+
+struct QuantStackParams {
+    int n;
+    int pad_;
+    QuantStackEntry e[kMaxQuantStack];
+};
+
+cudaError_t launch_quant_rows(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
+                              int M, int K, cudaStream_t stream);
+cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream);
+
+// ------------------------------------------------- streaming GEMV (M <= 4)
+// One entry = one projection. The projection's packed rows are cut into
+// tiles of `rows_per_tile` consecutive packed rows (a contiguous byte range);
+// global tile t of the launch belongs to the entry with the largest
+// tile_begin <= t. Each row of a tile is cut into `ksplit` pieces along K,
+// so that rows_per_tile * ksplit work items keep every consumer warp busy.
+struct StreamEntry {
+    const uint8_t *packed;  // [N4, K]
+    const int8_t *xq;       // [M, K]
+    const float *x_scale;   // [M]
+    const int32_t *x_sum;   // [M]
+    float *y;               // [M, 4*N4]
+    int32_t *acc_out;       // [M, 4*N4] or null
+    float w_scale;
+    int N4;
+    int K;
+    int rows_per_tile;
+    int ksplit;
+    int tile_begin;
+};
+
+constexpr int kStreamMaxTokens = 4;     // tokens per launch of the streaming kernel
+constexpr int kStreamMaxRows = 16;      // rows_per_tile upper bound
+constexpr int kStreamMaxK = 32768;
+
+template <int MaxE>
+struct StreamParams {
+    int n_entries;
+    int total_tiles;
+    int M;             // tokens, 1..kStreamMaxTokens
+    int x_slot;        // bytes of a stage reserved for activations (>= M * K of every entry)
+    int w_slot;        // bytes of a stage reserved for weights (>= rows_per_tile * K)
+    int stages;
+    int overlap_prev;  // start weight copies before the previous grid completes
+    int pad_;
+    unsigned *err;     // the library's device error word
+    StreamEntry e[MaxE];
+};
+
+constexpr int kStreamStackMax = 384;  // entries per launch (kernel parameters <= 32 KB)
+
+struct StreamLaunch {
+    int grid;
+    int consumer_warps;
+    size_t smem_bytes;
+};
+
+// Plan tiles for a set of entries (fills rows_per_tile, ksplit, tile_begin,
+// total_tiles, x_slot, w_slot, stages) and launch. `single` selects the
+// small-launch heuristics for one projection.
+cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_prev,
+                               bool single, cudaStream_t stream);
+
+int device_sm_count();
+
+// Device address of the library's error word on the current device.
+unsigned *device_error_word();
+
+}  // namespace tq

@@ -1,0 +1,49 @@
+"""GPU parity of tq_gemm_prefill (M = 512 prompt processing) against the oracle.
+
+Full outputs at M = 128 and 256 for the FFN shapes; at M = 512 on the three
+prefill shapes (including the 27B-scale 17408 x 5120) a sample of token rows,
+first and last included, is checked on all N outputs. Ragged M and N exercise
+partial tiles.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests._gpu import assert_parity, gpu_forward, host_pack, oracle_forward
+from workloads import PREFILL_M, PREFILL_SHAPES, activations_bf16, make_projections, \
+    stored_weight_scale, ternary_weights
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M", [128, 256])
+def test_prefill_full_outputs(cuda_device, M):
+    for p in make_projections(PREFILL_SHAPES[:2], M=M, seed=77 + M):
+        P = host_pack(p.w)
+        assert_parity(gpu_forward(P, p.N, p.w_scale, p.x_bf16),
+                      oracle_forward(p.w, p.w_scale, p.x_bf16), f"{p.name} M={M}")
+
+
+def test_prefill_m512_sampled_rows(cuda_device):
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, PREFILL_M - 1], rng.choice(PREFILL_M, 30, replace=False)]))
+    for p in make_projections(PREFILL_SHAPES, M=PREFILL_M, seed=0):
+        P = host_pack(p.w)
+        q, xs, xsum, acc, y = gpu_forward(P, p.N, p.w_scale, p.x_bf16)
+        rq, rxs, rxsum = oracle.quant(p.x_bf16)
+        assert (q == rq).all() and (xs.view(np.uint32) == rxs.view(np.uint32)).all()
+        assert (xsum == rxsum).all()
+        sub = (q[rows], xs[rows], xsum[rows], acc[rows], y[rows])
+        ref = oracle_forward(p.w, p.w_scale, p.x_bf16[rows])
+        assert_parity(sub, ref, p.name)
+
+
+@pytest.mark.parametrize("N,K,M", [(516, 272, 130), (4, 16, 129), (2048, 1024, 384),
+                                   (260, 2560, 200)])
+def test_prefill_ragged(cuda_device, N, K, M):
+    rng = np.random.default_rng(N + K + M)
+    w = ternary_weights(rng, N, K)
+    xb = activations_bf16(rng, M, K)
+    ws = stored_weight_scale(w)
+    assert_parity(gpu_forward(host_pack(w), N, ws, xb), oracle_forward(w, ws, xb),
+                  f"{N}x{K} M={M}")
