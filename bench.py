@@ -1,0 +1,460 @@
+"""Benchmark of the ternary GEMV hot path on B200 (one JSON line on rank 0).
+
+Default workload (the headline): the decode layer stack -- 30 independently
+seeded copies of a BitNet-b1.58-2B-4T decoder layer, 7 ternary projections
+each (210 projections, 2.08e9 weights, 521 MB packed), M = 1. One step is one
+pass of the whole path over that stack: absmax-int8 quantisation of 210 fresh
+bf16 activation vectors (one launch) and the 210 GEMVs with their scale
+epilogues (one persistent launch). The weight stream is larger than L2, so no
+flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME]
+
+value  = algorithmic bytes of a step (all ranks) / device time per step, GB/s
+e2e    = the same metric through the same calls with host buffers: each step
+         copies the activations in from pinned host memory and the outputs back
+roofline = the stack GEMV kernel alone (its algorithmic bytes / its average
+         CUDA-event duration inside the timed region) against the measured HBM
+         copy bandwidth.
+--impl reference times the oracle (plain C, one host thread) on a bounded
+sample of the same workload; it is the CPU baseline, not a GPU arm.
+With N > 1 (torchrun) every rank runs its own replica of the workload
+(replicas only: the path has no exchange step); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import (WORKLOADS, algorithmic_bytes, make_projections)  # noqa: E402
+
+METRIC = ("ternary GEMV achieved HBM GB/s (% of B200 peak) at M=1; layer-stack passes/s")
+PEAK_FALLBACK_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+STACK_KERNEL_SRC = os.path.join(ROOT, "ternary_absmax_int8_b200", "csrc", "gemv_stream.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+DESCRIPTIONS = {
+    "stack30_m1": "decode layer stack: 30 x BitNet-b1.58-2B-4T decoder layer (q,k,v,o,gate,up,"
+                  "down ternary projections), M=1, 210 projections, 2.08e9 weights",
+    "layer_m1": "one BitNet-b1.58-2B-4T decoder layer, 7 ternary projections, M=1",
+    "single_640x2560_m1": "one ternary projection N=640 K=2560, M=1",
+    "prefill_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120",
+}
+
+
+def quant_bytes(K: int, M: int) -> int:
+    """bf16 in, int8 out, fp32 scale + int32 sum out."""
+    return M * K * 2 + M * K + M * 8
+
+
+def step_bytes(projs) -> int:
+    return sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
+
+
+# ----------------------------------------------------------------- helpers
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"tq_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 10:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        busy = [r for r in rows if r[4].isdigit() and int(r[4]) > 0] or rows
+        sm = [int(r[1]) for r in busy if r[1].isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": int(rows[0][2]) if rows[0][2].isdigit() else None,
+                "reasons": reasons, "samples": len(busy)}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return PEAK_FALLBACK_GBS, "fallback"
+
+
+def stack_kernel_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("gemv_stream.cu", "tq_device.cuh", "tq_internal.h"):
+        h.update(open(os.path.join(os.path.dirname(STACK_KERNEL_SRC), name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the stack kernel from a committed ncu summary,
+    scaled to this workload; None if absent or taken on another kernel version."""
+    try:
+        d = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_sha") != stack_kernel_sha() or workload != "stack30_m1":
+        return None
+    return float(d["bytes_per_packed_byte"]) * d["full_packed_bytes"]
+
+
+# -------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int):
+    import torch
+
+    import ternary_absmax_int8_b200 as tq
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    shapes, M = WORKLOADS[args.workload]
+    projs = list(make_projections(shapes, M=M, seed=args.seed))
+    stack = args.workload.startswith("stack") and M == 1
+    sb = step_bytes(projs)
+    gemv_bytes = sum(algorithmic_bytes(p.N, p.K, p.M) for p in projs)
+    packed_bytes = sum(p.N * p.K // 4 for p in projs)
+
+    # Weights: packed on the host by the library's packer, then resident in
+    # HBM. Small workloads rotate several copies so a step's weights are never
+    # still in L2 from the previous step.
+    copies = 1 if packed_bytes > 2 * L2_BYTES else -(-2 * L2_BYTES // packed_bytes)
+    packed = []
+    for p in projs:
+        P = np.empty((p.N // 4, p.K), dtype=np.uint8)
+        tq.tq_pack_host(p.w, P, p.M, p.N, p.K)
+        packed.append([torch.from_numpy(P).cuda() for _ in range(copies)])
+    w_scales = [float(p.w_scale) for p in projs]
+
+    # Activations and outputs: one contiguous buffer each, per-projection views.
+    kx = [p.M * p.K for p in projs]
+    ny = [p.M * p.N for p in projs]
+    ox = np.concatenate([[0], np.cumsum(kx)]).astype(np.int64)
+    oy = np.concatenate([[0], np.cumsum(ny)]).astype(np.int64)
+    x_host = torch.empty(int(ox[-1]), dtype=torch.int16).pin_memory()
+    for j, p in enumerate(projs):
+        x_host[ox[j]:ox[j + 1]] = torch.from_numpy(p.x_bf16.view(np.int16).reshape(-1))
+    x_dev = x_host.cuda()
+    xq = torch.empty(int(ox[-1]), dtype=torch.int8, device="cuda")
+    y_dev = torch.empty(int(oy[-1]), dtype=torch.float32, device="cuda")
+    y_host = torch.empty(int(oy[-1]), dtype=torch.float32).pin_memory()
+    moff = np.concatenate([[0], np.cumsum([p.M for p in projs])]).astype(np.int64)
+    xs = torch.empty(int(moff[-1]), dtype=torch.float32, device="cuda")
+    xsum = torch.empty(int(moff[-1]), dtype=torch.int32, device="cuda")
+
+    def table(c):
+        return [tq.make_proj(packed=packed[j][c], x=x_dev.data_ptr() + 2 * int(ox[j]),
+                             xq=xq.data_ptr() + int(ox[j]),
+                             x_scale=xs.data_ptr() + 4 * int(moff[j]),
+                             x_sum=xsum.data_ptr() + 4 * int(moff[j]),
+                             y=y_dev.data_ptr() + 4 * int(oy[j]), w_scale=w_scales[j],
+                             N=p.N, K=p.K) for j, p in enumerate(projs)]
+
+    tables = [table(c) for c in range(copies)]
+    stream = torch.cuda.current_stream()
+
+    def quant(c):
+        if stack:
+            tq.tq_quantize_act_stack(tables[c], stream=stream)
+        else:
+            for j, p in enumerate(projs):
+                t = tables[c][j]
+                tq.tq_quantize_act(t.x, t.xq, t.x_scale, t.x_sum, p.M, p.N, p.K, stream=stream)
+
+    def gemv(c):
+        if stack:
+            tq.tq_gemv_stack(tables[c], flags=tq.TQ_STACK_OVERLAP_PREV, stream=stream)
+        else:
+            for j, p in enumerate(projs):
+                t = tables[c][j]
+                call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
+                call(t.packed, t.w_scale, t.xq, t.x_scale, t.x_sum, t.y, None, p.M, p.N, p.K,
+                     stream=stream)
+
+    launches_per_step = 2 if stack else sum(1 + gemv_launches(p.M) for p in projs)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for i in range(args.warmup):
+        quant(i % copies)
+        gemv(i % copies)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        c = i % copies
+        ev[i][0].record(stream)
+        quant(c)
+        ev[i][1].record(stream)
+        gemv(c)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    gemv_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+
+    # End to end: host activations in, host outputs out, every step. At least
+    # half a second of it, so that the clock samples see the GPU under load.
+    e2e_steps = max(K, int(0.5e3 / max(total_ms / K, 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        quant(i % copies)
+        gemv(i % copies)
+        y_host.copy_(y_dev, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        quant(i % copies)
+        gemv(i % copies)
+        y_host.copy_(y_dev, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    time.sleep(0.3)
+    clk = clocks.stop()
+    assert tq.tq_device_error(reset=True) == 0, "a kernel reported a device error"
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    if rank != 0:
+        return None
+
+    ms_step = total_ms / K
+    value = world * sb / (ms_step * 1e6)
+    peak, peak_kind = measured_peak()
+    gemv_avg = statistics.mean(gemv_ms)
+    achieved = gemv_bytes / (gemv_avg * 1e6)
+    traffic = recorded_traffic(args.workload)
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8 (bf16 activations in, int8 x ternary -> int32, fp32 out)",
+        "data": "synthetic (seeded ternary weights P=0.3/0.4/0.3, bf16 N(0,1) activations "
+                "with 1% x20 outliers)",
+        "config": {
+            "workload": f"{args.workload}: {DESCRIPTIONS.get(args.workload, args.workload)}",
+            "projections": len(projs),
+            "tokens_M": M,
+            "packed_weight_bytes": packed_bytes,
+            "step_bytes": sb,
+            "weight_copies_rotated": copies,
+            "l2": ("inputs larger than L2 (weight stream > 126 MB), no flush" if copies == 1 else
+                   f"{copies} rotated weight copies, {copies * packed_bytes / 2**20:.0f} MiB > L2"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "seed": args.seed,
+        },
+        "passes_per_s": round(world * 1e3 / ms_step, 1),
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "us_per_projection": round(ms_step * 1e3 / len(projs), 4),
+        "quant_us_per_step": round(statistics.mean(quant_ms) * 1e3, 3),
+        "gemv_us_per_step": round(gemv_avg * 1e3, 3),
+        "roofline": {
+            "kernel": "stream_gemv_kernel" if stack else "per-projection kernels",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": gemv_bytes,
+        },
+        "e2e": {
+            "value": round(world * sb / (e2e_ms / e2e_steps * 1e6), 1),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+            "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
+            "ms_per_step": round(e2e_ms / e2e_steps, 5),
+        },
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+        "impl": "ours",
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(projs, args, budget_s=args.cpu_seconds)
+    return out
+
+
+def gemv_launches(M: int) -> int:
+    """Kernel launches of one tq_gemv / tq_gemm_prefill call at M tokens."""
+    return -(-M // 4)
+
+
+# ------------------------------------------------------------ CPU / oracle
+def cpu_baseline(projs, args, budget_s: float = 10.0):
+    """Time the oracle (one host thread) on whole passes over the workload's
+    projections until budget_s has elapsed (at least one pass); report GB/s
+    with the same algorithmic-byte count as the GPU arm. Prefill keeps the
+    first 16 tokens of each projection so one pass stays within seconds."""
+    import oracle
+
+    sp = projs
+    if projs[0].M > 24:
+        import copy
+        sp = []
+        for p in projs:
+            q = copy.copy(p)
+            q.M, q.x_bf16 = 16, p.x_bf16[:16]
+            sp.append(q)
+    packed = [(oracle.pack(p.w), p) for p in sp]
+    sb = step_bytes(sp)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        for P, p in packed:
+            oracle.forward(P, p.N, p.w_scale, p.x_bf16, threads=1)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": round(sb * passes / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{passes} full pass(es) of the oracle over {len(sp)} projections of "
+                      f"{args.workload} ({sb} algorithmic bytes per pass) in {el:.1f} s, "
+                      f"one thread, on {os.cpu_count()} host cores",
+            "passes_per_s": round(passes / el, 4)}
+
+
+def run_reference(args, rank: int, world: int):
+    """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
+    if rank != 0:
+        return None
+    import oracle
+
+    shapes, M = WORKLOADS[args.workload]
+    # One decoder layer's projections (or the whole workload if smaller) per step.
+    sample = shapes[:7] if len(shapes) > 7 else shapes
+    if M > 24:  # prefill: a 16-token slice per step keeps a step to seconds
+        M = 16
+    sp = list(make_projections(sample, M=M, seed=args.seed))
+    packed = [(oracle.pack(p.w), p) for p in sp]
+    sb = step_bytes(sp)
+
+    def step():
+        for P, p in packed:
+            oracle.forward(P, p.N, p.w_scale, p.x_bf16, threads=1)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    ms = el * 1e3 / args.steps
+    value = sb / (ms * 1e6)
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 (oracle: int32 accumulate, fp64 epilogue)", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {DESCRIPTIONS.get(args.workload, '')}",
+                   "sample_per_step": f"{len(sp)} projections, M={M}",
+                   "parallelism": "host, one thread"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{len(sp)} projections (M={M}) of {args.workload} per step, "
+                                   f"one thread, on {os.cpu_count()} host cores"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="stack30_m1")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_ours(args, rank, world) if args.impl == "ours" else \
+            run_reference(args, rank, world)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -5,8 +5,9 @@ in its CUDA kernels. Tensors are passed as raw pointers (``data_ptr()``), an
 ``int`` is taken as a raw pointer, ``None`` as NULL. ``stream`` defaults to
 PyTorch's current CUDA stream. A non-OK status raises :class:`TQError`.
 
-There is no fallback: if ``libtq.so`` is missing, importing this package fails.
-Build it with ``python -m ternary_absmax_int8_b200.build``.
+There is no fallback: if ``libtq.so`` is missing, every call raises (the
+package itself still imports, so that its ``build`` module can run). Build it
+with ``python -m ternary_absmax_int8_b200.build``.
 """
 from __future__ import annotations
 
@@ -23,13 +24,6 @@ __all__ = [
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libtq.so")
 
-if not os.path.exists(lib_path):
-    raise ImportError(
-        f"{lib_path} is missing: build it with `python -m ternary_absmax_int8_b200.build` "
-        "(there is no CPU fallback)")
-
-_lib = ctypes.CDLL(lib_path)
-
 TQ_STACK_OVERLAP_PREV = 1
 _STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN",
            4: "TQ_ERR_VALUE", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_UNSUPPORTED"}
@@ -40,6 +34,9 @@ class TQError(RuntimeError):
         self.status = status
         self.name = _STATUS.get(status, f"status {status}")
         super().__init__(f"{self.name}: {message}")
+
+
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 
 
 class TqProj(ctypes.Structure):
@@ -58,8 +55,7 @@ class TqProj(ctypes.Structure):
     ]
 
 
-_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-_sigs = {
+_SIGS = {
     "tq_pack_host": [_vp, _vp, _i, _i, _i, _vp],
     "tq_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "tq_gemv": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
@@ -68,14 +64,28 @@ _sigs = {
     "tq_gemv_stack": [ctypes.POINTER(TqProj), _i, ctypes.c_uint, _vp],
     "tq_device_error": [ctypes.POINTER(ctypes.c_uint32), _i],
 }
-for _name, _args in _sigs.items():
-    _fn = getattr(_lib, _name)
-    _fn.argtypes = _args
-    _fn.restype = ctypes.c_int
-_lib.tq_status_string.argtypes = [ctypes.c_int]
-_lib.tq_status_string.restype = ctypes.c_char_p
-_lib.tq_last_error.argtypes = []
-_lib.tq_last_error.restype = ctypes.c_char_p
+_lib_handle = None
+
+
+def _load():
+    """Load libtq.so once; raise loudly if it has not been built."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(
+                f"{lib_path} is missing: build it with `python -m ternary_absmax_int8_b200.build`"
+                " (there is no CPU fallback)")
+        lib = ctypes.CDLL(lib_path)
+        for name, args in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        lib.tq_status_string.argtypes = [ctypes.c_int]
+        lib.tq_status_string.restype = ctypes.c_char_p
+        lib.tq_last_error.argtypes = []
+        lib.tq_last_error.restype = ctypes.c_char_p
+        _lib_handle = lib
+    return _lib_handle
 
 
 def _ptr(t):
@@ -103,36 +113,36 @@ def _stream(stream):
 
 def _check(rc: int):
     if rc != 0:
-        raise TQError(rc, _lib.tq_last_error().decode())
+        raise TQError(rc, _load().tq_last_error().decode())
 
 
 def tq_status_string(status: int) -> str:
-    return _lib.tq_status_string(status).decode()
+    return _load().tq_status_string(status).decode()
 
 
 def tq_last_error() -> str:
-    return _lib.tq_last_error().decode()
+    return _load().tq_last_error().decode()
 
 
 def tq_pack_host(w, packed, M: int, N: int, K: int, stream=0) -> None:
     """Host packing: w int8 [N,K] (CPU tensor or numpy) -> packed uint8 [N/4,K]."""
-    _check(_lib.tq_pack_host(_ptr(w), _ptr(packed), M, N, K, None))
+    _check(_load().tq_pack_host(_ptr(w), _ptr(packed), M, N, K, None))
 
 
 def tq_quantize_act(x, xq, x_scale, x_sum, M: int, N: int, K: int, stream=None) -> None:
-    _check(_lib.tq_quantize_act(_ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, N, K,
+    _check(_load().tq_quantize_act(_ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, N, K,
                                 _stream(stream)))
 
 
 def tq_gemv(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int, K: int,
             stream=None) -> None:
-    _check(_lib.tq_gemv(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale), _ptr(x_sum),
+    _check(_load().tq_gemv(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale), _ptr(x_sum),
                         _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
 
 
 def tq_gemm_prefill(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int,
                     K: int, stream=None) -> None:
-    _check(_lib.tq_gemm_prefill(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
+    _check(_load().tq_gemm_prefill(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
                                 _ptr(x_sum), _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
 
 
@@ -149,15 +159,15 @@ def _proj_array(projs):
 
 def tq_quantize_act_stack(projs, stream=None) -> None:
     arr, n = _proj_array(projs)
-    _check(_lib.tq_quantize_act_stack(arr, n, _stream(stream)))
+    _check(_load().tq_quantize_act_stack(arr, n, _stream(stream)))
 
 
 def tq_gemv_stack(projs, flags: int = 0, stream=None) -> None:
     arr, n = _proj_array(projs)
-    _check(_lib.tq_gemv_stack(arr, n, int(flags), _stream(stream)))
+    _check(_load().tq_gemv_stack(arr, n, int(flags), _stream(stream)))
 
 
 def tq_device_error(reset: bool = False) -> int:
     code = ctypes.c_uint32(0)
-    _check(_lib.tq_device_error(ctypes.byref(code), 1 if reset else 0))
+    _check(_load().tq_device_error(ctypes.byref(code), 1 if reset else 0))
     return int(code.value)

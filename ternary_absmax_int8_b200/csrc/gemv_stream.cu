@@ -45,62 +45,64 @@ namespace tq {
 namespace {
 
 constexpr int kMaxStages = 8;
-constexpr int kWTargetBytes = 20480;  // weight bytes per tile, aim
+constexpr int kWTargetBytes = 40960;  // weight bytes per tile, aim (default)
 
 // Dynamic shared memory a CTA may use when `cps` CTAs share an SM (228 KB per
 // SM, 1 KB of it reserved per CTA).
 constexpr size_t smem_budget(int cps) { return cps == 1 ? 227 * 1024 : 112 * 1024; }
 
-__device__ __forceinline__ void dot16(const uint4 w, const uint4 x, int32_t (&a)[4])
+// Accumulators of one token: a[e][slot]. With u a packed word, byte b of u
+// is c0 + 4 c1 + 16 c2 + 64 c3 (the four planes' codes at column k + b), so
+// one dp4a each on u & 0x03030303, u & 0x0F0F0F0F, u & 0x3F3F3F3F and u
+// itself (unsigned codes x signed int8) gives the nested sums
+//   E0 = P0, E1 = P0 + 4 P1, E2 = P0 + 4 P1 + 16 P2, E3 = E2 + 64 P3,
+// with P_p = sum_k c_p q. Differences recover 4^p P_p exactly (fold). Three
+// logic ops and four dp4a per word; both share one half-rate pipe on sm_100,
+// so the fourth mask saved is 1/8 of the inner loop. Word j of a 16-byte
+// chunk goes to slot j % J, so each chunk feeds 4*J independent dp4a chains
+// (J = 4 for one token, fewer when several tokens already give independent
+// chains).
+template <int J>
+__device__ __forceinline__ void dot16(const uint4 w, const uint4 x, int32_t (&a)[4][J])
 {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        a[0] = dp4a_us(ws[j] & 0x03030303u, xs[j], a[0]);
-        a[1] = dp4a_us(ws[j] & 0x0C0C0C0Cu, xs[j], a[1]);
-        a[2] = dp4a_us(ws[j] & 0x30303030u, xs[j], a[2]);
-        a[3] = dp4a_us(ws[j] & 0xC0C0C0C0u, xs[j], a[3]);
+        const int s = j % J;
+        a[0][s] = dp4a_us(ws[j] & 0x03030303u, xs[j], a[0][s]);
+        a[1][s] = dp4a_us(ws[j] & 0x0F0F0F0Fu, xs[j], a[1][s]);
+        a[2][s] = dp4a_us(ws[j] & 0x3F3F3F3Fu, xs[j], a[2][s]);
+        a[3][s] = dp4a_us(ws[j], xs[j], a[3][s]);
     }
 }
 
-// Sum four per-lane values over the warp; lane L returns the total of value
-// (L >> 3) & 3. Six shuffles instead of twenty.
-__device__ __forceinline__ int32_t reduce4(const int32_t (&v)[4], int lane)
+// Sum the slots and turn the nested sums into out[p] = 4^p * P_p.
+template <int J>
+__device__ __forceinline__ void fold(const int32_t (&a)[4][J], int32_t (&out)[4])
 {
-    const bool hi = lane & 16;
-    int32_t k0 = hi ? v[2] : v[0], k1 = hi ? v[3] : v[1];
-    const int32_t s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
-    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    const bool b3 = lane & 8;
-    int32_t c = b3 ? k1 : k0;
-    const int32_t d = b3 ? k0 : k1;
-    c += __shfl_xor_sync(0xffffffffu, d, 8);
-    c += __shfl_xor_sync(0xffffffffu, c, 4);
-    c += __shfl_xor_sync(0xffffffffu, c, 2);
-    c += __shfl_xor_sync(0xffffffffu, c, 1);
-    return c;
+    int32_t e[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        int32_t v = a[p][0];
+#pragma unroll
+        for (int s = 1; s < J; ++s)
+            v += a[p][s];
+        e[p] = v;
+    }
+    out[0] = e[0];
+    out[1] = e[1] - e[0];
+    out[2] = e[2] - e[1];
+    out[3] = e[3] - e[2];
 }
 
-struct TileInfo {
-    int entry;
-    int row0;
-    int rows;
+// What the producer tells the consumers about the tile in a stage.
+struct StageDesc {
+    int entry;  // index into the entry table
+    int row0;   // first packed row of the tile
+    int rows;   // packed rows in the tile
+    int x_off;  // byte offset of the tile's activations inside the stage
 };
-
-template <int MaxE>
-__device__ __forceinline__ TileInfo locate(const StreamParams<MaxE> &p, int t, int &cursor)
-{
-    while (cursor + 1 < p.n_entries && p.e[cursor + 1].tile_begin <= t)
-        ++cursor;
-    const StreamEntry &e = p.e[cursor];
-    TileInfo ti;
-    ti.entry = cursor;
-    ti.row0 = (t - e.tile_begin) * e.rows_per_tile;
-    ti.rows = min(e.rows_per_tile, e.N4 - ti.row0);
-    return ti;
-}
 
 template <int MT>
 __device__ __forceinline__ float pick(const float (&a)[MT], int m)
@@ -122,31 +124,65 @@ __device__ __forceinline__ int32_t pick(const int32_t (&a)[MT], int m)
     return r;
 }
 
+// reduce4 within each 16-lane half of the warp: lane (half, sub) returns the
+// half's total of value (sub >> 2) & 3. Five shuffles serve both halves.
+__device__ __forceinline__ int32_t reduce4_half(const int32_t (&v)[4], int sub)
+{
+    const bool hi = sub & 8;
+    int32_t k0 = hi ? v[2] : v[0], k1 = hi ? v[3] : v[1];
+    const int32_t s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 8);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 8);
+    const bool b2 = sub & 4;
+    int32_t c = b2 ? k1 : k0;
+    const int32_t d = b2 ? k0 : k1;
+    c += __shfl_xor_sync(0xffffffffu, d, 4);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    return c;
+}
+
 // Shared-memory plan of one CTA (byte offsets from the dynamic base):
+//   [head_bytes]          the entry table (copied once from the launch
+//                         parameters, which are far larger than the constant
+//                         cache) and, per entry and token, w_scale * x_scale
+//                         and x_sum (loaded once the previous grid is done)
 //   [x_slot]              resident activations (one-projection launches only)
-//   [stages * stage]      the ring; a stage is [x_slot (stack launches)][w_slot]
+//   [stages * stage]      the ring; a stage holds a tile's packed rows and,
+//                         in stack launches, the projection's activations
+//   desc[8]               StageDesc per stage
 //   full[8], empty[8], xbar
 //   part[8][16][MT][4]    int32 partial sums of rows split across warps
 //   cnt[8][16]            how many warps have added into each row's partials
 template <int MT>
 struct SmemTail {
+    static constexpr int kDesc = kMaxStages * int(sizeof(StageDesc));
     static constexpr int kBars = 2 * kMaxStages + 1;
     static constexpr int kPart = kMaxStages * kStreamMaxRows * MT * 4;
     static constexpr int kCnt = kMaxStages * kStreamMaxRows;
-    static constexpr size_t bytes() { return kBars * 8 + (kPart + kCnt) * 4; }
+    static constexpr size_t bytes() { return kDesc + kBars * 8 + (kPart + kCnt) * 4; }
 };
 
-template <int W, int MaxE, int MT, int CPS>
-__global__ void __launch_bounds__((W + 1) * 32, CPS)
+// W consumer warps per group, G groups: group g consumes the CTA's tiles
+// g, g + G, ... (stages g, g + G, ...), so G tiles are worked on at once
+// while the other stages are in flight.
+template <int W, int G, int MaxE, int MT, int CPS>
+__global__ void __launch_bounds__((W * G + 1) * 32, CPS)
 stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
 {
+    constexpr int WC = W * G;  // consumer warps
     extern __shared__ __align__(128) uint8_t smem[];
     const int stages = p.stages;
-    const bool resident_x = p.n_entries == 1;
-    const int stage_bytes = (resident_x ? 0 : p.x_slot) + p.w_slot;
-    uint8_t *xres = smem;
-    uint8_t *ring = smem + (resident_x ? p.x_slot : 0);
-    uint64_t *full = reinterpret_cast<uint64_t *>(ring + stages * stage_bytes);
+    const int n_entries = p.n_entries;
+    const int total = p.total_tiles;
+    const bool resident_x = n_entries == 1;
+    const int stage_bytes = p.w_slot;
+    StreamEntry *tab = reinterpret_cast<StreamEntry *>(smem);
+    float2 *scl = reinterpret_cast<float2 *>(smem + n_entries * sizeof(StreamEntry));
+    uint8_t *xres = smem + p.head_bytes;
+    uint8_t *ring = xres + (resident_x ? p.x_slot : 0);
+    StageDesc *desc = reinterpret_cast<StageDesc *>(ring + stages * stage_bytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(desc + kMaxStages);
     uint64_t *empty = full + kMaxStages;
     uint64_t *xbar = empty + kMaxStages;
     int32_t *part = reinterpret_cast<int32_t *>(xbar + 1);
@@ -156,6 +192,14 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
 
     for (int i = threadIdx.x; i < SmemTail<MT>::kPart + SmemTail<MT>::kCnt; i += blockDim.x)
         part[i] = 0;
+    {
+        static_assert(sizeof(StreamEntry) % 8 == 0, "entry size");
+        const uint64_t *src = reinterpret_cast<const uint64_t *>(&p.e[0]);
+        uint64_t *dst = reinterpret_cast<uint64_t *>(tab);
+        const int n64 = n_entries * int(sizeof(StreamEntry) / 8);
+        for (int i = threadIdx.x; i < n64; i += blockDim.x)
+            dst[i] = src[i];
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
@@ -166,158 +210,194 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
     }
     __syncthreads();
 
-    if (warp == W) {
+    if (warp == WC) {
         // ------------------------------------------------------ producer
         if (lane != 0)
             return;
         const uint64_t pol_w = policy_evict_first();  // weights: read once
         const uint64_t pol_x = policy_evict_last();   // activations: reread by many CTAs
+        const uint32_t xbytes_m = uint32_t(p.M);
         bool waited = !p.overlap_prev;
         if (waited)
             pdl_wait();
         if (resident_x && waited) {
-            const StreamEntry &e = p.e[0];
-            mbar_arrive_expect_tx(xbar, uint32_t(p.M * e.K));
-            bulk_g2s(xres, e.xq, uint32_t(p.M * e.K), xbar, pol_x);
+            mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
+            bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
         }
-        int deferred[kMaxStages];
-        int n_def = 0;
-        int cursor = 0, it = 0;
-        for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
-            const TileInfo ti = locate(p, t, cursor);
-            const StreamEntry &e = p.e[ti.entry];
-            const int stage = it % stages;
-            const int use = it / stages;
+        int cursor = 0, it = 0, stage = 0;
+        uint32_t phase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            while (cursor + 1 < n_entries && tab[cursor + 1].tile_begin <= t)
+                ++cursor;
+            const StreamEntry &e = tab[cursor];
+            const int K = e.K;
+            const int row0 = (t - e.tile_begin) * e.rows_per_tile;
+            const int rows = min(e.rows_per_tile, e.N4 - row0);
             if (!waited && it == stages) {
                 // The ring is full of weight copies issued before the
                 // previous grid finished; activations may be read now.
                 pdl_wait();
                 waited = true;
                 if (resident_x) {
-                    mbar_arrive_expect_tx(xbar, uint32_t(p.M * e.K));
-                    bulk_g2s(xres, e.xq, uint32_t(p.M * e.K), xbar, pol_x);
+                    mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
+                    bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
                 } else {
-                    for (int d = 0; d < n_def; ++d) {
-                        const StreamEntry &ed = p.e[deferred[d]];
-                        bulk_g2s(ring + d * stage_bytes, ed.xq, uint32_t(p.M * ed.K), &full[d],
-                                 pol_x);
+                    for (int d = 0; d < stages; ++d) {
+                        const StageDesc dd = desc[d];
+                        const StreamEntry &ed = tab[dd.entry];
+                        bulk_g2s(ring + d * stage_bytes + dd.x_off, ed.xq, xbytes_m * ed.K,
+                                 &full[d], pol_x);
                     }
                 }
             }
-            if (use > 0 && !mbar_wait(&empty[stage], uint32_t((use - 1) & 1), p.err))
+            if (it >= stages && !mbar_wait(&empty[stage], phase ^ 1u, p.err))
                 break;
+            const uint32_t wbytes = uint32_t(rows) * uint32_t(K);
+            const uint32_t xbytes = resident_x ? 0u : xbytes_m * K;
+            desc[stage] = StageDesc{cursor, row0, rows, int(wbytes)};
             uint8_t *st = ring + stage * stage_bytes;
-            const uint32_t wbytes = uint32_t(ti.rows) * uint32_t(e.K);
-            const uint32_t xbytes = resident_x ? 0u : uint32_t(p.M * e.K);
             mbar_arrive_expect_tx(&full[stage], wbytes + xbytes);
-            bulk_g2s(st + (resident_x ? 0 : p.x_slot), e.packed + size_t(ti.row0) * e.K, wbytes,
-                     &full[stage], pol_w);
-            if (!resident_x) {
-                if (waited)
-                    bulk_g2s(st, e.xq, xbytes, &full[stage], pol_x);
-                else
-                    deferred[n_def++] = ti.entry;
+            bulk_g2s(st, e.packed + size_t(row0) * K, wbytes, &full[stage], pol_w);
+            if (!resident_x && waited)
+                bulk_g2s(st + wbytes, e.xq, xbytes, &full[stage], pol_x);
+            if (++stage == stages) {
+                stage = 0;
+                phase ^= 1u;
             }
         }
         if (!waited) {
-            // Issue the activation copies still owed, even after a failed
-            // wait, so that every stage barrier can complete.
+            // Issue the activation copies still owed (also after a failed
+            // wait, so that every stage barrier can complete).
             pdl_wait();
             if (resident_x) {
-                const StreamEntry &e = p.e[0];
-                mbar_arrive_expect_tx(xbar, uint32_t(p.M * e.K));
-                bulk_g2s(xres, e.xq, uint32_t(p.M * e.K), xbar, pol_x);
+                mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
+                bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
             } else {
-                for (int d = 0; d < n_def; ++d) {
-                    const StreamEntry &ed = p.e[deferred[d]];
-                    bulk_g2s(ring + d * stage_bytes, ed.xq, uint32_t(p.M * ed.K), &full[d], pol_x);
+                const int owed = min(it, stages);
+                for (int d = 0; d < owed; ++d) {
+                    const StageDesc dd = desc[d];
+                    const StreamEntry &ed = tab[dd.entry];
+                    bulk_g2s(ring + d * stage_bytes + dd.x_off, ed.xq, xbytes_m * ed.K, &full[d],
+                             pol_x);
                 }
             }
         }
         // Do not let the CTA retire while a copy this thread issued is in
-        // flight (matters only when a wait gave up).
-        const int used = min(it, stages);
-        for (int s = 0; s < used; ++s)
-            mbar_wait(&full[s], uint32_t(((it - 1 - s) / stages) & 1), p.err);
-        if (resident_x && used > 0)
+        // flight (matters only when a wait gave up). Stage s was last used
+        // in this round (parity phase) if s < stage, else in the previous one.
+        for (int s = 0; s < stages; ++s) {
+            if (s < stage)
+                mbar_wait(&full[s], phase, p.err);
+            else if (it >= stages)
+                mbar_wait(&full[s], phase ^ 1u, p.err);
+        }
+        if (resident_x && it > 0)
             mbar_wait(xbar, 0, p.err);
         return;
     }
 
     // ---------------------------------------------------------- consumers
-    // Each consumer warp walks the ring on its own (no CTA barrier): it waits
-    // for a stage, takes items warp, warp + W, ... of that tile, and releases
-    // the stage. A row split over several warps is finished by whichever warp
-    // adds the last partial sum.
+    // Each consumer warp walks the ring on its own (no CTA barrier in the
+    // loop): it waits for a stage, takes items warp, warp + W, ... of that
+    // tile, and releases the stage. A row split over several warps is
+    // finished by whichever warp adds the last partial sum.
     pdl_wait();  // x_scale and x_sum are read below
-    if (resident_x && p.total_tiles > int(blockIdx.x) && !mbar_wait_warp(xbar, 0, p.err))
+    for (int i = threadIdx.x; i < n_entries * p.M; i += WC * 32) {
+        const int j = i / p.M, m = i - j * p.M;
+        const StreamEntry &e = tab[j];
+        scl[j * MT + m] = make_float2(__fmul_rn(e.w_scale, __ldg(e.x_scale + m)),
+                                      __int_as_float(__ldg(e.x_sum + m)));
+    }
+    named_bar_sync(1, WC * 32);
+    if (resident_x && total > int(blockIdx.x) && !mbar_wait_warp(xbar, 0, p.err))
         return;
 
-    int cursor = 0, it = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
-        const TileInfo ti = locate(p, t, cursor);
-        const StreamEntry &e = p.e[ti.entry];
-        const int stage = it % stages;
-        const int use = it / stages;
-
-        // Epilogue scales, fetched before the wait so their latency hides.
+    const int grp = warp / W, wg = warp - grp * W;
+    int stage = grp;  // stages % G == 0, so the group keeps to stages grp + k*G
+    uint32_t phase = 0;
+    for (int t = blockIdx.x + grp * gridDim.x; t < total; t += G * gridDim.x) {
+        if (!mbar_wait_warp(&full[stage], phase, p.err))
+            return;
+        const StageDesc d = desc[stage];
+        const StreamEntry &e = tab[d.entry];
+        const int K = e.K;
+        const int C = K >> 4;
+        const int lg = e.ksplit;  // log2 of the pieces per row
+        const int N4 = e.N4;
+        const int N = N4 * 4;
+        float *const y = e.y;
+        int32_t *const acc_out = e.acc_out;
         float tsc[MT];
         int32_t xsm[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            tsc[m] = 0.0f;
-            xsm[m] = 0;
-            if (m < p.M) {
-                tsc[m] = __fmul_rn(e.w_scale, __ldg(e.x_scale + m));
-                xsm[m] = __ldg(e.x_sum + m);
-            }
+            const float2 v = scl[d.entry * MT + m];
+            tsc[m] = v.x;
+            xsm[m] = __float_as_int(v.y);
         }
 
-        if (!mbar_wait_warp(&full[stage], uint32_t(use & 1), p.err))
-            return;
-
-        const uint8_t *st = ring + stage * stage_bytes;
-        const uint8_t *sx = resident_x ? xres : st;
-        const uint8_t *sw = resident_x ? st : st + p.x_slot;
-        const int K = e.K;
-        const int C = K >> 4;
-        const int ks = e.ksplit;
-        const int N = e.N4 * 4;
-        const int n_items = ti.rows * ks;
-        for (int item = warp; item < n_items; item += W) {
-            const int r = item / ks;
-            const int piece = item - r * ks;
-            const int c0 = (piece * C) / ks, c1 = ((piece + 1) * C) / ks;
+        const uint8_t *sw = ring + stage * stage_bytes;
+        const uint8_t *sx = resident_x ? xres : sw + d.x_off;
+        // A work item is a pair of rows (half-warp each, 16 lanes per row)
+        // times one of 2^lg pieces of K.
+        const int half = lane >> 4, sub = lane & 15;
+        const int n_items = ((d.rows + 1) >> 1) << lg;
+        bool released = false;
+        for (int item = wg; item < n_items; item += W) {
+            const int pr = item >> lg;
+            const int piece = item & ((1 << lg) - 1);
+            const int r = 2 * pr + half;
+            const bool valid = r < d.rows;
+            const int c0 = (piece * C) >> lg;
+            const int c1 = valid ? ((piece + 1) * C) >> lg : c0;
             const uint4 *wrow = reinterpret_cast<const uint4 *>(sw + size_t(r) * K);
-            int32_t a[MT][4];
+            constexpr int J = 4 / MT;
+            int32_t a[MT][4][J];
 #pragma unroll
             for (int m = 0; m < MT; ++m)
-                a[m][0] = a[m][1] = a[m][2] = a[m][3] = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int s2 = 0; s2 < J; ++s2)
+                        a[m][q][s2] = 0;
 #pragma unroll 4
-            for (int c = c0 + lane; c < c1; c += 32) {
+            for (int c = c0 + sub; c < c1; c += 16) {
                 const uint4 wv = wrow[c];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (m < p.M) {
                         const uint4 xv = reinterpret_cast<const uint4 *>(sx + m * K)[c];
-                        dot16(wv, xv, a[m]);
+                        dot16<J>(wv, xv, a[m]);
                     }
                 }
             }
-            const int row = ti.row0 + r;
-            if (ks == 1) {
-                // Whole row in this warp: lanes 0, 8, 16, 24 write planes 0..3.
+            if (lg == 0 && item + W >= n_items) {
+                // This warp's last whole-row item of the tile: its shared
+                // memory is no longer read (the partial-sum slots are used
+                // only by split rows), so hand the stage back before the
+                // reduction and epilogue.
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[stage]);
+                released = true;
+            }
+            const int row = d.row0 + r;
+            if (lg == 0) {
+                // Whole rows in this warp: in each half, sub 0, 4, 8, 12 write
+                // planes 0..3 of that half's row.
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (m < p.M) {
-                        const int32_t v = reduce4(a[m], lane);
-                        if ((lane & 7) == 0) {
-                            const int plane = lane >> 3;
+                        int32_t f[4];
+                        fold<J>(a[m], f);
+                        const int32_t v = reduce4_half(f, sub);
+                        if (valid && (sub & 3) == 0) {
+                            const int plane = sub >> 2;
                             const int32_t acc = (v >> (2 * plane)) - xsm[m];
-                            const size_t o = size_t(m) * N + row + plane * e.N4;
-                            e.y[o] = __fmul_rn(__int2float_rn(acc), tsc[m]);
-                            if (e.acc_out)
-                                e.acc_out[o] = acc;
+                            const size_t o = size_t(m) * N + row + plane * N4;
+                            y[o] = __fmul_rn(__int2float_rn(acc), tsc[m]);
+                            if (acc_out)
+                                acc_out[o] = acc;
                         }
                     }
                 }
@@ -326,44 +406,52 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (m < p.M) {
-                        const int32_t v = reduce4(a[m], lane);
-                        if ((lane & 7) == 0)
-                            atomicAdd(&slot[m * 4 + (lane >> 3)], v);
+                        int32_t f[4];
+                        fold<J>(a[m], f);
+                        const int32_t v = reduce4_half(f, sub);
+                        if (valid && (sub & 3) == 0)
+                            atomicAdd(&slot[m * 4 + (sub >> 2)], v);
                     }
                 }
                 __threadfence_block();  // partial sums before the count
                 __syncwarp();
                 int old = 0;
                 if (lane == 0)
-                    old = atomicAdd(&cnt[stage * kStreamMaxRows + r], 1);
+                    old = atomicAdd(&cnt[stage * kStreamMaxRows + pr], 1);
                 old = __shfl_sync(0xffffffffu, old, 0);
-                if (old == ks - 1) {
+                if (old == (1 << lg) - 1) {
+                    // Last piece of this pair: finish both rows.
                     __threadfence_block();
-                    if (lane < 4 * p.M) {
-                        const int m = lane >> 2, plane = lane & 3;
+                    if (valid && sub < 4 * p.M) {
+                        const int m = sub >> 2, plane = sub & 3;
                         const int32_t v = atomicExch(&slot[m * 4 + plane], 0);
                         const int32_t acc = (v >> (2 * plane)) - pick(xsm, m);
-                        const size_t o = size_t(m) * N + row + plane * e.N4;
-                        e.y[o] = __fmul_rn(__int2float_rn(acc), pick(tsc, m));
-                        if (e.acc_out)
-                            e.acc_out[o] = acc;
+                        const size_t o = size_t(m) * N + row + plane * N4;
+                        y[o] = __fmul_rn(__int2float_rn(acc), pick(tsc, m));
+                        if (acc_out)
+                            acc_out[o] = acc;
                     }
                     if (lane == 0)
-                        cnt[stage * kStreamMaxRows + r] = 0;
+                        cnt[stage * kStreamMaxRows + pr] = 0;
                 }
             }
         }
         __syncwarp();
-        if (lane == 0)
+        if (lane == 0 && !released)
             mbar_arrive(&empty[stage]);
+        stage += G;
+        if (stage >= stages) {
+            stage -= stages;
+            phase ^= 1u;
+        }
     }
 }
 
-template <int W, int MaxE, int MT, int CPS>
+template <int W, int G, int MaxE, int MT, int CPS>
 cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, bool pdl,
                             cudaStream_t stream)
 {
-    auto kern = stream_gemv_kernel<W, MaxE, MT, CPS>;
+    auto kern = stream_gemv_kernel<W, G, MaxE, MT, CPS>;
     static int configured_dev = -1;  // per instantiation
     int dev = 0;
     cudaGetDevice(&dev);
@@ -376,7 +464,7 @@ cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, 
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3((W + 1) * 32);
+    cfg.blockDim = dim3((W * G + 1) * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -390,11 +478,14 @@ cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, 
     return cudaGetLastError();
 }
 
-// Tuning knobs: consumer warps per CTA and CTAs per SM. TQ_STREAM_CFG="W,CPS"
-// picks another instantiated variant (for measurement); default 8,1.
+// Tuning knobs: warps per consumer group, groups, CTAs per SM and the tile
+// size aim. TQ_STREAM_CFG="W,G,CPS[,tile_bytes]" picks another instantiated
+// variant (for measurement).
 struct StreamCfg {
     int W = 8;
+    int G = 1;
     int CPS = 1;
+    int tile = kWTargetBytes;
 };
 
 StreamCfg stream_cfg()
@@ -402,13 +493,19 @@ StreamCfg stream_cfg()
     static StreamCfg cfg = [] {
         StreamCfg c;
         if (const char *s = getenv("TQ_STREAM_CFG")) {
-            int w = 0, cps = 0;
-            if (sscanf(s, "%d,%d", &w, &cps) == 2 &&
-                ((w == 8 && (cps == 1 || cps == 2)) || (w == 16 && cps == 1) ||
-                 (w == 4 && cps == 2))) {
+            int w = 0, g = 0, cps = 0, tile = 0;
+            const int n = sscanf(s, "%d,%d,%d,%d", &w, &g, &cps, &tile);
+            const bool known = (w == 8 && g == 1 && (cps == 1 || cps == 2)) ||
+                               (w == 8 && g == 2 && cps == 1) || (w == 4 && g == 2 && cps == 1) ||
+                               (w == 4 && g == 4 && cps == 1) || (w == 4 && g == 2 && cps == 2) ||
+                               (w == 4 && g == 1 && cps == 2);
+            if (n >= 3 && known) {
                 c.W = w;
+                c.G = g;
                 c.CPS = cps;
             }
+            if (n == 4 && tile >= 4096 && tile <= 65536)
+                c.tile = tile;
         }
         return c;
     }();
@@ -419,13 +516,19 @@ template <int MaxE, int MT>
 cudaError_t launch_variant(const StreamCfg &c, const StreamParams<MaxE> &p, int grid, size_t smem,
                            bool pdl, cudaStream_t stream)
 {
-    if (c.W == 8 && c.CPS == 2)
-        return launch_instance<8, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    if (c.W == 16)
-        return launch_instance<16, MaxE, MT, 1>(p, grid, smem, pdl, stream);
-    if (c.W == 4)
-        return launch_instance<4, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    return launch_instance<8, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.W == 8 && c.G == 1 && c.CPS == 2)
+        return launch_instance<8, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
+    if (c.W == 8 && c.G == 2)
+        return launch_instance<8, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.W == 4 && c.G == 2 && c.CPS == 1)
+        return launch_instance<4, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.W == 4 && c.G == 4)
+        return launch_instance<4, 4, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.W == 4 && c.G == 2 && c.CPS == 2)
+        return launch_instance<4, 2, MaxE, MT, 2>(p, grid, smem, pdl, stream);
+    if (c.W == 4 && c.G == 1)
+        return launch_instance<4, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
+    return launch_instance<8, 1, MaxE, MT, 1>(p, grid, smem, pdl, stream);
 }
 
 template <int MaxE>
@@ -437,51 +540,54 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     const StreamCfg cfg = stream_cfg();
     const int sms = device_sm_count();
     const int W = cfg.W;
-    int total = 0, kmax = 0, wmax = 0;
+    const bool resident = n == 1;
+    int total = 0, kmax = 0, stage_max = 0;
     for (int j = 0; j < n; ++j) {
         StreamEntry &e = entries[j];
         const int K = e.K;
         int R = kStreamMaxRows;
-        while (R > 1 && R * K > kWTargetBytes)
+        while (R > 1 && R * K > cfg.tile)
             R >>= 1;
         if (single)
             while (R > 1 && (e.N4 + R - 1) / R < 2 * sms * cfg.CPS)
                 R >>= 1;
+        // pieces per row pair: enough items for every warp, each piece >= 16 chunks
         const int C = K >> 4;
-        int ks = std::max(1, W / R);
-        ks = std::min(ks, std::max(1, C / 16));
+        int lg = 0;
+        while ((((R + 1) >> 1) << lg) < W && (C >> (lg + 1)) >= 16)
+            ++lg;
         e.rows_per_tile = R;
-        e.ksplit = ks;
+        e.ksplit = lg;
         e.tile_begin = total;
         total += (e.N4 + R - 1) / R;
         kmax = std::max(kmax, K);
-        wmax = std::max(wmax, R * K);
+        stage_max = std::max(stage_max, R * K + (resident ? 0 : M * K));
         p.e[j] = e;
     }
     p.n_entries = n;
     p.total_tiles = total;
     p.M = M;
-    p.x_slot = (M * kmax + 127) / 128 * 128;
-    p.w_slot = (wmax + 127) / 128 * 128;
+    p.x_slot = resident ? (M * kmax + 127) / 128 * 128 : 0;
+    p.w_slot = (stage_max + 127) / 128 * 128;
     p.overlap_prev = overlap_prev ? 1 : 0;
+    const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
+    p.head_bytes = int((n * sizeof(StreamEntry) + size_t(n) * mt * sizeof(float2) + 127) / 128 * 128);
     p.err = device_error_word();
     if (!p.err)
         return cudaErrorUnknown;
-    const bool resident = n == 1;
-    const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
     const size_t tail = mt == 1 ? SmemTail<1>::bytes()
                                 : (mt == 2 ? SmemTail<2>::bytes() : SmemTail<4>::bytes());
-    const size_t fixed = tail + (resident ? p.x_slot : 0);
-    const int stage_bytes = (resident ? 0 : p.x_slot) + p.w_slot;
+    const size_t fixed = tail + p.head_bytes + p.x_slot;
     const size_t budget = smem_budget(cfg.CPS);
-    int stages = budget > fixed ? int((budget - fixed) / size_t(stage_bytes)) : 0;
+    int stages = budget > fixed ? int((budget - fixed) / size_t(p.w_slot)) : 0;
     stages = std::min(stages, kMaxStages);
+    stages -= stages % cfg.G;  // each consumer group keeps to its own stages
     if (total == 0)
         return cudaSuccess;
-    if (stages < 2)
+    if (stages < 2 * cfg.G)
         return cudaErrorInvalidValue;
     p.stages = stages;
-    const size_t smem = fixed + size_t(stages) * stage_bytes;
+    const size_t smem = fixed + size_t(stages) * p.w_slot;
     const int grid = std::min(total, sms * cfg.CPS);
     switch (mt) {
     case 1: return launch_variant<MaxE, 1>(cfg, p, grid, smem, overlap_prev, stream);

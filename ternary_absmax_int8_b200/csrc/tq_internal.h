@@ -35,8 +35,8 @@ cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream);
 // One entry = one projection. The projection's packed rows are cut into
 // tiles of `rows_per_tile` consecutive packed rows (a contiguous byte range);
 // global tile t of the launch belongs to the entry with the largest
-// tile_begin <= t. Each row of a tile is cut into `ksplit` pieces along K,
-// so that rows_per_tile * ksplit work items keep every consumer warp busy.
+// tile_begin <= t. Each row of a tile is cut into 2^ksplit pieces along K,
+// so that rows_per_tile << ksplit work items keep every consumer warp busy.
 struct StreamEntry {
     const uint8_t *packed;  // [N4, K]
     const int8_t *xq;       // [M, K]
@@ -48,7 +48,7 @@ struct StreamEntry {
     int N4;
     int K;
     int rows_per_tile;
-    int ksplit;
+    int ksplit;             // log2 of the pieces each row is cut into along K
     int tile_begin;
 };
 
@@ -61,11 +61,11 @@ struct StreamParams {
     int n_entries;
     int total_tiles;
     int M;             // tokens, 1..kStreamMaxTokens
-    int x_slot;        // bytes of a stage reserved for activations (>= M * K of every entry)
-    int w_slot;        // bytes of a stage reserved for weights (>= rows_per_tile * K)
+    int x_slot;        // bytes of resident activations (one-entry launches), else 0
+    int w_slot;        // bytes of a ring stage (a tile's packed rows + activations)
     int stages;
     int overlap_prev;  // start weight copies before the previous grid completes
-    int pad_;
+    int head_bytes;    // shared memory for the entry table and the per-token scales
     unsigned *err;     // the library's device error word
     StreamEntry e[MaxE];
 };
