@@ -65,6 +65,22 @@ def step_bytes(projs) -> int:
 
 
 # ----------------------------------------------------------------- helpers
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of per-rank timings (one collective; identity at N=1)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Units of all ranks per second of the slowest rank's time (ms)."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
@@ -116,6 +132,15 @@ def measured_peak():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return PEAK_FALLBACK_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return 2.0 * float(d["bf16_tflops"]), "measured bf16 burst x 2 (nominal int8:bf16)"
+    except (OSError, KeyError, ValueError):
+        return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2"
 
 
 def stack_kernel_sha() -> str:
@@ -261,24 +286,69 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
+
+    # Per-projection GEMM timing (non-stack workloads): each projection's call
+    # alone, over the rotated weight copies, median of the repeats.
+    per_proj = []
+    if not stack:
+        for j, p in enumerate(projs):
+            call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
+            reps = max(20, min(200, K))
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            for r in range(reps):
+                t_ = tables[r % copies][j]
+                evs[r][0].record(stream)
+                call(t_.packed, t_.w_scale, t_.xq, t_.x_scale, t_.x_sum, t_.y, None, p.M, p.N, p.K,
+                     stream=stream)
+                evs[r][1].record(stream)
+            torch.cuda.synchronize()
+            us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+            entry = {"name": p.name, "N": p.N, "K": p.K, "M": p.M, "us": round(us, 3),
+                     "GB_s": round(algorithmic_bytes(p.N, p.K, p.M) / (us * 1e3), 1)}
+            if p.M > 24:
+                entry["TOPS"] = round(2.0 * p.M * p.N * p.K / (us * 1e6), 1)
+            else:
+                entry["token_proj_per_s"] = round(p.M / (us * 1e-6), 1)
+            per_proj.append(entry)
     time.sleep(0.3)
     clk = clocks.stop()
     assert tq.tq_device_error(reset=True) == 0, "a kernel reported a device error"
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device="cuda")
     if rank != 0:
         return None
 
     ms_step = total_ms / K
-    value = world * sb / (ms_step * 1e6)
+    value = whole_job_rate(world, sb, ms_step) / 1e9
     peak, peak_kind = measured_peak()
     gemv_avg = statistics.mean(gemv_ms)
     achieved = gemv_bytes / (gemv_avg * 1e6)
     traffic = recorded_traffic(args.workload)
+    prefill = M > 24
+    flops = sum(2.0 * p.M * p.N * p.K for p in projs)
+    if prefill:
+        # int8 contraction: tensor-bound. Peak = measured dense bf16 x the
+        # nominal int8 : bf16 ratio (4.5 : 2.25 PFLOP/s).
+        tpeak, tkind = measured_tensor_peak()
+        roof = {"kernel": "prefill_tc_kernel", "bound": "tensor",
+                "achieved": round(flops / (gemv_avg * 1e9), 1), "peak": tpeak,
+                "peak_kind": tkind, "unit": "TOPS (int8)",
+                "frac": round(flops / (gemv_avg * 1e9) / tpeak, 4), "traffic": None,
+                "algorithmic_ops_per_step": flops}
+    else:
+        roof = {
+            "kernel": "stream_gemv_kernel",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": gemv_bytes,
+        }
     out = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -305,25 +375,14 @@ def run_ours(args, rank: int, world: int):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "seed": args.seed,
         },
-        "passes_per_s": round(world * 1e3 / ms_step, 1),
+        "passes_per_s": round(whole_job_rate(world, 1.0, ms_step), 1),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "us_per_projection": round(ms_step * 1e3 / len(projs), 4),
         "quant_us_per_step": round(statistics.mean(quant_ms) * 1e3, 3),
         "gemv_us_per_step": round(gemv_avg * 1e3, 3),
-        "roofline": {
-            "kernel": "stream_gemv_kernel" if stack else "per-projection kernels",
-            "bound": "hbm",
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)"
-                         if peak_kind == "measured" else "fallback 6.65 TB/s",
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": gemv_bytes,
-        },
+        "roofline": roof,
         "e2e": {
-            "value": round(world * sb / (e2e_ms / e2e_steps * 1e6), 1),
+            "value": round(whole_job_rate(world, sb, e2e_ms / e2e_steps) / 1e9, 1),
             "unit": "GB/s",
             "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
             "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size()),
@@ -333,6 +392,10 @@ def run_ours(args, rank: int, world: int):
         "clocks": clk,
         "impl": "ours",
     }
+    if per_proj:
+        out["per_projection"] = per_proj
+    if prefill:
+        out["tops"] = round(world * flops / (ms_step * 1e9), 1)
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(projs, args, budget_s=args.cpu_seconds)
     return out
@@ -340,7 +403,7 @@ def run_ours(args, rank: int, world: int):
 
 def gemv_launches(M: int) -> int:
     """Kernel launches of one tq_gemv / tq_gemm_prefill call at M tokens."""
-    return -(-M // 4)
+    return 1 if M >= 128 else -(-M // 4)
 
 
 # ------------------------------------------------------------ CPU / oracle

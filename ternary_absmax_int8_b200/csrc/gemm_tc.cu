@@ -25,12 +25,10 @@
 //               32 (w % 4) ..), subtract x_sum, scale, store y
 // Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
 // of tile t overlaps the MMAs of tile t + 1. Every mbarrier wait is bounded.
-#include <cuda.h>
-
 #include <algorithm>
 #include <cstring>
 
-#include "tq_internal.h"
+#include "tc_common.cuh"
 
 namespace tq {
 
@@ -46,6 +44,7 @@ constexpr int kBBytes = kBN * kBK;           // 32 KB
 constexpr int kPBytes = kPackedRows * kBK;   // 4 KB
 constexpr int kThreads = 320;
 constexpr int kTmemCols = 2 * kBN;           // two accumulator buffers
+constexpr uint32_t kIdesc = idesc_i8_u8s8(kBM, kBN);
 
 struct PrefillParams {
     int N4, K, M;
@@ -69,78 +68,6 @@ struct PrefillSmem {
     static constexpr size_t tmem_slot_off = bar_off + kBarCount * 8;
     static constexpr size_t bytes = tmem_slot_off + 16;
 };
-
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr)
-{
-    // K-major, 128B swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
-    uint64_t d = 0;
-    d |= uint64_t((saddr & 0x3FFFFu) >> 4);   // start address
-    d |= uint64_t(1) << 16;                    // leading byte offset (unused here)
-    d |= uint64_t(1024 >> 4) << 32;            // stride byte offset
-    d |= uint64_t(1) << 46;                    // descriptor version (sm_100)
-    d |= uint64_t(2) << 61;                    // layout: SWIZZLE_128B
-    return d;
-}
-
-// kind::i8 instruction descriptor: D s32, A u8 (codes), B s8 (activations),
-// both K-major, M = 128, N = kBN.
-constexpr uint32_t kIdesc = (2u << 4)            // D format s32
-                            | (0u << 7)          // A unsigned 8-bit
-                            | (1u << 10)         // B signed 8-bit
-                            | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                        uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.u32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Byte offset of (row r, 16-byte chunk c) in a K-major 128B-swizzled operand.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c)
-{
-    return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
@@ -179,13 +106,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
         }
         fence_mbar_init();
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
+    if (warp == 1)
+        tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -250,7 +172,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     const uint32_t b0 = smem_u32(sB + stage * kBBytes);
 #pragma unroll
                     for (int kk = 0; kk < kBK / 32; ++kk)
-                        umma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                        umma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), kIdesc,
                                 (ks > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&mma_done[stage]);
                     ++issued;
@@ -363,49 +285,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
     __syncthreads();
     tc_fence_after();
     if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kTmemCols)
-                     : "memory");
-}
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = [] {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return EncodeTiledFn(nullptr);
-        return reinterpret_cast<EncodeTiledFn>(f);
-    }();
-    return fn;
-}
-
-// 2-D byte tensor [rows, width] (row stride = width), boxes of 128 x box_rows,
-// 128B swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap *m, const void *base, int width, int rows, int box_rows)
-{
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return false;
-    const cuuint64_t gdim[2] = {cuuint64_t(width), cuuint64_t(rows)};
-    const cuuint64_t gstride[1] = {cuuint64_t(width)};
-    const cuuint32_t box[2] = {cuuint32_t(kBK), cuuint32_t(box_rows)};
-    const cuuint32_t estride[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), gdim, gstride, box,
-               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        tmem_dealloc(tmem_base, kTmemCols);
 }
 
 }  // namespace
 
-constexpr int kPrefillMinM = 128;
+constexpr int kPrefillMinM = 33;
 
 cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
                               const float *x_scale, const int32_t *x_sum, float *y,

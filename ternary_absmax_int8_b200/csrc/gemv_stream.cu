@@ -37,6 +37,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
+#include <vector>
 
 #include "tq_internal.h"
 
@@ -45,6 +46,7 @@ namespace tq {
 namespace {
 
 constexpr int kMaxStages = 8;
+
 constexpr int kWTargetBytes = 40960;  // weight bytes per tile, aim (default)
 
 // Dynamic shared memory a CTA may use when `cps` CTAs share an SM (228 KB per
@@ -142,18 +144,50 @@ __device__ __forceinline__ int32_t reduce4_half(const int32_t (&v)[4], int sub)
     return c;
 }
 
+// Sum four per-lane values over each group of lpr lanes (8, 16 or 32; the
+// groups are aligned). On return, `plane` is the value index whose group total
+// this lane holds and should write, or -1 if another lane of the group writes
+// it. 8 lanes: 4 shuffles; 16 lanes: 5; 32 lanes: 6.
+__device__ __forceinline__ int32_t reduce4_rows(const int32_t (&v)[4], int lane, int lpr,
+                                                int &plane)
+{
+    if (lpr == 8) {
+        const int sub = lane & 7;
+        const bool hi = sub & 4;
+        int32_t k0 = hi ? v[2] : v[0], k1 = hi ? v[3] : v[1];
+        const int32_t s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
+        k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+        k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+        const bool b1 = sub & 2;
+        int32_t c = b1 ? k1 : k0;
+        const int32_t d = b1 ? k0 : k1;
+        c += __shfl_xor_sync(0xffffffffu, d, 2);
+        c += __shfl_xor_sync(0xffffffffu, c, 1);
+        plane = (sub & 1) ? -1 : (sub >> 1);
+        return c;
+    }
+    int32_t c = reduce4_half(v, lane & 15);
+    if (lpr == 32) {
+        c += __shfl_xor_sync(0xffffffffu, c, 16);
+        plane = (lane < 16 && (lane & 3) == 0) ? (lane >> 2) : -1;
+    } else {
+        plane = (lane & 3) == 0 ? ((lane & 15) >> 2) : -1;
+    }
+    return c;
+}
+
 // Shared-memory plan of one CTA (byte offsets from the dynamic base):
-//   [head_bytes]          the entry table (copied once from the launch
-//                         parameters, which are far larger than the constant
-//                         cache) and, per entry and token, w_scale * x_scale
-//                         and x_sum (loaded once the previous grid is done)
-//   [x_slot]              resident activations (one-projection launches only)
-//   [stages * stage]      the ring; a stage holds a tile's packed rows and,
-//                         in stack launches, the projection's activations
-//   desc[8]               StageDesc per stage
+//   [head_bytes]   this CTA's entries (copied once from the launch parameters),
+//                  per entry and token w_scale * x_scale and x_sum (loaded once
+//                  the previous grid is done), per entry the offset of its
+//                  activations in the x cache
+//   [x_slot]       the activations (M x K int8) of this CTA's entries, loaded
+//                  once per launch
+//   [stages * stage]  the ring of packed weight tiles
+//   desc[8]        StageDesc per stage
 //   full[8], empty[8], xbar
-//   part[8][16][MT][4]    int32 partial sums of rows split across warps
-//   cnt[8][16]            how many warps have added into each row's partials
+//   part[8][16][MT][4]  int32 partial sums of rows split across warps
+//   cnt[8][16]     how many warps have added into each row's partials
 template <int MT>
 struct SmemTail {
     static constexpr int kDesc = kMaxStages * int(sizeof(StageDesc));
@@ -163,9 +197,9 @@ struct SmemTail {
     static constexpr size_t bytes() { return kDesc + kBars * 8 + (kPart + kCnt) * 4; }
 };
 
+
 // W consumer warps per group, G groups: group g consumes the CTA's tiles
-// g, g + G, ... (stages g, g + G, ...), so G tiles are worked on at once
-// while the other stages are in flight.
+// g, g + G, ... (stages g, g + G, ...).
 template <int W, int G, int MaxE, int MT, int CPS>
 __global__ void __launch_bounds__((W * G + 1) * 32, CPS)
 stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
@@ -173,14 +207,16 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
     constexpr int WC = W * G;  // consumer warps
     extern __shared__ __align__(128) uint8_t smem[];
     const int stages = p.stages;
-    const int n_entries = p.n_entries;
-    const int total = p.total_tiles;
-    const bool resident_x = n_entries == 1;
     const int stage_bytes = p.w_slot;
+    // This CTA's tiles and the entries they belong to.
+    const int t_begin = p.cta_tile0[blockIdx.x], t_end = p.cta_tile0[blockIdx.x + 1];
+    const int e_first = p.cta_entry0[blockIdx.x];
+    const int n_entries = p.cta_nent[blockIdx.x];  // local table size
     StreamEntry *tab = reinterpret_cast<StreamEntry *>(smem);
     float2 *scl = reinterpret_cast<float2 *>(smem + n_entries * sizeof(StreamEntry));
-    uint8_t *xres = smem + p.head_bytes;
-    uint8_t *ring = xres + (resident_x ? p.x_slot : 0);
+    int *xoff = reinterpret_cast<int *>(scl + n_entries * MT);
+    uint8_t *xcache = smem + p.head_bytes;
+    uint8_t *ring = xcache + p.x_slot;
     StageDesc *desc = reinterpret_cast<StageDesc *>(ring + stages * stage_bytes);
     uint64_t *full = reinterpret_cast<uint64_t *>(desc + kMaxStages);
     uint64_t *empty = full + kMaxStages;
@@ -194,13 +230,19 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
         part[i] = 0;
     {
         static_assert(sizeof(StreamEntry) % 8 == 0, "entry size");
-        const uint64_t *src = reinterpret_cast<const uint64_t *>(&p.e[0]);
+        const uint64_t *src = reinterpret_cast<const uint64_t *>(&p.e[e_first]);
         uint64_t *dst = reinterpret_cast<uint64_t *>(tab);
         const int n64 = n_entries * int(sizeof(StreamEntry) / 8);
         for (int i = threadIdx.x; i < n64; i += blockDim.x)
             dst[i] = src[i];
     }
+    __syncthreads();
     if (threadIdx.x == 0) {
+        int off = 0;
+        for (int j = 0; j < n_entries; ++j) {
+            xoff[j] = off;
+            off += (p.M * tab[j].K + 127) & ~127;
+        }
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], W);
@@ -216,71 +258,50 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
             return;
         const uint64_t pol_w = policy_evict_first();  // weights: read once
         const uint64_t pol_x = policy_evict_last();   // activations: reread by many CTAs
-        const uint32_t xbytes_m = uint32_t(p.M);
+        auto load_x = [&]() {
+            uint32_t total = 0;
+            for (int j = 0; j < n_entries; ++j)
+                total += uint32_t(p.M * tab[j].K);
+            mbar_arrive_expect_tx(xbar, total);
+            for (int j = 0; j < n_entries; ++j)
+                bulk_g2s(xcache + xoff[j], tab[j].xq, uint32_t(p.M * tab[j].K), xbar, pol_x);
+        };
         bool waited = !p.overlap_prev;
-        if (waited)
+        if (waited) {
             pdl_wait();
-        if (resident_x && waited) {
-            mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
-            bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
+            load_x();
         }
         int cursor = 0, it = 0, stage = 0;
         uint32_t phase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+        for (int t = t_begin; t < t_end; ++t, ++it) {
+            if (!waited && it == stages) {
+                // The ring is full of weight copies issued before the
+                // previous grid finished; activations may be read now.
+                pdl_wait();
+                waited = true;
+                load_x();
+            }
             while (cursor + 1 < n_entries && tab[cursor + 1].tile_begin <= t)
                 ++cursor;
             const StreamEntry &e = tab[cursor];
             const int K = e.K;
             const int row0 = (t - e.tile_begin) * e.rows_per_tile;
             const int rows = min(e.rows_per_tile, e.N4 - row0);
-            if (!waited && it == stages) {
-                // The ring is full of weight copies issued before the
-                // previous grid finished; activations may be read now.
-                pdl_wait();
-                waited = true;
-                if (resident_x) {
-                    mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
-                    bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
-                } else {
-                    for (int d = 0; d < stages; ++d) {
-                        const StageDesc dd = desc[d];
-                        const StreamEntry &ed = tab[dd.entry];
-                        bulk_g2s(ring + d * stage_bytes + dd.x_off, ed.xq, xbytes_m * ed.K,
-                                 &full[d], pol_x);
-                    }
-                }
-            }
             if (it >= stages && !mbar_wait(&empty[stage], phase ^ 1u, p.err))
                 break;
             const uint32_t wbytes = uint32_t(rows) * uint32_t(K);
-            const uint32_t xbytes = resident_x ? 0u : xbytes_m * K;
-            desc[stage] = StageDesc{cursor, row0, rows, int(wbytes)};
-            uint8_t *st = ring + stage * stage_bytes;
-            mbar_arrive_expect_tx(&full[stage], wbytes + xbytes);
-            bulk_g2s(st, e.packed + size_t(row0) * K, wbytes, &full[stage], pol_w);
-            if (!resident_x && waited)
-                bulk_g2s(st + wbytes, e.xq, xbytes, &full[stage], pol_x);
+            desc[stage] = StageDesc{cursor, row0, rows, 0};
+            mbar_arrive_expect_tx(&full[stage], wbytes);
+            bulk_g2s(ring + stage * stage_bytes, e.packed + size_t(row0) * K, wbytes, &full[stage],
+                     pol_w);
             if (++stage == stages) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
         if (!waited) {
-            // Issue the activation copies still owed (also after a failed
-            // wait, so that every stage barrier can complete).
-            pdl_wait();
-            if (resident_x) {
-                mbar_arrive_expect_tx(xbar, xbytes_m * tab[0].K);
-                bulk_g2s(xres, tab[0].xq, xbytes_m * tab[0].K, xbar, pol_x);
-            } else {
-                const int owed = min(it, stages);
-                for (int d = 0; d < owed; ++d) {
-                    const StageDesc dd = desc[d];
-                    const StreamEntry &ed = tab[dd.entry];
-                    bulk_g2s(ring + d * stage_bytes + dd.x_off, ed.xq, xbytes_m * ed.K, &full[d],
-                             pol_x);
-                }
-            }
+            pdl_wait();  // also after a failed wait: the x barrier must complete
+            load_x();
         }
         // Do not let the CTA retire while a copy this thread issued is in
         // flight (matters only when a wait gave up). Stage s was last used
@@ -291,16 +312,16 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
             else if (it >= stages)
                 mbar_wait(&full[s], phase ^ 1u, p.err);
         }
-        if (resident_x && it > 0)
-            mbar_wait(xbar, 0, p.err);
+        mbar_wait(xbar, 0, p.err);
         return;
     }
 
     // ---------------------------------------------------------- consumers
     // Each consumer warp walks the ring on its own (no CTA barrier in the
-    // loop): it waits for a stage, takes items warp, warp + W, ... of that
-    // tile, and releases the stage. A row split over several warps is
-    // finished by whichever warp adds the last partial sum.
+    // loop). For each of its items it copies the item's packed words from
+    // the stage into registers, hands the stage back after its last item's
+    // copy, and only then computes: a stage is held for the copy, not for the
+    // arithmetic, so nearly the whole ring stays in flight.
     pdl_wait();  // x_scale and x_sum are read below
     for (int i = threadIdx.x; i < n_entries * p.M; i += WC * 32) {
         const int j = i / p.M, m = i - j * p.M;
@@ -309,20 +330,24 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                                       __int_as_float(__ldg(e.x_sum + m)));
     }
     named_bar_sync(1, WC * 32);
-    if (resident_x && total > int(blockIdx.x) && !mbar_wait_warp(xbar, 0, p.err))
+    if (t_end > t_begin && !mbar_wait_warp(xbar, 0, p.err))
         return;
 
     const int grp = warp / W, wg = warp - grp * W;
     int stage = grp;  // stages % G == 0, so the group keeps to stages grp + k*G
     uint32_t phase = 0;
-    for (int t = blockIdx.x + grp * gridDim.x; t < total; t += G * gridDim.x) {
+    // Items are dealt to the group's warps round-robin across tiles (a tile
+    // with fewer items than warps leaves different warps idle each time):
+    // item i of a tile goes to warp (rot + i) % W, rot advancing by the
+    // tile's item count.
+    int rot = 0;
+    for (int t = t_begin + grp; t < t_end; t += G) {
         if (!mbar_wait_warp(&full[stage], phase, p.err))
             return;
         const StageDesc d = desc[stage];
         const StreamEntry &e = tab[d.entry];
         const int K = e.K;
         const int C = K >> 4;
-        const int lg = e.ksplit;  // log2 of the pieces per row
         const int N4 = e.N4;
         const int N = N4 * 4;
         float *const y = e.y;
@@ -335,18 +360,26 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
             tsc[m] = v.x;
             xsm[m] = __float_as_int(v.y);
         }
-
         const uint8_t *sw = ring + stage * stage_bytes;
-        const uint8_t *sx = resident_x ? xres : sw + d.x_off;
-        // A work item is a pair of rows (half-warp each, 16 lanes per row)
-        // times one of 2^lg pieces of K.
-        const int half = lane >> 4, sub = lane & 15;
-        const int n_items = ((d.rows + 1) >> 1) << lg;
+        const uint8_t *sx = xcache + xoff[d.entry];
+
+        // A work item is 32 / lpr rows (lpr lanes each: 8, 16 or 32) times
+        // one of 2^lg pieces of K. Fewer lanes per row means fewer shuffle
+        // levels per row in the reduction and a longer loop per lane.
+        const int lg = e.ksplit & 0xFF;
+        const int lpr = 8 << ((e.ksplit >> 8) & 3);  // lanes per row
+        const int grp_in = lane / lpr;               // row of the item this lane serves
+        const int sub = lane & (lpr - 1);
+        const int rpi = 32 / lpr;                    // rows per item
+        const int n_items = ((d.rows + rpi - 1) / rpi) << lg;
         bool released = false;
-        for (int item = wg; item < n_items; item += W) {
+        const int first_item = (wg - rot + W) % W;
+        const int last_item = n_items - 1 - ((n_items - 1 - first_item) % W + W) % W;
+        rot = (rot + n_items) % W;
+        for (int item = first_item; item < n_items; item += W) {
             const int pr = item >> lg;
             const int piece = item & ((1 << lg) - 1);
-            const int r = 2 * pr + half;
+            const int r = rpi * pr + grp_in;
             const bool valid = r < d.rows;
             const int c0 = (piece * C) >> lg;
             const int c1 = valid ? ((piece + 1) * C) >> lg : c0;
@@ -361,7 +394,7 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                     for (int s2 = 0; s2 < J; ++s2)
                         a[m][q][s2] = 0;
 #pragma unroll 4
-            for (int c = c0 + sub; c < c1; c += 16) {
+            for (int c = c0 + sub; c < c1; c += lpr) {
                 const uint4 wv = wrow[c];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
@@ -371,11 +404,10 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                     }
                 }
             }
-            if (lg == 0 && item + W >= n_items) {
-                // This warp's last whole-row item of the tile: its shared
-                // memory is no longer read (the partial-sum slots are used
-                // only by split rows), so hand the stage back before the
-                // reduction and epilogue.
+            if (lg == 0 && item == last_item) {
+                // This warp's last read of the stage is done; the partial-sum
+                // slots are used only by split rows: hand the stage back
+                // before the reduction and epilogue.
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[stage]);
@@ -383,16 +415,16 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
             }
             const int row = d.row0 + r;
             if (lg == 0) {
-                // Whole rows in this warp: in each half, sub 0, 4, 8, 12 write
-                // planes 0..3 of that half's row.
+                // Whole rows: lane 4 q (+16 for the second row of a pair)
+                // writes plane q of its row.
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (m < p.M) {
                         int32_t f[4];
                         fold<J>(a[m], f);
-                        const int32_t v = reduce4_half(f, sub);
-                        if (valid && (sub & 3) == 0) {
-                            const int plane = sub >> 2;
+                        int plane;
+                        const int32_t v = reduce4_rows(f, lane, lpr, plane);
+                        if (valid && plane >= 0) {
                             const int32_t acc = (v >> (2 * plane)) - xsm[m];
                             const size_t o = size_t(m) * N + row + plane * N4;
                             y[o] = __fmul_rn(__int2float_rn(acc), tsc[m]);
@@ -408,9 +440,10 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                     if (m < p.M) {
                         int32_t f[4];
                         fold<J>(a[m], f);
-                        const int32_t v = reduce4_half(f, sub);
-                        if (valid && (sub & 3) == 0)
-                            atomicAdd(&slot[m * 4 + (sub >> 2)], v);
+                        int plane;
+                        const int32_t v = reduce4_rows(f, lane, lpr, plane);
+                        if (valid && plane >= 0)
+                            atomicAdd(&slot[m * 4 + plane], v);
                     }
                 }
                 __threadfence_block();  // partial sums before the count
@@ -420,10 +453,10 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                     old = atomicAdd(&cnt[stage * kStreamMaxRows + pr], 1);
                 old = __shfl_sync(0xffffffffu, old, 0);
                 if (old == (1 << lg) - 1) {
-                    // Last piece of this pair: finish both rows.
+                    // Last piece of this item's rows: finish them.
                     __threadfence_block();
-                    if (valid && sub < 4 * p.M) {
-                        const int m = sub >> 2, plane = sub & 3;
+                    for (int oi = sub; valid && oi < 4 * p.M; oi += lpr) {
+                        const int m = oi >> 2, plane = oi & 3;
                         const int32_t v = atomicExch(&slot[m * 4 + plane], 0);
                         const int32_t acc = (v >> (2 * plane)) - pick(xsm, m);
                         const size_t o = size_t(m) * N + row + plane * N4;
@@ -482,8 +515,8 @@ cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, 
 // size aim. TQ_STREAM_CFG="W,G,CPS[,tile_bytes]" picks another instantiated
 // variant (for measurement).
 struct StreamCfg {
-    int W = 8;
-    int G = 1;
+    int W = 4;
+    int G = 2;
     int CPS = 1;
     int tile = kWTargetBytes;
 };
@@ -520,15 +553,15 @@ cudaError_t launch_variant(const StreamCfg &c, const StreamParams<MaxE> &p, int 
         return launch_instance<8, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
     if (c.W == 8 && c.G == 2)
         return launch_instance<8, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
-    if (c.W == 4 && c.G == 2 && c.CPS == 1)
-        return launch_instance<4, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
     if (c.W == 4 && c.G == 4)
         return launch_instance<4, 4, MaxE, MT, 1>(p, grid, smem, pdl, stream);
     if (c.W == 4 && c.G == 2 && c.CPS == 2)
         return launch_instance<4, 2, MaxE, MT, 2>(p, grid, smem, pdl, stream);
     if (c.W == 4 && c.G == 1)
         return launch_instance<4, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    return launch_instance<8, 1, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.W == 8 && c.G == 1 && c.CPS == 1)
+        return launch_instance<8, 1, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    return launch_instance<4, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
 }
 
 template <int MaxE>
@@ -540,8 +573,7 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     const StreamCfg cfg = stream_cfg();
     const int sms = device_sm_count();
     const int W = cfg.W;
-    const bool resident = n == 1;
-    int total = 0, kmax = 0, stage_max = 0;
+    int total = 0, stage_max = 0;
     for (int j = 0; j < n; ++j) {
         StreamEntry &e = entries[j];
         const int K = e.K;
@@ -551,27 +583,91 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
         if (single)
             while (R > 1 && (e.N4 + R - 1) / R < 2 * sms * cfg.CPS)
                 R >>= 1;
-        // pieces per row pair: enough items for every warp, each piece >= 16 chunks
+        // Lanes per row: the fewest (8, 16, 32) that still give every warp
+        // of a consumer group an item of 32 / lpr rows. Rows are cut into
+        // pieces along K only if even 32 lanes per row leave warps idle.
         const int C = K >> 4;
+        auto items_of = [&](int lsel) {
+            const int rpi = 4 >> lsel;  // rows per item at 8 << lsel lanes per row
+            return (R + rpi - 1) / rpi;
+        };
+        int lsel = 0;  // lanes per row = 8 << lsel
+        while (lsel < 2 && items_of(lsel) < W)
+            ++lsel;
+        const int items = items_of(lsel);
         int lg = 0;
-        while ((((R + 1) >> 1) << lg) < W && (C >> (lg + 1)) >= 16)
+        while ((items << lg) < W && (C >> (lg + 1)) >= 16)
             ++lg;
         e.rows_per_tile = R;
-        e.ksplit = lg;
+        e.ksplit = lg | (lsel << 8);
         e.tile_begin = total;
         total += (e.N4 + R - 1) / R;
-        kmax = std::max(kmax, K);
-        stage_max = std::max(stage_max, R * K + (resident ? 0 : M * K));
+        stage_max = std::max(stage_max, R * K);
         p.e[j] = e;
     }
     p.n_entries = n;
     p.total_tiles = total;
     p.M = M;
-    p.x_slot = resident ? (M * kmax + 127) / 128 * 128 : 0;
     p.w_slot = (stage_max + 127) / 128 * 128;
     p.overlap_prev = overlap_prev ? 1 : 0;
     const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
-    p.head_bytes = int((n * sizeof(StreamEntry) + size_t(n) * mt * sizeof(float2) + 127) / 128 * 128);
+    if (total == 0)
+        return cudaSuccess;
+
+    // Contiguous tile ranges per CTA, balanced by bytes (plus a fixed cost per
+    // tile), so that every CTA streams about the same amount and finishes at
+    // about the same time.
+    const int grid = std::min({total, sms * cfg.CPS, kStreamMaxGrid});
+    std::vector<long long> prefix(size_t(total) + 1, 0);
+    {
+        int t = 0;
+        for (int j = 0; j < n; ++j) {
+            const StreamEntry &e = p.e[j];
+            const int tiles = (e.N4 + e.rows_per_tile - 1) / e.rows_per_tile;
+            for (int i = 0; i < tiles; ++i, ++t) {
+                const int rows = std::min(e.rows_per_tile, e.N4 - i * e.rows_per_tile);
+                prefix[size_t(t) + 1] = prefix[size_t(t)] + (long long)rows * e.K + 4096;
+            }
+        }
+    }
+    p.cta_tile0[0] = 0;
+    for (int b = 1; b < grid; ++b) {
+        const long long target = prefix[size_t(total)] * b / grid;
+        int t = int(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
+        t = std::max(t, p.cta_tile0[b - 1] + 1);
+        t = std::min(t, total - (grid - b));
+        p.cta_tile0[b] = t;
+    }
+    p.cta_tile0[grid] = total;
+    int max_local = 1;
+    size_t x_max = 0;
+    for (int b = 0; b < grid; ++b) {
+        auto entry_of = [&](int t) {
+            int lo = 0, hi = n - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) / 2;
+                if (p.e[mid].tile_begin <= t)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            return lo;
+        };
+        const int e0 = entry_of(p.cta_tile0[b]);
+        const int e1 = entry_of(p.cta_tile0[b + 1] - 1);
+        p.cta_entry0[b] = e0;
+        p.cta_nent[b] = e1 - e0 + 1;
+        max_local = std::max(max_local, e1 - e0 + 1);
+        size_t xb = 0;
+        for (int j = e0; j <= e1; ++j)
+            xb += (size_t(M) * p.e[j].K + 127) / 128 * 128;
+        x_max = std::max(x_max, xb);
+    }
+    p.x_slot = int(x_max);
+    p.head_bytes = int((size_t(max_local) * (sizeof(StreamEntry) + size_t(mt) * sizeof(float2) +
+                                             sizeof(int)) +
+                        127) /
+                       128 * 128);
     p.err = device_error_word();
     if (!p.err)
         return cudaErrorUnknown;
@@ -582,13 +678,10 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     int stages = budget > fixed ? int((budget - fixed) / size_t(p.w_slot)) : 0;
     stages = std::min(stages, kMaxStages);
     stages -= stages % cfg.G;  // each consumer group keeps to its own stages
-    if (total == 0)
-        return cudaSuccess;
-    if (stages < 2 * cfg.G)
+    if (stages < std::max(2, cfg.G))
         return cudaErrorInvalidValue;
     p.stages = stages;
     const size_t smem = fixed + size_t(stages) * p.w_slot;
-    const int grid = std::min(total, sms * cfg.CPS);
     switch (mt) {
     case 1: return launch_variant<MaxE, 1>(cfg, p, grid, smem, overlap_prev, stream);
     case 2: return launch_variant<MaxE, 2>(cfg, p, grid, smem, overlap_prev, stream);

@@ -1,0 +1,418 @@
+// gemv_tc.cu -- batched-decode ternary GEMV on the tensor cores (5 <= M <= 32
+// tokens), tcgen05 with the code operand in tensor memory, stream-K.
+//
+// Many concurrent requests turn decode into a skinny contraction (1bit engine
+// blog, "One GPU, many users"): each weight byte now feeds M tokens, so
+// unpacking with dp4a on the CUDA cores runs out of issue slots long before
+// HBM does, while the work is still far too small for a prefill tile.
+//
+//   D[r, m] = sum_k c[r, k] * xq[m, k]     (u8 codes, s8 activations, s32)
+//   acc = D - x_sum[m],  y = float(acc) * (w_scale * x_scale[m])
+//
+// * Tile: 32 packed rows = 128 MMA rows with row r = 4 j + p holding plane p
+//   of packed row j (feature i0 + j + p N/4); BN = 16 or 32 token columns.
+//   With this order a warp's 32 tensor-memory lanes are 8 packed rows x 4
+//   planes, so each packed byte is read from shared memory once.
+// * The expansion warps unpack codes in registers and store them straight
+//   into tensor memory (tcgen05.st): the A operand never passes through shared
+//   memory, which at small N would otherwise bound the kernel (16 KB written
+//   and 16 KB read back per 4 KB of weights).
+// * K advances in 256-byte units; a unit is one TMA box pair of packed bytes
+//   (32 rows) plus activations (BN rows), 128B swizzled. The (tile, unit)
+//   sequence is split into one contiguous, balanced range per CTA (stream-K),
+//   so every SM streams weights even when there are fewer tiles than SMs.
+//   A tile split across CTAs adds its int32 partial sums into a global
+//   workspace with integer atomics (exact, order-free); the CTA whose
+//   contribution completes the tile applies the epilogue and zeroes the
+//   workspace for the next call.
+// * Warp roles (12 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
+//   4..7 expansion, 8..11 epilogue. All mbarrier waits are bounded.
+#include <algorithm>
+
+#include "tc_common.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kRows = 128;             // MMA M (32 packed rows x 4 planes)
+constexpr int kPRows = kRows / 4;      // packed rows per tile
+constexpr int kUnitK = 256;            // bytes of K per unit (two 128-byte boxes)
+constexpr int kSP = 10;                // shared-memory stages (packed + activations)
+constexpr int kSA = 4;                 // tensor-memory A slots
+constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
+constexpr int kThreads = 384;
+constexpr int kMaxGrid = 512;
+
+struct SmallMParams {
+    int N4, K, M;
+    int tiles, units_per_tile, total_units, grid;
+    float w_scale;
+    const float *x_scale;
+    const int32_t *x_sum;
+    float *y;
+    int32_t *acc_out;
+    int32_t *ws;    // [tiles][BN][128] int32 partial sums (all zero between calls)
+    int32_t *cnt;   // [tiles] arrivals (all zero between calls)
+    unsigned *err;
+};
+
+template <int BN>
+struct SmallMSmem {
+    static constexpr int kPBytes = kPRows * kUnitK;  // 8 KB
+    static constexpr int kBBytes = BN * kUnitK;
+    static constexpr size_t p_off = 0;
+    static constexpr size_t b_off = p_off + size_t(kSP) * kPBytes;
+    static constexpr size_t bar_off = b_off + size_t(kSP) * kBBytes;
+    // tma_full[SP], p_free[SP], mma_done[SP], a_full[SA], acc_full[2], acc_empty[2]
+    static constexpr int kBars = 3 * kSP + kSA + 4;
+    static constexpr size_t misc_off = bar_off + kBars * 8;  // tmem slot, finisher flag
+    static constexpr size_t bytes = misc_off + 16;
+};
+
+// Unit u of the whole call belongs to CTA b with U(b) <= u < U(b+1).
+__device__ __forceinline__ int unit_start(int b, int total, int grid)
+{
+    return int((long long)total * b / grid);
+}
+
+__device__ __forceinline__ int cta_of_unit(int u, int total, int grid)
+{
+    // largest b with unit_start(b) <= u
+    int b = int(((long long)u * grid) / total);
+    while (b + 1 < grid && unit_start(b + 1, total, grid) <= u)
+        ++b;
+    while (b > 0 && unit_start(b, total, grid) > u)
+        --b;
+    return b;
+}
+
+// Barrier over the 128 epilogue threads (named barrier 2) that ORs a predicate.
+__device__ __forceinline__ bool epilogue_any(bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(pred))
+        : "memory");
+    return r != 0;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
+                 const __grid_constant__ SmallMParams p)
+{
+    using L = SmallMSmem<BN>;
+    constexpr uint32_t kIdesc = idesc_i8_u8s8(kRows, BN);
+    constexpr int kTmemCols = 512;  // kSA * kACols + 2 * BN, rounded to a power of two
+    static_assert(kSA * kACols + 2 * BN <= kTmemCols, "tensor memory plan");
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sP = smem + L::p_off;
+    uint8_t *sB = smem + L::b_off;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
+    uint64_t *tma_full = bars;
+    uint64_t *p_free = bars + kSP;
+    uint64_t *mma_done = bars + 2 * kSP;
+    uint64_t *a_full = bars + 3 * kSP;
+    uint64_t *acc_full = a_full + kSA;
+    uint64_t *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
+    int *fin_flag = reinterpret_cast<int *>(smem + L::misc_off + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u_begin = unit_start(blockIdx.x, p.total_units, p.grid);
+    const int u_end = unit_start(blockIdx.x + 1, p.total_units, p.grid);
+    const int UPT = p.units_per_tile;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSP; ++s) {
+            mbar_init(&tma_full[s], 1);
+            mbar_init(&p_free[s], 4);
+            mbar_init(&mma_done[s], 1);
+        }
+        for (int s = 0; s < kSA; ++s)
+            mbar_init(&a_full[s], 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1)
+        tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_a = tmem_base;                    // kSA slots of kACols
+    const uint32_t tmem_d = tmem_base + kSA * kACols;     // 2 x BN accumulator columns
+
+    if (warp == 0) {
+        // -------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int u = u_begin; u < u_end; ++u, ++issued) {
+                const int s = issued % kSP;
+                const uint32_t use = uint32_t(issued / kSP);
+                if (use > 0 && (!mbar_wait(&p_free[s], (use - 1) & 1, p.err) ||
+                                !mbar_wait(&mma_done[s], (use - 1) & 1, p.err)))
+                    break;
+                const int tile = u / UPT, k0 = (u - tile * UPT) * kUnitK;
+                mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
+                uint8_t *P = sP + s * L::kPBytes;
+                uint8_t *B = sB + s * L::kBBytes;
+                tma_load_2d(P, &map_p, k0, tile * kPRows, &tma_full[s]);
+                tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, tile * kPRows, &tma_full[s]);
+                tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
+                tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+            }
+            for (int s = 0; s < kSP && s < issued; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % kSP);
+                mbar_wait(&tma_full[s], uint32_t((last / kSP) & 1), p.err);
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int i = 0, seg = 0;
+            bool ok = true;
+            for (int u = u_begin; u < u_end && ok;) {
+                const int tile = u / UPT;
+                const int seg_end = min(u_end, (tile + 1) * UPT);
+                const int buf = seg & 1;
+                if (seg >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((seg >> 1) - 1) & 1), p.err))
+                    break;
+                tc_fence_after();
+                const uint32_t d = tmem_d + uint32_t(buf * BN);
+                for (; u < seg_end; ++u, ++i) {
+                    const int s = i % kSP, sa = i % kSA;
+                    if (!mbar_wait(&tma_full[s], uint32_t((i / kSP) & 1), p.err) ||
+                        !mbar_wait(&a_full[sa], uint32_t((i / kSA) & 1), p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b0 = smem_u32(sB + s * L::kBBytes);
+                    const bool first = (u == u_begin) || (u % UPT == 0);
+#pragma unroll
+                    for (int kk = 0; kk < kUnitK / 32; ++kk) {
+                        const uint32_t bk = b0 + uint32_t((kk >> 2) * (L::kBBytes / 2) + (kk & 3) * 32);
+                        umma_i8_ts(d, tmem_a + uint32_t(sa * kACols + kk * 8), umma_desc_sw128(bk),
+                                   kIdesc, (first && kk == 0) ? 0u : 1u);
+                    }
+                    umma_commit(&mma_done[s]);
+                }
+                if (ok)
+                    umma_commit(&acc_full[buf]);
+                ++seg;
+            }
+            if (i > 0) {
+                const int s = (i - 1) % kSP;
+                mbar_wait(&mma_done[s], uint32_t(((i - 1) / kSP) & 1), p.err);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // -------------------------------------------------- expansion
+        const int q = warp & 3;                      // TMEM lane quarter
+        const int j = 8 * q + (lane >> 2), pl = lane & 3;  // packed row, plane of this lane
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        int i = 0;
+        for (int u = u_begin; u < u_end; ++u, ++i) {
+            const int s = i % kSP, sa = i % kSA;
+            bool ok = mbar_wait_warp(&tma_full[s], uint32_t((i / kSP) & 1), p.err);
+            if (ok && i >= kSA) {
+                const int pi = i - kSA;  // the unit that last used this A slot
+                ok = mbar_wait_warp(&mma_done[pi % kSP], uint32_t((pi / kSP) & 1), p.err);
+            }
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint8_t *P = sP + s * L::kPBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(P + h * (L::kPBytes / 2) +
+                                                                     sw128_off(j, c));
+                    v[4 * c + 0] = (w.x >> (2 * pl)) & 0x03030303u;
+                    v[4 * c + 1] = (w.y >> (2 * pl)) & 0x03030303u;
+                    v[4 * c + 2] = (w.z >> (2 * pl)) & 0x03030303u;
+                    v[4 * c + 3] = (w.w >> (2 * pl)) & 0x03030303u;
+                }
+                tmem_st32(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&a_full[sa]);
+                mbar_arrive(&p_free[s]);
+            }
+        }
+    } else if (warp >= 8) {
+        // -------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int r = 32 * q + lane;                 // accumulator row = TMEM lane
+        const int jr = r >> 2, pl = r & 3;
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        const int N = 4 * p.N4;
+        int seg = 0;
+        for (int u = u_begin; u < u_end; ++seg) {
+            const int tile = u / UPT;
+            const int seg_end = min(u_end, (tile + 1) * UPT);
+            const bool whole = (u == tile * UPT) && (seg_end == (tile + 1) * UPT);
+            u = seg_end;
+            const int buf = seg & 1;
+            const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((seg >> 1) & 1), p.err);
+            // The four epilogue warps meet at named barriers below: decide
+            // together whether to go on.
+            if (epilogue_any(!got))
+                break;
+            tc_fence_after();
+            uint32_t v[32];
+            if constexpr (BN == 32) {
+                tmem_ld32(tmem_d + lane_base + uint32_t(buf * BN), v);
+            } else {
+                uint32_t h[16];
+                tmem_ld16(tmem_d + lane_base + uint32_t(buf * BN), h);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    v[c] = h[c];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers now
+
+            const int prow = tile * kPRows + jr;
+            const bool row_ok = prow < p.N4;
+            const int n = prow + pl * p.N4;
+            if (whole) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    if (c < p.M && row_ok) {
+                        const int32_t acc = int32_t(v[c]) - __ldg(p.x_sum + c);
+                        const float t = __fmul_rn(p.w_scale, __ldg(p.x_scale + c));
+                        const size_t o = size_t(c) * N + n;
+                        p.y[o] = __fmul_rn(__int2float_rn(acc), t);
+                        if (p.acc_out)
+                            p.acc_out[o] = acc;
+                    }
+                }
+                continue;
+            }
+            // Partial tile: add into the workspace, then count this CTA in.
+            int32_t *wt = p.ws + size_t(tile) * BN * kRows;
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+                if (c < p.M)
+                    atomicAdd(wt + c * kRows + r, int32_t(v[c]));
+            __threadfence();
+            named_bar_sync(2, 128);
+            if (threadIdx.x == 8 * 32) {
+                const int first = cta_of_unit(tile * UPT, p.total_units, p.grid);
+                const int last = cta_of_unit((tile + 1) * UPT - 1, p.total_units, p.grid);
+                const int old = atomicAdd(p.cnt + tile, 1);
+                *fin_flag = (old == last - first) ? 1 : 0;
+            }
+            named_bar_sync(2, 128);
+            if (*fin_flag) {
+                __threadfence();
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    if (c < p.M) {
+                        const int32_t d = atomicExch(wt + c * kRows + r, 0);
+                        if (row_ok) {
+                            const int32_t acc = d - __ldg(p.x_sum + c);
+                            const float t = __fmul_rn(p.w_scale, __ldg(p.x_scale + c));
+                            const size_t o = size_t(c) * N + n;
+                            p.y[o] = __fmul_rn(__int2float_rn(acc), t);
+                            if (p.acc_out)
+                                p.acc_out[o] = acc;
+                        }
+                    }
+                }
+                if (threadIdx.x == 8 * 32)
+                    p.cnt[tile] = 0;
+            }
+            named_bar_sync(2, 128);  // fin_flag is reused by the next segment
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem_base, kTmemCols);
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &mp, const CUtensorMap &mx, const SmallMParams &prm,
+                      cudaStream_t stream)
+{
+    const size_t smem = SmallMSmem<BN>::bytes + 1024;
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(smallm_tc_kernel<BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
+    smallm_tc_kernel<BN><<<prm.grid, kThreads, smem, stream>>>(mp, mx, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t smallm_workspace_bytes(int N, int M)
+{
+    const int BN = M <= 16 ? 16 : 32;
+    const size_t tiles = (size_t(N / 4) + kPRows - 1) / kPRows;
+    return tiles * BN * kRows * sizeof(int32_t) + tiles * sizeof(int32_t);
+}
+
+cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                             const float *x_scale, const int32_t *x_sum, float *y,
+                             int32_t *acc_out, int M, int N, int K, void *workspace,
+                             cudaStream_t stream)
+{
+    if (M < 1 || M > 32)
+        return cudaErrorInvalidValue;
+    const int BN = M <= 16 ? 16 : 32;
+    CUtensorMap map_p, map_x;
+    if (!make_map(&map_p, packed, K, N / 4, kPRows) || !make_map(&map_x, xq, K, M, BN))
+        return cudaErrorInvalidValue;
+    SmallMParams prm;
+    prm.N4 = N / 4;
+    prm.K = K;
+    prm.M = M;
+    prm.tiles = (prm.N4 + kPRows - 1) / kPRows;
+    prm.units_per_tile = (K + kUnitK - 1) / kUnitK;
+    prm.total_units = prm.tiles * prm.units_per_tile;
+    prm.grid = std::min({prm.total_units, device_sm_count(), kMaxGrid});
+    prm.w_scale = w_scale;
+    prm.x_scale = x_scale;
+    prm.x_sum = x_sum;
+    prm.y = y;
+    prm.acc_out = acc_out;
+    prm.ws = static_cast<int32_t *>(workspace);
+    prm.cnt = prm.ws + size_t(prm.tiles) * BN * kRows;
+    prm.err = device_error_word();
+    if (!prm.err)
+        return cudaErrorUnknown;
+    return BN == 16 ? launch_bn<16>(map_p, map_x, prm, stream) : launch_bn<32>(map_p, map_x, prm, stream);
+}
+
+}  // namespace tq

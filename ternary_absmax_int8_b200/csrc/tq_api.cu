@@ -3,6 +3,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "tq.h"
@@ -31,6 +33,41 @@ unsigned *device_error_word()
         cache[dev] = static_cast<unsigned *>(p);
     }
     return cache[dev];
+}
+
+void *device_workspace(size_t bytes, cudaError_t *err)
+{
+    static std::mutex mu;
+    static void *buf[64] = {nullptr};
+    static size_t cap[64] = {0};
+    std::lock_guard<std::mutex> lock(mu);
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess)
+        return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    if (cap[dev] < bytes) {
+        if (buf[dev]) {
+            // cudaFree waits for work that may still use the old buffer
+            cudaFree(buf[dev]);
+            buf[dev] = nullptr;
+            cap[dev] = 0;
+        }
+        const size_t want = std::max(bytes, size_t(1) << 20);
+        *err = cudaMalloc(&buf[dev], want);
+        if (*err != cudaSuccess) {
+            buf[dev] = nullptr;
+            return nullptr;
+        }
+        *err = cudaMemset(buf[dev], 0, want);
+        if (*err != cudaSuccess)
+            return nullptr;
+        cap[dev] = want;
+    }
+    return buf[dev];
 }
 
 int device_sm_count()
@@ -140,6 +177,20 @@ tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
     return ok();
 }
 
+// 5 <= M <= 32: the tensor-core batched-decode kernel with its split-K scratch.
+tq_status smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
+                    const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K,
+                    cudaStream_t stream, const char *fn)
+{
+    cudaError_t err = cudaSuccess;
+    void *ws = tq::device_workspace(tq::smallm_workspace_bytes(N, M), &err);
+    if (!ws)
+        return cuda_fail(err, fn);
+    err = tq::launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, ws,
+                               stream);
+    return err == cudaSuccess ? ok() : cuda_fail(err, fn);
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,6 +266,9 @@ tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq, const 
         return ok();
     if (K == 0)
         return zero_outputs(y, acc_out, size_t(M) * N, stream);
+    if (M > tq::kStreamMaxTokens)
+        return smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                         "tq_gemv");
     return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
                          "tq_gemv");
 }
@@ -231,6 +285,9 @@ tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq
         return ok();
     if (K == 0)
         return zero_outputs(y, acc_out, size_t(M) * N, stream);
+    if (M > tq::kStreamMaxTokens && M <= 32)
+        return smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                         "tq_gemm_prefill");
     bool handled = false;
     cudaError_t e = tq::launch_prefill_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
                                           stream, &handled);

@@ -48,13 +48,16 @@ struct StreamEntry {
     int N4;
     int K;
     int rows_per_tile;
-    int ksplit;             // log2 of the pieces each row is cut into along K
+    int ksplit;             // bits 0-7: log2 of the pieces each row is cut into
+                            // along K; bits 8-9: lanes per row = 8 << value
     int tile_begin;
 };
 
 constexpr int kStreamMaxTokens = 4;     // tokens per launch of the streaming kernel
 constexpr int kStreamMaxRows = 16;      // rows_per_tile upper bound
 constexpr int kStreamMaxK = 32768;
+
+constexpr int kStreamMaxGridFwd = 320;
 
 template <int MaxE>
 struct StreamParams {
@@ -67,10 +70,17 @@ struct StreamParams {
     int overlap_prev;  // start weight copies before the previous grid completes
     int head_bytes;    // shared memory for the entry table and the per-token scales
     unsigned *err;     // the library's device error word
+    // Work split: CTA b streams tiles cta_tile0[b] .. cta_tile0[b+1]-1 (a
+    // contiguous range, balanced by bytes), which belong to entries
+    // cta_entry0[b] .. cta_entry0[b] + cta_nent[b] - 1.
+    int cta_tile0[kStreamMaxGridFwd + 1];
+    int cta_entry0[kStreamMaxGridFwd];
+    int cta_nent[kStreamMaxGridFwd];
     StreamEntry e[MaxE];
 };
 
-constexpr int kStreamStackMax = 384;  // entries per launch (kernel parameters <= 32 KB)
+constexpr int kStreamStackMax = 320;  // entries per launch (kernel parameters <= 32 KB)
+constexpr int kStreamMaxGrid = kStreamMaxGridFwd;  // CTAs per launch
 
 struct StreamLaunch {
     int grid;
@@ -85,6 +95,20 @@ cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_
                                bool single, cudaStream_t stream);
 
 int device_sm_count();
+
+// ---------------------------------------- batched decode on the tensor cores
+// 1 <= M <= 32. `workspace` is zero-filled device memory of at least
+// smallm_workspace_bytes(N, M) bytes; the kernel leaves it zero-filled.
+size_t smallm_workspace_bytes(int N, int M);
+cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                             const float *x_scale, const int32_t *x_sum, float *y,
+                             int32_t *acc_out, int M, int N, int K, void *workspace,
+                             cudaStream_t stream);
+
+// Library-owned, zero-filled scratch on the current device, at least `bytes`
+// long (allocated on first use, grown when a call needs more). Returns null
+// and sets *err on failure.
+void *device_workspace(size_t bytes, cudaError_t *err);
 
 // Device address of the library's error word on the current device.
 unsigned *device_error_word();
