@@ -163,6 +163,28 @@ tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t s
 tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream);
 
 /*
+ * tq_gemv_noalloc -- tq_gemv for 5 <= M <= 32 tokens that allocates no device
+ * memory at all. No passage of the method corresponds to this call; it exists
+ * for callers that cannot call cudaMalloc: a host process whose device memory
+ * is all owned by another allocator (a framework's caching pool, a
+ * pre-reserved arena) or a latency-critical loop that cannot afford the
+ * implicit device synchronisation of an allocation. tq_gemv's path for these M
+ * keeps its split-K partial sums in library-allocated scratch; this one uses
+ * a fixed 4 MiB device array compiled into the library instead, so it works
+ * for N up to the size that fits there (TQ_ERR_UNSUPPORTED beyond it; at
+ * M <= 16 that is N <= 65,408, at 17 <= M <= 32 N <= 32,640).
+ *   Same arguments, results and alignment rules as tq_gemv.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call shares the one array: the part a call uses is zero-filled on
+ *   `stream` before its kernel, but calls whose work overlaps on the GPU
+ *   (e.g. on two streams) race on it and must be serialised by the caller.
+ */
+tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                          const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
+                          int M, int N, int K, cudaStream_t stream);
+
+/*
  * tq_device_error -- read (and if reset != 0, clear) the library's device
  * error word on the current device. Synchronises the device. 0 means no
  * kernel has reported an error. A nonzero value means a kernel gave up a

@@ -17,7 +17,7 @@ import os
 __all__ = [
     "TQError", "TQ_STACK_OVERLAP_PREV", "TqProj", "lib_path",
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
-    "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error",
+    "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj",
 ]
 
@@ -60,6 +60,7 @@ _SIGS = {
     "tq_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "tq_gemv": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "tq_gemm_prefill": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_gemv_noalloc": [_vp, _f, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "tq_quantize_act_stack": [ctypes.POINTER(TqProj), _i, _vp],
     "tq_gemv_stack": [ctypes.POINTER(TqProj), _i, ctypes.c_uint, _vp],
     "tq_device_error": [ctypes.POINTER(ctypes.c_uint32), _i],
@@ -143,6 +144,13 @@ def tq_gemv(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: i
 def tq_gemm_prefill(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int,
                     K: int, stream=None) -> None:
     _check(_load().tq_gemm_prefill(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
+                                _ptr(x_sum), _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
+
+
+def tq_gemv_noalloc(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: int, N: int,
+                    K: int, stream=None) -> None:
+    """tq_gemv for 5 <= M <= 32 on fixed library scratch (allocates nothing)."""
+    _check(_load().tq_gemv_noalloc(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
                                 _ptr(x_sum), _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
 
 

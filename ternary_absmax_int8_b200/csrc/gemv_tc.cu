@@ -374,6 +374,12 @@ cudaError_t launch_bn(const CUtensorMap &mp, const CUtensorMap &mx, const SmallM
     return cudaGetLastError();
 }
 
+// Fixed scratch for tq_gemv_noalloc: the stream-K partial sums and tile
+// counters live here instead of in library-allocated memory. Every GPU that
+// loads the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
+
 }  // namespace
 
 size_t smallm_workspace_bytes(int N, int M)
@@ -413,6 +419,41 @@ cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t 
     if (!prm.err)
         return cudaErrorUnknown;
     return BN == 16 ? launch_bn<16>(map_p, map_x, prm, stream) : launch_bn<32>(map_p, map_x, prm, stream);
+}
+
+size_t noalloc_scratch_capacity() { return kNoAllocScratchBytes; }
+
+// The same kernel with the fixed scratch above. The device address of the
+// scratch array is looked up once per device (on that device's first call)
+// with cudaGetSymbolAddress; host code cannot use the array's name as a
+// device pointer. The part the call uses is zero-filled on `stream` before
+// the kernel, so a call never depends on what an earlier call left there.
+cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                                     const float *x_scale, const int32_t *x_sum, float *y,
+                                     int32_t *acc_out, int M, int N, int K, cudaStream_t stream)
+{
+    static void *scratch[64] = {nullptr};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    const size_t need = smallm_workspace_bytes(N, M);
+    if (need > kNoAllocScratchBytes)
+        return cudaErrorInvalidValue;
+    if (!scratch[dev]) {
+        void *ptr = nullptr;
+        err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (err != cudaSuccess)
+            return err;
+        scratch[dev] = ptr;
+    }
+    err = cudaMemsetAsync(scratch[dev], 0, need, stream);
+    if (err != cudaSuccess)
+        return err;
+    return launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
+                            scratch[dev], stream);
 }
 
 }  // namespace tq

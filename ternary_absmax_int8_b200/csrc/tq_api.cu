@@ -397,6 +397,32 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
     return ok();
 }
 
+tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                          const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
+                          int M, int N, int K, cudaStream_t stream)
+{
+    tq_status st =
+        check_gemv_args("tq_gemv_noalloc", packed, xq, x_scale, x_sum, y, acc_out, M, N, K);
+    if (st != TQ_OK)
+        return st;
+    if (M == 0 || N == 0)
+        return ok();
+    if (M < 5 || M > 32)
+        return fail(TQ_ERR_UNSUPPORTED,
+                    "tq_gemv_noalloc: M=%d outside 5..32 (tq_gemv needs no scratch for M <= 4)", M);
+    if (K == 0)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_gemv_noalloc: K=0 (use tq_gemv)");
+    const size_t need = tq::smallm_workspace_bytes(N, M);
+    if (need > tq::noalloc_scratch_capacity())
+        return fail(TQ_ERR_UNSUPPORTED,
+                    "tq_gemv_noalloc: N=%d at M=%d needs %zu bytes of scratch, more than the fixed "
+                    "%zu",
+                    N, M, need, tq::noalloc_scratch_capacity());
+    cudaError_t e = tq::launch_smallm_tc_noalloc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M,
+                                                 N, K, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "tq_gemv_noalloc");
+}
+
 tq_status tq_device_error(uint32_t *code, int reset)
 {
     if (!code)

@@ -105,6 +105,14 @@ cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t 
                              int32_t *acc_out, int M, int N, int K, void *workspace,
                              cudaStream_t stream);
 
+// The same kernel on a fixed, statically allocated device scratch (no
+// allocation by anyone); cudaErrorInvalidValue when the shape needs more than
+// noalloc_scratch_capacity() bytes of it.
+size_t noalloc_scratch_capacity();
+cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                                     const float *x_scale, const int32_t *x_sum, float *y,
+                                     int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
+
 // Library-owned, zero-filled scratch on the current device, at least `bytes`
 // long (allocated on first use, grown when a call needs more). Returns null
 // and sets *err on failure.
