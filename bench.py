@@ -49,6 +49,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 DESCRIPTIONS = {
     "stack30_m1": "decode layer stack: 30 x BitNet-b1.58-2B-4T decoder layer (q,k,v,o,gate,up,"
                   "down ternary projections), M=1, 210 projections, 2.08e9 weights",
+    "stack10_m1": "decode layer stack: 10 x BitNet-b1.58-2B-4T decoder layer, M=1 "
+                  "(profiling case)",
     "layer_m1": "one BitNet-b1.58-2B-4T decoder layer, 7 ternary projections, M=1",
     "single_640x2560_m1": "one ternary projection N=640 K=2560, M=1",
     "prefill_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120",

@@ -128,6 +128,9 @@ WORKLOADS = {
     "single_640x2560_m1": ([("proj", 640, 2560)], 1),
     "layer_m1": (list(DECODER_LAYER), 1),
     "stack30_m1": (stack_shapes(STACK_LAYERS), 1),
+    # a 10-layer stack (175 MB of weights, still larger than L2): the small case
+    # for profiler captures of the stack kernel
+    "stack10_m1": (stack_shapes(10), 1),
 }
 for _m in SMALL_M_VALUES:
     WORKLOADS[f"ffn_m{_m}"] = (list(SMALL_M_SHAPES), _m)
