@@ -7,33 +7,34 @@
 // numbers": their HIP ternary GEMV at 92% of memory-bandwidth peak on
 // gfx1151). Design for sm_100a:
 //
-//  * Persistent CTAs, one per SM, each a producer warp plus W consumer warps.
+//  * Persistent CTAs, one per SM, each a producer warp plus G groups of W
+//    consumer warps.
 //  * The packed weights of a projection, uint8 [N/4, K] row-major, are cut
 //    into tiles of R consecutive packed rows: one contiguous R*K-byte range,
 //    moved by a single 1-D bulk copy (TMA engine, cp.async.bulk, no
-//    multicast) into a ring of shared-memory stages guarded by mbarriers. The
-//    ring keeps ~100-200 KB per SM in flight, which is what HBM3e's latency x
-//    bandwidth product asks for. Tiles of all projections of a launch form one
-//    sequence, dealt round-robin to the CTAs, so a stack of projections is
-//    streamed back to back in projection order with no drain in between.
-//  * Activations (int8, M x K) either stay resident in shared memory for the
-//    whole launch (one projection) or ride along with each tile (a stack).
+//    multicast) into a ring of shared-memory stages guarded by mbarriers.
+//    Tiles of all projections of a launch form one sequence, cut into one
+//    contiguous, byte-balanced range per CTA, so a stack of projections is
+//    streamed back to back with no drain in between. Group g consumes the
+//    CTA's tiles g, g + G, ...
+//  * The int8 activations of the CTA's projections are copied once into a
+//    resident shared-memory cache.
 //  * Consumers read 16-byte words of packed weights and activations from
 //    shared memory. A 32-bit word u holds, for output row i + p*N/4 (p =
-//    0..3), the codes of 4 consecutive k in its bytes' bit fields 2p..2p+1;
-//    u & (0x03030303 << 2p) isolates them, scaled by 4^p, and one dp4a
-//    (unsigned codes x signed int8) accumulates them: acc'_p = 4^p * sum c*q.
-//    No shifts are needed in the loop; the 4^p is removed once per output.
+//    0..3), the codes of 4 consecutive k in its bytes' bit fields 2p..2p+1.
+//    Four dp4a (unsigned codes x signed int8) on nested masks of u give
+//    nested sums from which 4^p * sum_k c*q follows by differences; the 4^p
+//    is removed once per output.
 //  * Since w = c - 1, acc = sum c*q - sum q = acc' - x_sum (x_sum comes from
 //    the quantiser), so no per-element subtraction is needed either.
-//  * A butterfly reduction gathers each warp's 4 partial sums per token in
-//    six shuffles; warps that share a row add into shared memory with integer
-//    atomics (exact, order-free); one named barrier per tile, then the
-//    epilogue writes y = float(acc) * (w_scale * x_scale) for the tile's rows.
+//  * A butterfly over the lanes of a row (8, 16 or 32) reduces the four
+//    partial sums per token; the epilogue writes y = float(acc) * (w_scale *
+//    x_scale). Single-projection launches may cut rows along K over several
+//    warps, which then add into shared memory with integer atomics (exact,
+//    order-free) and the last warp finishes the row.
 //  * Every mbarrier wait is bounded (2 s of global time); on a timeout the
-//    kernel records an error bit, all consumer warps agree to stop through a
-//    barrier reduction, and the producer waits (bounded) for its copies in
-//    flight before the CTA exits.
+//    kernel records an error bit and winds down, the producer first waiting
+//    (bounded) for its copies in flight.
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -398,7 +399,7 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                 const uint4 wv = wrow[c];
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    if (m < p.M) {
+                    if (MT == 1 || m < p.M) {
                         const uint4 xv = reinterpret_cast<const uint4 *>(sx + m * K)[c];
                         dot16<J>(wv, xv, a[m]);
                     }
@@ -419,7 +420,7 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                 // writes plane q of its row.
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    if (m < p.M) {
+                    if (MT == 1 || m < p.M) {
                         int32_t f[4];
                         fold<J>(a[m], f);
                         int plane;
@@ -437,7 +438,7 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                 int32_t *slot = part + (stage * kStreamMaxRows + r) * MT * 4;
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    if (m < p.M) {
+                    if (MT == 1 || m < p.M) {
                         int32_t f[4];
                         fold<J>(a[m], f);
                         int plane;
@@ -515,7 +516,7 @@ cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, 
 // size aim. TQ_STREAM_CFG="W,G,CPS[,tile_bytes]" picks another instantiated
 // variant (for measurement).
 struct StreamCfg {
-    int W = 4;
+    int W = 8;
     int G = 2;
     int CPS = 1;
     int tile = kWTargetBytes;
@@ -528,10 +529,8 @@ StreamCfg stream_cfg()
         if (const char *s = getenv("TQ_STREAM_CFG")) {
             int w = 0, g = 0, cps = 0, tile = 0;
             const int n = sscanf(s, "%d,%d,%d,%d", &w, &g, &cps, &tile);
-            const bool known = (w == 8 && g == 1 && (cps == 1 || cps == 2)) ||
-                               (w == 8 && g == 2 && cps == 1) || (w == 4 && g == 2 && cps == 1) ||
-                               (w == 4 && g == 4 && cps == 1) || (w == 4 && g == 2 && cps == 2) ||
-                               (w == 4 && g == 1 && cps == 2);
+            const bool known = cps == 1 && ((g == 2 && (w == 4 || w == 6 || w == 7 || w == 8)) ||
+                                            (g == 3 && w == 4) || (g == 4 && w == 4));
             if (n >= 3 && known) {
                 c.W = w;
                 c.G = g;
@@ -549,18 +548,16 @@ template <int MaxE, int MT>
 cudaError_t launch_variant(const StreamCfg &c, const StreamParams<MaxE> &p, int grid, size_t smem,
                            bool pdl, cudaStream_t stream)
 {
-    if (c.W == 8 && c.G == 1 && c.CPS == 2)
-        return launch_instance<8, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    if (c.W == 8 && c.G == 2)
+    if (c.G == 2 && c.W == 8)
         return launch_instance<8, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
-    if (c.W == 4 && c.G == 4)
+    if (c.G == 2 && c.W == 7)
+        return launch_instance<7, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.G == 2 && c.W == 6)
+        return launch_instance<6, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.G == 3)
+        return launch_instance<4, 3, MaxE, MT, 1>(p, grid, smem, pdl, stream);
+    if (c.G == 4)
         return launch_instance<4, 4, MaxE, MT, 1>(p, grid, smem, pdl, stream);
-    if (c.W == 4 && c.G == 2 && c.CPS == 2)
-        return launch_instance<4, 2, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    if (c.W == 4 && c.G == 1)
-        return launch_instance<4, 1, MaxE, MT, 2>(p, grid, smem, pdl, stream);
-    if (c.W == 8 && c.G == 1 && c.CPS == 1)
-        return launch_instance<8, 1, MaxE, MT, 1>(p, grid, smem, pdl, stream);
     return launch_instance<4, 2, MaxE, MT, 1>(p, grid, smem, pdl, stream);
 }
 
@@ -595,8 +592,11 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
         while (lsel < 2 && items_of(lsel) < W)
             ++lsel;
         const int items = items_of(lsel);
+        // Rows are cut into pieces along K only in single-projection
+        // launches, where a CTA holds too few tiles for the round-robin deal
+        // to keep its warps busy.
         int lg = 0;
-        while ((items << lg) < W && (C >> (lg + 1)) >= 16)
+        while (single && (items << lg) < W && (C >> (lg + 1)) >= 16)
             ++lg;
         e.rows_per_tile = R;
         e.ksplit = lg | (lsel << 8);
@@ -677,7 +677,11 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     const size_t budget = smem_budget(cfg.CPS);
     int stages = budget > fixed ? int((budget - fixed) / size_t(p.w_slot)) : 0;
     stages = std::min(stages, kMaxStages);
-    stages -= stages % cfg.G;  // each consumer group keeps to its own stages
+    // Each consumer group must see every phase of the stages it uses: with
+    // stages % G != 0 a group would wait for phase k of a stage whose phase
+    // k - 1 (another group's tile) has not completed yet, and a parity wait
+    // cannot tell those apart.
+    stages -= stages % cfg.G;
     if (stages < std::max(2, cfg.G))
         return cudaErrorInvalidValue;
     p.stages = stages;
