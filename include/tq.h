@@ -144,6 +144,12 @@ typedef struct tq_proj {
                                     before the previous kernel on the stream ends
                                     (programmatic dependent launch); activations,
                                     scales and sums are read only after it ends. */
+#define TQ_STACK_QUANTIZE 2u     /* the same launch also quantises: x (bf16, 16-byte
+                                    aligned) is the input, and xq, x_scale and x_sum
+                                    are written with exactly the values
+                                    tq_quantize_act_stack would write, instead of
+                                    being read. One launch per call replaces the
+                                    quantiser launch and the GEMV launch. */
 
 /*
  * tq_quantize_act_stack -- tq_quantize_act for each projection's single
@@ -154,25 +160,30 @@ tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t s
 
 /*
  * tq_gemv_stack -- tq_gemv (M = 1) for every projection, in one persistent
- * launch per 384 projections that streams all their weights back to back, in
+ * launch per 320 projections that streams all their weights back to back, in
  * projection order, with no drain between projections. projs is a HOST array
  * (read during the call only; the table travels in the launch parameters).
- * flags: 0 or TQ_STACK_OVERLAP_PREV. Projections are independent: y of one
- * must not be another's input within the same call.
+ * flags: any of TQ_STACK_OVERLAP_PREV and TQ_STACK_QUANTIZE. Without
+ * TQ_STACK_QUANTIZE, xq, x_scale and x_sum are inputs (from
+ * tq_quantize_act_stack); with it, x is the input and they are outputs.
+ * Projections are independent: y of one must not be another's input within
+ * the same call, and no buffer may be shared between two entries.
  */
 tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream);
 
 /*
- * tq_gemv_noalloc -- tq_gemv for 5 <= M <= 32 tokens that allocates no device
+ * tq_gemv_noalloc -- tq_gemv for 5 <= M <= 32 tokens computed by the
+ * stream-K formulation of the batched-decode kernel, which allocates no device
  * memory at all. No passage of the method corresponds to this call; it exists
  * for callers that cannot call cudaMalloc: a host process whose device memory
  * is all owned by another allocator (a framework's caching pool, a
  * pre-reserved arena) or a latency-critical loop that cannot afford the
- * implicit device synchronisation of an allocation. tq_gemv's path for these M
- * keeps its split-K partial sums in library-allocated scratch; this one uses
- * a fixed 4 MiB device array compiled into the library instead, so it works
- * for N up to the size that fits there (TQ_ERR_UNSUPPORTED beyond it; at
- * M <= 16 that is N <= 65,408, at 17 <= M <= 32 N <= 32,640).
+ * implicit device synchronisation of an allocation. tq_gemv splits K inside
+ * thread-block clusters and needs no scratch; the stream-K formulation spreads
+ * every projection over all SMs and keeps its split-K partial sums in a fixed
+ * 4 MiB device array compiled into the library, so it works for N up to the
+ * size that fits there (TQ_ERR_UNSUPPORTED beyond it; at M <= 16 that is
+ * N <= 65,408, at 17 <= M <= 32 N <= 32,640).
  *   Same arguments, results and alignment rules as tq_gemv.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.

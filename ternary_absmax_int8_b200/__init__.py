@@ -15,7 +15,7 @@ import ctypes
 import os
 
 __all__ = [
-    "TQError", "TQ_STACK_OVERLAP_PREV", "TqProj", "lib_path",
+    "TQError", "TQ_STACK_OVERLAP_PREV", "TQ_STACK_QUANTIZE", "TqProj", "lib_path",
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
     "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj",
@@ -25,6 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libtq.so")
 
 TQ_STACK_OVERLAP_PREV = 1
+TQ_STACK_QUANTIZE = 2
 _STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN",
            4: "TQ_ERR_VALUE", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_UNSUPPORTED"}
 

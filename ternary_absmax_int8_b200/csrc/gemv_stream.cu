@@ -40,6 +40,7 @@
 #include <cstdlib>
 #include <vector>
 
+#include "quant_core.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -195,7 +196,35 @@ struct SmemTail {
     static constexpr int kBars = 2 * kMaxStages + 1;
     static constexpr int kPart = kMaxStages * kStreamMaxRows * MT * 4;
     static constexpr int kCnt = kMaxStages * kStreamMaxRows;
-    static constexpr size_t bytes() { return kDesc + kBars * 8 + (kPart + kCnt) * 4; }
+    static constexpr int kRed = 32;
+    static constexpr size_t bytes() { return kDesc + kBars * 8 + (kPart + kCnt + kRed) * 4; }
+};
+
+// Max / sum over the WC consumer warps (named barrier 1). Every thread gets
+// the result; `red` holds one slot per warp. Both are exact in any order
+// (max of non-NaN floats, integer sum).
+template <int WC, typename T, typename Op>
+__device__ __forceinline__ T consumer_reduce(T v, Op op, T *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = v;
+    named_bar_sync(1, WC * 32);
+    T r = red[0];
+#pragma unroll
+    for (int w = 1; w < WC; ++w)
+        r = op(r, red[w]);
+    named_bar_sync(1, WC * 32);  // red is reused by the next reduction
+    return r;
+}
+
+struct FMax {
+    __device__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct IAdd {
+    __device__ int operator()(int a, int b) const { return a + b; }
 };
 
 
@@ -224,10 +253,19 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
     uint64_t *xbar = empty + kMaxStages;
     int32_t *part = reinterpret_cast<int32_t *>(xbar + 1);
     int32_t *cnt = part + SmemTail<MT>::kPart;
+    int32_t *red = cnt + SmemTail<MT>::kCnt;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    for (int i = threadIdx.x; i < SmemTail<MT>::kPart + SmemTail<MT>::kCnt; i += blockDim.x)
+    // A dependent grid launched with programmatic serialisation (the next
+    // call's stack GEMV) may start its prologue and weight copies as soon as
+    // SMs free up; it reads nothing this grid writes before its own
+    // griddepcontrol.wait.
+    if (threadIdx.x == 0)
+        pdl_launch_dependents();
+
+    for (int i = threadIdx.x; i < SmemTail<MT>::kPart + SmemTail<MT>::kCnt + SmemTail<MT>::kRed;
+         i += blockDim.x)
         part[i] = 0;
     {
         static_assert(sizeof(StreamEntry) % 8 == 0, "entry size");
@@ -260,6 +298,11 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
         const uint64_t pol_w = policy_evict_first();  // weights: read once
         const uint64_t pol_x = policy_evict_last();   // activations: reread by many CTAs
         auto load_x = [&]() {
+            if (p.quant) {
+                // The consumers write the activation cache themselves.
+                mbar_arrive(xbar);
+                return;
+            }
             uint32_t total = 0;
             for (int j = 0; j < n_entries; ++j)
                 total += uint32_t(p.M * tab[j].K);
@@ -323,12 +366,47 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
     // the stage into registers, hands the stage back after its last item's
     // copy, and only then computes: a stage is held for the copy, not for the
     // arithmetic, so nearly the whole ring stays in flight.
-    pdl_wait();  // x_scale and x_sum are read below
-    for (int i = threadIdx.x; i < n_entries * p.M; i += WC * 32) {
-        const int j = i / p.M, m = i - j * p.M;
-        const StreamEntry &e = tab[j];
-        scl[j * MT + m] = make_float2(__fmul_rn(e.w_scale, __ldg(e.x_scale + m)),
-                                      __int_as_float(__ldg(e.x_sum + m)));
+    pdl_wait();  // activations, x_scale and x_sum are read below
+    if (MT == 1 && p.quant) {
+        // Quantise the CTA's activations (one token per projection) straight
+        // into the activation cache. The CTA that streams a projection's
+        // first tile also writes xq, x_scale and x_sum to global memory.
+        for (int j = 0; j < n_entries; ++j) {
+            const StreamEntry &e = tab[j];
+            const uint4 *xv = reinterpret_cast<const uint4 *>(e.xb);
+            const int nvec = e.K >> 3;  // 8 bf16 per 16-byte vector
+            float amax = 0.0f;
+            for (int v = threadIdx.x; v < nvec; v += WC * 32)
+                amax = fmaxf(amax, absmax8(__ldg(xv + v)));
+            amax = consumer_reduce<WC>(amax, FMax(), reinterpret_cast<float *>(red));
+            const float s = quant_inv_scale(amax);
+            const bool owner = e.tile_begin >= t_begin;
+            uint2 *qc = reinterpret_cast<uint2 *>(xcache + xoff[j]);
+            uint2 *qg = reinterpret_cast<uint2 *>(e.xq);
+            int sum = 0;
+            for (int v = threadIdx.x; v < nvec; v += WC * 32) {
+                const uint2 o = quant8(__ldg(xv + v), s, &sum);
+                qc[v] = o;
+                if (owner)
+                    qg[v] = o;
+            }
+            sum = consumer_reduce<WC>(sum, IAdd(), red);
+            if (threadIdx.x == 0) {
+                const float xs = quant_scale(amax);
+                scl[j * MT] = make_float2(__fmul_rn(e.w_scale, xs), __int_as_float(sum));
+                if (owner) {
+                    *e.x_scale = xs;
+                    *e.x_sum = sum;
+                }
+            }
+        }
+    } else {
+        for (int i = threadIdx.x; i < n_entries * p.M; i += WC * 32) {
+            const int j = i / p.M, m = i - j * p.M;
+            const StreamEntry &e = tab[j];
+            scl[j * MT + m] = make_float2(__fmul_rn(e.w_scale, __ldg(e.x_scale + m)),
+                                          __int_as_float(__ldg(e.x_sum + m)));
+        }
     }
     named_bar_sync(1, WC * 32);
     if (t_end > t_begin && !mbar_wait_warp(xbar, 0, p.err))
@@ -563,7 +641,7 @@ cudaError_t launch_variant(const StreamCfg &c, const StreamParams<MaxE> &p, int 
 
 template <int MaxE>
 cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, bool single,
-                         cudaStream_t stream)
+                         bool quant, cudaStream_t stream)
 {
     StreamParams<MaxE> p;  // host staging of the launch parameters
     static_assert(sizeof(StreamParams<MaxE>) <= 32000, "kernel parameters exceed 32 KB");
@@ -610,6 +688,7 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     p.M = M;
     p.w_slot = (stage_max + 127) / 128 * 128;
     p.overlap_prev = overlap_prev ? 1 : 0;
+    p.quant = quant ? 1 : 0;
     const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
     if (total == 0)
         return cudaSuccess;
@@ -696,17 +775,17 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
 }  // namespace
 
 cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_prev, bool single,
-                               cudaStream_t stream)
+                               bool quant, cudaStream_t stream)
 {
     if (n <= 0)
         return cudaSuccess;
-    if (M < 1 || M > kStreamMaxTokens || n > kStreamStackMax)
+    if (M < 1 || M > kStreamMaxTokens || n > kStreamStackMax || (quant && M != 1))
         return cudaErrorInvalidValue;
     if (n == 1)
-        return launch_sized<1>(entries, n, M, overlap_prev, single, stream);
+        return launch_sized<1>(entries, n, M, overlap_prev, single, quant, stream);
     if (n <= 16)
-        return launch_sized<16>(entries, n, M, overlap_prev, single, stream);
-    return launch_sized<kStreamStackMax>(entries, n, M, overlap_prev, single, stream);
+        return launch_sized<16>(entries, n, M, overlap_prev, single, quant, stream);
+    return launch_sized<kStreamStackMax>(entries, n, M, overlap_prev, single, quant, stream);
 }
 
 }  // namespace tq

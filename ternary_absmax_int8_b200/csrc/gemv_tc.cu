@@ -1,5 +1,5 @@
 // gemv_tc.cu -- batched-decode ternary GEMV on the tensor cores (5 <= M <= 32
-// tokens), tcgen05 with the code operand in tensor memory, stream-K.
+// tokens), tcgen05 with the code operand in tensor memory.
 //
 // Many concurrent requests turn decode into a skinny contraction (1bit engine
 // blog, "One GPU, many users"): each weight byte now feeds M tokens, so
@@ -18,16 +18,25 @@
 //   memory, which at small N would otherwise bound the kernel (16 KB written
 //   and 16 KB read back per 4 KB of weights).
 // * K advances in 256-byte units; a unit is one TMA box pair of packed bytes
-//   (32 rows) plus activations (BN rows), 128B swizzled. The (tile, unit)
-//   sequence is split into one contiguous, balanced range per CTA (stream-K),
-//   so every SM streams weights even when there are fewer tiles than SMs.
-//   A tile split across CTAs adds its int32 partial sums into a global
-//   workspace with integer atomics (exact, order-free); the CTA whose
-//   contribution completes the tile applies the epilogue and zeroes the
-//   workspace for the next call.
+//   (32 rows) plus activations (BN rows), 128B swizzled. A CTA works through
+//   segments (tile, first unit, end unit); two plans decide which:
+//   - cluster plan (tq_gemv): with fewer tiles than SMs, the C CTAs of a
+//     thread-block cluster split one tile's K range; the other CTAs add their
+//     int32 partial sums into the leader CTA's shared memory (red on
+//     shared::cluster, exact and order-free) and signal its mbarrier; the
+//     leader applies the epilogue. With many tiles, C = 1 and each CTA takes
+//     whole tiles.
+//   - stream-K plan (tq_gemv_noalloc): the (tile, unit) sequence is cut into
+//     one contiguous, balanced range per CTA; a tile split across CTAs adds
+//     its partial sums into a global scratch with integer atomics, and the
+//     CTA whose contribution completes the tile applies the epilogue and
+//     zeroes the scratch for the next call.
 // * Warp roles (12 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
 //   4..7 expansion, 8..11 epilogue. All mbarrier waits are bounded.
 #include <algorithm>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 #include "tc_common.cuh"
 
@@ -44,17 +53,47 @@ constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per c
 constexpr int kThreads = 384;
 constexpr int kMaxGrid = 512;
 
+constexpr int kPlanStreamK = 0;
+constexpr int kPlanCluster = 1;
+constexpr int kMaxCluster = 8;
+
 struct SmallMParams {
     int N4, K, M;
     int tiles, units_per_tile, total_units, grid;
+    int plan;   // kPlanStreamK or kPlanCluster
+    int csize;  // CTAs per cluster (cluster plan)
     float w_scale;
     const float *x_scale;
     const int32_t *x_sum;
     float *y;
     int32_t *acc_out;
-    int32_t *ws;    // [tiles][BN][128] int32 partial sums (all zero between calls)
-    int32_t *cnt;   // [tiles] arrivals (all zero between calls)
+    int32_t *ws;    // stream-K: [tiles][BN][128] int32 partial sums (all zero between calls)
+    int32_t *cnt;   // stream-K: [tiles] arrivals (all zero between calls)
     unsigned *err;
+};
+
+// A run of consecutive K units [k0, k1) of one tile.
+struct Seg {
+    int tile, k0, k1;
+};
+
+// The segments one CTA works through, in order.
+struct CtaWork {
+    int nseg;
+    int u_begin, u_end;  // stream-K: this CTA's global unit range
+    int rank;            // cluster plan: rank in the cluster
+
+    __device__ Seg seg(const SmallMParams &p, int s) const
+    {
+        const int U = p.units_per_tile;
+        if (p.plan == kPlanStreamK) {
+            const int t = u_begin / U + s;
+            return Seg{t, s == 0 ? u_begin - t * U : 0, min(U, u_end - t * U)};
+        }
+        if (p.csize == 1)
+            return Seg{int(blockIdx.x) + s * int(gridDim.x), 0, U};
+        return Seg{int(blockIdx.x) / p.csize, U * rank / p.csize, U * (rank + 1) / p.csize};
+    }
 };
 
 template <int BN>
@@ -63,12 +102,85 @@ struct SmallMSmem {
     static constexpr int kBBytes = BN * kUnitK;
     static constexpr size_t p_off = 0;
     static constexpr size_t b_off = p_off + size_t(kSP) * kPBytes;
-    static constexpr size_t bar_off = b_off + size_t(kSP) * kBBytes;
-    // tma_full[SP], p_free[SP], mma_done[SP], a_full[SA], acc_full[2], acc_empty[2]
-    static constexpr int kBars = 3 * kSP + kSA + 4;
+    // cluster plan: the leader's sum of the other CTAs' partials, [BN][128]
+    static constexpr size_t red_off = b_off + size_t(kSP) * kBBytes;
+    static constexpr size_t bar_off = red_off + size_t(BN) * kRows * 4;
+    // tma_full[SP], p_free[SP], mma_done[SP], a_full[SA], acc_full[2],
+    // acc_empty[2], red_done
+    static constexpr int kBars = 3 * kSP + kSA + 5;
     static constexpr size_t misc_off = bar_off + kBars * 8;  // tmem slot, finisher flag
     static constexpr size_t bytes = misc_off + 16;
 };
+
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_cluster(uint32_t raddr, int32_t v)
+{
+    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" ::"r"(raddr), "r"(v)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait_warp with cluster-scope acquire (the arrivals come from other
+// CTAs of the cluster, after their red operations on this CTA's memory).
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
+                                                       unsigned *err)
+{
+    bool done = mbar_try_wait_cluster(bar, parity);
+    if (__all_sync(0xffffffffu, done))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        done = done || mbar_try_wait_cluster(bar, parity);
+        if (__all_sync(0xffffffffu, done))
+            return true;
+        if ((i & 255u) == 0) {
+            const bool late = global_ns() - t0 > kWaitLimitNs;
+            if (__any_sync(0xffffffffu, late)) {
+                if ((threadIdx.x & 31) == 0)
+                    atomicOr(err, kErrWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
 
 // Unit u of the whole call belongs to CTA b with U(b) <= u < U(b+1).
 __device__ __forceinline__ int unit_start(int b, int total, int grid)
@@ -117,6 +229,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sP = smem + L::p_off;
     uint8_t *sB = smem + L::b_off;
+    int32_t *red_buf = reinterpret_cast<int32_t *>(smem + L::red_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
     uint64_t *tma_full = bars;
     uint64_t *p_free = bars + kSP;
@@ -124,13 +237,26 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
     uint64_t *a_full = bars + 3 * kSP;
     uint64_t *acc_full = a_full + kSA;
     uint64_t *acc_empty = acc_full + 2;
+    uint64_t *red_done = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
     int *fin_flag = reinterpret_cast<int *>(smem + L::misc_off + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int u_begin = unit_start(blockIdx.x, p.total_units, p.grid);
-    const int u_end = unit_start(blockIdx.x + 1, p.total_units, p.grid);
-    const int UPT = p.units_per_tile;
+    const int U = p.units_per_tile;
+    const bool split_cluster = p.plan == kPlanCluster && p.csize > 1;
+    CtaWork cw;
+    cw.rank = split_cluster ? int(cluster_ctarank()) : 0;
+    if (p.plan == kPlanStreamK) {
+        cw.u_begin = unit_start(blockIdx.x, p.total_units, p.grid);
+        cw.u_end = unit_start(blockIdx.x + 1, p.total_units, p.grid);
+        cw.nseg = cw.u_end > cw.u_begin ? (cw.u_end - 1) / U - cw.u_begin / U + 1 : 0;
+    } else {
+        cw.u_begin = cw.u_end = 0;
+        cw.nseg = split_cluster ? 1
+                                : (p.tiles > int(blockIdx.x)
+                                       ? (p.tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1
+                                       : 0);
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSP; ++s) {
@@ -144,13 +270,22 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
+        // every epilogue thread of every other CTA of the cluster arrives once
+        mbar_init(red_done, split_cluster ? uint32_t(kRows * (p.csize - 1)) : 1u);
         fence_mbar_init();
     }
+    if (split_cluster && cw.rank == 0)
+        for (int i = threadIdx.x; i < BN * kRows; i += kThreads)
+            red_buf[i] = 0;
     if (warp == 1)
         tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The leader's barrier and zeroed sum must exist before any CTA of the
+    // cluster touches them.
+    if (split_cluster)
+        cluster_sync_all();
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t tmem_a = tmem_base;                    // kSA slots of kACols
     const uint32_t tmem_d = tmem_base + kSA * kACols;     // 2 x BN accumulator columns
@@ -159,20 +294,26 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         // -------------------------------------------------- TMA producer
         if (lane == 0) {
             int issued = 0;
-            for (int u = u_begin; u < u_end; ++u, ++issued) {
-                const int s = issued % kSP;
-                const uint32_t use = uint32_t(issued / kSP);
-                if (use > 0 && (!mbar_wait(&p_free[s], (use - 1) & 1, p.err) ||
-                                !mbar_wait(&mma_done[s], (use - 1) & 1, p.err)))
-                    break;
-                const int tile = u / UPT, k0 = (u - tile * UPT) * kUnitK;
-                mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
-                uint8_t *P = sP + s * L::kPBytes;
-                uint8_t *B = sB + s * L::kBBytes;
-                tma_load_2d(P, &map_p, k0, tile * kPRows, &tma_full[s]);
-                tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, tile * kPRows, &tma_full[s]);
-                tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
-                tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+            bool ok = true;
+            for (int sg = 0; sg < cw.nseg && ok; ++sg) {
+                const Seg g = cw.seg(p, sg);
+                for (int k = g.k0; k < g.k1; ++k, ++issued) {
+                    const int s = issued % kSP;
+                    const uint32_t use = uint32_t(issued / kSP);
+                    if (use > 0 && (!mbar_wait(&p_free[s], (use - 1) & 1, p.err) ||
+                                    !mbar_wait(&mma_done[s], (use - 1) & 1, p.err))) {
+                        ok = false;
+                        break;
+                    }
+                    const int k0 = k * kUnitK;
+                    mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
+                    uint8_t *P = sP + s * L::kPBytes;
+                    uint8_t *B = sB + s * L::kBBytes;
+                    tma_load_2d(P, &map_p, k0, g.tile * kPRows, &tma_full[s]);
+                    tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, g.tile * kPRows, &tma_full[s]);
+                    tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
+                    tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+                }
             }
             for (int s = 0; s < kSP && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % kSP);
@@ -182,17 +323,16 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
     } else if (warp == 1) {
         // -------------------------------------------------- MMA issuer
         if (lane == 0) {
-            int i = 0, seg = 0;
+            int i = 0;
             bool ok = true;
-            for (int u = u_begin; u < u_end && ok;) {
-                const int tile = u / UPT;
-                const int seg_end = min(u_end, (tile + 1) * UPT);
-                const int buf = seg & 1;
-                if (seg >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((seg >> 1) - 1) & 1), p.err))
+            for (int sg = 0; sg < cw.nseg && ok; ++sg) {
+                const Seg g = cw.seg(p, sg);
+                const int buf = sg & 1;
+                if (sg >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((sg >> 1) - 1) & 1), p.err))
                     break;
                 tc_fence_after();
                 const uint32_t d = tmem_d + uint32_t(buf * BN);
-                for (; u < seg_end; ++u, ++i) {
+                for (int k = g.k0; k < g.k1; ++k, ++i) {
                     const int s = i % kSP, sa = i % kSA;
                     if (!mbar_wait(&tma_full[s], uint32_t((i / kSP) & 1), p.err) ||
                         !mbar_wait(&a_full[sa], uint32_t((i / kSA) & 1), p.err)) {
@@ -201,18 +341,16 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                     }
                     tc_fence_after();
                     const uint32_t b0 = smem_u32(sB + s * L::kBBytes);
-                    const bool first = (u == u_begin) || (u % UPT == 0);
 #pragma unroll
                     for (int kk = 0; kk < kUnitK / 32; ++kk) {
                         const uint32_t bk = b0 + uint32_t((kk >> 2) * (L::kBBytes / 2) + (kk & 3) * 32);
                         umma_i8_ts(d, tmem_a + uint32_t(sa * kACols + kk * 8), umma_desc_sw128(bk),
-                                   kIdesc, (first && kk == 0) ? 0u : 1u);
+                                   kIdesc, (k == g.k0 && kk == 0) ? 0u : 1u);
                     }
                     umma_commit(&mma_done[s]);
                 }
                 if (ok)
                     umma_commit(&acc_full[buf]);
-                ++seg;
             }
             if (i > 0) {
                 const int s = (i - 1) % kSP;
@@ -225,36 +363,40 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         const int j = 8 * q + (lane >> 2), pl = lane & 3;  // packed row, plane of this lane
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int i = 0;
-        for (int u = u_begin; u < u_end; ++u, ++i) {
-            const int s = i % kSP, sa = i % kSA;
-            bool ok = mbar_wait_warp(&tma_full[s], uint32_t((i / kSP) & 1), p.err);
-            if (ok && i >= kSA) {
-                const int pi = i - kSA;  // the unit that last used this A slot
-                ok = mbar_wait_warp(&mma_done[pi % kSP], uint32_t((pi / kSP) & 1), p.err);
-            }
-            if (!ok)
-                break;
-            tc_fence_after();
-            const uint8_t *P = sP + s * L::kPBytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t v[32];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(P + h * (L::kPBytes / 2) +
-                                                                     sw128_off(j, c));
-                    v[4 * c + 0] = (w.x >> (2 * pl)) & 0x03030303u;
-                    v[4 * c + 1] = (w.y >> (2 * pl)) & 0x03030303u;
-                    v[4 * c + 2] = (w.z >> (2 * pl)) & 0x03030303u;
-                    v[4 * c + 3] = (w.w >> (2 * pl)) & 0x03030303u;
+        bool ok = true;
+        for (int sg = 0; sg < cw.nseg && ok; ++sg) {
+            const Seg g = cw.seg(p, sg);
+            for (int k = g.k0; k < g.k1; ++k, ++i) {
+                const int s = i % kSP, sa = i % kSA;
+                ok = mbar_wait_warp(&tma_full[s], uint32_t((i / kSP) & 1), p.err);
+                if (ok && i >= kSA) {
+                    const int pi = i - kSA;  // the unit that last used this A slot
+                    ok = mbar_wait_warp(&mma_done[pi % kSP], uint32_t((pi / kSP) & 1), p.err);
                 }
-                tmem_st32(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&a_full[sa]);
-                mbar_arrive(&p_free[s]);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const uint8_t *P = sP + s * L::kPBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(P + h * (L::kPBytes / 2) +
+                                                                         sw128_off(j, c));
+                        v[4 * c + 0] = (w.x >> (2 * pl)) & 0x03030303u;
+                        v[4 * c + 1] = (w.y >> (2 * pl)) & 0x03030303u;
+                        v[4 * c + 2] = (w.z >> (2 * pl)) & 0x03030303u;
+                        v[4 * c + 3] = (w.w >> (2 * pl)) & 0x03030303u;
+                    }
+                    tmem_st32(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&a_full[sa]);
+                    mbar_arrive(&p_free[s]);
+                }
             }
         }
     } else if (warp >= 8) {
@@ -264,14 +406,12 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         const int jr = r >> 2, pl = r & 3;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         const int N = 4 * p.N4;
-        int seg = 0;
-        for (int u = u_begin; u < u_end; ++seg) {
-            const int tile = u / UPT;
-            const int seg_end = min(u_end, (tile + 1) * UPT);
-            const bool whole = (u == tile * UPT) && (seg_end == (tile + 1) * UPT);
-            u = seg_end;
-            const int buf = seg & 1;
-            const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((seg >> 1) & 1), p.err);
+        for (int sg = 0; sg < cw.nseg; ++sg) {
+            const Seg g = cw.seg(p, sg);
+            const int tile = g.tile;
+            const bool whole = g.k0 == 0 && g.k1 == U;
+            const int buf = sg & 1;
+            const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((sg >> 1) & 1), p.err);
             // The four epilogue warps meet at named barriers below: decide
             // together whether to go on.
             if (epilogue_any(!got))
@@ -295,7 +435,26 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
             const int prow = tile * kPRows + jr;
             const bool row_ok = prow < p.N4;
             const int n = prow + pl * p.N4;
-            if (whole) {
+            if (split_cluster) {
+                if (cw.rank != 0) {
+                    // Add this CTA's partial sums into the leader's buffer,
+                    // then tell the leader (release: the adds come first).
+                    const uint32_t base = map_to_rank(smem_u32(red_buf), 0u);
+#pragma unroll
+                    for (int c = 0; c < BN; ++c)
+                        if (c < p.M)
+                            red_add_cluster(base + uint32_t((c * kRows + r) * 4), int32_t(v[c]));
+                    mbar_arrive_remote(map_to_rank(smem_u32(red_done), 0u));
+                    continue;
+                }
+                // Leader: wait for the other CTAs' sums, then finish the tile.
+                if (!mbar_wait_cluster_warp(red_done, 0u, p.err))
+                    continue;
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    v[c] += uint32_t(red_buf[c * kRows + r]);
+            }
+            if (whole || split_cluster) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
                     if (c < p.M && row_ok) {
@@ -309,7 +468,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                 }
                 continue;
             }
-            // Partial tile: add into the workspace, then count this CTA in.
+            // Stream-K partial tile: add into the workspace, then count this
+            // CTA in.
             int32_t *wt = p.ws + size_t(tile) * BN * kRows;
 #pragma unroll
             for (int c = 0; c < BN; ++c)
@@ -318,8 +478,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
             __threadfence();
             named_bar_sync(2, 128);
             if (threadIdx.x == 8 * 32) {
-                const int first = cta_of_unit(tile * UPT, p.total_units, p.grid);
-                const int last = cta_of_unit((tile + 1) * UPT - 1, p.total_units, p.grid);
+                const int first = cta_of_unit(tile * U, p.total_units, p.grid);
+                const int last = cta_of_unit((tile + 1) * U - 1, p.total_units, p.grid);
                 const int old = atomicAdd(p.cnt + tile, 1);
                 *fin_flag = (old == last - first) ? 1 : 0;
             }
@@ -353,25 +513,148 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
     tc_fence_after();
     if (warp == 1)
         tmem_dealloc(tmem_base, kTmemCols);
+    // No CTA leaves while another may still address its shared memory.
+    if (split_cluster)
+        cluster_sync_all();
+}
+
+template <int BN>
+cudaError_t configure_bn()
+{
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (configured_dev != dev) {
+        e = cudaFuncSetAttribute(smallm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(SmallMSmem<BN>::bytes + 1024));
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
+    return cudaSuccess;
 }
 
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap &mp, const CUtensorMap &mx, const SmallMParams &prm,
                       cudaStream_t stream)
 {
-    const size_t smem = SmallMSmem<BN>::bytes + 1024;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(smallm_tc_kernel<BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess)
-            return e;
-        configured_dev = dev;
+    cudaError_t e = configure_bn<BN>();
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SmallMSmem<BN>::bytes + 1024;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (prm.plan == kPlanCluster && prm.csize > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = unsigned(prm.csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
     }
-    smallm_tc_kernel<BN><<<prm.grid, kThreads, smem, stream>>>(mp, mx, prm);
-    return cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, smallm_tc_kernel<BN>, mp, mx, prm);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Largest cluster size C <= min(8, units per tile) such that tiles x C CTAs
+// fit the GPU in one wave as whole clusters (the occupancy API counts how
+// many clusters of C CTAs can be resident at once); 1 if none does.
+template <int BN>
+int pick_cluster(int tiles, int units)
+{
+    struct Key {
+        int dev, tiles, units;
+    };
+    static std::mutex mu;
+    static std::vector<std::pair<Key, int>> memo;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto &kv : memo)
+            if (kv.first.dev == dev && kv.first.tiles == tiles && kv.first.units == units)
+                return kv.second;
+    }
+    int best = 1;
+    const int sms = device_sm_count();
+    if (configure_bn<BN>() == cudaSuccess) {
+        for (int c = std::min(kMaxCluster, units); c >= 2; --c) {
+            if (tiles * c > sms)
+                continue;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(tiles * c);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = SmallMSmem<BN>::bytes + 1024;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = unsigned(c);
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int active = 0;
+            if (cudaOccupancyMaxActiveClusters(&active, smallm_tc_kernel<BN>, &cfg) ==
+                    cudaSuccess &&
+                active >= tiles) {
+                best = c;
+                break;
+            }
+            cudaGetLastError();  // an unsupported size is not an error of the call
+        }
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    memo.push_back({Key{dev, tiles, units}, best});
+    return best;
+}
+
+bool fill_params(SmallMParams &prm, CUtensorMap &map_p, CUtensorMap &map_x,
+                 const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
+                 const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K)
+{
+    const int BN = M <= 16 ? 16 : 32;
+    if (!make_map(&map_p, packed, K, N / 4, kPRows) || !make_map(&map_x, xq, K, M, BN))
+        return false;
+    prm = SmallMParams{};
+    prm.N4 = N / 4;
+    prm.K = K;
+    prm.M = M;
+    prm.tiles = (prm.N4 + kPRows - 1) / kPRows;
+    prm.units_per_tile = (K + kUnitK - 1) / kUnitK;
+    prm.total_units = prm.tiles * prm.units_per_tile;
+    prm.w_scale = w_scale;
+    prm.x_scale = x_scale;
+    prm.x_sum = x_sum;
+    prm.y = y;
+    prm.acc_out = acc_out;
+    prm.err = device_error_word();
+    return prm.err != nullptr;
+}
+
+// The stream-K plan on caller-provided, zero-filled scratch.
+cudaError_t launch_smallm_streamk(const uint8_t *packed, float w_scale, const int8_t *xq,
+                                  const float *x_scale, const int32_t *x_sum, float *y,
+                                  int32_t *acc_out, int M, int N, int K, void *workspace,
+                                  cudaStream_t stream)
+{
+    if (M < 1 || M > 32)
+        return cudaErrorInvalidValue;
+    const int BN = M <= 16 ? 16 : 32;
+    CUtensorMap map_p, map_x;
+    SmallMParams prm;
+    if (!fill_params(prm, map_p, map_x, packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K))
+        return cudaErrorInvalidValue;
+    prm.plan = kPlanStreamK;
+    prm.csize = 1;
+    prm.grid = std::min({prm.total_units, device_sm_count(), kMaxGrid});
+    prm.ws = static_cast<int32_t *>(workspace);
+    prm.cnt = prm.ws + size_t(prm.tiles) * BN * kRows;
+    return BN == 16 ? launch_bn<16>(map_p, map_x, prm, stream) : launch_bn<32>(map_p, map_x, prm, stream);
 }
 
 // Fixed scratch for tq_gemv_noalloc: the stream-K partial sums and tile
@@ -391,39 +674,26 @@ size_t smallm_workspace_bytes(int N, int M)
 
 cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
                              const float *x_scale, const int32_t *x_sum, float *y,
-                             int32_t *acc_out, int M, int N, int K, void *workspace,
-                             cudaStream_t stream)
+                             int32_t *acc_out, int M, int N, int K, cudaStream_t stream)
 {
     if (M < 1 || M > 32)
         return cudaErrorInvalidValue;
     const int BN = M <= 16 ? 16 : 32;
     CUtensorMap map_p, map_x;
-    if (!make_map(&map_p, packed, K, N / 4, kPRows) || !make_map(&map_x, xq, K, M, BN))
-        return cudaErrorInvalidValue;
     SmallMParams prm;
-    prm.N4 = N / 4;
-    prm.K = K;
-    prm.M = M;
-    prm.tiles = (prm.N4 + kPRows - 1) / kPRows;
-    prm.units_per_tile = (K + kUnitK - 1) / kUnitK;
-    prm.total_units = prm.tiles * prm.units_per_tile;
-    prm.grid = std::min({prm.total_units, device_sm_count(), kMaxGrid});
-    prm.w_scale = w_scale;
-    prm.x_scale = x_scale;
-    prm.x_sum = x_sum;
-    prm.y = y;
-    prm.acc_out = acc_out;
-    prm.ws = static_cast<int32_t *>(workspace);
-    prm.cnt = prm.ws + size_t(prm.tiles) * BN * kRows;
-    prm.err = device_error_word();
-    if (!prm.err)
-        return cudaErrorUnknown;
+    if (!fill_params(prm, map_p, map_x, packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K))
+        return cudaErrorInvalidValue;
+    prm.plan = kPlanCluster;
+    prm.csize = BN == 16 ? pick_cluster<16>(prm.tiles, prm.units_per_tile)
+                         : pick_cluster<32>(prm.tiles, prm.units_per_tile);
+    prm.grid = prm.csize > 1 ? prm.tiles * prm.csize
+                             : std::min({prm.tiles, device_sm_count(), kMaxGrid});
     return BN == 16 ? launch_bn<16>(map_p, map_x, prm, stream) : launch_bn<32>(map_p, map_x, prm, stream);
 }
 
 size_t noalloc_scratch_capacity() { return kNoAllocScratchBytes; }
 
-// The same kernel with the fixed scratch above. The device address of the
+// The stream-K plan with the fixed scratch above. The device address of the
 // scratch array is looked up once per device (on that device's first call)
 // with cudaGetSymbolAddress; host code cannot use the array's name as a
 // device pointer. The part the call uses is zero-filled on `stream` before
@@ -452,8 +722,8 @@ cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const
     err = cudaMemsetAsync(scratch[dev], 0, need, stream);
     if (err != cudaSuccess)
         return err;
-    return launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
-                            scratch[dev], stream);
+    return launch_smallm_streamk(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
+                                 scratch[dev], stream);
 }
 
 }  // namespace tq

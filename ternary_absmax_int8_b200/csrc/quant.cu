@@ -2,15 +2,15 @@
 //
 // BitNet b1.58 quantises activations to 8 bits per token by their largest
 // magnitude (1bit.systems post "the full arc ...", paper list item 1). The
-// pages give no formula; the one used (shared with the header tq.h):
+// per-element arithmetic (quant_core.cuh, shared with the stack GEMV's fused
+// quantiser):
 //   amax = max_k |x|, s = fl32(127/amax), q = clamp(rne(fl32(x*s)), -127, 127),
 //   x_scale = fl32(amax/127), x_sum = sum q; amax == 0 gives zeros.
-// Each rounding is an explicit _rn intrinsic, so the result does not depend
-// on compiler contraction or fast-math settings.
 //
 // One CTA per token row. Pass 1 reads the row as 16-byte vectors and reduces
 // |x| to amax; pass 2 re-reads it (an L1/L2 hit), converts and writes 8 codes
 // per vector, and reduces the code sum. HBM traffic: 2K bytes in, K + 8 out.
+#include "quant_core.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -18,34 +18,6 @@ namespace tq {
 namespace {
 
 constexpr int kQuantThreads = 256;
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ float absmax8(uint4 u)
-{
-    float a = fmaxf(fabsf(bf16_lo(u.x)), fabsf(bf16_hi(u.x)));
-    a = fmaxf(a, fmaxf(fabsf(bf16_lo(u.y)), fabsf(bf16_hi(u.y))));
-    a = fmaxf(a, fmaxf(fabsf(bf16_lo(u.z)), fabsf(bf16_hi(u.z))));
-    a = fmaxf(a, fmaxf(fabsf(bf16_lo(u.w)), fabsf(bf16_hi(u.w))));
-    return a;
-}
-
-__device__ __forceinline__ int code_of(float v, float s)
-{
-    int r = __float2int_rn(__fmul_rn(v, s));  // one fp32 rounding, then ties-to-even
-    return min(max(r, -127), 127);
-}
-
-// Quantise two bf16 values held in one 32-bit word; returns two int8 codes in
-// the low 16 bits and adds them to *sum.
-__device__ __forceinline__ uint32_t quant2(uint32_t w, float s, int *sum)
-{
-    int a = code_of(bf16_lo(w), s);
-    int b = code_of(bf16_hi(w), s);
-    *sum += a + b;
-    return (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8);
-}
 
 // Reduce v over the block with op; `identity` is op's neutral element (it
 // fills the lanes of the final warp that have no partial to contribute).
@@ -93,19 +65,14 @@ __device__ void quant_row(const uint16_t *__restrict__ x, int8_t *__restrict__ x
         amax = fmaxf(amax, absmax8(__ldg(xv + v)));
     amax = block_reduce(amax, MaxOp(), 0.0f, red_f);
 
-    const float s = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const float s = quant_inv_scale(amax);
     int sum = 0;
     uint2 *qv = reinterpret_cast<uint2 *>(xq);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        const uint4 u = __ldg(xv + v);
-        uint2 o;
-        o.x = quant2(u.x, s, &sum) | (quant2(u.y, s, &sum) << 16);
-        o.y = quant2(u.z, s, &sum) | (quant2(u.w, s, &sum) << 16);
-        qv[v] = o;
-    }
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x)
+        qv[v] = quant8(__ldg(xv + v), s, &sum);
     sum = block_reduce(sum, AddOp(), 0, red_i);
     if (threadIdx.x == 0) {
-        *x_scale = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+        *x_scale = quant_scale(amax);
         if (x_sum)
             *x_sum = sum;
     }

@@ -35,41 +35,6 @@ unsigned *device_error_word()
     return cache[dev];
 }
 
-void *device_workspace(size_t bytes, cudaError_t *err)
-{
-    static std::mutex mu;
-    static void *buf[64] = {nullptr};
-    static size_t cap[64] = {0};
-    std::lock_guard<std::mutex> lock(mu);
-    int dev = 0;
-    *err = cudaGetDevice(&dev);
-    if (*err != cudaSuccess)
-        return nullptr;
-    if (dev < 0 || dev >= 64) {
-        *err = cudaErrorInvalidDevice;
-        return nullptr;
-    }
-    if (cap[dev] < bytes) {
-        if (buf[dev]) {
-            // cudaFree waits for work that may still use the old buffer
-            cudaFree(buf[dev]);
-            buf[dev] = nullptr;
-            cap[dev] = 0;
-        }
-        const size_t want = std::max(bytes, size_t(1) << 20);
-        *err = cudaMalloc(&buf[dev], want);
-        if (*err != cudaSuccess) {
-            buf[dev] = nullptr;
-            return nullptr;
-        }
-        *err = cudaMemset(buf[dev], 0, want);
-        if (*err != cudaSuccess)
-            return nullptr;
-        cap[dev] = want;
-    }
-    return buf[dev];
-}
-
 int device_sm_count()
 {
     static int cache[64] = {0};
@@ -144,6 +109,14 @@ tq_status check_gemv_args(const char *fn, const uint8_t *packed, const int8_t *x
     return TQ_OK;
 }
 
+// Host staging of the stack quantiser's launch parameters (too large for
+// the stack), one per calling thread.
+tq::QuantStackParams *quant_params()
+{
+    static thread_local tq::QuantStackParams params;
+    return &params;
+}
+
 // K == 0: every accumulator is 0 and so is every output.
 tq_status zero_outputs(float *y, int32_t *acc_out, size_t count, cudaStream_t s)
 {
@@ -162,32 +135,29 @@ tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
         const int mg = M - m0 < tq::kStreamMaxTokens ? M - m0 : tq::kStreamMaxTokens;
         tq::StreamEntry e = {};
         e.packed = packed;
-        e.xq = xq + size_t(m0) * K;
-        e.x_scale = x_scale + m0;
-        e.x_sum = x_sum + m0;
+        // Inputs only: a launch that does not quantise never writes them.
+        e.xq = const_cast<int8_t *>(xq) + size_t(m0) * K;
+        e.x_scale = const_cast<float *>(x_scale) + m0;
+        e.x_sum = const_cast<int32_t *>(x_sum) + m0;
         e.y = y + size_t(m0) * N;
         e.acc_out = acc_out ? acc_out + size_t(m0) * N : nullptr;
         e.w_scale = w_scale;
         e.N4 = N / 4;
         e.K = K;
-        cudaError_t err = tq::launch_stream_gemv(&e, 1, mg, false, true, stream);
+        cudaError_t err = tq::launch_stream_gemv(&e, 1, mg, false, true, false, stream);
         if (err != cudaSuccess)
             return cuda_fail(err, fn);
     }
     return ok();
 }
 
-// 5 <= M <= 32: the tensor-core batched-decode kernel with its split-K scratch.
+// 5 <= M <= 32: the tensor-core batched-decode kernel.
 tq_status smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
                     const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K,
                     cudaStream_t stream, const char *fn)
 {
-    cudaError_t err = cudaSuccess;
-    void *ws = tq::device_workspace(tq::smallm_workspace_bytes(N, M), &err);
-    if (!ws)
-        return cuda_fail(err, fn);
-    err = tq::launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, ws,
-                               stream);
+    cudaError_t err = tq::launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N,
+                                           K, stream);
     return err == cudaSuccess ? ok() : cuda_fail(err, fn);
 }
 
@@ -334,7 +304,7 @@ tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t s
         q.K = p.K;
         list.push_back(q);
     }
-    static thread_local tq::QuantStackParams params;
+    tq::QuantStackParams &params = *quant_params();
     for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
         const size_t n = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
         params.n = int(n);
@@ -350,12 +320,13 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
 {
     if (n_proj < 0)
         return fail(TQ_ERR_SHAPE, "tq_gemv_stack: n_proj=%d", n_proj);
-    if (flags & ~unsigned(TQ_STACK_OVERLAP_PREV))
+    if (flags & ~unsigned(TQ_STACK_OVERLAP_PREV | TQ_STACK_QUANTIZE))
         return fail(TQ_ERR_VALUE, "tq_gemv_stack: unknown flags 0x%x", flags);
     if (n_proj == 0)
         return ok();
     if (!projs)
         return fail(TQ_ERR_NULL, "tq_gemv_stack: projs is NULL");
+    const bool quant = (flags & TQ_STACK_QUANTIZE) != 0;
     std::vector<tq::StreamEntry> list;
     list.reserve(size_t(n_proj));
     for (int j = 0; j < n_proj; ++j) {
@@ -366,16 +337,40 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
             check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, 1, p.N, p.K);
         if (st != TQ_OK)
             return st;
-        if (p.N == 0)
+        if (quant && p.K > 0 && !p.x)
+            return fail(TQ_ERR_NULL, "%s: x is NULL (TQ_STACK_QUANTIZE)", fn);
+        if (quant && p.K > 0 && !aligned(p.x, 16))
+            return fail(TQ_ERR_ALIGN, "%s: x must be 16-byte aligned", fn);
+        if (p.N == 0 && !quant)
             continue;
         if (p.K == 0) {
+            // Every accumulator is 0; a quantising call also reports the
+            // empty token's scale and sum as 0.
+            cudaError_t e = cudaSuccess;
+            if (quant)
+                e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
+            if (e == cudaSuccess && quant)
+                e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, fn);
             st = zero_outputs(p.y, p.acc_out, size_t(p.N), stream);
             if (st != TQ_OK)
                 return st;
             continue;
         }
+        if (p.N == 0) {
+            // Nothing to multiply, but the quantiser's outputs are owed.
+            tq::QuantStackParams *qp = quant_params();
+            qp->n = 1;
+            qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
+            cudaError_t e = tq::launch_quant_stack(*qp, stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, fn);
+            continue;
+        }
         tq::StreamEntry e = {};
         e.packed = p.packed;
+        e.xb = p.x;
         e.xq = p.xq;
         e.x_scale = p.x_scale;
         e.x_sum = p.x_sum;
@@ -390,7 +385,7 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
     for (size_t base = 0; base < list.size(); base += tq::kStreamStackMax) {
         const int n = int(std::min(list.size() - base, size_t(tq::kStreamStackMax)));
         cudaError_t e = tq::launch_stream_gemv(list.data() + base, n, 1, overlap && base == 0,
-                                               false, stream);
+                                               false, quant, stream);
         if (e != cudaSuccess)
             return cuda_fail(e, "tq_gemv_stack");
     }

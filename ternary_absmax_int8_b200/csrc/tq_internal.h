@@ -39,9 +39,10 @@ cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream);
 // so that rows_per_tile << ksplit work items keep every consumer warp busy.
 struct StreamEntry {
     const uint8_t *packed;  // [N4, K]
-    const int8_t *xq;       // [M, K]
-    const float *x_scale;   // [M]
-    const int32_t *x_sum;   // [M]
+    const uint16_t *xb;     // [M, K] bf16 (read only when the launch quantises)
+    int8_t *xq;             // [M, K] (written when the launch quantises, else read)
+    float *x_scale;         // [M]    (likewise)
+    int32_t *x_sum;         // [M]    (likewise)
     float *y;               // [M, 4*N4]
     int32_t *acc_out;       // [M, 4*N4] or null
     float w_scale;
@@ -68,6 +69,7 @@ struct StreamParams {
     int w_slot;        // bytes of a ring stage (a tile's packed rows + activations)
     int stages;
     int overlap_prev;  // start weight copies before the previous grid completes
+    int quant;         // quantise each entry's bf16 activations in the launch (M == 1)
     int head_bytes;    // shared memory for the entry table and the per-token scales
     unsigned *err;     // the library's device error word
     // Work split: CTA b streams tiles cta_tile0[b] .. cta_tile0[b+1]-1 (a
@@ -90,33 +92,32 @@ struct StreamLaunch {
 
 // Plan tiles for a set of entries (fills rows_per_tile, ksplit, tile_begin,
 // total_tiles, x_slot, w_slot, stages) and launch. `single` selects the
-// small-launch heuristics for one projection.
+// small-launch heuristics for one projection. With `quant` (M == 1 only) the
+// kernel quantises each entry's bf16 activations itself and writes xq,
+// x_scale and x_sum as the standalone quantiser would.
 cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_prev,
-                               bool single, cudaStream_t stream);
+                               bool single, bool quant, cudaStream_t stream);
 
 int device_sm_count();
 
 // ---------------------------------------- batched decode on the tensor cores
-// 1 <= M <= 32. `workspace` is zero-filled device memory of at least
-// smallm_workspace_bytes(N, M) bytes; the kernel leaves it zero-filled.
-size_t smallm_workspace_bytes(int N, int M);
+// 1 <= M <= 32. Thread-block clusters split a tile's K range when there are
+// fewer tiles than SMs; no scratch memory is involved.
 cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
                              const float *x_scale, const int32_t *x_sum, float *y,
-                             int32_t *acc_out, int M, int N, int K, void *workspace,
-                             cudaStream_t stream);
+                             int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
 
-// The same kernel on a fixed, statically allocated device scratch (no
-// allocation by anyone); cudaErrorInvalidValue when the shape needs more than
-// noalloc_scratch_capacity() bytes of it.
+// Bytes of zero-filled scratch the stream-K formulation of the same kernel
+// needs (its split-K partial sums and per-tile counters).
+size_t smallm_workspace_bytes(int N, int M);
+
+// The stream-K formulation on a fixed, statically allocated device scratch
+// (no allocation by anyone); cudaErrorInvalidValue when the shape needs more
+// than noalloc_scratch_capacity() bytes of it.
 size_t noalloc_scratch_capacity();
 cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
                                      const float *x_scale, const int32_t *x_sum, float *y,
                                      int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
-
-// Library-owned, zero-filled scratch on the current device, at least `bytes`
-// long (allocated on first use, grown when a call needs more). Returns null
-// and sets *err on failure.
-void *device_workspace(size_t bytes, cudaError_t *err);
 
 // Device address of the library's error word on the current device.
 unsigned *device_error_word();

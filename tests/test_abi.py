@@ -128,6 +128,15 @@ def test_stack_argument_checks():
     with pytest.raises(tq.TQError) as e:
         tq.tq_quantize_act_stack([tq.make_proj(**dict(good, K=20))], stream=0)
     assert e.value.name == "TQ_ERR_SHAPE"
+    # the quantising launch needs the bf16 activations, 16-byte aligned
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**dict(good, x=None))], flags=tq.TQ_STACK_QUANTIZE,
+                         stream=0)
+    assert e.value.name == "TQ_ERR_NULL" and "x is NULL" in str(e.value)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**dict(good, x=A + 8))], flags=tq.TQ_STACK_QUANTIZE,
+                         stream=0)
+    assert e.value.name == "TQ_ERR_ALIGN"
     tq.tq_gemv_stack([], stream=0)
     tq.tq_quantize_act_stack([], stream=0)
 

@@ -1,7 +1,8 @@
-"""GPU parity of the grouped decode calls (tq_quantize_act_stack +
-tq_gemv_stack) on the full 30-layer stack (210 projections, M = 1), in the
-launch configuration the bench times (one quantise launch, then one stack
-launch allowed to overlap it), against the oracle on every output."""
+"""GPU parity of the grouped decode calls on the full 30-layer stack (210
+projections, M = 1) against the oracle on every output: the one-launch form
+the bench times (tq_gemv_stack with TQ_STACK_QUANTIZE: quantise and multiply
+in the same launch) and the two-launch form (tq_quantize_act_stack, then
+tq_gemv_stack, allowed to overlap it)."""
 import numpy as np
 import pytest
 import torch
@@ -38,6 +39,15 @@ class Stack:
         tq.tq_gemv_stack(self.table, flags=flags)
         torch.cuda.synchronize()
 
+    def run_fused(self):
+        # Poison the quantiser's outputs first: the fused launch must write them.
+        for q in self.xq:
+            q.fill_(-128)
+        self.xs.fill_(float("nan"))
+        self.xsum.fill_(-(2 ** 31))
+        tq.tq_gemv_stack(self.table, flags=tq.TQ_STACK_QUANTIZE)
+        torch.cuda.synchronize()
+
 
 def _oracle(p):
     P = oracle.pack(p.w)
@@ -64,20 +74,47 @@ def test_layer_stack_small(cuda_device):
     for flags in (0, tq.TQ_STACK_OVERLAP_PREV):
         st.run(flags)
         _check(st, refs)
+    st.run_fused()
+    _check(st, refs)
 
 
-def test_full_stack_30_layers(cuda_device):
+def test_full_stack_30_layers_fused(cuda_device):
+    # The bench's launch: one tq_gemv_stack(TQ_STACK_QUANTIZE) for all 210.
+    projs = list(make_projections(stack_shapes(30), M=1, seed=0))
+    st = Stack(projs)
+    refs = parallel_map(_oracle, projs)
+    st.run_fused()
+    _check(st, refs)
+    # repeat: byte-identical outputs
+    y0 = [y.clone() for y in st.y]
+    st.run_fused()
+    for a, b in zip(y0, st.y):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    assert tq.tq_device_error(reset=True) == 0
+
+
+def test_full_stack_30_layers_two_launches(cuda_device):
     projs = list(make_projections(stack_shapes(30), M=1, seed=0))
     st = Stack(projs)
     refs = parallel_map(_oracle, projs)
     st.run(tq.TQ_STACK_OVERLAP_PREV)
     _check(st, refs)
-    # repeat: byte-identical outputs
-    y0 = [y.clone() for y in st.y]
-    st.run(tq.TQ_STACK_OVERLAP_PREV)
-    for a, b in zip(y0, st.y):
-        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
     assert tq.tq_device_error(reset=True) == 0
+
+
+def test_fused_stack_degenerate_rows(cuda_device):
+    # An all-zero token (amax = 0), a token whose every entry is +-max, and
+    # all-zero / all-(+1) weights, through the quantising launch.
+    projs = list(make_projections([("a", 640, 2560), ("b", 2560, 6912), ("c", 64, 512)],
+                                  M=1, seed=5))
+    projs[0].x_bf16[:] = 0
+    projs[1].x_bf16[:] = np.where(np.arange(6912) % 2 == 0, 0x4120, 0xC120).astype(np.uint16)
+    projs[2].w[:] = 1
+    projs[0].w[: 320] = 0
+    st = Stack(projs)
+    refs = parallel_map(_oracle, projs)
+    st.run_fused()
+    _check(st, refs)
 
 
 def test_mixed_stack_more_than_one_launch(cuda_device):
@@ -87,4 +124,6 @@ def test_mixed_stack_more_than_one_launch(cuda_device):
     st = Stack(projs)
     refs = parallel_map(_oracle, projs)
     st.run(0)
+    _check(st, refs)
+    st.run_fused()
     _check(st, refs)

@@ -1,8 +1,9 @@
 """tq_gemv_noalloc, the entry point for callers that cannot allocate device
 memory (their device memory belongs to another allocator, or an allocation's
-implicit synchronisation is not acceptable on their path). It must give the
-same results as tq_gemv, which keeps the same kernel's split-K partial sums in
-library-allocated scratch, on consecutive calls that share its fixed scratch.
+implicit synchronisation is not acceptable on their path). It runs the
+stream-K formulation of the batched-decode kernel on a fixed device array and
+must give the same results as tq_gemv (the cluster formulation, no scratch) on
+consecutive calls that share that array.
 
 Collected last on purpose (file name), so that a run stopping at the first
 failure has already run every other test; it also passes alone in a fresh
