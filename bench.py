@@ -4,9 +4,10 @@ Default workload (the headline): the decode layer stack -- 30 independently
 seeded copies of a BitNet-b1.58-2B-4T decoder layer, 7 ternary projections
 each (210 projections, 2.08e9 weights, 521 MB packed), M = 1. One step is one
 pass of the whole path over that stack: absmax-int8 quantisation of 210 fresh
-bf16 activation vectors (one launch) and the 210 GEMVs with their scale
-epilogues (one persistent launch). The weight stream is larger than L2, so no
-flush is needed between steps.
+bf16 activation vectors and the 210 GEMVs with their scale epilogues, in one
+persistent launch (tq_gemv_stack with TQ_STACK_QUANTIZE). The weight stream is
+larger than L2, so no flush is needed between steps. Other workloads run one
+quantiser launch and one GEMV launch per projection.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME]
@@ -14,9 +15,10 @@ flush is needed between steps.
 value  = algorithmic bytes of a step (all ranks) / device time per step, GB/s
 e2e    = the same metric through the same calls with host buffers: each step
          copies the activations in from pinned host memory and the outputs back
-roofline = the stack GEMV kernel alone (its algorithmic bytes / its average
-         CUDA-event duration inside the timed region) against the measured HBM
-         copy bandwidth.
+roofline = the dominant kernel (the quantising stack GEMV for the stack; the
+         GEMV or prefill GEMM otherwise): its algorithmic bytes (or int8 ops)
+         over its average CUDA-event duration inside the timed region, against
+         the measured HBM copy bandwidth (or int8 tensor peak).
 --impl reference times the oracle (plain C, one host thread) on a bounded
 sample of the same workload; it is the CPU baseline, not a GPU arm.
 With N > 1 (torchrun) every rank runs its own replica of the workload
@@ -63,7 +65,24 @@ def quant_bytes(K: int, M: int) -> int:
 
 
 def step_bytes(projs) -> int:
+    """Quantiser launch + GEMV launch per projection."""
     return sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
+
+
+def is_stack(workload: str, M: int) -> bool:
+    return workload.startswith("stack") and M == 1
+
+
+def workload_step_bytes(workload: str, projs) -> int:
+    """Algorithmic bytes of one step of `workload` over `projs` (both arms)."""
+    return fused_step_bytes(projs) if is_stack(workload, projs[0].M) else step_bytes(projs)
+
+
+def fused_step_bytes(projs) -> int:
+    """One quantising GEMV launch per projection: the GEMV's bytes with bf16
+    activations read (2K) and int8 codes written (K) instead of int8 codes
+    read (K), plus the scale and sum written (8) instead of read (8)."""
+    return sum(algorithmic_bytes(p.N, p.K, p.M) + 2 * p.M * p.K for p in projs)
 
 
 # ----------------------------------------------------------------- helpers
@@ -147,7 +166,7 @@ def measured_tensor_peak():
 
 def stack_kernel_sha() -> str:
     h = hashlib.sha256()
-    for name in ("gemv_stream.cu", "tq_device.cuh", "tq_internal.h"):
+    for name in ("gemv_stream.cu", "quant_core.cuh", "tq_device.cuh", "tq_internal.h"):
         h.update(open(os.path.join(os.path.dirname(STACK_KERNEL_SRC), name), "rb").read())
     return h.hexdigest()[:16]
 
@@ -174,9 +193,11 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.set_device(dev)
     shapes, M = WORKLOADS[args.workload]
     projs = list(make_projections(shapes, M=M, seed=args.seed))
-    stack = args.workload.startswith("stack") and M == 1
-    sb = step_bytes(projs)
-    gemv_bytes = sum(algorithmic_bytes(p.N, p.K, p.M) for p in projs)
+    stack = is_stack(args.workload, M)
+    # The stack quantises inside its GEMV launch; the other workloads run the
+    # standalone quantiser first.
+    sb = workload_step_bytes(args.workload, projs)
+    gemv_bytes = sb if stack else sum(algorithmic_bytes(p.N, p.K, p.M) for p in projs)
     packed_bytes = sum(p.N * p.K // 4 for p in projs)
 
     # Weights: packed on the host by the library's packer, then resident in
@@ -217,25 +238,31 @@ def run_ours(args, rank: int, world: int):
     tables = [table(c) for c in range(copies)]
     stream = torch.cuda.current_stream()
 
-    def quant(c):
+    def quant(c, s):
         if stack:
-            tq.tq_quantize_act_stack(tables[c], stream=stream)
-        else:
-            for j, p in enumerate(projs):
-                t = tables[c][j]
-                tq.tq_quantize_act(t.x, t.xq, t.x_scale, t.x_sum, p.M, p.N, p.K, stream=stream)
+            return  # quantised inside the stack launch
+        for j, p in enumerate(projs):
+            t = tables[c][j]
+            tq.tq_quantize_act(t.x, t.xq, t.x_scale, t.x_sum, p.M, p.N, p.K, stream=s)
 
-    def gemv(c):
+    def gemv(c, s, first=True):
         if stack:
-            tq.tq_gemv_stack(tables[c], flags=tq.TQ_STACK_OVERLAP_PREV, stream=stream)
-        else:
-            for j, p in enumerate(projs):
-                t = tables[c][j]
-                call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
-                call(t.packed, t.w_scale, t.xq, t.x_scale, t.x_sum, t.y, None, p.M, p.N, p.K,
-                     stream=stream)
+            # Consecutive stack launches may overlap (the next one streams
+            # weights while the previous one drains); the first launch of a
+            # captured sequence has no predecessor to overlap.
+            flags = tq.TQ_STACK_QUANTIZE | (0 if first else tq.TQ_STACK_OVERLAP_PREV)
+            tq.tq_gemv_stack(tables[c], flags=flags, stream=s)
+            return
+        for j, p in enumerate(projs):
+            t = tables[c][j]
+            call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
+            call(t.packed, t.w_scale, t.xq, t.x_scale, t.x_sum, t.y, None, p.M, p.N, p.K, stream=s)
 
-    launches_per_step = 2 if stack else sum(1 + gemv_launches(p.M) for p in projs)
+    def step(c, s, first=True):
+        quant(c, s)
+        gemv(c, s, first)
+
+    launches_per_step = 1 if stack else sum(1 + gemv_launches(p.M) for p in projs)
 
     def barrier():
         if world > 1:
@@ -243,69 +270,103 @@ def run_ours(args, rank: int, world: int):
             dist.barrier()
 
     for i in range(args.warmup):
-        quant(i % copies)
-        gemv(i % copies)
+        step(i % copies, stream)
+    torch.cuda.synchronize()
+
+    # The timed steps replay CUDA graphs of the same library calls, so host
+    # launch overhead does not stretch the device time: a chunk graph holds
+    # S consecutive steps (a multiple of the rotated weight copies), and
+    # single-step graphs cover a remainder, so exactly K steps run.
+    K = args.steps
+    S = copies * max(1, 16 // copies)
+    n_chunks, rem = divmod(K, S)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=cs):
+            fn(cs)
+        return g
+
+    chunk_graph = capture(lambda cs: [step(i % copies, cs, first=(i == 0)) for i in range(S)])
+    single = [capture(lambda cs, c=c: step(c, cs)) for c in range(copies)] if rem else []
+    chunk_graph.replay()
+    for g in single:
+        g.replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(dev)
     clocks.start()
     time.sleep(0.3)
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    for i in range(K):
-        c = i % copies
-        ev[i][0].record(stream)
-        quant(c)
-        ev[i][1].record(stream)
-        gemv(c)
-        ev[i][2].record(stream)
+    t0.record(stream)
+    for _ in range(n_chunks):
+        chunk_graph.replay()
+    for i in range(rem):
+        single[(n_chunks * S + i) % copies].replay()
+    t1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
-    gemv_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    total_ms = t0.elapsed_time(t1)
 
-    # End to end: host activations in, host outputs out, every step. At least
-    # half a second of it, so that the clock samples see the GPU under load.
+    # The split between quantiser and GEMV launches (non-stack workloads):
+    # graphs of S steps' quantiser calls alone and GEMV calls alone.
+    def graph_ms(fn, reps=3):
+        g = capture(fn)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    if stack:
+        quant_ms_step, gemv_ms_step = 0.0, total_ms / K
+    else:
+        quant_ms_step = graph_ms(lambda cs: [quant(i % copies, cs) for i in range(S)]) / S
+        gemv_ms_step = graph_ms(lambda cs: [gemv(i % copies, cs) for i in range(S)]) / S
+
+    # End to end through the library calls themselves (no graph): host
+    # activations in, host outputs out, every step. At least half a second of
+    # it, so that the clock samples see the GPU under load.
     e2e_steps = max(K, int(0.5e3 / max(total_ms / K, 1e-3)))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(3):
         x_dev.copy_(x_host, non_blocking=True)
-        quant(i % copies)
-        gemv(i % copies)
+        step(i % copies, stream)
         y_host.copy_(y_dev, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
     e0.record(stream)
     for i in range(e2e_steps):
         x_dev.copy_(x_host, non_blocking=True)
-        quant(i % copies)
-        gemv(i % copies)
+        step(i % copies, stream)  # copies sit between launches: no overlap
         y_host.copy_(y_dev, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    # Per-projection GEMM timing (non-stack workloads): each projection's call
-    # alone, over the rotated weight copies, median of the repeats.
+    # Per-projection GEMM timing (non-stack workloads): a graph of R calls of
+    # one projection over the rotated weight copies, time per call.
     per_proj = []
     if not stack:
+        R = copies * max(1, 32 // copies)
         for j, p in enumerate(projs):
             call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
-            reps = max(20, min(200, K))
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(reps)]
-            for r in range(reps):
-                t_ = tables[r % copies][j]
-                evs[r][0].record(stream)
-                call(t_.packed, t_.w_scale, t_.xq, t_.x_scale, t_.x_sum, t_.y, None, p.M, p.N, p.K,
-                     stream=stream)
-                evs[r][1].record(stream)
-            torch.cuda.synchronize()
-            us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+
+            def proj_calls(cs, j=j, p=p, call=call):
+                for r in range(R):
+                    t_ = tables[r % copies][j]
+                    call(t_.packed, t_.w_scale, t_.xq, t_.x_scale, t_.x_sum, t_.y, None, p.M,
+                         p.N, p.K, stream=cs)
+
+            us = graph_ms(proj_calls) / R * 1e3
             entry = {"name": p.name, "N": p.N, "K": p.K, "M": p.M, "us": round(us, 3),
                      "GB_s": round(algorithmic_bytes(p.N, p.K, p.M) / (us * 1e3), 1)}
             if p.M > 24:
@@ -324,7 +385,7 @@ def run_ours(args, rank: int, world: int):
     ms_step = total_ms / K
     value = whole_job_rate(world, sb, ms_step) / 1e9
     peak, peak_kind = measured_peak()
-    gemv_avg = statistics.mean(gemv_ms)
+    gemv_avg = gemv_ms_step
     achieved = gemv_bytes / (gemv_avg * 1e6)
     traffic = recorded_traffic(args.workload)
     prefill = M > 24
@@ -380,8 +441,9 @@ def run_ours(args, rank: int, world: int):
         "passes_per_s": round(whole_job_rate(world, 1.0, ms_step), 1),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "us_per_projection": round(ms_step * 1e3 / len(projs), 4),
-        "quant_us_per_step": round(statistics.mean(quant_ms) * 1e3, 3),
+        "quant_us_per_step": round(quant_ms_step * 1e3, 3),
         "gemv_us_per_step": round(gemv_avg * 1e3, 3),
+        "quantiser": "fused into the stack launch" if stack else "separate launch",
         "roofline": roof,
         "e2e": {
             "value": round(whole_job_rate(world, sb, e2e_ms / e2e_steps) / 1e9, 1),
@@ -404,8 +466,10 @@ def run_ours(args, rank: int, world: int):
 
 
 def gemv_launches(M: int) -> int:
-    """Kernel launches of one tq_gemv / tq_gemm_prefill call at M tokens."""
-    return 1 if M >= 128 else -(-M // 4)
+    """Kernel launches of one tq_gemv / tq_gemm_prefill call at M tokens: one
+    (the streaming kernel up to 4 tokens, the batched-decode tensor-core
+    kernel up to 32, the prefill GEMM beyond)."""
+    return 1
 
 
 # ------------------------------------------------------------ CPU / oracle
@@ -425,7 +489,7 @@ def cpu_baseline(projs, args, budget_s: float = 10.0):
             q.M, q.x_bf16 = 16, p.x_bf16[:16]
             sp.append(q)
     packed = [(oracle.pack(p.w), p) for p in sp]
-    sb = step_bytes(sp)
+    sb = workload_step_bytes(args.workload, sp)
     passes, t0 = 0, time.perf_counter()
     while True:
         for P, p in packed:
@@ -455,7 +519,7 @@ def run_reference(args, rank: int, world: int):
         M = 16
     sp = list(make_projections(sample, M=M, seed=args.seed))
     packed = [(oracle.pack(p.w), p) for p in sp]
-    sb = step_bytes(sp)
+    sb = workload_step_bytes(args.workload, sp)
 
     def step():
         for P, p in packed:
