@@ -31,8 +31,9 @@
 //     its partial sums into a global scratch with integer atomics, and the
 //     CTA whose contribution completes the tile applies the epilogue and
 //     zeroes the scratch for the next call.
-// * Warp roles (12 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
-//   4..7 expansion, 8..11 epilogue. All mbarrier waits are bounded.
+// * Warp roles (16 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
+//   4..11 expansion (two sets of four warps, one TMEM lane quarter each,
+//   taking alternate units), 12..15 epilogue. All mbarrier waits are bounded.
 #include <algorithm>
 #include <mutex>
 #include <utility>
@@ -50,7 +51,10 @@ constexpr int kUnitK = 256;            // bytes of K per unit (two 128-byte boxe
 constexpr int kSP = 10;                // shared-memory stages (packed + activations)
 constexpr int kSA = 4;                 // tensor-memory A slots
 constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kExpandWarp0 = 4;        // expansion warps 4..11: two sets of four
+constexpr int kExpandSets = 2;         // set s expands the CTA's units s, s + 2, ...
+constexpr int kEpiWarp0 = 4 + 4 * kExpandSets;  // epilogue warps 12..15
 constexpr int kMaxGrid = 512;
 
 constexpr int kPlanStreamK = 0;
@@ -357,9 +361,10 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                 mbar_wait(&mma_done[s], uint32_t(((i - 1) / kSP) & 1), p.err);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= kExpandWarp0 && warp < kEpiWarp0) {
         // -------------------------------------------------- expansion
         const int q = warp & 3;                      // TMEM lane quarter
+        const int set = (warp - kExpandWarp0) >> 2;  // this warp's units: set, set + 2, ...
         const int j = 8 * q + (lane >> 2), pl = lane & 3;  // packed row, plane of this lane
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int i = 0;
@@ -367,6 +372,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         for (int sg = 0; sg < cw.nseg && ok; ++sg) {
             const Seg g = cw.seg(p, sg);
             for (int k = g.k0; k < g.k1; ++k, ++i) {
+                if (i % kExpandSets != set)
+                    continue;
                 const int s = i % kSP, sa = i % kSA;
                 ok = mbar_wait_warp(&tma_full[s], uint32_t((i / kSP) & 1), p.err);
                 if (ok && i >= kSA) {
@@ -389,8 +396,9 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                         v[4 * c + 2] = (w.z >> (2 * pl)) & 0x03030303u;
                         v[4 * c + 3] = (w.w >> (2 * pl)) & 0x03030303u;
                     }
-                    tmem_st32(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
+                    tmem_st32_async(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
                 }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -399,7 +407,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= kEpiWarp0) {
         // -------------------------------------------------- epilogue
         const int q = warp & 3;
         const int r = 32 * q + lane;                 // accumulator row = TMEM lane
@@ -477,7 +485,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                     atomicAdd(wt + c * kRows + r, int32_t(v[c]));
             __threadfence();
             named_bar_sync(2, 128);
-            if (threadIdx.x == 8 * 32) {
+            if (threadIdx.x == kEpiWarp0 * 32) {
                 const int first = cta_of_unit(tile * U, p.total_units, p.grid);
                 const int last = cta_of_unit((tile + 1) * U - 1, p.total_units, p.grid);
                 const int old = atomicAdd(p.cnt + tile, 1);
@@ -500,7 +508,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                         }
                     }
                 }
-                if (threadIdx.x == 8 * 32)
+                if (threadIdx.x == kEpiWarp0 * 32)
                     p.cnt[tile] = 0;
             }
             named_bar_sync(2, 128);  // fin_flag is reused by the next segment
