@@ -1,4 +1,4 @@
-// gemm_tc.cu -- prompt-processing (M >= 128 tokens) ternary GEMM on the
+// gemm_tc.cu -- prompt-processing (M >= 33 tokens) ternary GEMM on the
 // 5th-generation tensor cores (tcgen05, int8, accumulators in tensor memory).
 //
 // Prompt processing is bound by the GPU's matrix units rather than by bytes
@@ -11,20 +11,27 @@
 //   acc[m, n] = D[n, m] - x_sum[m]          (since w = c - 1)
 //   y[m, n] = float(acc) * (w_scale * x_scale[m])
 //
-// Tile: 128 output features x BN = 256 tokens, K in stages of 128 bytes.
-// The 128 features of a tile are 32 packed rows i0 .. i0+31 times the four
-// planes: MMA row r = 32 p + j is feature i0 + j + p N/4. So one 4 KB tile of
-// packed bytes (TMA, 128B-swizzled) expands into the 16 KB A operand.
+// Tile: G x 128 output features x BN tokens, K in stages of 128 bytes; G (1
+// or 2) MMA groups of 128 rows share each activation stage, so the
+// activation operand is read from L2 once per G x 128 features. In group g,
+// MMA row r = 32 p + j is feature i0 + 32 g + j + p N/4: one TMA tile of
+// G x 32 packed rows (128B-swizzled) expands into the G A operands of 16 KB.
+// The host picks (G, BN) in {(2,256), (2,128), (1,128), (1,64)} for the
+// fewest waves of tile work over the SMs (larger tiles on ties), since a
+// 512-token prompt through a 2560-feature projection makes only 20 tiles of
+// the largest shape.
 //
-// Warp roles (10 warps, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer: packed tile + activation tile per K stage
-//   warp 1      TMEM allocator; lane 0 issues the MMAs and commits
-//   warps 2..5  expand the codes into the A stage (canonical K-major,
-//               128B swizzle), fence to the async proxy, signal the MMA
-//   warps 6..9  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//               32 (w % 4) ..), subtract x_sum, scale, store y
-// Accumulators are double-buffered in TMEM (2 x 256 columns) so the epilogue
-// of tile t overlaps the MMAs of tile t + 1. Every mbarrier wait is bounded.
+// Warp roles (14 warps, one CTA per SM, persistent over tiles):
+//   warp 0       TMA producer: packed tile + activation tile per K stage
+//   warp 1       TMEM allocator; lane 0 issues the MMAs and commits
+//   warps 2..5   expand the codes into the A stage (canonical K-major, 128B
+//                swizzle), fence to the async proxy, signal the MMA
+//   warps 6..13  epilogue: warp w reads TMEM lane quarter w % 4 of its group
+//                (G = 2) or of its half of the columns (G = 1), subtracts
+//                x_sum, scales, stores y
+// The accumulator (G x BN columns) is single-buffered: a CTA's next tile
+// starts its MMAs once the epilogue has drained it. Every mbarrier wait is
+// bounded; loads never use cluster multicast.
 #include <algorithm>
 #include <cstring>
 
@@ -34,17 +41,13 @@ namespace tq {
 
 namespace {
 
-constexpr int kBM = 128;         // features per tile (MMA M)
-constexpr int kBN = 256;         // tokens per tile (MMA N)
-constexpr int kBK = 128;         // bytes of K per stage
-constexpr int kStages = 4;
-constexpr int kPackedRows = kBM / 4;
-constexpr int kABytes = kBM * kBK;           // 16 KB
-constexpr int kBBytes = kBN * kBK;           // 32 KB
-constexpr int kPBytes = kPackedRows * kBK;   // 4 KB
-constexpr int kThreads = 320;
-constexpr int kTmemCols = 2 * kBN;           // two accumulator buffers
-constexpr uint32_t kIdesc = idesc_i8_u8s8(kBM, kBN);
+constexpr int kGM = 128;                // MMA M: rows of one group
+constexpr int kBK = 128;                // bytes of K per stage
+constexpr int kAGroupBytes = kGM * kBK; // 16 KB
+constexpr int kThreads = 448;
+constexpr int kEpiWarp0 = 6;
+constexpr int kEpiWarps = 8;
+constexpr size_t kSmemLimit = 227 * 1024;
 
 struct PrefillParams {
     int N4, K, M;
@@ -57,57 +60,88 @@ struct PrefillParams {
     unsigned *err;
 };
 
-struct PrefillSmem {
+template <int G, int BN>
+struct PrefillShape {
+    static constexpr int kPackedRows = 32 * G;          // packed rows per tile
+    static constexpr int kABytes = G * kAGroupBytes;
+    static constexpr int kBBytes = BN * kBK;
+    static constexpr int kPBytes = kPackedRows * kBK;
+    static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+    static constexpr int kBarCount_(int s) { return 4 * s + 2; }
+    // as many stages as fit next to the barriers and the 1 KB alignment slack
+    static constexpr int kStages =
+        int((kSmemLimit - 1024 - 256) / size_t(kStageBytes)) > 6
+            ? 6
+            : int((kSmemLimit - 1024 - 256) / size_t(kStageBytes));
+    static constexpr int kAccCols = G * BN;
+    static constexpr int kTmemCols = kAccCols < 32 ? 32 : kAccCols;  // a power of two here
     // 1024-byte aligned operand stages (the 128B swizzle atom is 1 KB)
     static constexpr size_t a_off = 0;
     static constexpr size_t b_off = a_off + size_t(kStages) * kABytes;
     static constexpr size_t p_off = b_off + size_t(kStages) * kBBytes;
     static constexpr size_t bar_off = p_off + size_t(kStages) * kPBytes;
-    // barriers: tma_full, a_full, mma_done, p_free per stage; acc_full, acc_empty x2
-    static constexpr int kBarCount = 4 * kStages + 4;
-    static constexpr size_t tmem_slot_off = bar_off + kBarCount * 8;
+    // barriers: tma_full, a_full, mma_done, p_free per stage; acc_full, acc_empty
+    static constexpr size_t tmem_slot_off = bar_off + size_t(kBarCount_(kStages)) * 8;
     static constexpr size_t bytes = tmem_slot_off + 16;
+    static_assert(kStages >= 2, "two stages at least");
+    static_assert(bytes + 1024 <= kSmemLimit, "shared memory");
+    static_assert((kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512, "tensor memory");
 };
 
+// One output element: y (and the exact accumulator when asked).
+__device__ __forceinline__ void store_out(const PrefillParams &p, int m, int n, int32_t d,
+                                          float t, int32_t xs)
+{
+    const int32_t acc = d - xs;
+    const size_t o = size_t(m) * (4 * size_t(p.N4)) + n;
+    p.y[o] = __fmul_rn(__int2float_rn(acc), t);
+    if (p.acc_out)
+        p.acc_out[o] = acc;
+}
+
+template <int G, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
                   const __grid_constant__ PrefillParams p)
 {
+    using S = PrefillShape<G, BN>;
+    constexpr int kStages = S::kStages;
+    constexpr uint32_t kIdesc = idesc_i8_u8s8(kGM, BN);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the dynamic base is only guaranteed 16-byte aligned: round up to 1 KB
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem + PrefillSmem::a_off;
-    uint8_t *sB = smem + PrefillSmem::b_off;
-    uint8_t *sP = smem + PrefillSmem::p_off;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PrefillSmem::bar_off);
+    uint8_t *sA = smem + S::a_off;
+    uint8_t *sB = smem + S::b_off;
+    uint8_t *sP = smem + S::p_off;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::bar_off);
     uint64_t *tma_full = bars;
     uint64_t *a_full = bars + kStages;
     uint64_t *mma_done = bars + 2 * kStages;
     uint64_t *p_free = bars + 3 * kStages;
     uint64_t *acc_full = bars + 4 * kStages;
-    uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PrefillSmem::tmem_slot_off);
+    uint64_t *acc_empty = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = p.feat_tiles * p.tok_tiles;
     const int KS = p.k_stages;
 
     if (threadIdx.x == 0) {
+        prefetch_tensormap(&map_p);
+        prefetch_tensormap(&map_x);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&tma_full[s], 1);
             mbar_init(&a_full[s], 4);
             mbar_init(&mma_done[s], 1);
             mbar_init(&p_free[s], 4);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
-        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
         fence_mbar_init();
     }
     if (warp == 1)
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(tmem_slot, S::kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -130,10 +164,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                             break;
                         }
                     }
-                    mbar_arrive_expect_tx(&tma_full[stage], kPBytes + kBBytes);
-                    tma_load_2d(sP + stage * kPBytes, &map_p, ks * kBK, ft * kPackedRows,
+                    mbar_arrive_expect_tx(&tma_full[stage], S::kPBytes + S::kBBytes);
+                    tma_load_2d(sP + stage * S::kPBytes, &map_p, ks * kBK, ft * S::kPackedRows,
                                 &tma_full[stage]);
-                    tma_load_2d(sB + stage * kBBytes, &map_x, ks * kBK, tt * kBN, &tma_full[stage]);
+                    tma_load_2d(sB + stage * S::kBBytes, &map_x, ks * kBK, tt * BN, &tma_full[stage]);
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -156,11 +190,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
             bool ok = true;
             int issued = 0;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
-                const int buf = local & 1;
-                if (local >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((local >> 1) - 1) & 1), p.err))
+                if (local >= 1 && !mbar_wait(acc_empty, uint32_t((local - 1) & 1), p.err))
                     break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + uint32_t(buf * kBN);
                 for (int ks = 0; ks < KS; ++ks) {
                     if (!mbar_wait(&tma_full[stage], phase, p.err) ||
                         !mbar_wait(&a_full[stage], phase, p.err)) {
@@ -168,12 +200,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * kABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * kBBytes);
+                    const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
+                    const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk)
-                        umma_i8(d_tmem, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32), kIdesc,
-                                (ks > 0 || kk > 0) ? 1u : 0u);
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 32; ++kk)
+                            umma_i8(tmem_base + uint32_t(g * BN),
+                                    umma_desc_sw128(a0 + uint32_t(g * kAGroupBytes + kk * 32)),
+                                    umma_desc_sw128(b0 + uint32_t(kk * 32)), kIdesc,
+                                    (ks > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&mma_done[stage]);
                     ++issued;
                     if (++stage == kStages) {
@@ -182,7 +218,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     }
                 }
                 if (ok)
-                    umma_commit(&acc_full[buf]);
+                    umma_commit(acc_full);
             }
             // the last commit tracks every MMA this thread issued
             if (issued > 0) {
@@ -190,7 +226,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                 mbar_wait(&mma_done[s], uint32_t(((issued - 1) / kStages) & 1), p.err);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------ code expansion
         const int et = threadIdx.x - 64;  // 0..127
         int stage = 0;
@@ -205,13 +241,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     ok = false;
                     break;
                 }
-                const uint8_t *P = sP + stage * kPBytes;
-                uint8_t *A = sA + stage * kABytes;
+                const uint8_t *P = sP + stage * S::kPBytes;
+                uint8_t *A = sA + stage * S::kABytes;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int idx = et + h * 128;  // (packed row j, chunk c)
+                for (int h = 0; h < 2 * G; ++h) {
+                    const int idx = et + h * 128;  // (packed row j of the tile, chunk c)
                     const int j = idx >> 3, c = idx & 7;
+                    const int g = j >> 5, jj = j & 31;
                     const uint4 v = *reinterpret_cast<const uint4 *>(P + sw128_off(j, c));
+                    uint8_t *Ag = A + g * kAGroupBytes;
 #pragma unroll
                     for (int pl = 0; pl < 4; ++pl) {
                         uint4 o;
@@ -219,7 +257,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                         o.y = (v.y >> (2 * pl)) & 0x03030303u;
                         o.z = (v.z >> (2 * pl)) & 0x03030303u;
                         o.w = (v.w >> (2 * pl)) & 0x03030303u;
-                        *reinterpret_cast<uint4 *>(A + sw128_off(j + 32 * pl, c)) = o;
+                        *reinterpret_cast<uint4 *>(Ag + sw128_off(jj + 32 * pl, c)) = o;
                     }
                 }
                 fence_proxy_async_smem();  // make the codes visible to the tensor cores
@@ -237,21 +275,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
         }
     } else {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access = plane
+        const int q = warp & 3;                  // TMEM lane quarter = plane
+        const int sub = (warp - kEpiWarp0) >> 2;
+        const int g = G == 2 ? sub : 0;          // MMA group of this warp
+        const int cb = G == 2 ? 0 : sub * (BN / 2);  // its columns: [cb, cb + ncol)
+        constexpr int ncol = G == 2 ? BN : BN / 2;
         int local = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
             const int ft = t / p.tok_tiles, tt = t - ft * p.tok_tiles;
-            const int buf = local & 1;
-            if (!mbar_wait_warp(&acc_full[buf], uint32_t((local >> 1) & 1), p.err))
+            if (!mbar_wait_warp(acc_full, uint32_t(local & 1), p.err))
                 break;
             tc_fence_after();
-            const int prow = ft * kPackedRows + lane;  // packed row of this lane
+            const int prow = ft * S::kPackedRows + g * 32 + lane;  // packed row of this lane
             const bool row_ok = prow < p.N4;
             const int n = prow + q * p.N4;
-            const int N = 4 * p.N4;
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * kBN);
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
-                const int mbase = tt * kBN + c0;
+            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(g * BN + cb);
+            for (int c0 = 0; c0 < ncol; c0 += 32) {
+                const int mbase = tt * BN + cb + c0;
                 if (mbase >= p.M)
                     break;
                 uint32_t v[32];
@@ -263,20 +303,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                 for (int i = 0; i < 32; ++i) {
                     const float ts = __shfl_sync(0xffffffffu, my_t, i);
                     const int32_t xs = __shfl_sync(0xffffffffu, my_s, i);
-                    const int m = mbase + i;
-                    if (row_ok && m < p.M) {
-                        const int32_t acc = int32_t(v[i]) - xs;
-                        const size_t o = size_t(m) * N + n;
-                        p.y[o] = __fmul_rn(__int2float_rn(acc), ts);
-                        if (p.acc_out)
-                            p.acc_out[o] = acc;
-                    }
+                    if (row_ok && mbase + i < p.M)
+                        store_out(p, mbase + i, n, int32_t(v[i]), ts, xs);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&acc_empty[buf]);
+                mbar_arrive(acc_empty);
         }
     }
 
@@ -285,7 +319,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
     __syncthreads();
     tc_fence_after();
     if (warp == 1)
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, S::kTmemCols);
+}
+
+template <int G, int BN>
+cudaError_t launch_shape(const uint8_t *packed, const int8_t *xq, PrefillParams prm,
+                         cudaStream_t stream)
+{
+    using S = PrefillShape<G, BN>;
+    CUtensorMap map_p, map_x;
+    if (!make_map(&map_p, packed, prm.K, prm.N4, S::kPackedRows) ||
+        !make_map(&map_x, xq, prm.K, prm.M, BN))
+        return cudaErrorInvalidValue;
+    prm.feat_tiles = (prm.N4 + S::kPackedRows - 1) / S::kPackedRows;
+    prm.tok_tiles = (prm.M + BN - 1) / BN;
+    const size_t smem = S::bytes + 1024;  // + alignment slack
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<G, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
+    const int tiles = prm.feat_tiles * prm.tok_tiles;
+    const int grid = std::min(tiles, device_sm_count());
+    prefill_tc_kernel<G, BN><<<grid, kThreads, smem, stream>>>(map_p, map_x, prm);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -300,15 +362,10 @@ cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t
     *handled = false;
     if (M < kPrefillMinM)
         return cudaSuccess;
-    CUtensorMap map_p, map_x;
-    if (!make_map(&map_p, packed, K, N / 4, kPackedRows) || !make_map(&map_x, xq, K, M, kBN))
-        return cudaErrorInvalidValue;
-    PrefillParams prm;
+    PrefillParams prm = {};
     prm.N4 = N / 4;
     prm.K = K;
     prm.M = M;
-    prm.feat_tiles = (prm.N4 + kPackedRows - 1) / kPackedRows;
-    prm.tok_tiles = (M + kBN - 1) / kBN;
     prm.k_stages = (K + kBK - 1) / kBK;
     prm.w_scale = w_scale;
     prm.x_scale = x_scale;
@@ -318,21 +375,33 @@ cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t
     prm.err = device_error_word();
     if (!prm.err)
         return cudaErrorUnknown;
-    const size_t smem = PrefillSmem::bytes + 1024;  // + alignment slack
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess)
-            return e;
-        configured_dev = dev;
+    // Tile shape: the least estimated time = waves of tiles over the SMs x
+    // cycles per K stage of one tile. A stage costs its MMAs (2 G BN cycles
+    // at the int8 rate), or the code expansion when that is longer (about
+    // 160 G cycles of shared-memory stores), plus ~100 cycles of pipeline
+    // overhead. The larger tile wins ties (fewer operand re-reads from L2).
+    const int sms = device_sm_count();
+    const int shapes[4][2] = {{2, 256}, {2, 128}, {1, 128}, {1, 64}};
+    int best = 0;
+    long long best_cost = -1;
+    for (int i = 0; i < 4; ++i) {
+        const int G = shapes[i][0], BN = shapes[i][1];
+        const long long tiles =
+            (long long)((prm.N4 + 32 * G - 1) / (32 * G)) * ((M + BN - 1) / BN);
+        const long long stage = std::max(2 * G * BN, 160 * G) + 100;
+        const long long cost = (tiles + sms - 1) / sms * stage;
+        if (best_cost < 0 || cost < best_cost) {
+            best = i;
+            best_cost = cost;
+        }
     }
-    const int tiles = prm.feat_tiles * prm.tok_tiles;
-    const int grid = std::min(tiles, device_sm_count());
-    prefill_tc_kernel<<<grid, kThreads, smem, stream>>>(map_p, map_x, prm);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    switch (best) {
+    case 0: e = launch_shape<2, 256>(packed, xq, prm, stream); break;
+    case 1: e = launch_shape<2, 128>(packed, xq, prm, stream); break;
+    case 2: e = launch_shape<1, 128>(packed, xq, prm, stream); break;
+    default: e = launch_shape<1, 64>(packed, xq, prm, stream); break;
+    }
     if (e == cudaSuccess)
         *handled = true;
     return e;

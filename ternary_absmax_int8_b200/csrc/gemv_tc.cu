@@ -21,10 +21,10 @@
 //   (32 rows) plus activations (BN rows), 128B swizzled. A CTA works through
 //   segments (tile, first unit, end unit); two plans decide which:
 //   - cluster plan (tq_gemv): with fewer tiles than SMs, the C CTAs of a
-//     thread-block cluster split one tile's K range; the other CTAs add their
-//     int32 partial sums into the leader CTA's shared memory (red on
-//     shared::cluster, exact and order-free) and signal its mbarrier; the
-//     leader applies the epilogue. With many tiles, C = 1 and each CTA takes
+//     thread-block cluster split one tile's K range; the other CTAs store
+//     their int32 partial sums into slots in the leader CTA's shared memory
+//     (16-byte st.shared::cluster) and signal its mbarrier; the leader adds
+//     them (exact, order-free) and applies the epilogue. With many tiles, C = 1 and each CTA takes
 //     whole tiles.
 //   - stream-K plan (tq_gemv_noalloc): the (tile, unit) sequence is cut into
 //     one contiguous, balanced range per CTA; a tile split across CTAs adds
@@ -48,7 +48,10 @@ namespace {
 constexpr int kRows = 128;             // MMA M (32 packed rows x 4 planes)
 constexpr int kPRows = kRows / 4;      // packed rows per tile
 constexpr int kUnitK = 256;            // bytes of K per unit (two 128-byte boxes)
-constexpr int kSP = 10;                // shared-memory stages (packed + activations)
+// Shared-memory stages (packed bytes + activations): fewer at BN = 32, whose
+// stages and cluster slots are twice as large.
+template <int BN>
+constexpr int kStagesOf = BN == 16 ? 10 : 6;
 constexpr int kSA = 4;                 // tensor-memory A slots
 constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
 constexpr int kThreads = 512;
@@ -102,46 +105,22 @@ struct CtaWork {
 
 template <int BN>
 struct SmallMSmem {
+    static constexpr int kSP = kStagesOf<BN>;
     static constexpr int kPBytes = kPRows * kUnitK;  // 8 KB
     static constexpr int kBBytes = BN * kUnitK;
     static constexpr size_t p_off = 0;
     static constexpr size_t b_off = p_off + size_t(kSP) * kPBytes;
-    // cluster plan: the leader's sum of the other CTAs' partials, [BN][128]
-    static constexpr size_t red_off = b_off + size_t(kSP) * kBBytes;
-    static constexpr size_t bar_off = red_off + size_t(BN) * kRows * 4;
+    // cluster plan: one slot per other CTA of the cluster for its partial
+    // sums, [rank - 1][BN / 4][128 rows] x 16 bytes, in the leader
+    static constexpr size_t slot_off = b_off + size_t(kSP) * kBBytes;
+    static constexpr size_t kSlotBytes = size_t(kRows) * BN * 4;
+    static constexpr size_t bar_off = slot_off + size_t(kMaxCluster - 1) * kSlotBytes;
     // tma_full[SP], p_free[SP], mma_done[SP], a_full[SA], acc_full[2],
     // acc_empty[2], red_done
     static constexpr int kBars = 3 * kSP + kSA + 5;
     static constexpr size_t misc_off = bar_off + kBars * 8;  // tmem slot, finisher flag
     static constexpr size_t bytes = misc_off + 16;
 };
-
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync_all()
-{
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void red_add_cluster(uint32_t raddr, int32_t v)
-{
-    asm volatile("red.relaxed.cluster.shared::cluster.add.s32 [%0], %1;" ::"r"(raddr), "r"(v)
-                 : "memory");
-}
 
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr)
 {
@@ -224,6 +203,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                  const __grid_constant__ SmallMParams p)
 {
     using L = SmallMSmem<BN>;
+    constexpr int kSP = L::kSP;
     constexpr uint32_t kIdesc = idesc_i8_u8s8(kRows, BN);
     constexpr int kTmemCols = 512;  // kSA * kACols + 2 * BN, rounded to a power of two
     static_assert(kSA * kACols + 2 * BN <= kTmemCols, "tensor memory plan");
@@ -233,7 +213,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sP = smem + L::p_off;
     uint8_t *sB = smem + L::b_off;
-    int32_t *red_buf = reinterpret_cast<int32_t *>(smem + L::red_off);
+    uint4 *slots = reinterpret_cast<uint4 *>(smem + L::slot_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
     uint64_t *tma_full = bars;
     uint64_t *p_free = bars + kSP;
@@ -262,7 +242,22 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                                        : 0);
     }
 
+    // The producer's copies, unit by unit in the CTA's order.
+    auto issue = [&](int issued, const Seg &g, int k) {
+        const int s = issued % kSP;
+        const int k0 = k * kUnitK;
+        mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
+        uint8_t *P = sP + s * L::kPBytes;
+        uint8_t *B = sB + s * L::kBBytes;
+        tma_load_2d(P, &map_p, k0, g.tile * kPRows, &tma_full[s]);
+        tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, g.tile * kPRows, &tma_full[s]);
+        tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
+        tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+    };
+    int early = 0;  // copies thread 0 issued before the CTA barrier
     if (threadIdx.x == 0) {
+        prefetch_tensormap(&map_p);
+        prefetch_tensormap(&map_x);
         for (int s = 0; s < kSP; ++s) {
             mbar_init(&tma_full[s], 1);
             mbar_init(&p_free[s], 4);
@@ -277,10 +272,14 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         // every epilogue thread of every other CTA of the cluster arrives once
         mbar_init(red_done, split_cluster ? uint32_t(kRows * (p.csize - 1)) : 1u);
         fence_mbar_init();
+        // Start the first stages' copies now: their latency overlaps the
+        // tensor-memory allocation and the barriers below.
+        for (int sg = 0; sg < cw.nseg && early < kSP; ++sg) {
+            const Seg g = cw.seg(p, sg);
+            for (int k = g.k0; k < g.k1 && early < kSP; ++k)
+                issue(early++, g, k);
+        }
     }
-    if (split_cluster && cw.rank == 0)
-        for (int i = threadIdx.x; i < BN * kRows; i += kThreads)
-            red_buf[i] = 0;
     if (warp == 1)
         tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -302,6 +301,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
             for (int sg = 0; sg < cw.nseg && ok; ++sg) {
                 const Seg g = cw.seg(p, sg);
                 for (int k = g.k0; k < g.k1; ++k, ++issued) {
+                    if (issued < early)
+                        continue;  // issued before the CTA barrier
                     const int s = issued % kSP;
                     const uint32_t use = uint32_t(issued / kSP);
                     if (use > 0 && (!mbar_wait(&p_free[s], (use - 1) & 1, p.err) ||
@@ -309,14 +310,7 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                         ok = false;
                         break;
                     }
-                    const int k0 = k * kUnitK;
-                    mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
-                    uint8_t *P = sP + s * L::kPBytes;
-                    uint8_t *B = sB + s * L::kBBytes;
-                    tma_load_2d(P, &map_p, k0, g.tile * kPRows, &tma_full[s]);
-                    tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, g.tile * kPRows, &tma_full[s]);
-                    tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
-                    tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+                    issue(issued, g, k);
                 }
             }
             for (int s = 0; s < kSP && s < issued; ++s) {
@@ -445,22 +439,34 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
             const int n = prow + pl * p.N4;
             if (split_cluster) {
                 if (cw.rank != 0) {
-                    // Add this CTA's partial sums into the leader's buffer,
-                    // then tell the leader (release: the adds come first).
-                    const uint32_t base = map_to_rank(smem_u32(red_buf), 0u);
+                    // Store this CTA's partial sums into its slot in the
+                    // leader, then tell the leader (release: the stores come
+                    // first).
+                    const uint32_t base = map_to_rank(smem_u32(slots), 0u) +
+                                          uint32_t((cw.rank - 1) * L::kSlotBytes);
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (c < p.M)
-                            red_add_cluster(base + uint32_t((c * kRows + r) * 4), int32_t(v[c]));
+                    for (int c4 = 0; c4 < BN / 4; ++c4)
+                        st_cluster_v4(base + uint32_t((c4 * kRows + r) * 16),
+                                      make_uint4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2],
+                                                 v[4 * c4 + 3]));
                     mbar_arrive_remote(map_to_rank(smem_u32(red_done), 0u));
                     continue;
                 }
-                // Leader: wait for the other CTAs' sums, then finish the tile.
+                // Leader: wait for the other CTAs' sums, add them (integer
+                // adds, exact in any order), then finish the tile.
                 if (!mbar_wait_cluster_warp(red_done, 0u, p.err))
                     continue;
+                for (int k = 0; k < p.csize - 1; ++k) {
+                    const uint4 *sl = slots + size_t(k) * (L::kSlotBytes / 16);
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    v[c] += uint32_t(red_buf[c * kRows + r]);
+                    for (int c4 = 0; c4 < BN / 4; ++c4) {
+                        const uint4 a = sl[c4 * kRows + r];
+                        v[4 * c4] += a.x;
+                        v[4 * c4 + 1] += a.y;
+                        v[4 * c4 + 2] += a.z;
+                        v[4 * c4 + 3] += a.w;
+                    }
+                }
             }
             if (whole || split_cluster) {
 #pragma unroll

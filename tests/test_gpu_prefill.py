@@ -3,7 +3,9 @@
 Full outputs at M = 128 and 256 for the FFN shapes; at M = 512 on the three
 prefill shapes (including the 27B-scale 17408 x 5120) a sample of token rows,
 first and last included, is checked on all N outputs. Ragged M and N exercise
-partial tiles.
+partial tiles; the shapes cover both work splits of the kernel: whole tiles per
+CTA (including CTAs that take a second tile) and K split over the CTAs of a
+thread-block cluster with a reduce-scatter of the partial sums.
 """
 import numpy as np
 import pytest
@@ -39,7 +41,7 @@ def test_prefill_m512_sampled_rows(cuda_device):
 
 
 @pytest.mark.parametrize("N,K,M", [(516, 272, 130), (4, 16, 129), (2048, 1024, 384),
-                                   (260, 2560, 200)])
+                                   (260, 2560, 200), (512, 128, 33), (2564, 6928, 64)])
 def test_prefill_ragged(cuda_device, N, K, M):
     rng = np.random.default_rng(N + K + M)
     w = ternary_weights(rng, N, K)
@@ -47,3 +49,18 @@ def test_prefill_ragged(cuda_device, N, K, M):
     ws = stored_weight_scale(w)
     assert_parity(gpu_forward(host_pack(w), N, ws, xb), oracle_forward(w, ws, xb),
                   f"{N}x{K} M={M}")
+
+
+def test_prefill_second_tile_per_cta(cuda_device):
+    # 68 x 4 = 272 tiles of 256 features x 256 tokens on 148 SMs: most CTAs
+    # take two tiles, so the accumulator is drained and refilled; sampled
+    # token rows from every token tile, all N outputs.
+    N, K, M = 17408, 512, 1024
+    rng = np.random.default_rng(5)
+    w = ternary_weights(rng, N, K)
+    xb = activations_bf16(rng, M, K)
+    ws = stored_weight_scale(w)
+    q, xs, xsum, acc, y = gpu_forward(host_pack(w), N, ws, xb)
+    rows = np.array([0, 255, 256, 300, 511, 512, 700, 767, 768, 1000, 1023])
+    sub = (q[rows], xs[rows], xsum[rows], acc[rows], y[rows])
+    assert_parity(sub, oracle_forward(w, ws, xb[rows]), "17408x512 M=1024")
