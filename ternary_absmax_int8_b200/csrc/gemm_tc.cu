@@ -16,21 +16,24 @@
 // activation operand is read from L2 once per G x 128 features. In group g,
 // MMA row r = 32 p + j is feature i0 + 32 g + j + p N/4: one TMA tile of
 // G x 32 packed rows (128B-swizzled) expands into the G A operands of 16 KB.
-// The host picks (G, BN) in {(2,256), (2,128), (1,128), (1,64)} for the
-// fewest waves of tile work over the SMs (larger tiles on ties), since a
-// 512-token prompt through a 2560-feature projection makes only 20 tiles of
-// the largest shape.
+// The host picks (G, BN) in {(2,256), (1,256), (1,128)} for the least
+// estimated time (waves of tiles over the SMs x cycles per K stage;
+// larger tiles on ties), since a 512-token prompt through a 2560-feature
+// projection makes only 20 tiles of the largest shape.
 //
 // Warp roles (14 warps, one CTA per SM, persistent over tiles):
 //   warp 0       TMA producer: packed tile + activation tile per K stage
 //   warp 1       TMEM allocator; lane 0 issues the MMAs and commits
-//   warps 2..5   expand the codes into the A stage (canonical K-major, 128B
+//   warps 2..13  expand the codes into the A stage (canonical K-major, 128B
 //                swizzle), fence to the async proxy, signal the MMA
-//   warps 6..13  epilogue: warp w reads TMEM lane quarter w % 4 of its group
-//                (G = 2) or of its half of the columns (G = 1), subtracts
-//                x_sum, scales, stores y
+//   warps 6..13  then run the tile's epilogue: warp w reads TMEM lane
+//                quarter w % 4 of its group (G = 2) or of its half of the
+//                columns (G = 1), subtracts x_sum, scales, stores y
 // The accumulator (G x BN columns) is single-buffered: a CTA's next tile
-// starts its MMAs once the epilogue has drained it. Every mbarrier wait is
+// starts its MMAs once the epilogue has drained it, so the epilogue warps
+// are free to expand codes during the main loop (expansion, 16 bytes of
+// shared-memory stores per 4 bytes of weights, is what bounds a stage
+// otherwise). Every mbarrier wait is
 // bounded; loads never use cluster multicast.
 #include <algorithm>
 #include <cstring>
@@ -45,7 +48,9 @@ constexpr int kGM = 128;                // MMA M: rows of one group
 constexpr int kBK = 128;                // bytes of K per stage
 constexpr int kAGroupBytes = kGM * kBK; // 16 KB
 constexpr int kThreads = 448;
-constexpr int kEpiWarp0 = 6;
+constexpr int kExpWarp0 = 2;             // warps 2..13 expand codes
+constexpr int kExpWarps = 12;
+constexpr int kEpiWarp0 = 6;             // warps 6..13 also run the epilogue
 constexpr int kEpiWarps = 8;
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -132,9 +137,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
         prefetch_tensormap(&map_x);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&tma_full[s], 1);
-            mbar_init(&a_full[s], 4);
+            mbar_init(&a_full[s], kExpWarps);
             mbar_init(&mma_done[s], 1);
-            mbar_init(&p_free[s], 4);
+            mbar_init(&p_free[s], kExpWarps);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
@@ -200,15 +205,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
-                    const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
+                    // one descriptor per operand and stage, advanced by adds
+                    const uint64_t da = umma_desc_sw128(smem_u32(sA + stage * S::kABytes));
+                    const uint64_t db = umma_desc_sw128(smem_u32(sB + stage * S::kBBytes));
 #pragma unroll
                     for (int g = 0; g < G; ++g)
 #pragma unroll
                         for (int kk = 0; kk < kBK / 32; ++kk)
                             umma_i8(tmem_base + uint32_t(g * BN),
-                                    umma_desc_sw128(a0 + uint32_t(g * kAGroupBytes + kk * 32)),
-                                    umma_desc_sw128(b0 + uint32_t(kk * 32)), kIdesc,
+                                    umma_desc_advance(da, uint32_t(g * kAGroupBytes + kk * 32)),
+                                    umma_desc_advance(db, uint32_t(kk * 32)), kIdesc,
                                     (ks > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&mma_done[stage]);
                     ++issued;
@@ -226,14 +232,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                 mbar_wait(&mma_done[s], uint32_t(((issued - 1) / kStages) & 1), p.err);
             }
         }
-    } else if (warp < kEpiWarp0) {
-        // ------------------------------------------------ code expansion
-        const int et = threadIdx.x - 64;  // 0..127
+    } else {
+        // -------------------------- code expansion, then (warps 6..13) epilogue
+        const int et = threadIdx.x - kExpWarp0 * 32;  // 0..383
+        const bool epi = warp >= kEpiWarp0;
+        const int q = warp & 3;                  // TMEM lane quarter = plane
+        const int sub = (warp - kEpiWarp0) >> 2;
+        const int eg = G == 2 ? sub : 0;         // MMA group of this epilogue warp
+        const int cb = G == 2 ? 0 : sub * (BN / 2);  // its columns: [cb, cb + ncol)
+        constexpr int ncol = G == 2 ? BN : BN / 2;
+        constexpr int kUnits = S::kPackedRows * 8;   // 16-byte chunks of packed bytes per stage
         int stage = 0;
         uint32_t phase = 0;
         int seen = 0;
+        int local = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
             for (int ks = 0; ks < KS; ++ks) {
                 bool w1 = mbar_wait_warp(&tma_full[stage], phase, p.err);
                 bool w2 = w1 && (seen < kStages || mbar_wait_warp(&mma_done[stage], phase ^ 1u, p.err));
@@ -244,20 +258,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                 const uint8_t *P = sP + stage * S::kPBytes;
                 uint8_t *A = sA + stage * S::kABytes;
 #pragma unroll
-                for (int h = 0; h < 2 * G; ++h) {
-                    const int idx = et + h * 128;  // (packed row j of the tile, chunk c)
-                    const int j = idx >> 3, c = idx & 7;
-                    const int g = j >> 5, jj = j & 31;
-                    const uint4 v = *reinterpret_cast<const uint4 *>(P + sw128_off(j, c));
-                    uint8_t *Ag = A + g * kAGroupBytes;
+                for (int h = 0; h < (kUnits + kExpWarps * 32 - 1) / (kExpWarps * 32); ++h) {
+                    const int idx = et + h * kExpWarps * 32;  // (packed row j of the tile, chunk c)
+                    if (idx < kUnits) {
+                        const int j = idx >> 3, c = idx & 7;
+                        const int g = j >> 5, jj = j & 31;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(P + sw128_off(j, c));
+                        uint8_t *Ag = A + g * kAGroupBytes;
 #pragma unroll
-                    for (int pl = 0; pl < 4; ++pl) {
-                        uint4 o;
-                        o.x = (v.x >> (2 * pl)) & 0x03030303u;
-                        o.y = (v.y >> (2 * pl)) & 0x03030303u;
-                        o.z = (v.z >> (2 * pl)) & 0x03030303u;
-                        o.w = (v.w >> (2 * pl)) & 0x03030303u;
-                        *reinterpret_cast<uint4 *>(Ag + sw128_off(jj + 32 * pl, c)) = o;
+                        for (int pl = 0; pl < 4; ++pl) {
+                            uint4 o;
+                            o.x = (v.x >> (2 * pl)) & 0x03030303u;
+                            o.y = (v.y >> (2 * pl)) & 0x03030303u;
+                            o.z = (v.z >> (2 * pl)) & 0x03030303u;
+                            o.w = (v.w >> (2 * pl)) & 0x03030303u;
+                            *reinterpret_cast<uint4 *>(Ag + sw128_off(jj + 32 * pl, c)) = o;
+                        }
                     }
                 }
                 fence_proxy_async_smem();  // make the codes visible to the tensor cores
@@ -272,24 +288,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     phase ^= 1u;
                 }
             }
-        }
-    } else {
-        // ------------------------------------------------ epilogue
-        const int q = warp & 3;                  // TMEM lane quarter = plane
-        const int sub = (warp - kEpiWarp0) >> 2;
-        const int g = G == 2 ? sub : 0;          // MMA group of this warp
-        const int cb = G == 2 ? 0 : sub * (BN / 2);  // its columns: [cb, cb + ncol)
-        constexpr int ncol = G == 2 ? BN : BN / 2;
-        int local = 0;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
+            if (!epi || !ok)
+                continue;
+            // ---- epilogue of tile t
             const int ft = t / p.tok_tiles, tt = t - ft * p.tok_tiles;
             if (!mbar_wait_warp(acc_full, uint32_t(local & 1), p.err))
                 break;
             tc_fence_after();
-            const int prow = ft * S::kPackedRows + g * 32 + lane;  // packed row of this lane
+            const int prow = ft * S::kPackedRows + eg * 32 + lane;  // packed row of this lane
             const bool row_ok = prow < p.N4;
             const int n = prow + q * p.N4;
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(g * BN + cb);
+            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(eg * BN + cb);
             for (int c0 = 0; c0 < ncol; c0 += 32) {
                 const int mbase = tt * BN + cb + c0;
                 if (mbase >= p.M)
@@ -376,19 +385,20 @@ cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t
     if (!prm.err)
         return cudaErrorUnknown;
     // Tile shape: the least estimated time = waves of tiles over the SMs x
-    // cycles per K stage of one tile. A stage costs its MMAs (2 G BN cycles
-    // at the int8 rate), or the code expansion when that is longer (about
-    // 160 G cycles of shared-memory stores), plus ~100 cycles of pipeline
-    // overhead. The larger tile wins ties (fewer operand re-reads from L2).
+    // cycles per K stage of one tile. A stage is 4 G MMAs of K = 32, each
+    // costing its execution (BN / 2 cycles at the int8 rate) or its issue by
+    // the single MMA thread (~100 cycles, measured), whichever is longer,
+    // plus ~100 cycles of pipeline overhead. The larger tile wins ties (fewer
+    // operand re-reads from L2).
     const int sms = device_sm_count();
-    const int shapes[4][2] = {{2, 256}, {2, 128}, {1, 128}, {1, 64}};
+    const int shapes[3][2] = {{2, 256}, {1, 256}, {1, 128}};
     int best = 0;
     long long best_cost = -1;
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 3; ++i) {
         const int G = shapes[i][0], BN = shapes[i][1];
         const long long tiles =
             (long long)((prm.N4 + 32 * G - 1) / (32 * G)) * ((M + BN - 1) / BN);
-        const long long stage = std::max(2 * G * BN, 160 * G) + 100;
+        const long long stage = 4LL * G * std::max(BN / 2, 100) + 100;
         const long long cost = (tiles + sms - 1) / sms * stage;
         if (best_cost < 0 || cost < best_cost) {
             best = i;
@@ -398,9 +408,8 @@ cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t
     cudaError_t e;
     switch (best) {
     case 0: e = launch_shape<2, 256>(packed, xq, prm, stream); break;
-    case 1: e = launch_shape<2, 128>(packed, xq, prm, stream); break;
-    case 2: e = launch_shape<1, 128>(packed, xq, prm, stream); break;
-    default: e = launch_shape<1, 64>(packed, xq, prm, stream); break;
+    case 1: e = launch_shape<1, 256>(packed, xq, prm, stream); break;
+    default: e = launch_shape<1, 128>(packed, xq, prm, stream); break;
     }
     if (e == cudaSuccess)
         *handled = true;

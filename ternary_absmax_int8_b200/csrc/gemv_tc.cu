@@ -338,13 +338,15 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b0 = smem_u32(sB + s * L::kBBytes);
+                    // one descriptor per unit, advanced by adds
+                    const uint64_t db = umma_desc_sw128(smem_u32(sB + s * L::kBBytes));
+                    const uint32_t ta = tmem_a + uint32_t(sa * kACols);
 #pragma unroll
-                    for (int kk = 0; kk < kUnitK / 32; ++kk) {
-                        const uint32_t bk = b0 + uint32_t((kk >> 2) * (L::kBBytes / 2) + (kk & 3) * 32);
-                        umma_i8_ts(d, tmem_a + uint32_t(sa * kACols + kk * 8), umma_desc_sw128(bk),
+                    for (int kk = 0; kk < kUnitK / 32; ++kk)
+                        umma_i8_ts(d, ta + uint32_t(kk * 8),
+                                   umma_desc_advance(db, uint32_t((kk >> 2) * (L::kBBytes / 2) +
+                                                                  (kk & 3) * 32)),
                                    kIdesc, (k == g.k0 && kk == 0) ? 0u : 1u);
-                    }
                     umma_commit(&mma_done[s]);
                 }
                 if (ok)

@@ -23,6 +23,15 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr)
     return d;
 }
 
+// The same operand advanced by `bytes` (a multiple of 16) inside its
+// swizzle atom or by whole atoms: the start address is the descriptor's low
+// 14-bit field in units of 16 bytes, so no other field changes as long as
+// the address stays within shared memory.
+__device__ __forceinline__ uint64_t umma_desc_advance(uint64_t desc, uint32_t bytes)
+{
+    return desc + uint64_t(bytes >> 4);
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar)
 {
