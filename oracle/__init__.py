@@ -49,8 +49,13 @@ def _load():
             lib.oracle_quant.argtypes = [p, i64, i64, p, p, p]
             lib.oracle_gemv.argtypes = [p, i64, i64, p, i64, i64, i64, p]
             lib.oracle_epilogue.argtypes = [p, i64, i64, ctypes.c_float, p, p]
+            lib.oracle_quant_f32.argtypes = [p, i64, i64, p, p, p]
+            lib.oracle_rmsnorm.argtypes = [p, i64, i64, p, ctypes.c_float, p]
+            lib.oracle_relu2_mul.argtypes = [p, p, i64, p]
+            lib.oracle_absmean.argtypes = [p, i64, i64, p, p]
             for f in (lib.oracle_pack, lib.oracle_unpack, lib.oracle_quant,
-                      lib.oracle_gemv, lib.oracle_epilogue):
+                      lib.oracle_gemv, lib.oracle_epilogue, lib.oracle_quant_f32,
+                      lib.oracle_rmsnorm, lib.oracle_relu2_mul, lib.oracle_absmean):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -166,3 +171,44 @@ def forward(P: np.ndarray, N: int, w_scale: float, x_bf16: np.ndarray, threads: 
     acc = gemv(P, N, q) if threads == 1 else gemv_threads(P, N, q, threads)
     y = epilogue(acc, w_scale, xs)
     return q, xs, xsum, acc, y
+
+
+def quant_f32(h: np.ndarray):
+    """Absmax int8 quantisation of fp32 rows h [M, K] -> (q, x_scale, x_sum)."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    M, K = h.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty(M, np.float32)
+    t = np.empty(M, np.int32)
+    _check(_load().oracle_quant_f32(_ptr(h), M, K, _ptr(q), _ptr(s), _ptr(t)), "quant_f32")
+    return q, s, t
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm of fp32 rows x [M, K] with gain g [K] -> fp32 [M, K]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    M, K = x.shape
+    h = np.empty((M, K), np.float32)
+    _check(_load().oracle_rmsnorm(_ptr(x), M, K, _ptr(g), float(eps), _ptr(h)), "rmsnorm")
+    return h
+
+
+def relu2_mul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """relu(a)^2 * b elementwise, fp32."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    b = np.ascontiguousarray(b, dtype=np.float32)
+    h = np.empty(a.shape, np.float32)
+    _check(_load().oracle_relu2_mul(_ptr(a), _ptr(b), a.size, _ptr(h)), "relu2_mul")
+    return h
+
+
+def absmean(W_bf16: np.ndarray):
+    """Absmean ternary quantisation of bf16 latent weights [N, K] ->
+    (w int8 [N, K] in {-1, 0, 1}, gamma fp32)."""
+    W = np.ascontiguousarray(W_bf16, dtype=np.uint16)
+    N, K = W.shape
+    w = np.empty((N, K), np.int8)
+    g = np.empty(1, np.float32)
+    _check(_load().oracle_absmean(_ptr(W), N, K, _ptr(w), _ptr(g)), "absmean")
+    return w, g[0]

@@ -34,12 +34,31 @@
  *    per-tensor weight scale (issue above, "What We Need" item 2, the
  *    .weight_scale keys). Computed in fp64 here.
  *
+ *
+ * The steps on either side of the GEMV in a BitNet decoder layer (the
+ * lemon-mlx-engine issue, section "Architecture": a Llama variant with
+ * relu_squared instead of silu and sub-layer norms, attn_sub_norm before
+ * o_proj and ffn_sub_norm before down_proj; RMSNorm is named among the ops
+ * that pass) and the absmean weight quantiser (1bit.systems post "the full
+ * arc ...", read-more item "Training-Runs -- absmean QAT"; the stored scale is
+ * the .weight_scale of "What We Need" item 2). The pages print none of their
+ * formulas. Readings taken:
+ *  - RMSNorm of a row x [K] with gain g [K] and epsilon e: the mean of x^2
+ *    is accumulated in fp64 (each square exact), r = 1 / sqrt(mean + e) in
+ *    fp64 rounded once to fp32, h[k] = fl32(fl32(x[k] * r) * g[k]).
+ *  - relu_squared(a) * b = fl32(fl32(max(a,0) * max(a,0)) * b), fp32.
+ *  - absmean: gamma = fl32(sum |W| / (N K)) with the sum in fp64;
+ *    w = clamp(rint(fl32(W / gamma)), -1, 1) (ties to even); gamma == 0
+ *    gives w = 0. The packed weights then follow oracle_pack, and gamma is
+ *    the stored per-tensor scale.
+ *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared.
  * Status codes: 0 ok; 1 a value outside the domain (a weight not in
  * {-1,0,1}, or a packed code 3); 2 a bad shape.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 static float bf16_to_float(uint16_t b)
@@ -98,38 +117,118 @@ int oracle_unpack(const uint8_t *P, int8_t *w, int64_t N, int64_t K)
     return 0;
 }
 
+/* Absmax int8 quantisation of one fp32 row (the reading above). */
+static void quant_row(const float *row, int64_t K, int8_t *q, float *x_scale, int32_t *x_sum)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(row[k]);
+        if (a > amax)
+            amax = a;
+    }
+    int32_t sum = 0;
+    if (amax == 0.0f) {
+        for (int64_t k = 0; k < K; ++k)
+            q[k] = 0;
+        *x_scale = 0.0f;
+    } else {
+        volatile float s = 127.0f / amax; /* one fp32 rounding */
+        for (int64_t k = 0; k < K; ++k) {
+            volatile float t = row[k] * s; /* one fp32 rounding */
+            float r = rintf(t); /* default mode: nearest, ties to even */
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            q[k] = (int8_t)r;
+            sum += (int32_t)r;
+        }
+        *x_scale = amax / 127.0f;
+    }
+    *x_sum = sum;
+}
+
 /* Per-token absmax int8 quantisation of x [M,K] (bf16 bit patterns). */
 int oracle_quant(const uint16_t *x, int64_t M, int64_t K,
                  int8_t *q, float *x_scale, int32_t *x_sum)
 {
     if (M < 0 || K < 0)
         return 2;
+    float *row = malloc((size_t)(K > 0 ? K : 1) * sizeof(float));
+    if (!row)
+        return 2;
     for (int64_t m = 0; m < M; ++m) {
-        const uint16_t *row = x + m * K;
-        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k)
+            row[k] = bf16_to_float(x[m * K + k]); /* exact */
+        quant_row(row, K, q + m * K, &x_scale[m], &x_sum[m]);
+    }
+    free(row);
+    return 0;
+}
+
+/* The same quantisation of fp32 rows h [M,K]. */
+int oracle_quant_f32(const float *h, int64_t M, int64_t K,
+                     int8_t *q, float *x_scale, int32_t *x_sum)
+{
+    if (M < 0 || K < 0)
+        return 2;
+    for (int64_t m = 0; m < M; ++m)
+        quant_row(h + m * K, K, q + m * K, &x_scale[m], &x_sum[m]);
+    return 0;
+}
+
+/* RMSNorm of each row of x [M,K] with gain g [K] (the reading above). */
+int oracle_rmsnorm(const float *x, int64_t M, int64_t K, const float *g, float eps, float *h)
+{
+    if (M < 0 || K <= 0)
+        return 2;
+    for (int64_t m = 0; m < M; ++m) {
+        const float *row = x + m * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            ss += (double)row[k] * (double)row[k]; /* each square exact in fp64 */
+        const float r = (float)(1.0 / sqrt(ss / (double)K + (double)eps));
         for (int64_t k = 0; k < K; ++k) {
-            float a = fabsf(bf16_to_float(row[k]));
-            if (a > amax)
-                amax = a;
+            volatile float t = row[k] * r; /* one fp32 rounding */
+            h[m * K + k] = t * g[k];
         }
-        int32_t sum = 0;
-        if (amax == 0.0f) {
-            for (int64_t k = 0; k < K; ++k)
-                q[m * K + k] = 0;
-            x_scale[m] = 0.0f;
-        } else {
-            volatile float s = 127.0f / amax; /* one fp32 rounding */
-            for (int64_t k = 0; k < K; ++k) {
-                volatile float t = bf16_to_float(row[k]) * s; /* one fp32 rounding */
-                float r = rintf(t); /* default mode: nearest, ties to even */
-                if (r > 127.0f) r = 127.0f;
-                if (r < -127.0f) r = -127.0f;
-                q[m * K + k] = (int8_t)r;
-                sum += (int32_t)r;
-            }
-            x_scale[m] = amax / 127.0f;
+    }
+    return 0;
+}
+
+/* h[i] = relu(a[i])^2 * b[i] for n elements (the reading above). */
+int oracle_relu2_mul(const float *a, const float *b, int64_t n, float *h)
+{
+    if (n < 0)
+        return 2;
+    for (int64_t i = 0; i < n; ++i) {
+        const float r = a[i] > 0.0f ? a[i] : 0.0f;
+        volatile float sq = r * r; /* one fp32 rounding */
+        h[i] = sq * b[i];
+    }
+    return 0;
+}
+
+/* Absmean ternary quantisation of latent weights W [N,K] (bf16 bit
+ * patterns): w [N,K] in {-1,0,1} and the per-tensor scale gamma. */
+int oracle_absmean(const uint16_t *W, int64_t N, int64_t K, int8_t *w, float *gamma)
+{
+    if (N < 0 || K < 0)
+        return 2;
+    const int64_t n = N * K;
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i)
+        s += fabs((double)bf16_to_float(W[i]));
+    const float g = n > 0 ? (float)(s / (double)n) : 0.0f;
+    *gamma = g;
+    for (int64_t i = 0; i < n; ++i) {
+        if (g == 0.0f) {
+            w[i] = 0;
+            continue;
         }
-        x_sum[m] = sum;
+        volatile float t = bf16_to_float(W[i]) / g; /* one fp32 rounding */
+        float r = rintf(t);
+        if (r > 1.0f) r = 1.0f;
+        if (r < -1.0f) r = -1.0f;
+        w[i] = (int8_t)r;
     }
     return 0;
 }
