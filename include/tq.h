@@ -196,6 +196,53 @@ tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq
                           int M, int N, int K, cudaStream_t stream);
 
 /*
+ * The steps either side of the GEMV in a BitNet decoder layer, each fused
+ * with the activation quantiser so that only int8 codes leave the kernel
+ * (lemon-mlx-engine issue, section "Architecture": relu_squared in place of
+ * silu, sub-layer norms attn_sub_norm before o_proj and ffn_sub_norm before
+ * down_proj, RMSNorm). The pages give no formulas; the reading:
+ *   r = fl32(1 / sqrt(sum_k v^2 / K + eps))   (the sum and root in fp64)
+ *   h[k] = fl32(fl32(v[k] * r) * gain[k]),  then the absmax quantiser of
+ *   tq_quantize_act on h (xq, x_scale, x_sum as there).
+ * One CTA per token row. Host checks: 0 <= M, 0 < K <= 32768, K % 16 == 0,
+ * eps >= 0 and finite; byte tensors and fp32 rows 16-byte aligned, vectors
+ * 4-byte aligned. M == 0 is a no-op.
+ *
+ * tq_rmsnorm_quantize -- v = x: exactly one of x_bf16 [M, K] (bf16 bits) and
+ * x_f32 [M, K] is non-NULL (TQ_ERR_VALUE otherwise). gain fp32 [K].
+ */
+tq_status tq_rmsnorm_quantize(const uint16_t *x_bf16, const float *x_f32, const float *gain,
+                              float eps, int8_t *xq, float *x_scale, int32_t *x_sum, int M,
+                              int K, cudaStream_t stream);
+
+/*
+ * tq_relu2_mul_rmsnorm_quantize -- the FFN's down_proj input: v =
+ * fl32(fl32(relu(gate)^2) * up) from the gate and up projections' fp32
+ * outputs gate, up [M, K], then RMSNorm (ffn_sub_norm, gain [K]) and the
+ * quantiser, in one pass over the rows.
+ */
+tq_status tq_relu2_mul_rmsnorm_quantize(const float *gate, const float *up, const float *gain,
+                                        float eps, int8_t *xq, float *x_scale, int32_t *x_sum,
+                                        int M, int K, cudaStream_t stream);
+
+/*
+ * tq_absmean_pack -- quantise latent (or pre-dequantised) weights to ternary
+ * by absmean and pack them (1bit.systems post "the full arc ...", read-more
+ * item "Training-Runs": absmean; the result is the packed tensor and its
+ * .weight_scale). Reading: gamma = fl32(sum |W| / (N K)) with the sum in
+ * fp64, w = clamp(rne(fl32(W / gamma)), -1, 1) (gamma == 0: w = 0), codes
+ * w + 1 packed as tq_pack_host does.
+ *   w_bf16  device, bf16 bits [N, K], 16-byte aligned
+ *   packed  device, uint8 [N/4, K], 16-byte aligned (written)
+ *   w_scale device, fp32 [1] (written: gamma)
+ * N % 4 == 0, K % 16 == 0. Two launches (reduction, then quantise-and-pack);
+ * the reduction's partial sums live in a fixed device array, so calls that
+ * overlap on the GPU (on several streams) race on it.
+ */
+tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scale, int N, int K,
+                          cudaStream_t stream);
+
+/*
  * tq_device_error -- read (and if reset != 0, clear) the library's device
  * error word on the current device. Synchronises the device. 0 means no
  * kernel has reported an error. A nonzero value means a kernel gave up a

@@ -18,7 +18,8 @@ __all__ = [
     "TQError", "TQ_STACK_OVERLAP_PREV", "TQ_STACK_QUANTIZE", "TqProj", "lib_path",
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
     "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error", "tq_gemv_noalloc",
-    "tq_status_string", "tq_last_error", "make_proj",
+    "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
+    "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +66,9 @@ _SIGS = {
     "tq_quantize_act_stack": [ctypes.POINTER(TqProj), _i, _vp],
     "tq_gemv_stack": [ctypes.POINTER(TqProj), _i, ctypes.c_uint, _vp],
     "tq_device_error": [ctypes.POINTER(ctypes.c_uint32), _i],
+    "tq_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
+    "tq_relu2_mul_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
+    "tq_absmean_pack": [_vp, _vp, _vp, _i, _i, _vp],
 }
 _lib_handle = None
 
@@ -153,6 +157,28 @@ def tq_gemv_noalloc(packed, w_scale: float, xq, x_scale, x_sum, y, acc_out, M: i
     """tq_gemv for 5 <= M <= 32 on fixed library scratch (allocates nothing)."""
     _check(_load().tq_gemv_noalloc(_ptr(packed), float(w_scale), _ptr(xq), _ptr(x_scale),
                                 _ptr(x_sum), _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
+
+
+def tq_rmsnorm_quantize(x_bf16, x_f32, gain, eps: float, xq, x_scale, x_sum, M: int, K: int,
+                        stream=None) -> None:
+    """RMSNorm (gain, eps) then the absmax quantiser; exactly one of x_bf16 / x_f32."""
+    _check(_load().tq_rmsnorm_quantize(_ptr(x_bf16), _ptr(x_f32), _ptr(gain), float(eps),
+                                    _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, K,
+                                    _stream(stream)))
+
+
+def tq_relu2_mul_rmsnorm_quantize(gate, up, gain, eps: float, xq, x_scale, x_sum, M: int,
+                                  K: int, stream=None) -> None:
+    """relu(gate)^2 * up, RMSNorm (gain, eps), then the absmax quantiser."""
+    _check(_load().tq_relu2_mul_rmsnorm_quantize(_ptr(gate), _ptr(up), _ptr(gain), float(eps),
+                                              _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, K,
+                                              _stream(stream)))
+
+
+def tq_absmean_pack(w_bf16, packed, w_scale, N: int, K: int, stream=None) -> None:
+    """Absmean ternary quantisation of bf16 weights [N,K] -> packed [N/4,K], w_scale [1]."""
+    _check(_load().tq_absmean_pack(_ptr(w_bf16), _ptr(packed), _ptr(w_scale), N, K,
+                                _stream(stream)))
 
 
 def make_proj(packed=None, x=None, xq=None, x_scale=None, x_sum=None, y=None, acc_out=None,

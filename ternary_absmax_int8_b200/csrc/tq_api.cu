@@ -1,5 +1,6 @@
 // tq_api.cu -- the C ABI of libtq (declared in include/tq.h): argument
 // checks, then kernel launches. Nothing here allocates device memory.
+#include <cfloat>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -416,6 +417,64 @@ tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq
     cudaError_t e = tq::launch_smallm_tc_noalloc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M,
                                                  N, K, stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "tq_gemv_noalloc");
+}
+
+static tq_status rms_quant_call(const char *fn, int input, const uint16_t *x_bf16,
+                                const float *x_f32, const float *up, const float *gain, float eps,
+                                int8_t *xq, float *x_scale, int32_t *x_sum, int M, int K,
+                                cudaStream_t stream)
+{
+    if (M < 0 || K <= 0 || K % 16 != 0)
+        return fail(TQ_ERR_SHAPE, "%s: M=%d K=%d (need M >= 0, K > 0, K %% 16 == 0)", fn, M, K);
+    if (K > tq::kStreamMaxK)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: K=%d exceeds %d", fn, K, tq::kStreamMaxK);
+    if (!(eps >= 0.0f) || eps > FLT_MAX)
+        return fail(TQ_ERR_VALUE, "%s: eps must be finite and >= 0", fn);
+    if (M == 0)
+        return ok();
+    const void *x = input == 0 ? static_cast<const void *>(x_bf16) : static_cast<const void *>(x_f32);
+    if (!x || !gain || !xq || !x_scale || !x_sum || (input == 2 && !up))
+        return fail(TQ_ERR_NULL, "%s: a required pointer is NULL", fn);
+    if (!aligned(x, 16) || !aligned(xq, 16) || (up && !aligned(up, 16)) || !aligned(gain, 4) ||
+        !aligned(x_scale, 4) || !aligned(x_sum, 4))
+        return fail(TQ_ERR_ALIGN, "%s: rows and codes must be 16-byte aligned, vectors 4-byte",
+                    fn);
+    cudaError_t e = tq::launch_rms_quant(input, x_bf16, x_f32, up, gain, eps, xq, x_scale, x_sum,
+                                         M, K, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, fn);
+}
+
+tq_status tq_rmsnorm_quantize(const uint16_t *x_bf16, const float *x_f32, const float *gain,
+                              float eps, int8_t *xq, float *x_scale, int32_t *x_sum, int M, int K,
+                              cudaStream_t stream)
+{
+    if ((x_bf16 != nullptr) == (x_f32 != nullptr) && M > 0)
+        return fail(TQ_ERR_VALUE, "tq_rmsnorm_quantize: give exactly one of x_bf16 and x_f32");
+    return rms_quant_call("tq_rmsnorm_quantize", x_bf16 ? 0 : 1, x_bf16, x_f32, nullptr, gain,
+                          eps, xq, x_scale, x_sum, M, K, stream);
+}
+
+tq_status tq_relu2_mul_rmsnorm_quantize(const float *gate, const float *up, const float *gain,
+                                        float eps, int8_t *xq, float *x_scale, int32_t *x_sum,
+                                        int M, int K, cudaStream_t stream)
+{
+    return rms_quant_call("tq_relu2_mul_rmsnorm_quantize", 2, nullptr, gate, up, gain, eps, xq,
+                          x_scale, x_sum, M, K, stream);
+}
+
+tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scale, int N, int K,
+                          cudaStream_t stream)
+{
+    if (N < 0 || K < 0 || N % 4 != 0 || K % 16 != 0)
+        return fail(TQ_ERR_SHAPE, "tq_absmean_pack: N=%d K=%d (need N %% 4 == 0, K %% 16 == 0)",
+                    N, K);
+    if (!w_scale || (N > 0 && K > 0 && (!w_bf16 || !packed)))
+        return fail(TQ_ERR_NULL, "tq_absmean_pack: a required pointer is NULL");
+    if ((w_bf16 && !aligned(w_bf16, 16)) || (packed && !aligned(packed, 16)) ||
+        !aligned(w_scale, 4))
+        return fail(TQ_ERR_ALIGN, "tq_absmean_pack: weights and packed bytes 16-byte aligned");
+    cudaError_t e = tq::launch_absmean_pack(w_bf16, packed, w_scale, N, K, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "tq_absmean_pack");
 }
 
 tq_status tq_device_error(uint32_t *code, int reset)

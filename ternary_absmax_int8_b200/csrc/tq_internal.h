@@ -119,6 +119,14 @@ cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const
                                      const float *x_scale, const int32_t *x_sum, float *y,
                                      int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
 
+// ------------------------------------------ decoder-layer neighbours, absmean
+// input: 0 = bf16 x, 1 = fp32 x, 2 = relu(x_f32)^2 * up. One CTA per row.
+cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f32,
+                             const float *up, const float *gain, float eps, int8_t *xq,
+                             float *x_scale, int32_t *x_sum, int M, int K, cudaStream_t stream);
+cudaError_t launch_absmean_pack(const uint16_t *w, uint8_t *packed, float *w_scale, int N, int K,
+                                cudaStream_t stream);
+
 // Device address of the library's error word on the current device.
 unsigned *device_error_word();
 

@@ -144,3 +144,38 @@ def test_stack_argument_checks():
 def test_tq_proj_layout_matches_header():
     # 7 pointers, a float and two ints: 7*8 + 4 + 4 + 4 = 68, padded to 72
     assert ctypes.sizeof(tq.TqProj) == 72
+
+
+def test_layer_op_argument_checks():
+    rq = tq.tq_rmsnorm_quantize
+    with pytest.raises(tq.TQError) as e:
+        rq(A, None, A, 1e-5, A, A, A, 1, 20, stream=0)
+    assert e.value.name == "TQ_ERR_SHAPE"
+    with pytest.raises(tq.TQError) as e:
+        rq(A, A, A, 1e-5, A, A, A, 1, 32, stream=0)          # both inputs
+    assert e.value.name == "TQ_ERR_VALUE"
+    with pytest.raises(tq.TQError) as e:
+        rq(A, None, A, -1.0, A, A, A, 1, 32, stream=0)       # negative eps
+    assert e.value.name == "TQ_ERR_VALUE"
+    with pytest.raises(tq.TQError) as e:
+        rq(A, None, None, 1e-5, A, A, A, 1, 32, stream=0)    # no gain
+    assert e.value.name == "TQ_ERR_NULL"
+    with pytest.raises(tq.TQError) as e:
+        rq(A + 8, None, A, 1e-5, A, A, A, 1, 32, stream=0)
+    assert e.value.name == "TQ_ERR_ALIGN"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_relu2_mul_rmsnorm_quantize(A, None, A, 1e-5, A, A, A, 2, 64, stream=0)
+    assert e.value.name == "TQ_ERR_NULL"
+    rq(None, None, None, 1e-5, None, None, None, 0, 32, stream=0)  # M = 0: no-op
+
+
+def test_absmean_pack_argument_checks():
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_absmean_pack(A, A, A, 6, 32, stream=0)
+    assert e.value.name == "TQ_ERR_SHAPE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_absmean_pack(A, None, A, 8, 32, stream=0)
+    assert e.value.name == "TQ_ERR_NULL"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_absmean_pack(A + 4, A, A, 8, 32, stream=0)
+    assert e.value.name == "TQ_ERR_ALIGN"
