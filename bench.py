@@ -551,13 +551,297 @@ def run_reference(args, rank: int, world: int):
     }
 
 
+# ------------------------------------------------ decoder-layer chains
+CHAIN_WORKLOADS = {
+    "ffn_block30_m1": "30 x BitNet-b1.58-2B-4T FFN block, M=1, real dependencies, two launches "
+                      "per layer: [input RMSNorm + quantiser + gate and up GEMVs] -> "
+                      "[relu^2(gate)*up + ffn_sub_norm + quantiser + down GEMV, weights "
+                      "streamed while the first drains]; 90 projections, 398 MB packed",
+    "absmean_pack_27b": "absmean ternary quantisation + packing of bf16 latent weights "
+                        "17408x5120 (N(0, 0.02)), two passes",
+}
+FFN_H, FFN_I, FFN_LAYERS, RMS_EPS = 2560, 6912, 30, 1e-5
+
+
+def ffn_block_bytes(M: int) -> int:
+    """Algorithmic bytes of one FFN block: rms+quant (x bf16, gain, codes,
+    scale+sum), gate and up GEMVs, relu^2*up + sub-norm + quant (two fp32
+    rows, gain, codes, scale+sum), down GEMV."""
+    H, I = FFN_H, FFN_I
+    rms = M * H * 2 + H * 4 + M * H + M * 8
+    relu = 2 * M * I * 4 + I * 4 + M * I + M * 8
+    return rms + 2 * algorithmic_bytes(I, H, M) + relu + algorithmic_bytes(H, I, M)
+
+
+def absmean_bytes(N: int, K: int) -> int:
+    """Two reads of the bf16 weights (the sum must be complete before any
+    weight is quantised and 178 MB does not stay on chip), the packed bytes
+    and the scale."""
+    return 2 * 2 * N * K + N * K // 4 + 4
+
+
+def run_chain(args, rank: int, world: int):
+    """The decoder-layer chain or the absmean packer: same JSON line as the
+    stack; CUDA-graph replays, e2e through the library calls with host
+    buffers, the oracle on a bounded sample as the CPU baseline."""
+    import torch
+
+    import ternary_absmax_int8_b200 as tq
+
+    dev_i = int(os.environ.get("LOCAL_RANK", "0"))
+    rng = np.random.default_rng(args.seed)
+    if args.impl == "reference" and rank != 0:
+        return None
+    if args.impl == "ours":
+        torch.cuda.set_device(dev_i)
+    stream = torch.cuda.current_stream() if args.impl == "ours" else None
+    if args.workload == "ffn_block30_m1":
+        M, H, I, L = 1, FFN_H, FFN_I, FFN_LAYERS
+        shapes = [(f"L{l}.{n}", a, b) for l in range(L)
+                  for (n, a, b) in (("gate_proj", I, H), ("up_proj", I, H), ("down_proj", H, I))]
+        projs = list(make_projections(shapes, M=M, seed=args.seed))
+        g_in = rng.uniform(0.5, 1.5, (L, H)).astype(np.float32)
+        g_ffn = rng.uniform(0.5, 1.5, (L, I)).astype(np.float32)
+        sb = L * ffn_block_bytes(M)
+        if args.impl == "reference":
+            return chain_reference(args, projs, g_in, g_ffn, sb, world)
+        packed = []
+        for p in projs:
+            P = np.empty((p.N // 4, p.K), np.uint8)
+            tq.tq_pack_host(p.w, P, M, p.N, p.K)
+            packed.append(torch.from_numpy(P).cuda())
+        x_host = torch.from_numpy(np.stack([projs[3 * l].x_bf16.view(np.int16)
+                                            for l in range(L)])).pin_memory()
+        x_dev = x_host.cuda()
+        gi, gf = torch.from_numpy(g_in).cuda(), torch.from_numpy(g_ffn).cuda()
+        xq = torch.empty((L, M, H), dtype=torch.int8, device="cuda")
+        xs = torch.empty((L, M), device="cuda")
+        xsum = torch.empty((L, M), dtype=torch.int32, device="cuda")
+        yg = torch.empty((L, M, I), device="cuda")
+        yu = torch.empty((L, M, I), device="cuda")
+        xq2 = torch.empty((L, M, I), dtype=torch.int8, device="cuda")
+        xs2 = torch.empty((L, M), device="cuda")
+        xsum2 = torch.empty((L, M), dtype=torch.int32, device="cuda")
+        yd = torch.empty((L, M, H), device="cuda")
+        y_host = torch.empty_like(yd, device="cpu").pin_memory()
+        tabs = [[tq.make_proj(packed=packed[3 * l + j], xq=xq[l], x_scale=xs[l], x_sum=xsum[l],
+                              y=(yg if j == 0 else yu)[l], w_scale=projs[3 * l + j].w_scale,
+                              N=I, K=H) for j in (0, 1)] for l in range(L)]
+        xq_b = torch.empty((L, M, H), dtype=torch.int8, device="cuda")
+        xs_b = torch.empty((L, M), device="cuda")
+        xsum_b = torch.empty((L, M), dtype=torch.int32, device="cuda")
+        # gate + up: one launch that normalises (gain g_in) and quantises the
+        # shared input itself; down: one launch that computes relu^2(gate) *
+        # up, normalises (g_ffn) and quantises, streaming its weights while
+        # the first launch drains.
+        tabs = [[tq.make_proj(packed=packed[3 * l], x=x_dev[l], xq=xq[l], x_scale=xs[l],
+                              x_sum=xsum[l], y=yg[l], w_scale=projs[3 * l].w_scale, N=I, K=H,
+                              gain=gi[l], eps=RMS_EPS),
+                 tq.make_proj(packed=packed[3 * l + 1], x=x_dev[l], xq=xq_b[l], x_scale=xs_b[l],
+                              x_sum=xsum_b[l], y=yu[l], w_scale=projs[3 * l + 1].w_scale, N=I,
+                              K=H, gain=gi[l], eps=RMS_EPS)] for l in range(L)]
+        dtabs = [[tq.make_proj(packed=packed[3 * l + 2], x_f32=yg[l], up=yu[l], xq=xq2[l],
+                               x_scale=xs2[l], x_sum=xsum2[l], y=yd[l],
+                               w_scale=projs[3 * l + 2].w_scale, N=H, K=I, gain=gf[l],
+                               eps=RMS_EPS)] for l in range(L)]
+        ov = tq.TQ_STACK_OVERLAP_PREV
+
+        def step(s_):
+            for l in range(L):
+                tq.tq_gemv_stack(tabs[l], flags=tq.TQ_STACK_RMSNORM, stream=s_)
+                tq.tq_gemv_stack(dtabs[l], flags=tq.TQ_STACK_RELU2_MUL | ov, stream=s_)
+
+        launches, kernel = 2 * L, "stream_gemv_kernel (normalising + quantising prologue)"
+        bytes_in = int(x_host.numel() * x_host.element_size())
+        bytes_out = int(y_host.numel() * y_host.element_size())
+        config = {"layers": L, "projections": 3 * L, "tokens_M": M,
+                  "packed_weight_bytes": sum(p.N * p.K // 4 for p in projs), "rms_eps": RMS_EPS,
+                  "l2": "inputs larger than L2 (weight stream 398 MB), no flush"}
+    else:
+        N, K = 17408, 5120
+        W = (rng.standard_normal((N, K), dtype=np.float32) * 0.02)
+        Wb = torch.from_numpy(W).to(torch.bfloat16)
+        sb = absmean_bytes(N, K)
+        if args.impl == "reference":
+            return absmean_reference(args, Wb.view(torch.int16).numpy().view(np.uint16), sb)
+        x_host = Wb.view(torch.int16).pin_memory()
+        x_dev = x_host.cuda()
+        packed_dev = torch.empty((N // 4, K), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(1, device="cuda")
+        y_host = torch.empty((N // 4, K), dtype=torch.uint8).pin_memory()
+        yd = packed_dev
+
+        def step(s_):
+            tq.tq_absmean_pack(x_dev, packed_dev, ws, N, K, stream=s_)
+
+        launches, kernel = 2, "absmean_sum_kernel + absmean_pack_kernel"
+        bytes_in = int(x_host.numel() * 2)
+        bytes_out = int(y_host.numel())
+        config = {"N": N, "K": K, "weight_bytes_bf16": 2 * N * K,
+                  "l2": "weights (178 MB) larger than L2; the second pass re-reads them, part "
+                        "from L2"}
+
+    for _ in range(args.warmup):
+        step(stream)
+    torch.cuda.synchronize()
+    K_ = args.steps
+    S = 4 if args.workload == "ffn_block30_m1" else 8
+    n_chunks, rem = divmod(K_, S)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=cs):
+            fn(cs)
+        return g
+
+    chunk = capture(lambda cs: [step(cs) for _ in range(S)])
+    single = capture(step) if rem else None
+    chunk.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev_i)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(n_chunks):
+        chunk.replay()
+    for _ in range(rem):
+        single.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    e2e_steps = max(K_, int(0.5e3 / max(total_ms / K_, 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(stream)
+        y_host.copy_(yd, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    time.sleep(0.3)
+    clk = clocks.stop()
+    assert tq.tq_device_error(reset=True) == 0, "a kernel reported a device error"
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device="cuda")
+    if rank != 0:
+        return None
+    ms_step = total_ms / K_
+    value = whole_job_rate(world, sb, ms_step) / 1e9
+    peak, peak_kind = measured_peak()
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K_, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 codes / ternary (bf16 and fp32 rows in, fp64 norm statistics)",
+        "data": "synthetic (seeded ternary weights P=0.3/0.4/0.3, bf16 N(0,1) activations "
+                "with 1% x20 outliers; gains U(0.5,1.5); latent weights N(0,0.02))",
+        "config": {"workload": f"{args.workload}: {CHAIN_WORKLOADS[args.workload]}",
+                   "step_bytes": sb, "parallelism": "single GPU" if world == 1 else
+                   f"replicas x{world}", "seed": args.seed, **config},
+        "roofline": {"kernel": kernel, "bound": "hbm", "achieved": round(value / world, 1),
+                     "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy "
+                                                f"bandwidth)", "unit": "GB/s",
+                     "frac": round(value / world / peak, 4), "traffic": None,
+                     "algorithmic_bytes_per_step": sb},
+        "e2e": {"value": round(whole_job_rate(world, sb, e2e_ms / e2e_steps) / 1e9, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": bytes_out,
+                "ms_per_step": round(e2e_ms / e2e_steps, 5)},
+        "gpu_launches": launches * K_,
+        "clocks": clk,
+        "impl": "ours",
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        sample = dict(args.__dict__)
+        sample["impl"] = "reference"
+        sample["steps"], sample["warmup"] = 1, 0
+        ref = run_chain(argparse.Namespace(**sample), 0, 1)
+        out["cpu_baseline"] = dict(ref["cpu_baseline"])
+    return out
+
+
+def chain_reference(args, projs, g_in, g_ffn, sb, world):
+    """The oracle on one FFN block per step (a bounded sample), the same chain
+    as the GPU step."""
+    import oracle
+
+    H, I = FFN_H, FFN_I
+    gate, up, down = projs[0], projs[1], projs[2]
+    P = [oracle.pack(p.w) for p in (gate, up, down)]
+    xb = gate.x_bf16
+    f32 = (xb.astype(np.uint32) << 16).view(np.float32)
+
+    def one():
+        q, s, t = oracle.quant_f32(oracle.rmsnorm(f32, g_in[0], RMS_EPS))
+        yg = oracle.epilogue(oracle.gemv(P[0], I, q), gate.w_scale, s).astype(np.float32)
+        yu = oracle.epilogue(oracle.gemv(P[1], I, q), up.w_scale, s).astype(np.float32)
+        q2, s2, t2 = oracle.quant_f32(oracle.rmsnorm(oracle.relu2_mul(yg, yu), g_ffn[0],
+                                                     RMS_EPS))
+        oracle.epilogue(oracle.gemv(P[2], H, q2), down.w_scale, s2)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    n = max(1, args.steps)
+    for _ in range(n):
+        one()
+    el = time.perf_counter() - t0
+    per_block = sb // FFN_LAYERS
+    value = per_block * n / el / 1e9
+    return _ref_line(args, world, value, el / n * 1e3,
+                     f"one FFN block (layer 0) of {args.workload} per step, one thread, on "
+                     f"{os.cpu_count()} host cores")
+
+
+def absmean_reference(args, Wb, sb):
+    """The oracle absmean + pack on a 1/16 row slice per step (bounded)."""
+    import oracle
+
+    rows = Wb.shape[0] // 16
+    sub = np.ascontiguousarray(Wb[:rows])
+    for _ in range(args.warmup):
+        oracle.pack(oracle.absmean(sub)[0])
+    t0 = time.perf_counter()
+    n = max(1, args.steps)
+    for _ in range(n):
+        oracle.pack(oracle.absmean(sub)[0])
+    el = time.perf_counter() - t0
+    value = (sb / 16) * n / el / 1e9
+    return _ref_line(args, 1, value, el / n * 1e3,
+                     f"rows 0..{rows - 1} of the 17408x5120 weights per step, one thread, on "
+                     f"{os.cpu_count()} host cores")
+
+
+def _ref_line(args, world, value, ms, sample):
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "oracle (int32 accumulate, fp64 statistics)", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {CHAIN_WORKLOADS[args.workload]}",
+                   "parallelism": "host, one thread"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="stack30_m1")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CHAIN_WORKLOADS),
+                    default="stack30_m1")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -575,8 +859,12 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        out = run_ours(args, rank, world) if args.impl == "ours" else \
-            run_reference(args, rank, world)
+        if args.workload in CHAIN_WORKLOADS:
+            out = run_chain(args, rank, world)
+        elif args.impl == "ours":
+            out = run_ours(args, rank, world)
+        else:
+            out = run_reference(args, rank, world)
     finally:
         if world > 1 and args.impl == "ours":
             import torch.distributed as dist

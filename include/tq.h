@@ -136,6 +136,12 @@ typedef struct tq_proj {
     float w_scale;
     int N;
     int K;
+    /* TQ_STACK_RMSNORM / TQ_STACK_RELU2_MUL only (else ignored): */
+    const float *gain;      /* fp32 [K] RMSNorm gain */
+    const float *x_f32;     /* fp32 [K] TQ_STACK_RELU2_MUL: the gate projection's output */
+    const float *up;        /* fp32 [K] TQ_STACK_RELU2_MUL: the up projection's output */
+    float eps;              /* RMSNorm epsilon, finite, >= 0 */
+    int reserved;           /* set to 0 */
 } tq_proj;
 
 /* Flags for tq_gemv_stack. */
@@ -150,6 +156,18 @@ typedef struct tq_proj {
                                     tq_quantize_act_stack would write, instead of
                                     being read. One launch per call replaces the
                                     quantiser launch and the GEMV launch. */
+#define TQ_STACK_RMSNORM 4u      /* as TQ_STACK_QUANTIZE, with RMSNorm (gain, eps)
+                                    applied to x first: the values
+                                    tq_rmsnorm_quantize would write. */
+#define TQ_STACK_RELU2_MUL 8u    /* as TQ_STACK_RMSNORM on v = relu(x_f32)^2 * up
+                                    (fp32 rows, 16-byte aligned): the values
+                                    tq_relu2_mul_rmsnorm_quantize would write.
+                                    With TQ_STACK_OVERLAP_PREV the launch streams
+                                    weights while the kernel producing x_f32 and up
+                                    finishes. At most one of the three quantising
+                                    flags; the launch quantises its own inputs, so
+                                    entries sharing one input each write identical
+                                    xq, x_scale and x_sum. */
 
 /*
  * tq_quantize_act_stack -- tq_quantize_act for each projection's single
@@ -160,12 +178,13 @@ tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t s
 
 /*
  * tq_gemv_stack -- tq_gemv (M = 1) for every projection, in one persistent
- * launch per 320 projections that streams all their weights back to back, in
+ * launch per 256 projections that streams all their weights back to back, in
  * projection order, with no drain between projections. projs is a HOST array
  * (read during the call only; the table travels in the launch parameters).
- * flags: any of TQ_STACK_OVERLAP_PREV and TQ_STACK_QUANTIZE. Without
- * TQ_STACK_QUANTIZE, xq, x_scale and x_sum are inputs (from
- * tq_quantize_act_stack); with it, x is the input and they are outputs.
+ * flags: TQ_STACK_OVERLAP_PREV, and at most one of TQ_STACK_QUANTIZE,
+ * TQ_STACK_RMSNORM, TQ_STACK_RELU2_MUL. Without those, xq, x_scale and x_sum
+ * are inputs (from tq_quantize_act_stack); with one, the launch computes
+ * them from x (or x_f32 and up) and writes them.
  * Projections are independent: y of one must not be another's input within
  * the same call, and no buffer may be shared between two entries.
  */
@@ -204,7 +223,11 @@ tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq
  *   r = fl32(1 / sqrt(sum_k v^2 / K + eps))   (the sum and root in fp64)
  *   h[k] = fl32(fl32(v[k] * r) * gain[k]),  then the absmax quantiser of
  *   tq_quantize_act on h (xq, x_scale, x_sum as there).
- * One CTA per token row. Host checks: 0 <= M, 0 < K <= 32768, K % 16 == 0,
+ * One CTA per token row, launched with programmatic stream serialisation:
+ * the kernel waits for the previous kernel on the stream to complete before
+ * it touches memory, and lets the next one start early (a tq_gemv_stack with
+ * TQ_STACK_OVERLAP_PREV streams weights meanwhile).
+ * Host checks: 0 <= M, 0 < K <= 32768, K % 16 == 0,
  * eps >= 0 and finite; byte tensors and fp32 rows 16-byte aligned, vectors
  * 4-byte aligned. M == 0 is a no-op.
  *

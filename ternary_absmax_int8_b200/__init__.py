@@ -15,7 +15,8 @@ import ctypes
 import os
 
 __all__ = [
-    "TQError", "TQ_STACK_OVERLAP_PREV", "TQ_STACK_QUANTIZE", "TqProj", "lib_path",
+    "TQError", "TQ_STACK_OVERLAP_PREV", "TQ_STACK_QUANTIZE", "TQ_STACK_RMSNORM",
+    "TQ_STACK_RELU2_MUL", "TqProj", "lib_path",
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
     "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
@@ -27,6 +28,8 @@ lib_path = os.path.join(_HERE, "libtq.so")
 
 TQ_STACK_OVERLAP_PREV = 1
 TQ_STACK_QUANTIZE = 2
+TQ_STACK_RMSNORM = 4
+TQ_STACK_RELU2_MUL = 8
 _STATUS = {0: "TQ_OK", 1: "TQ_ERR_NULL", 2: "TQ_ERR_SHAPE", 3: "TQ_ERR_ALIGN",
            4: "TQ_ERR_VALUE", 5: "TQ_ERR_CUDA", 6: "TQ_ERR_UNSUPPORTED"}
 
@@ -54,6 +57,11 @@ class TqProj(ctypes.Structure):
         ("w_scale", ctypes.c_float),
         ("N", ctypes.c_int),
         ("K", ctypes.c_int),
+        ("gain", ctypes.c_void_p),
+        ("x_f32", ctypes.c_void_p),
+        ("up", ctypes.c_void_p),
+        ("eps", ctypes.c_float),
+        ("reserved", ctypes.c_int),
     ]
 
 
@@ -182,9 +190,11 @@ def tq_absmean_pack(w_bf16, packed, w_scale, N: int, K: int, stream=None) -> Non
 
 
 def make_proj(packed=None, x=None, xq=None, x_scale=None, x_sum=None, y=None, acc_out=None,
-              w_scale: float = 0.0, N: int = 0, K: int = 0) -> TqProj:
+              w_scale: float = 0.0, N: int = 0, K: int = 0, gain=None, x_f32=None, up=None,
+              eps: float = 0.0) -> TqProj:
     return TqProj(_ptr(packed), _ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), _ptr(y),
-                  _ptr(acc_out), float(w_scale), int(N), int(K))
+                  _ptr(acc_out), float(w_scale), int(N), int(K), _ptr(gain), _ptr(x_f32),
+                  _ptr(up), float(eps), 0)
 
 
 def _proj_array(projs):

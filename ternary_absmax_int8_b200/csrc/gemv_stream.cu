@@ -226,6 +226,9 @@ struct FMax {
 struct IAdd {
     __device__ int operator()(int a, int b) const { return a + b; }
 };
+struct DAdd {
+    __device__ double operator()(double a, double b) const { return a + b; }
+};
 
 
 // W consumer warps per group, G groups: group g consumes the CTA's tiles
@@ -362,18 +365,17 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
 
     // ---------------------------------------------------------- consumers
     // Each consumer warp walks the ring on its own (no CTA barrier in the
-    // loop). For each of its items it copies the item's packed words from
-    // the stage into registers, hands the stage back after its last item's
-    // copy, and only then computes: a stage is held for the copy, not for the
-    // arithmetic, so nearly the whole ring stays in flight.
+    // loop): for each of its items it reads the packed words from the stage
+    // while it computes, and hands the stage back after its last item's K
+    // loop (rows split over warps: after their partial sums are in).
     pdl_wait();  // activations, x_scale and x_sum are read below
-    if (MT == 1 && p.quant) {
+    if (MT == 1 && p.quant == 1) {
         // Quantise the CTA's activations (one token per projection) straight
         // into the activation cache. The CTA that streams a projection's
         // first tile also writes xq, x_scale and x_sum to global memory.
         for (int j = 0; j < n_entries; ++j) {
             const StreamEntry &e = tab[j];
-            const uint4 *xv = reinterpret_cast<const uint4 *>(e.xb);
+            const uint4 *xv = reinterpret_cast<const uint4 *>(e.xin);
             const int nvec = e.K >> 3;  // 8 bf16 per 16-byte vector
             float amax = 0.0f;
             for (int v = threadIdx.x; v < nvec; v += WC * 32)
@@ -389,6 +391,79 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                 qc[v] = o;
                 if (owner)
                     qg[v] = o;
+            }
+            sum = consumer_reduce<WC>(sum, IAdd(), red);
+            if (threadIdx.x == 0) {
+                const float xs = quant_scale(amax);
+                scl[j * MT] = make_float2(__fmul_rn(e.w_scale, xs), __int_as_float(sum));
+                if (owner) {
+                    *e.x_scale = xs;
+                    *e.x_sum = sum;
+                }
+            }
+        }
+    } else if (MT == 1 && p.quant >= 2) {
+        // RMSNorm (gain, eps) of the token -- of bf16 x (mode 2) or of
+        // relu(gate)^2 * up from fp32 rows (mode 3) -- then the same
+        // quantiser, with the arithmetic of the standalone normalising
+        // kernels: r = fl32(1 / sqrt(sum v^2 / K + eps)) from an fp64 sum,
+        // h = fl32(fl32(v * r) * gain). Three passes over the row (from L2).
+        static_assert(WC <= 16, "one fp64 reduction slot per consumer warp");
+        for (int j = 0; j < n_entries; ++j) {
+            const StreamEntry &e = tab[j];
+            const int K = e.K;
+            auto v4 = [&](int k) -> float4 {
+                if (p.quant == 2) {
+                    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(
+                        static_cast<const uint16_t *>(e.xin) + k));
+                    return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+                }
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(
+                    static_cast<const float *>(e.xin) + k));
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(e.up + k));
+                auto r2 = [](float g, float u) {
+                    const float r = fmaxf(g, 0.0f);
+                    return __fmul_rn(__fmul_rn(r, r), u);
+                };
+                return make_float4(r2(a.x, b.x), r2(a.y, b.y), r2(a.z, b.z), r2(a.w, b.w));
+            };
+            double ss = 0.0;
+            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
+                const float4 v = v4(k);
+                ss += double(v.x) * v.x;  // each square exact in fp64
+                ss += double(v.y) * v.y;
+                ss += double(v.z) * v.z;
+                ss += double(v.w) * v.w;
+            }
+            ss = consumer_reduce<WC>(ss, DAdd(), reinterpret_cast<double *>(red));
+            const float r = __double2float_rn(1.0 / sqrt(ss / double(K) + double(e.eps)));
+            auto h_of = [&](float v, int k) {
+                return __fmul_rn(__fmul_rn(v, r), __ldg(e.gain + k));
+            };
+            float amax = 0.0f;
+            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
+                const float4 v = v4(k);
+                amax = fmaxf(amax, fabsf(h_of(v.x, k)));
+                amax = fmaxf(amax, fabsf(h_of(v.y, k + 1)));
+                amax = fmaxf(amax, fabsf(h_of(v.z, k + 2)));
+                amax = fmaxf(amax, fabsf(h_of(v.w, k + 3)));
+            }
+            amax = consumer_reduce<WC>(amax, FMax(), reinterpret_cast<float *>(red));
+            const float s = quant_inv_scale(amax);
+            const bool owner = e.tile_begin >= t_begin;
+            uint32_t *qc = reinterpret_cast<uint32_t *>(xcache + xoff[j]);
+            uint32_t *qg = reinterpret_cast<uint32_t *>(e.xq);
+            int sum = 0;
+            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
+                const float4 v = v4(k);
+                const int a = code_of(h_of(v.x, k), s), b = code_of(h_of(v.y, k + 1), s);
+                const int c = code_of(h_of(v.z, k + 2), s), d = code_of(h_of(v.w, k + 3), s);
+                sum += a + b + c + d;
+                const uint32_t word = (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) |
+                                      ((uint32_t(c) & 0xFFu) << 16) | ((uint32_t(d) & 0xFFu) << 24);
+                qc[k >> 2] = word;
+                if (owner)
+                    qg[k >> 2] = word;
             }
             sum = consumer_reduce<WC>(sum, IAdd(), red);
             if (threadIdx.x == 0) {
@@ -641,7 +716,7 @@ cudaError_t launch_variant(const StreamCfg &c, const StreamParams<MaxE> &p, int 
 
 template <int MaxE>
 cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, bool single,
-                         bool quant, cudaStream_t stream)
+                         int quant, cudaStream_t stream)
 {
     StreamParams<MaxE> p;  // host staging of the launch parameters
     static_assert(sizeof(StreamParams<MaxE>) <= 32000, "kernel parameters exceed 32 KB");
@@ -688,7 +763,7 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
     p.M = M;
     p.w_slot = (stage_max + 127) / 128 * 128;
     p.overlap_prev = overlap_prev ? 1 : 0;
-    p.quant = quant ? 1 : 0;
+    p.quant = quant;
     const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
     if (total == 0)
         return cudaSuccess;
@@ -775,11 +850,12 @@ cudaError_t launch_sized(StreamEntry *entries, int n, int M, bool overlap_prev, 
 }  // namespace
 
 cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_prev, bool single,
-                               bool quant, cudaStream_t stream)
+                               int quant, cudaStream_t stream)
 {
     if (n <= 0)
         return cudaSuccess;
-    if (M < 1 || M > kStreamMaxTokens || n > kStreamStackMax || (quant && M != 1))
+    if (M < 1 || M > kStreamMaxTokens || n > kStreamStackMax || quant < 0 || quant > 3 ||
+        (quant && M != 1))
         return cudaErrorInvalidValue;
     if (n == 1)
         return launch_sized<1>(entries, n, M, overlap_prev, single, quant, stream);

@@ -16,10 +16,14 @@
 //   absmean:  gamma = fl32(sum |W| / (N K)) (fp64 sum), w = clamp(rne(fl32(W
 //             / gamma)), -1, 1), code w + 1 packed four rows to a byte
 //
-// The normalise-and-quantise kernels take one CTA per token: pass 1 reduces
-// the sum of squares (fp64), pass 2 the largest |h| (exact), pass 3 writes
-// the codes and reduces their sum; passes 2 and 3 re-read the row from L1/L2
-// and recompute h, so nothing but the codes is written.
+// The normalise-and-quantise kernels take one CTA of 1024 threads per token:
+// pass 1 reads the row into shared memory and reduces the sum of squares
+// (fp64), pass 2 the largest |h| (exact), pass 3 writes the codes and
+// reduces their sum; passes 2 and 3 recompute h from shared memory, so the
+// row is read once and nothing but the codes is written. They are launched
+// with programmatic stream serialisation and wait for the previous grid
+// before any memory access, so a following stack GEMV launched with
+// TQ_STACK_OVERLAP_PREV streams its weights while they run.
 #include <algorithm>
 #include <cfloat>
 
@@ -30,7 +34,7 @@ namespace tq {
 
 namespace {
 
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 1024;
 
 enum RowInput : int { kInBf16 = 0, kInF32 = 1, kInRelu2Mul = 2 };
 
@@ -93,12 +97,20 @@ rms_quant_kernel(const RowParams p)
     __shared__ double red_d[kRowThreads / 32];
     __shared__ float red_f[kRowThreads / 32];
     __shared__ int red_i[kRowThreads / 32];
+    extern __shared__ float4 row[];  // the row's inputs v, K / 4 vectors
     const int K = p.K;
     const size_t base = size_t(blockIdx.x) * K;
+    // Launched with programmatic stream serialisation: let the next grid (a
+    // GEMV that streams weights first) start, and wait for the previous grid
+    // (which may produce this row) before touching memory.
+    pdl_launch_dependents();
+    pdl_wait();
 
+    // Pass 1 reads the row once from global memory into shared memory.
     double ss = 0.0;
     for (int k = 4 * threadIdx.x; k < K; k += 4 * kRowThreads) {
         const float4 v = load4<In>(p, base, k);
+        row[k >> 2] = v;
         ss += double(v.x) * v.x;  // each square exact in fp64
         ss += double(v.y) * v.y;
         ss += double(v.z) * v.z;
@@ -110,7 +122,7 @@ rms_quant_kernel(const RowParams p)
     auto h_of = [&](float v, int k) { return __fmul_rn(__fmul_rn(v, r), __ldg(p.gain + k)); };
     float amax = 0.0f;
     for (int k = 4 * threadIdx.x; k < K; k += 4 * kRowThreads) {
-        const float4 v = load4<In>(p, base, k);
+        const float4 v = row[k >> 2];
         amax = fmaxf(amax, fabsf(h_of(v.x, k)));
         amax = fmaxf(amax, fabsf(h_of(v.y, k + 1)));
         amax = fmaxf(amax, fabsf(h_of(v.z, k + 2)));
@@ -121,7 +133,7 @@ rms_quant_kernel(const RowParams p)
 
     int sum = 0;
     for (int k = 4 * threadIdx.x; k < K; k += 4 * kRowThreads) {
-        const float4 v = load4<In>(p, base, k);
+        const float4 v = row[k >> 2];
         const int a = code_of(h_of(v.x, k), s), b = code_of(h_of(v.y, k + 1), s);
         const int c = code_of(h_of(v.z, k + 2), s), d = code_of(h_of(v.w, k + 3), s);
         sum += a + b + c + d;
@@ -225,13 +237,41 @@ cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f
                              float *x_scale, int32_t *x_sum, int M, int K, cudaStream_t stream)
 {
     RowParams p{x_bf16, x_f32, up, gain, eps, xq, x_scale, x_sum, K};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(M);
+    cfg.blockDim = dim3(kRowThreads);
+    cfg.dynamicSmemBytes = size_t(K) * sizeof(float);
+    cfg.stream = stream;
+    static int configured_dev = -1;  // the row may need more than 48 KB
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        const int most = int(kStreamMaxK * sizeof(float));
+        cudaError_t e = cudaFuncSetAttribute(rms_quant_kernel<kInBf16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(rms_quant_kernel<kInF32>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(rms_quant_kernel<kInRelu2Mul>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     if (input == kInBf16)
-        rms_quant_kernel<kInBf16><<<M, kRowThreads, 0, stream>>>(p);
+        e = cudaLaunchKernelEx(&cfg, rms_quant_kernel<kInBf16>, p);
     else if (input == kInF32)
-        rms_quant_kernel<kInF32><<<M, kRowThreads, 0, stream>>>(p);
+        e = cudaLaunchKernelEx(&cfg, rms_quant_kernel<kInF32>, p);
     else
-        rms_quant_kernel<kInRelu2Mul><<<M, kRowThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+        e = cudaLaunchKernelEx(&cfg, rms_quant_kernel<kInRelu2Mul>, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_absmean_pack(const uint16_t *w, uint8_t *packed, float *w_scale, int N, int K,

@@ -145,7 +145,7 @@ tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
         e.w_scale = w_scale;
         e.N4 = N / 4;
         e.K = K;
-        cudaError_t err = tq::launch_stream_gemv(&e, 1, mg, false, true, false, stream);
+        cudaError_t err = tq::launch_stream_gemv(&e, 1, mg, false, true, 0, stream);
         if (err != cudaSuccess)
             return cuda_fail(err, fn);
     }
@@ -321,13 +321,18 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
 {
     if (n_proj < 0)
         return fail(TQ_ERR_SHAPE, "tq_gemv_stack: n_proj=%d", n_proj);
-    if (flags & ~unsigned(TQ_STACK_OVERLAP_PREV | TQ_STACK_QUANTIZE))
-        return fail(TQ_ERR_VALUE, "tq_gemv_stack: unknown flags 0x%x", flags);
+    const unsigned qflags = flags & (TQ_STACK_QUANTIZE | TQ_STACK_RMSNORM | TQ_STACK_RELU2_MUL);
+    if ((flags & ~(unsigned(TQ_STACK_OVERLAP_PREV) | qflags)) || (qflags & (qflags - 1)))
+        return fail(TQ_ERR_VALUE, "tq_gemv_stack: bad flags 0x%x", flags);
     if (n_proj == 0)
         return ok();
     if (!projs)
         return fail(TQ_ERR_NULL, "tq_gemv_stack: projs is NULL");
-    const bool quant = (flags & TQ_STACK_QUANTIZE) != 0;
+    // the launch's quantising mode: 1 absmax of bf16 x, 2 RMSNorm then absmax,
+    // 3 relu(x_f32)^2 * up, RMSNorm, absmax
+    const int mode = qflags == TQ_STACK_QUANTIZE ? 1
+                     : qflags == TQ_STACK_RMSNORM ? 2
+                     : qflags == TQ_STACK_RELU2_MUL ? 3 : 0;
     std::vector<tq::StreamEntry> list;
     list.reserve(size_t(n_proj));
     for (int j = 0; j < n_proj; ++j) {
@@ -338,19 +343,26 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
             check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, 1, p.N, p.K);
         if (st != TQ_OK)
             return st;
-        if (quant && p.K > 0 && !p.x)
-            return fail(TQ_ERR_NULL, "%s: x is NULL (TQ_STACK_QUANTIZE)", fn);
-        if (quant && p.K > 0 && !aligned(p.x, 16))
-            return fail(TQ_ERR_ALIGN, "%s: x must be 16-byte aligned", fn);
-        if (p.N == 0 && !quant)
+        const void *xin = mode == 3 ? static_cast<const void *>(p.x_f32)
+                                    : static_cast<const void *>(p.x);
+        if (mode && p.K > 0) {
+            if (!xin || (mode == 3 && !p.up) || (mode >= 2 && !p.gain))
+                return fail(TQ_ERR_NULL, "%s: x is NULL (or x_f32, up or gain for its mode)", fn);
+            if (!aligned(xin, 16) || (mode == 3 && !aligned(p.up, 16)) ||
+                (mode >= 2 && !aligned(p.gain, 4)))
+                return fail(TQ_ERR_ALIGN, "%s: x must be 16-byte aligned (x_f32, up too)", fn);
+            if (mode >= 2 && (!(p.eps >= 0.0f) || p.eps > FLT_MAX))
+                return fail(TQ_ERR_VALUE, "%s: eps must be finite and >= 0", fn);
+        }
+        if (p.N == 0 && !mode)
             continue;
         if (p.K == 0) {
             // Every accumulator is 0; a quantising call also reports the
             // empty token's scale and sum as 0.
             cudaError_t e = cudaSuccess;
-            if (quant)
+            if (mode)
                 e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
-            if (e == cudaSuccess && quant)
+            if (e == cudaSuccess && mode)
                 e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
             if (e != cudaSuccess)
                 return cuda_fail(e, fn);
@@ -361,17 +373,26 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
         }
         if (p.N == 0) {
             // Nothing to multiply, but the quantiser's outputs are owed.
-            tq::QuantStackParams *qp = quant_params();
-            qp->n = 1;
-            qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
-            cudaError_t e = tq::launch_quant_stack(*qp, stream);
+            cudaError_t e;
+            if (mode == 1) {
+                tq::QuantStackParams *qp = quant_params();
+                qp->n = 1;
+                qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
+                e = tq::launch_quant_stack(*qp, stream);
+            } else {
+                e = tq::launch_rms_quant(mode == 2 ? 0 : 2, p.x, p.x_f32, p.up, p.gain, p.eps,
+                                         p.xq, p.x_scale, p.x_sum, 1, p.K, stream);
+            }
             if (e != cudaSuccess)
                 return cuda_fail(e, fn);
             continue;
         }
         tq::StreamEntry e = {};
         e.packed = p.packed;
-        e.xb = p.x;
+        e.xin = xin;
+        e.gain = p.gain;
+        e.up = p.up;
+        e.eps = p.eps;
         e.xq = p.xq;
         e.x_scale = p.x_scale;
         e.x_sum = p.x_sum;
@@ -386,7 +407,7 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
     for (size_t base = 0; base < list.size(); base += tq::kStreamStackMax) {
         const int n = int(std::min(list.size() - base, size_t(tq::kStreamStackMax)));
         cudaError_t e = tq::launch_stream_gemv(list.data() + base, n, 1, overlap && base == 0,
-                                               false, quant, stream);
+                                               false, mode, stream);
         if (e != cudaSuccess)
             return cuda_fail(e, "tq_gemv_stack");
     }

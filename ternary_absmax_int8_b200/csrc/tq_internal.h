@@ -39,13 +39,16 @@ cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream);
 // so that rows_per_tile << ksplit work items keep every consumer warp busy.
 struct StreamEntry {
     const uint8_t *packed;  // [N4, K]
-    const uint16_t *xb;     // [M, K] bf16 (read only when the launch quantises)
+    const void *xin;        // [M, K] bf16 (quantising modes 1, 2) or fp32 gate (mode 3)
+    const float *gain;      // [K] RMSNorm gain (modes 2, 3)
+    const float *up;        // [M, K] fp32 up (mode 3)
     int8_t *xq;             // [M, K] (written when the launch quantises, else read)
     float *x_scale;         // [M]    (likewise)
     int32_t *x_sum;         // [M]    (likewise)
     float *y;               // [M, 4*N4]
     int32_t *acc_out;       // [M, 4*N4] or null
     float w_scale;
+    float eps;              // RMSNorm epsilon (modes 2, 3)
     int N4;
     int K;
     int rows_per_tile;
@@ -69,7 +72,9 @@ struct StreamParams {
     int w_slot;        // bytes of a ring stage (a tile's packed rows + activations)
     int stages;
     int overlap_prev;  // start weight copies before the previous grid completes
-    int quant;         // quantise each entry's bf16 activations in the launch (M == 1)
+    int quant;         // the launch quantises (M == 1): 0 no (xq is an input); 1 absmax of
+                       // bf16 x; 2 RMSNorm of bf16 x, then absmax; 3 relu(gate)^2 * up, then
+                       // RMSNorm and absmax
     int head_bytes;    // shared memory for the entry table and the per-token scales
     unsigned *err;     // the library's device error word
     // Work split: CTA b streams tiles cta_tile0[b] .. cta_tile0[b+1]-1 (a
@@ -81,7 +86,7 @@ struct StreamParams {
     StreamEntry e[MaxE];
 };
 
-constexpr int kStreamStackMax = 320;  // entries per launch (kernel parameters <= 32 KB)
+constexpr int kStreamStackMax = 256;  // entries per launch (kernel parameters <= 32 KB)
 constexpr int kStreamMaxGrid = kStreamMaxGridFwd;  // CTAs per launch
 
 struct StreamLaunch {
@@ -92,11 +97,12 @@ struct StreamLaunch {
 
 // Plan tiles for a set of entries (fills rows_per_tile, ksplit, tile_begin,
 // total_tiles, x_slot, w_slot, stages) and launch. `single` selects the
-// small-launch heuristics for one projection. With `quant` (M == 1 only) the
-// kernel quantises each entry's bf16 activations itself and writes xq,
-// x_scale and x_sum as the standalone quantiser would.
+// small-launch heuristics for one projection. With `quant` (M == 1 only; the
+// modes of StreamParams::quant) the kernel computes each entry's activation
+// codes itself and writes xq, x_scale and x_sum as the standalone kernels
+// would.
 cudaError_t launch_stream_gemv(StreamEntry *entries, int n, int M, bool overlap_prev,
-                               bool single, bool quant, cudaStream_t stream);
+                               bool single, int quant, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -123,7 +123,7 @@ def test_stack_argument_checks():
         tq.tq_gemv_stack([tq.make_proj(**good), tq.make_proj(**bad)], stream=0)
     assert e.value.name == "TQ_ERR_SHAPE" and "[1]" in str(e.value)
     with pytest.raises(tq.TQError) as e:
-        tq.tq_gemv_stack([tq.make_proj(**good)], flags=8, stream=0)
+        tq.tq_gemv_stack([tq.make_proj(**good)], flags=16, stream=0)   # no such flag
     assert e.value.name == "TQ_ERR_VALUE"
     with pytest.raises(tq.TQError) as e:
         tq.tq_quantize_act_stack([tq.make_proj(**dict(good, K=20))], stream=0)
@@ -137,13 +137,31 @@ def test_stack_argument_checks():
         tq.tq_gemv_stack([tq.make_proj(**dict(good, x=A + 8))], flags=tq.TQ_STACK_QUANTIZE,
                          stream=0)
     assert e.value.name == "TQ_ERR_ALIGN"
+    # the normalising modes need the gain (and x_f32, up for relu^2); one mode
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**good)], flags=tq.TQ_STACK_RMSNORM, stream=0)
+    assert e.value.name == "TQ_ERR_NULL"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**dict(good, gain=A))], flags=tq.TQ_STACK_RELU2_MUL,
+                         stream=0)
+    assert e.value.name == "TQ_ERR_NULL"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**dict(good, gain=A, eps=-1.0))],
+                         flags=tq.TQ_STACK_RMSNORM, stream=0)
+    assert e.value.name == "TQ_ERR_VALUE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack([tq.make_proj(**good)],
+                         flags=tq.TQ_STACK_QUANTIZE | tq.TQ_STACK_RMSNORM, stream=0)
+    assert e.value.name == "TQ_ERR_VALUE"
     tq.tq_gemv_stack([], stream=0)
     tq.tq_quantize_act_stack([], stream=0)
 
 
 def test_tq_proj_layout_matches_header():
-    # 7 pointers, a float and two ints: 7*8 + 4 + 4 + 4 = 68, padded to 72
-    assert ctypes.sizeof(tq.TqProj) == 72
+    # 7 pointers, a float and two ints (68, padded to 72), then 3 pointers, a
+    # float and an int: 72 + 24 + 8 = 104
+    assert ctypes.sizeof(tq.TqProj) == 104
+    assert tq.TqProj.gain.offset == 72 and tq.TqProj.eps.offset == 96
 
 
 def test_layer_op_argument_checks():

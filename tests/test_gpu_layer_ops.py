@@ -103,10 +103,12 @@ def y32(acc, w_scale, x_scale):
     return acc.astype(np.float32) * t[:, None]
 
 
-@pytest.mark.parametrize("M", [1, 4])
-def test_ffn_block_chain(cuda_device, M):
+@pytest.mark.parametrize("M,overlap", [(1, False), (4, False), (1, True)])
+def test_ffn_block_chain(cuda_device, M, overlap):
     # input RMSNorm + quantiser -> gate, up GEMVs -> relu^2(gate) * up,
     # ffn_sub_norm + quantiser -> down GEMV, each step consuming the last.
+    # overlap: the GEMVs as stack launches that stream their weights while
+    # the kernel before them runs (the bench's form).
     H, I = 2560, 6912
     gate_p, up_p, down_p = make_projections(
         [("gate_proj", I, H), ("up_proj", I, H), ("down_proj", H, I)], M=M, seed=31 + M)
@@ -122,15 +124,26 @@ def test_ffn_block_chain(cuda_device, M):
     tq.tq_rmsnorm_quantize(dev(xb.view(np.int16)), None, dev(g_in), EPS, xq, xs, xsum, M, H)
     yg = torch.empty((M, I), device="cuda")
     yu = torch.empty((M, I), device="cuda")
-    tq.tq_gemv(P[0], gate_p.w_scale, xq, xs, xsum, yg, None, M, I, H)
-    tq.tq_gemv(P[1], up_p.w_scale, xq, xs, xsum, yu, None, M, I, H)
     xq2 = torch.empty((M, I), dtype=torch.int8, device="cuda")
     xs2 = torch.empty(M, device="cuda")
     xsum2 = torch.empty(M, dtype=torch.int32, device="cuda")
-    tq.tq_relu2_mul_rmsnorm_quantize(yg, yu, dev(g_ffn), EPS, xq2, xs2, xsum2, M, I)
     yd = torch.empty((M, H), device="cuda")
     accd = torch.empty((M, H), dtype=torch.int32, device="cuda")
-    tq.tq_gemv(P[2], down_p.w_scale, xq2, xs2, xsum2, yd, accd, M, H, I)
+    if overlap:
+        ov = tq.TQ_STACK_OVERLAP_PREV
+        tq.tq_gemv_stack([tq.make_proj(packed=P[0], xq=xq, x_scale=xs, x_sum=xsum, y=yg,
+                                       w_scale=gate_p.w_scale, N=I, K=H),
+                          tq.make_proj(packed=P[1], xq=xq, x_scale=xs, x_sum=xsum, y=yu,
+                                       w_scale=up_p.w_scale, N=I, K=H)], flags=ov)
+        tq.tq_relu2_mul_rmsnorm_quantize(yg, yu, dev(g_ffn), EPS, xq2, xs2, xsum2, M, I)
+        tq.tq_gemv_stack([tq.make_proj(packed=P[2], xq=xq2, x_scale=xs2, x_sum=xsum2, y=yd,
+                                       acc_out=accd, w_scale=down_p.w_scale, N=H, K=I)],
+                         flags=ov)
+    else:
+        tq.tq_gemv(P[0], gate_p.w_scale, xq, xs, xsum, yg, None, M, I, H)
+        tq.tq_gemv(P[1], up_p.w_scale, xq, xs, xsum, yu, None, M, I, H)
+        tq.tq_relu2_mul_rmsnorm_quantize(yg, yu, dev(g_ffn), EPS, xq2, xs2, xsum2, M, I)
+        tq.tq_gemv(P[2], down_p.w_scale, xq2, xs2, xsum2, yd, accd, M, H, I)
     torch.cuda.synchronize()
 
     # ---- oracle, the same chain
@@ -178,3 +191,70 @@ def test_absmean_pack_dequantised_and_zero(cuda_device):
     assert ws == np.float32(0.375 * np.count_nonzero(p.w) / p.w.size)
     packed, ws = run_absmean(np.zeros((8, 64), np.uint16))
     assert ws == 0 and (packed == 0x55).all()   # every code 1 (weight 0)
+
+
+@pytest.mark.parametrize("layers", [1, 3])
+def test_ffn_block_fused_two_launches(cuda_device, layers):
+    # Per layer: one stack launch for gate + up that normalises (RMSNorm,
+    # gain g_in) and quantises x itself, then one stack launch for down that
+    # computes relu^2(gate) * up, normalises (g_ffn) and quantises -- and
+    # streams its weights while the first launch drains. Layers run one
+    # after another on the stream.
+    H, I = 2560, 6912
+    shapes = [(f"L{l}.{n}", a, b) for l in range(layers)
+              for (n, a, b) in (("gate_proj", I, H), ("up_proj", I, H), ("down_proj", H, I))]
+    projs = list(make_projections(shapes, M=1, seed=90 + layers))
+    rng = np.random.default_rng(5)
+    gin = [gains(rng, H) for _ in range(layers)]
+    gff = [gains(rng, I) for _ in range(layers)]
+    keep = []
+    out = []
+    ov = tq.TQ_STACK_OVERLAP_PREV
+    for l in range(layers):
+        gp, upp, dp = projs[3 * l:3 * l + 3]
+        P = [dev(host_pack(p.w)) for p in (gp, upp, dp)]
+        x = dev(gp.x_bf16.view(np.int16))
+        g1, g2 = dev(gin[l]), dev(gff[l])
+        xq = torch.empty(H, dtype=torch.int8, device="cuda")
+        xq_b = torch.empty(H, dtype=torch.int8, device="cuda")
+        xs = torch.empty(2, device="cuda")
+        xsum = torch.empty(2, dtype=torch.int32, device="cuda")
+        yg = torch.empty(I, device="cuda")
+        yu = torch.empty(I, device="cuda")
+        xq2 = torch.empty(I, dtype=torch.int8, device="cuda")
+        xs2 = torch.empty(1, device="cuda")
+        xsum2 = torch.empty(1, dtype=torch.int32, device="cuda")
+        yd = torch.empty(H, device="cuda")
+        accd = torch.empty(H, dtype=torch.int32, device="cuda")
+        keep += [P, x, g1, g2]
+        # gate and up each quantise the shared input into their own buffers
+        tq.tq_gemv_stack([
+            tq.make_proj(packed=P[0], x=x, xq=xq, x_scale=xs[0:1], x_sum=xsum[0:1], y=yg,
+                         w_scale=gp.w_scale, N=I, K=H, gain=g1, eps=EPS),
+            tq.make_proj(packed=P[1], x=x, xq=xq_b, x_scale=xs[1:2], x_sum=xsum[1:2], y=yu,
+                         w_scale=upp.w_scale, N=I, K=H, gain=g1, eps=EPS)],
+            flags=tq.TQ_STACK_RMSNORM | (ov if l else 0))
+        tq.tq_gemv_stack([
+            tq.make_proj(packed=P[2], x_f32=yg, up=yu, xq=xq2, x_scale=xs2, x_sum=xsum2, y=yd,
+                         acc_out=accd, w_scale=dp.w_scale, N=H, K=I, gain=g2, eps=EPS)],
+            flags=tq.TQ_STACK_RELU2_MUL | ov)
+        out.append((xq, xq_b, xs, xsum, xq2, xs2, xsum2, yd, accd))
+    torch.cuda.synchronize()
+    assert tq.tq_device_error(reset=True) == 0
+
+    for l in range(layers):
+        gp, upp, dp = projs[3 * l:3 * l + 3]
+        xq, xq_b, xs, xsum, xq2, xs2, xsum2, yd, accd = out[l]
+        q, s, t = oracle.quant_f32(oracle.rmsnorm(f32_of_bf16(gp.x_bf16), gin[l], EPS))
+        for qq, j in ((xq, 0), (xq_b, 1)):
+            assert_same((qq.cpu().numpy()[None], xs.cpu().numpy()[j:j + 1],
+                         xsum.cpu().numpy()[j:j + 1]), (q, s, t), f"layer {l} input codes")
+        acc_g = oracle.gemv_threads(oracle.pack(gp.w), I, q)
+        acc_u = oracle.gemv_threads(oracle.pack(upp.w), I, q)
+        h = oracle.relu2_mul(y32(acc_g, gp.w_scale, s), y32(acc_u, upp.w_scale, s))
+        q2, s2, t2 = oracle.quant_f32(oracle.rmsnorm(h, gff[l], EPS))
+        assert_same((xq2.cpu().numpy()[None], xs2.cpu().numpy(), xsum2.cpu().numpy()),
+                    (q2, s2, t2), f"layer {l} down codes")
+        acc_d = oracle.gemv_threads(oracle.pack(dp.w), H, q2)
+        assert np.array_equal(accd.cpu().numpy(), acc_d[0])
+        assert_y_close(yd.cpu().numpy()[None], oracle.epilogue(acc_d, dp.w_scale, s2))
