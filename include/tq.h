@@ -266,6 +266,16 @@ tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scal
                           cudaStream_t stream);
 
 /*
+ * tq_selftest_wait_timeout -- exercise the failure path of the kernels'
+ * bounded waits without a fault: one thread waits, with the same bounded
+ * wait the kernels use, on an mbarrier that nothing ever arrives on. After
+ * limit_us (1 .. 2,000,000) microseconds the wait gives up, sets bit 1 of the
+ * device error word and the kernel returns; the context stays usable. Read
+ * the result with tq_device_error. Asynchronous on `stream`.
+ */
+tq_status tq_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream);
+
+/*
  * tq_device_error -- read (and if reset != 0, clear) the library's device
  * error word on the current device. Synchronises the device. 0 means no
  * kernel has reported an error. A nonzero value means a kernel gave up a

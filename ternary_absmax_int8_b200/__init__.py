@@ -20,7 +20,7 @@ __all__ = [
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
     "tq_quantize_act_stack", "tq_gemv_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
-    "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack",
+    "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack", "tq_selftest_wait_timeout",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +77,7 @@ _SIGS = {
     "tq_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
     "tq_relu2_mul_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
     "tq_absmean_pack": [_vp, _vp, _vp, _i, _i, _vp],
+    "tq_selftest_wait_timeout": [ctypes.c_uint, _vp],
 }
 _lib_handle = None
 
@@ -187,6 +188,11 @@ def tq_absmean_pack(w_bf16, packed, w_scale, N: int, K: int, stream=None) -> Non
     """Absmean ternary quantisation of bf16 weights [N,K] -> packed [N/4,K], w_scale [1]."""
     _check(_load().tq_absmean_pack(_ptr(w_bf16), _ptr(packed), _ptr(w_scale), N, K,
                                 _stream(stream)))
+
+
+def tq_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """A bounded wait that nothing satisfies: sets the device error word."""
+    _check(_load().tq_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def make_proj(packed=None, x=None, xq=None, x_scale=None, x_sum=None, y=None, acc_out=None,

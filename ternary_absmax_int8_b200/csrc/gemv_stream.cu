@@ -407,7 +407,8 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
         // relu(gate)^2 * up from fp32 rows (mode 3) -- then the same
         // quantiser, with the arithmetic of the standalone normalising
         // kernels: r = fl32(1 / sqrt(sum v^2 / K + eps)) from an fp64 sum,
-        // h = fl32(fl32(v * r) * gain). Three passes over the row (from L2).
+        // h = fl32(fl32(v * r) * gain). Three passes over the row: sum of
+        // squares, largest |h|, codes.
         static_assert(WC <= 16, "one fp64 reduction slot per consumer warp");
         for (int j = 0; j < n_entries; ++j) {
             const StreamEntry &e = tab[j];
@@ -427,44 +428,74 @@ stream_gemv_kernel(const __grid_constant__ StreamParams<MaxE> p)
                 };
                 return make_float4(r2(a.x, b.x), r2(a.y, b.y), r2(a.z, b.z), r2(a.w, b.w));
             };
+            // Each thread keeps its first kNV groups of four inputs, and
+            // their gains, in registers across the three passes (all of a
+            // row up to K = 4 kNV x 32 WC); a tail beyond that is re-read.
+            constexpr int kNV = 4;
+            constexpr int stride = 4 * WC * 32;
+            auto g4 = [&](int k) {
+                return make_float4(__ldg(e.gain + k), __ldg(e.gain + k + 1),
+                                   __ldg(e.gain + k + 2), __ldg(e.gain + k + 3));
+            };
+            float4 vr[kNV], gr[kNV];
             double ss = 0.0;
-            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
-                const float4 v = v4(k);
+            auto add_sq = [&](const float4 &v) {
                 ss += double(v.x) * v.x;  // each square exact in fp64
                 ss += double(v.y) * v.y;
                 ss += double(v.z) * v.z;
                 ss += double(v.w) * v.w;
+            };
+#pragma unroll
+            for (int i = 0; i < kNV; ++i) {
+                const int k = 4 * threadIdx.x + i * stride;
+                if (k < K) {
+                    vr[i] = v4(k);
+                    gr[i] = g4(k);
+                    add_sq(vr[i]);
+                }
             }
+            for (int k = 4 * threadIdx.x + kNV * stride; k < K; k += stride)
+                add_sq(v4(k));
             ss = consumer_reduce<WC>(ss, DAdd(), reinterpret_cast<double *>(red));
             const float r = __double2float_rn(1.0 / sqrt(ss / double(K) + double(e.eps)));
-            auto h_of = [&](float v, int k) {
-                return __fmul_rn(__fmul_rn(v, r), __ldg(e.gain + k));
+            auto h4 = [&](const float4 &v, const float4 &g) {
+                return make_float4(__fmul_rn(__fmul_rn(v.x, r), g.x), __fmul_rn(__fmul_rn(v.y, r), g.y),
+                                   __fmul_rn(__fmul_rn(v.z, r), g.z), __fmul_rn(__fmul_rn(v.w, r), g.w));
+            };
+            auto amax4 = [](float m, const float4 &h) {
+                return fmaxf(fmaxf(fmaxf(m, fabsf(h.x)), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w)));
             };
             float amax = 0.0f;
-            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
-                const float4 v = v4(k);
-                amax = fmaxf(amax, fabsf(h_of(v.x, k)));
-                amax = fmaxf(amax, fabsf(h_of(v.y, k + 1)));
-                amax = fmaxf(amax, fabsf(h_of(v.z, k + 2)));
-                amax = fmaxf(amax, fabsf(h_of(v.w, k + 3)));
-            }
+#pragma unroll
+            for (int i = 0; i < kNV; ++i)
+                if (4 * threadIdx.x + i * stride < K)
+                    amax = amax4(amax, h4(vr[i], gr[i]));
+            for (int k = 4 * threadIdx.x + kNV * stride; k < K; k += stride)
+                amax = amax4(amax, h4(v4(k), g4(k)));
             amax = consumer_reduce<WC>(amax, FMax(), reinterpret_cast<float *>(red));
             const float s = quant_inv_scale(amax);
             const bool owner = e.tile_begin >= t_begin;
             uint32_t *qc = reinterpret_cast<uint32_t *>(xcache + xoff[j]);
             uint32_t *qg = reinterpret_cast<uint32_t *>(e.xq);
             int sum = 0;
-            for (int k = 4 * threadIdx.x; k < K; k += 4 * WC * 32) {
-                const float4 v = v4(k);
-                const int a = code_of(h_of(v.x, k), s), b = code_of(h_of(v.y, k + 1), s);
-                const int c = code_of(h_of(v.z, k + 2), s), d = code_of(h_of(v.w, k + 3), s);
+            auto put = [&](int k, const float4 &h) {
+                const int a = code_of(h.x, s), b = code_of(h.y, s);
+                const int c = code_of(h.z, s), d = code_of(h.w, s);
                 sum += a + b + c + d;
                 const uint32_t word = (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) |
                                       ((uint32_t(c) & 0xFFu) << 16) | ((uint32_t(d) & 0xFFu) << 24);
                 qc[k >> 2] = word;
                 if (owner)
                     qg[k >> 2] = word;
+            };
+#pragma unroll
+            for (int i = 0; i < kNV; ++i) {
+                const int k = 4 * threadIdx.x + i * stride;
+                if (k < K)
+                    put(k, h4(vr[i], gr[i]));
             }
+            for (int k = 4 * threadIdx.x + kNV * stride; k < K; k += stride)
+                put(k, h4(v4(k), g4(k)));
             sum = consumer_reduce<WC>(sum, IAdd(), red);
             if (threadIdx.x == 0) {
                 const float xs = quant_scale(amax);

@@ -162,6 +162,19 @@ tq_status smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq, cons
     return err == cudaSuccess ? ok() : cuda_fail(err, fn);
 }
 
+// One thread waits, with the library's bounded wait, on an mbarrier that
+// nothing ever arrives on: the wait gives up after limit_ns, records
+// kErrWaitTimeout in the error word and the kernel returns normally.
+__global__ void wait_selftest_kernel(unsigned *err, unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0)
+        return;
+    tq::mbar_init(&bar, 1);
+    tq::fence_mbar_init();
+    tq::mbar_wait(&bar, 0u, err, limit_ns);
+}
+
 }  // namespace
 
 extern "C" {
@@ -496,6 +509,18 @@ tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scal
         return fail(TQ_ERR_ALIGN, "tq_absmean_pack: weights and packed bytes 16-byte aligned");
     cudaError_t e = tq::launch_absmean_pack(w_bf16, packed, w_scale, N, K, stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "tq_absmean_pack");
+}
+
+tq_status tq_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream)
+{
+    if (limit_us == 0 || limit_us > 2000000u)
+        return fail(TQ_ERR_VALUE, "tq_selftest_wait_timeout: limit_us=%u (1..2000000)", limit_us);
+    unsigned *err = tq::device_error_word();
+    if (!err)
+        return fail(TQ_ERR_CUDA, "tq_selftest_wait_timeout: no device error word");
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(err, 1000ull * limit_us);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "tq_selftest_wait_timeout");
 }
 
 tq_status tq_device_error(uint32_t *code, int reset)

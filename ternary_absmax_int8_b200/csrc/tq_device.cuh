@@ -73,8 +73,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 
 // Wait until the phase with the given parity has completed. Returns false
 // (after recording kErrWaitTimeout in *err) if it does not complete within
-// the limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err)
+// limit_ns nanoseconds of global time.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err,
+                                          unsigned long long limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -82,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) {
             atomicOr(err, kErrWaitTimeout);
             return false;
         }
