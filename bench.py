@@ -6,8 +6,11 @@ each (210 projections, 2.08e9 weights, 521 MB packed), M = 1. One step is one
 pass of the whole path over that stack: absmax-int8 quantisation of 210 fresh
 bf16 activation vectors and the 210 GEMVs with their scale epilogues, in one
 persistent launch (tq_gemv_stack with TQ_STACK_QUANTIZE). The weight stream is
-larger than L2, so no flush is needed between steps. Other workloads run one
-quantiser launch and one GEMV launch per projection.
+larger than L2, so no flush is needed between steps. Other workloads of several
+projections group them the same way: one quantising stack launch at M = 1, the
+stack quantiser plus tq_gemv_stack_batch at M = 2..32 (the streaming kernel up
+to 4 tokens, the tensor-core group plan from 5); single projections and
+prefill run one quantiser launch and one GEMV launch per projection.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME]
@@ -69,13 +72,29 @@ def step_bytes(projs) -> int:
     return sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
 
 
-def is_stack(workload: str, M: int) -> bool:
-    return workload.startswith("stack") and M == 1
+def step_mode(projs) -> str:
+    """How a step launches: "fused" -- one quantising stack launch for every
+    projection (M = 1); "batch" -- the stack quantiser, then
+    tq_gemv_stack_batch (M = 2..32); "per_projection" -- a quantiser launch
+    and a GEMV launch per projection (a single projection, or prefill)."""
+    M = projs[0].M
+    if len(projs) > 1 and M == 1:
+        return "fused"
+    if len(projs) > 1 and M <= 32:
+        return "batch"
+    return "per_projection"
+
+
+def batch_launches(n: int, M: int) -> int:
+    """Kernel launches of tq_quantize_act_stack_batch + tq_gemv_stack_batch
+    over n projections of M tokens: 512 token rows per quantiser launch; 256
+    projections per streaming launch (M <= 4), 16 per tensor-core group launch."""
+    return -(-n * M // 512) + (-(-n // 256) if M <= 4 else -(-n // 16))
 
 
 def workload_step_bytes(workload: str, projs) -> int:
     """Algorithmic bytes of one step of `workload` over `projs` (both arms)."""
-    return fused_step_bytes(projs) if is_stack(workload, projs[0].M) else step_bytes(projs)
+    return fused_step_bytes(projs) if step_mode(projs) == "fused" else step_bytes(projs)
 
 
 def fused_step_bytes(projs) -> int:
@@ -193,9 +212,10 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.set_device(dev)
     shapes, M = WORKLOADS[args.workload]
     projs = list(make_projections(shapes, M=M, seed=args.seed))
-    stack = is_stack(args.workload, M)
-    # The stack quantises inside its GEMV launch; the other workloads run the
-    # standalone quantiser first.
+    mode = step_mode(projs)
+    stack = mode == "fused"
+    # The fused stack quantises inside its GEMV launch; the other modes run a
+    # quantiser launch first.
     sb = workload_step_bytes(args.workload, projs)
     gemv_bytes = sb if stack else sum(algorithmic_bytes(p.N, p.K, p.M) for p in projs)
     packed_bytes = sum(p.N * p.K // 4 for p in projs)
@@ -241,6 +261,9 @@ def run_ours(args, rank: int, world: int):
     def quant(c, s):
         if stack:
             return  # quantised inside the stack launch
+        if mode == "batch":
+            tq.tq_quantize_act_stack_batch(tables[c], M, stream=s)
+            return
         for j, p in enumerate(projs):
             t = tables[c][j]
             tq.tq_quantize_act(t.x, t.xq, t.x_scale, t.x_sum, p.M, p.N, p.K, stream=s)
@@ -253,6 +276,10 @@ def run_ours(args, rank: int, world: int):
             flags = tq.TQ_STACK_QUANTIZE | (0 if first else tq.TQ_STACK_OVERLAP_PREV)
             tq.tq_gemv_stack(tables[c], flags=flags, stream=s)
             return
+        if mode == "batch":
+            # weights may stream while the quantiser drains
+            tq.tq_gemv_stack_batch(tables[c], M, flags=tq.TQ_STACK_OVERLAP_PREV, stream=s)
+            return
         for j, p in enumerate(projs):
             t = tables[c][j]
             call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
@@ -262,7 +289,8 @@ def run_ours(args, rank: int, world: int):
         quant(c, s)
         gemv(c, s, first)
 
-    launches_per_step = 1 if stack else sum(1 + gemv_launches(p.M) for p in projs)
+    launches_per_step = {"fused": 1, "batch": batch_launches(len(projs), M)}.get(
+        mode, sum(1 + gemv_launches(p.M) for p in projs))
 
     def barrier():
         if world > 1:
@@ -352,7 +380,8 @@ def run_ours(args, rank: int, world: int):
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    # Per-projection GEMM timing (non-stack workloads): a graph of R calls of
+    # Per-projection GEMM timing (workloads of separate calls, and the small
+    # batches for comparison with their grouped launch): a graph of R calls of
     # one projection over the rotated weight copies, time per call.
     per_proj = []
     if not stack:
@@ -401,7 +430,8 @@ def run_ours(args, rank: int, world: int):
                 "algorithmic_ops_per_step": flops}
     else:
         roof = {
-            "kernel": "stream_gemv_kernel",
+            "kernel": "stream_gemv_kernel" if M <= 4 else
+                      ("smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -443,7 +473,12 @@ def run_ours(args, rank: int, world: int):
         "us_per_projection": round(ms_step * 1e3 / len(projs), 4),
         "quant_us_per_step": round(quant_ms_step * 1e3, 3),
         "gemv_us_per_step": round(gemv_avg * 1e3, 3),
-        "quantiser": "fused into the stack launch" if stack else "separate launch",
+        "quantiser": {"fused": "fused into the stack launch",
+                      "batch": "one stack quantiser launch for all projections"}.get(
+                          mode, "separate launch per projection"),
+        "launch_form": {"fused": "one quantising tq_gemv_stack launch",
+                        "batch": "tq_quantize_act_stack_batch + tq_gemv_stack_batch"}
+        .get(mode, "tq_quantize_act + tq_gemv / tq_gemm_prefill per projection"),
         "roofline": roof,
         "e2e": {
             "value": round(whole_job_rate(world, sb, e2e_ms / e2e_steps) / 1e9, 1),

@@ -118,10 +118,11 @@ tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq
                           int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
 
 /*
- * One projection of a decode layer stack (M = 1), for the grouped calls below.
- * All pointers are device pointers with the meanings they have in
- * tq_quantize_act / tq_gemv for M = 1. tq_quantize_act_stack reads x and
- * writes xq, x_scale, x_sum (packed, y, acc_out unused, may be NULL);
+ * One projection of a decode layer stack, for the grouped calls below. All
+ * pointers are device pointers with the meanings they have in
+ * tq_quantize_act / tq_gemv; the shapes below are for M = 1 and become
+ * [M, K], [M] and [M, N] in the _batch calls. tq_quantize_act_stack reads x
+ * and writes xq, x_scale, x_sum (packed, y, acc_out unused, may be NULL);
  * tq_gemv_stack reads packed, xq, x_scale, x_sum and writes y and, when not
  * NULL, acc_out (x unused, may be NULL).
  */
@@ -189,6 +190,33 @@ tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t s
  * the same call, and no buffer may be shared between two entries.
  */
 tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream);
+
+/*
+ * The same two calls for M tokens per projection (small-batch decode: each
+ * projection's weights streamed once for all M rows): x bf16 [M, K], xq int8
+ * [M, K], x_scale fp32 [M], x_sum int32 [M], y fp32 [M, N], acc_out int32
+ * [M, N] or NULL, row-major. tq_quantize_act_stack_batch quantises every row
+ * exactly as tq_quantize_act does (any M >= 0). tq_gemv_stack_batch takes
+ * 0 <= M <= 32 (TQ_ERR_UNSUPPORTED above); M == 0 is a no-op and M == 1 is
+ * tq_gemv_stack. The quantising flags need M == 1 (TQ_ERR_UNSUPPORTED
+ * otherwise); TQ_STACK_OVERLAP_PREV is accepted at every M.
+ *   M <= 4: the streaming kernel, one launch per 256 projections.
+ *   5 <= M <= 32: the tensor-core batched-decode kernel, one launch per 16
+ *   projections, its K work split evenly over the SMs across projection
+ *   boundaries (TQ_STACK_OVERLAP_PREV has no effect there). Tiles split between
+ *   CTAs finish through a fixed 8 MiB device array compiled into the library,
+ *   which every launch leaves zeroed; the first call on a device (make it
+ *   before any stream capture) and the first call after tq_device_error
+ *   reported a nonzero code zero-fill it on `stream` first. Calls whose work
+ *   overlaps on the GPU (two streams) race on that array and must be
+ *   serialised by the caller. A projection too large for the array
+ *   (N > 130,944 at M <= 16, N > 65,408 at M > 16) runs alone as tq_gemv
+ *   would run it.
+ */
+tq_status tq_quantize_act_stack_batch(const tq_proj *projs, int n_proj, int M,
+                                      cudaStream_t stream);
+tq_status tq_gemv_stack_batch(const tq_proj *projs, int n_proj, int M, unsigned flags,
+                              cudaStream_t stream);
 
 /*
  * tq_gemv_noalloc -- tq_gemv for 5 <= M <= 32 tokens computed by the

@@ -31,6 +31,11 @@
 //     its partial sums into a global scratch with integer atomics, and the
 //     CTA whose contribution completes the tile applies the epilogue and
 //     zeroes the scratch for the next call.
+//   - group plan (tq_gemv_stack_batch): the stream-K plan over the
+//     concatenated (projection, tile, unit) sequence of up to 16 projections
+//     of different shapes, one tensor map pair per projection, so that one
+//     launch balances, say, the 10-unit tiles of a 2560-wide projection
+//     against the 27-unit tiles of a 6912-wide one.
 // * Warp roles (16 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
 //   4..11 expansion (two sets of four warps, one TMEM lane quarter each,
 //   taking alternate units), 12..15 epilogue. All mbarrier waits are bounded.
@@ -53,6 +58,10 @@ constexpr int kUnitK = 256;            // bytes of K per unit (two 128-byte boxe
 template <int BN>
 constexpr int kStagesOf = BN == 16 ? 10 : 6;
 constexpr int kSA = 4;                 // tensor-memory A slots
+// Units whose copies thread 0 issues before the CTA barrier (their latency
+// overlaps the tensor-memory allocation); the producer warp issues the rest.
+// Few: every copy issued here delays the barrier the whole CTA waits on.
+constexpr int kEarlyUnits = 2;
 constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
 constexpr int kThreads = 512;
 constexpr int kExpandWarp0 = 4;        // expansion warps 4..11: two sets of four
@@ -63,6 +72,7 @@ constexpr int kMaxGrid = 512;
 constexpr int kPlanStreamK = 0;
 constexpr int kPlanCluster = 1;
 constexpr int kMaxCluster = 8;
+constexpr int kMaxGroup = 16;          // projections per group launch
 
 struct SmallMParams {
     int N4, K, M;
@@ -79,9 +89,30 @@ struct SmallMParams {
     unsigned *err;
 };
 
-// A run of consecutive K units [k0, k1) of one tile.
+// One projection of a group launch: its shape, where its tiles and units
+// start in the launch's sequence, and its epilogue operands.
+struct GroupProj {
+    int N4, U, tiles;    // packed rows, K units per tile, tiles
+    int tile0, unit0;    // first tile / unit of this projection in the launch
+    float w_scale;
+    const float *x_scale;
+    const int32_t *x_sum;
+    float *y;
+    int32_t *acc_out;
+};
+
+// The group launch's table (a kernel parameter; tensor maps 64-byte aligned).
+struct GroupTable {
+    CUtensorMap map_p[kMaxGroup];
+    CUtensorMap map_x[kMaxGroup];
+    GroupProj g[kMaxGroup];
+    int n;
+};
+
+// A run of consecutive K units [k0, k1) of one tile (of projection `proj`
+// in a group launch, else 0).
 struct Seg {
-    int tile, k0, k1;
+    int tile, k0, k1, proj;
 };
 
 // The segments one CTA works through, in order.
@@ -95,11 +126,39 @@ struct CtaWork {
         const int U = p.units_per_tile;
         if (p.plan == kPlanStreamK) {
             const int t = u_begin / U + s;
-            return Seg{t, s == 0 ? u_begin - t * U : 0, min(U, u_end - t * U)};
+            return Seg{t, s == 0 ? u_begin - t * U : 0, min(U, u_end - t * U), 0};
         }
         if (p.csize == 1)
-            return Seg{int(blockIdx.x) + s * int(gridDim.x), 0, U};
-        return Seg{int(blockIdx.x) / p.csize, U * rank / p.csize, U * (rank + 1) / p.csize};
+            return Seg{int(blockIdx.x) + s * int(gridDim.x), 0, U, 0};
+        return Seg{int(blockIdx.x) / p.csize, U * rank / p.csize, U * (rank + 1) / p.csize, 0};
+    }
+
+    // Group plan: the CTA's first segment, and the one after `g` (the next
+    // tile of the sequence, crossing into the next projection; every
+    // projection of the table has at least one tile).
+    __device__ Seg group_first(const GroupTable &t) const
+    {
+        int j = 0;
+        while (j + 1 < t.n && t.g[j + 1].unit0 <= u_begin)
+            ++j;
+        const GroupProj &q = t.g[j];
+        const int tile = (u_begin - q.unit0) / q.U;
+        const int u0 = q.unit0 + tile * q.U;
+        return Seg{tile, u_begin - u0, min(q.U, u_end - u0), j};
+    }
+
+    __device__ Seg group_next(const GroupTable &t, const Seg &g) const
+    {
+        int j = g.proj, tile = g.tile + 1;
+        if (tile == t.g[j].tiles) {
+            ++j;
+            tile = 0;
+        }
+        if (j >= t.n)
+            return Seg{0, 0, 0, j};
+        const GroupProj &q = t.g[j];
+        const int u0 = q.unit0 + tile * q.U;
+        return Seg{tile, 0, min(q.U, u_end - u0), j};
     }
 };
 
@@ -182,6 +241,19 @@ __device__ __forceinline__ int cta_of_unit(int u, int total, int grid)
     return b;
 }
 
+// Tile counter of the stream-K plans: release (the epilogue threads' partial
+// sums, ordered before this by the named barrier) and acquire (the other
+// CTAs' sums, for the CTA that completes the tile), at GPU scope.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+                 : "=r"(old)
+                 : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // Barrier over the 128 epilogue threads (named barrier 2) that ORs a predicate.
 __device__ __forceinline__ bool epilogue_any(bool pred)
 {
@@ -197,10 +269,11 @@ __device__ __forceinline__ bool epilogue_any(bool pred)
     return r != 0;
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
-smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
-                 const __grid_constant__ SmallMParams p)
+// The kernel body. maps_p / maps_x point at the launch's tensor maps in
+// parameter space (one pair, or one per projection of a group launch, gt).
+template <int BN, bool Group>
+__device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUtensorMap *maps_x,
+                                            const SmallMParams &p, const GroupTable *gt)
 {
     using L = SmallMSmem<BN>;
     constexpr int kSP = L::kSP;
@@ -233,7 +306,19 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
     if (p.plan == kPlanStreamK) {
         cw.u_begin = unit_start(blockIdx.x, p.total_units, p.grid);
         cw.u_end = unit_start(blockIdx.x + 1, p.total_units, p.grid);
-        cw.nseg = cw.u_end > cw.u_begin ? (cw.u_end - 1) / U - cw.u_begin / U + 1 : 0;
+        if constexpr (Group) {
+            cw.nseg = 0;
+            if (cw.u_end > cw.u_begin) {
+                for (Seg g = cw.group_first(*gt); g.proj < gt->n; g = cw.group_next(*gt, g)) {
+                    ++cw.nseg;
+                    const GroupProj &q = gt->g[g.proj];
+                    if (q.unit0 + g.tile * q.U + g.k1 >= cw.u_end)
+                        break;
+                }
+            }
+        } else {
+            cw.nseg = cw.u_end > cw.u_begin ? (cw.u_end - 1) / U - cw.u_begin / U + 1 : 0;
+        }
     } else {
         cw.u_begin = cw.u_end = 0;
         cw.nseg = split_cluster ? 1
@@ -242,6 +327,21 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                                        : 0);
     }
 
+    // The CTA's segments in order: segment 0, and the one after segment
+    // sg - 1 (= g).
+    auto first_seg = [&]() -> Seg {
+        if constexpr (Group)
+            return cw.group_first(*gt);
+        else
+            return cw.seg(p, 0);
+    };
+    auto next_seg = [&](const Seg &g, int sg) -> Seg {
+        if constexpr (Group)
+            return cw.group_next(*gt, g);
+        else
+            return cw.seg(p, sg);
+    };
+
     // The producer's copies, unit by unit in the CTA's order.
     auto issue = [&](int issued, const Seg &g, int k) {
         const int s = issued % kSP;
@@ -249,15 +349,19 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
         uint8_t *P = sP + s * L::kPBytes;
         uint8_t *B = sB + s * L::kBBytes;
-        tma_load_2d(P, &map_p, k0, g.tile * kPRows, &tma_full[s]);
-        tma_load_2d(P + L::kPBytes / 2, &map_p, k0 + 128, g.tile * kPRows, &tma_full[s]);
-        tma_load_2d(B, &map_x, k0, 0, &tma_full[s]);
-        tma_load_2d(B + L::kBBytes / 2, &map_x, k0 + 128, 0, &tma_full[s]);
+        const CUtensorMap *mp = maps_p + g.proj, *mx = maps_x + g.proj;
+        tma_load_2d(P, mp, k0, g.tile * kPRows, &tma_full[s]);
+        tma_load_2d(P + L::kPBytes / 2, mp, k0 + 128, g.tile * kPRows, &tma_full[s]);
+        tma_load_2d(B, mx, k0, 0, &tma_full[s]);
+        tma_load_2d(B + L::kBBytes / 2, mx, k0 + 128, 0, &tma_full[s]);
     };
     int early = 0;  // copies thread 0 issued before the CTA barrier
     if (threadIdx.x == 0) {
-        prefetch_tensormap(&map_p);
-        prefetch_tensormap(&map_x);
+        {
+            const int j0 = cw.nseg > 0 ? first_seg().proj : 0;
+            prefetch_tensormap(maps_p + j0);
+            prefetch_tensormap(maps_x + j0);
+        }
         for (int s = 0; s < kSP; ++s) {
             mbar_init(&tma_full[s], 1);
             mbar_init(&p_free[s], 4);
@@ -274,9 +378,9 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         fence_mbar_init();
         // Start the first stages' copies now: their latency overlaps the
         // tensor-memory allocation and the barriers below.
-        for (int sg = 0; sg < cw.nseg && early < kSP; ++sg) {
-            const Seg g = cw.seg(p, sg);
-            for (int k = g.k0; k < g.k1 && early < kSP; ++k)
+        Seg g = first_seg();
+        for (int sg = 0; sg < cw.nseg && early < kEarlyUnits; ++sg, g = next_seg(g, sg)) {
+            for (int k = g.k0; k < g.k1 && early < kEarlyUnits; ++k)
                 issue(early++, g, k);
         }
     }
@@ -298,8 +402,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
-            for (int sg = 0; sg < cw.nseg && ok; ++sg) {
-                const Seg g = cw.seg(p, sg);
+            Seg g = first_seg();
+            for (int sg = 0; sg < cw.nseg && ok; ++sg, g = next_seg(g, sg)) {
                 for (int k = g.k0; k < g.k1; ++k, ++issued) {
                     if (issued < early)
                         continue;  // issued before the CTA barrier
@@ -323,8 +427,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         if (lane == 0) {
             int i = 0;
             bool ok = true;
-            for (int sg = 0; sg < cw.nseg && ok; ++sg) {
-                const Seg g = cw.seg(p, sg);
+            Seg g = first_seg();
+            for (int sg = 0; sg < cw.nseg && ok; ++sg, g = next_seg(g, sg)) {
                 const int buf = sg & 1;
                 if (sg >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((sg >> 1) - 1) & 1), p.err))
                     break;
@@ -365,8 +469,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         int i = 0;
         bool ok = true;
-        for (int sg = 0; sg < cw.nseg && ok; ++sg) {
-            const Seg g = cw.seg(p, sg);
+        Seg g = first_seg();
+        for (int sg = 0; sg < cw.nseg && ok; ++sg, g = next_seg(g, sg)) {
             for (int k = g.k0; k < g.k1; ++k, ++i) {
                 if (i % kExpandSets != set)
                     continue;
@@ -409,11 +513,19 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
         const int r = 32 * q + lane;                 // accumulator row = TMEM lane
         const int jr = r >> 2, pl = r & 3;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        const int N = 4 * p.N4;
-        for (int sg = 0; sg < cw.nseg; ++sg) {
-            const Seg g = cw.seg(p, sg);
+        // the single projection of a plain launch, in the group's form
+        const GroupProj self{p.N4, U, p.tiles, 0, 0, p.w_scale, p.x_scale, p.x_sum, p.y,
+                             p.acc_out};
+        Seg g = first_seg();
+        for (int sg = 0; sg < cw.nseg; ++sg, g = next_seg(g, sg)) {
+            const GroupProj *pj;
+            if constexpr (Group)
+                pj = &gt->g[g.proj];
+            else
+                pj = &self;
+            const int N = 4 * pj->N4;
             const int tile = g.tile;
-            const bool whole = g.k0 == 0 && g.k1 == U;
+            const bool whole = g.k0 == 0 && g.k1 == pj->U;
             const int buf = sg & 1;
             const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((sg >> 1) & 1), p.err);
             // The four epilogue warps meet at named barriers below: decide
@@ -437,8 +549,8 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
                 mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers now
 
             const int prow = tile * kPRows + jr;
-            const bool row_ok = prow < p.N4;
-            const int n = prow + pl * p.N4;
+            const bool row_ok = prow < pj->N4;
+            const int n = prow + pl * pj->N4;
             if (split_cluster) {
                 if (cw.rank != 0) {
                     // Store this CTA's partial sums into its slot in the
@@ -474,50 +586,64 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
                     if (c < p.M && row_ok) {
-                        const int32_t acc = int32_t(v[c]) - __ldg(p.x_sum + c);
-                        const float t = __fmul_rn(p.w_scale, __ldg(p.x_scale + c));
+                        const int32_t acc = int32_t(v[c]) - __ldg(pj->x_sum + c);
+                        const float t = __fmul_rn(pj->w_scale, __ldg(pj->x_scale + c));
                         const size_t o = size_t(c) * N + n;
-                        p.y[o] = __fmul_rn(__int2float_rn(acc), t);
-                        if (p.acc_out)
-                            p.acc_out[o] = acc;
+                        pj->y[o] = __fmul_rn(__int2float_rn(acc), t);
+                        if (pj->acc_out)
+                            pj->acc_out[o] = acc;
                     }
                 }
                 continue;
             }
             // Stream-K partial tile: add into the workspace, then count this
-            // CTA in.
-            int32_t *wt = p.ws + size_t(tile) * BN * kRows;
+            // CTA in. (Tiles and units of a group launch are numbered across
+            // its projections.)
+            const int wtile = pj->tile0 + tile;
+            const int wunit = pj->unit0 + tile * pj->U;
+            int32_t *wt = p.ws + size_t(wtile) * BN * kRows;
 #pragma unroll
             for (int c = 0; c < BN; ++c)
                 if (c < p.M)
                     atomicAdd(wt + c * kRows + r, int32_t(v[c]));
-            __threadfence();
+            // One thread counts the CTA in once every epilogue thread has
+            // issued its adds (the barrier orders them before its release).
             named_bar_sync(2, 128);
             if (threadIdx.x == kEpiWarp0 * 32) {
-                const int first = cta_of_unit(tile * U, p.total_units, p.grid);
-                const int last = cta_of_unit((tile + 1) * U - 1, p.total_units, p.grid);
-                const int old = atomicAdd(p.cnt + tile, 1);
+                const int first = cta_of_unit(wunit, p.total_units, p.grid);
+                const int last = cta_of_unit(wunit + pj->U - 1, p.total_units, p.grid);
+                const int old = atom_add_acq_rel_gpu(p.cnt + wtile, 1);
                 *fin_flag = (old == last - first) ? 1 : 0;
             }
             named_bar_sync(2, 128);
             if (*fin_flag) {
-                __threadfence();
+                // Every CTA of the tile has added its sums (acquired above):
+                // read them all at once from L2, then leave the slots zeroed.
 #pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    if (c < p.M) {
-                        const int32_t d = atomicExch(wt + c * kRows + r, 0);
-                        if (row_ok) {
-                            const int32_t acc = d - __ldg(p.x_sum + c);
-                            const float t = __fmul_rn(p.w_scale, __ldg(p.x_scale + c));
-                            const size_t o = size_t(c) * N + n;
-                            p.y[o] = __fmul_rn(__int2float_rn(acc), t);
-                            if (p.acc_out)
-                                p.acc_out[o] = acc;
+                for (int h = 0; h < BN / 16; ++h) {
+                    int32_t d[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        d[c] = h * 16 + c < p.M ? __ldcg(wt + (h * 16 + c) * kRows + r) : 0;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (h * 16 + c < p.M)
+                            __stcg(wt + (h * 16 + c) * kRows + r, 0);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int m = h * 16 + c;
+                        if (m < p.M && row_ok) {
+                            const int32_t acc = d[c] - __ldg(pj->x_sum + m);
+                            const float t = __fmul_rn(pj->w_scale, __ldg(pj->x_scale + m));
+                            const size_t o = size_t(m) * N + n;
+                            pj->y[o] = __fmul_rn(__int2float_rn(acc), t);
+                            if (pj->acc_out)
+                                pj->acc_out[o] = acc;
                         }
                     }
                 }
                 if (threadIdx.x == kEpiWarp0 * 32)
-                    p.cnt[tile] = 0;
+                    p.cnt[wtile] = 0;
             }
             named_bar_sync(2, 128);  // fin_flag is reused by the next segment
         }
@@ -535,6 +661,21 @@ smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constan
 }
 
 template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+smallm_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
+                 const __grid_constant__ SmallMParams p)
+{
+    smallm_body<BN, false>(&map_p, &map_x, p, nullptr);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+smallm_group_kernel(const __grid_constant__ GroupTable gt, const __grid_constant__ SmallMParams p)
+{
+    smallm_body<BN, true>(gt.map_p, gt.map_x, p, &gt);
+}
+
+template <int BN>
 cudaError_t configure_bn()
 {
     static int configured_dev = -1;
@@ -545,6 +686,10 @@ cudaError_t configure_bn()
     if (configured_dev != dev) {
         e = cudaFuncSetAttribute(smallm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(SmallMSmem<BN>::bytes + 1024));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(smallm_group_kernel<BN>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(SmallMSmem<BN>::bytes + 1024));
         if (e != cudaSuccess)
             return e;
         configured_dev = dev;
@@ -679,6 +824,49 @@ cudaError_t launch_smallm_streamk(const uint8_t *packed, float w_scale, const in
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
+// Fixed scratch of the group plan. Unlike tq_gemv_noalloc's it is not
+// zero-filled before every call: every launch leaves the parts it used zero
+// (the CTA that completes a split tile zeroes its partial sums and counter),
+// so only the first call on a device, and the first one after a device error
+// was reported (a kernel that gave up a wait may have left sums behind), fill
+// it.
+constexpr size_t kGroupScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) int32_t g_group_scratch[kGroupScratchBytes / sizeof(int32_t)];
+
+struct GroupScratch {
+    std::mutex mu;
+    void *ptr[64] = {};
+    bool clean[64] = {};
+};
+
+GroupScratch &group_scratch()
+{
+    static GroupScratch gs;
+    return gs;
+}
+
+// Host staging of a group launch's table, one per calling thread.
+GroupTable *group_table()
+{
+    static thread_local GroupTable t;
+    return &t;
+}
+
+template <int BN>
+cudaError_t launch_group_bn(const GroupTable &gt, const SmallMParams &prm, cudaStream_t stream)
+{
+    cudaError_t e = configure_bn<BN>();
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SmallMSmem<BN>::bytes + 1024;
+    cfg.stream = stream;
+    e = cudaLaunchKernelEx(&cfg, smallm_group_kernel<BN>, gt, prm);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 }  // namespace
 
 size_t smallm_workspace_bytes(int N, int M)
@@ -708,6 +896,99 @@ cudaError_t launch_smallm_tc(const uint8_t *packed, float w_scale, const int8_t 
 }
 
 size_t noalloc_scratch_capacity() { return kNoAllocScratchBytes; }
+
+void group_scratch_mark_dirty()
+{
+    GroupScratch &gs = group_scratch();
+    std::lock_guard<std::mutex> lock(gs.mu);
+    for (bool &c : gs.clean)
+        c = false;
+}
+
+cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t stream)
+{
+    if (M < 5 || M > 32 || n < 0)
+        return cudaErrorInvalidValue;
+    if (n == 0)
+        return cudaSuccess;
+    const int BN = M <= 16 ? 16 : 32;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    int32_t *scratch = nullptr;
+    {
+        GroupScratch &gs = group_scratch();
+        std::lock_guard<std::mutex> lock(gs.mu);
+        if (!gs.ptr[dev]) {
+            err = cudaGetSymbolAddress(&gs.ptr[dev], g_group_scratch);
+            if (err != cudaSuccess)
+                return err;
+        }
+        if (!gs.clean[dev]) {
+            err = cudaMemsetAsync(gs.ptr[dev], 0, kGroupScratchBytes, stream);
+            if (err != cudaSuccess)
+                return err;
+            gs.clean[dev] = true;
+        }
+        scratch = static_cast<int32_t *>(gs.ptr[dev]);
+    }
+    // tiles whose partial sums (and counter) the scratch holds at once
+    const int cap_tiles = int(kGroupScratchBytes / (size_t(BN) * kRows * 4 + 4));
+    const int sms = device_sm_count();
+    int i = 0;
+    while (i < n) {
+        const int tiles_i = (e[i].N / 4 + kPRows - 1) / kPRows;
+        if (tiles_i > cap_tiles) {
+            // too large for the scratch: this projection alone, cluster plan
+            err = launch_smallm_tc(e[i].packed, e[i].w_scale, e[i].xq, e[i].x_scale, e[i].x_sum,
+                                   e[i].y, e[i].acc_out, M, e[i].N, e[i].K, stream);
+            if (err != cudaSuccess)
+                return err;
+            ++i;
+            continue;
+        }
+        GroupTable &gt = *group_table();
+        int j = 0, tiles = 0, units = 0;
+        while (i < n && j < kMaxGroup) {
+            const GroupEntry &x = e[i];
+            const int t = (x.N / 4 + kPRows - 1) / kPRows;
+            if (tiles + t > cap_tiles)
+                break;
+            const int U = (x.K + kUnitK - 1) / kUnitK;
+            if (!make_map(&gt.map_p[j], x.packed, x.K, x.N / 4, kPRows) ||
+                !make_map(&gt.map_x[j], x.xq, x.K, M, BN))
+                return cudaErrorInvalidValue;
+            gt.g[j] = GroupProj{x.N / 4, U, t, tiles, units, x.w_scale, x.x_scale, x.x_sum,
+                                x.y, x.acc_out};
+            tiles += t;
+            units += t * U;
+            ++j;
+            ++i;
+        }
+        gt.n = j;
+        SmallMParams prm = {};
+        prm.M = M;
+        prm.K = 0;
+        prm.plan = kPlanStreamK;
+        prm.csize = 1;
+        prm.tiles = tiles;
+        prm.units_per_tile = 1;  // unused by the group plan
+        prm.total_units = units;
+        prm.grid = std::min({units, sms, kMaxGrid});
+        prm.ws = scratch;
+        prm.cnt = scratch + size_t(tiles) * BN * kRows;
+        prm.err = device_error_word();
+        if (!prm.err)
+            return cudaErrorUnknown;
+        err = BN == 16 ? launch_group_bn<16>(gt, prm, stream) : launch_group_bn<32>(gt, prm, stream);
+        if (err != cudaSuccess)
+            return err;
+    }
+    return cudaSuccess;
+}
 
 // The stream-K plan with the fixed scratch above. The device address of the
 // scratch array is looked up once per device (on that device's first call)

@@ -84,6 +84,7 @@ tq_status cuda_fail(cudaError_t e, const char *where)
 bool aligned(const void *p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
 
 constexpr int kGemvMaxM = 24;
+constexpr int kStackMaxM = 32;  // tq_gemv_stack_batch
 
 // Shared checks of the GEMV-shaped calls.
 tq_status check_gemv_args(const char *fn, const uint8_t *packed, const int8_t *xq,
@@ -173,6 +174,171 @@ __global__ void wait_selftest_kernel(unsigned *err, unsigned long long limit_ns)
     tq::mbar_init(&bar, 1);
     tq::fence_mbar_init();
     tq::mbar_wait(&bar, 0u, err, limit_ns);
+}
+
+// The quantiser over M token rows of each projection: one entry of the stack
+// quantiser per row, all in one launch per kMaxQuantStack rows.
+tq_status quantize_stack_impl(const char *fname, const tq_proj *projs, int n_proj, int M,
+                              cudaStream_t stream)
+{
+    if (n_proj < 0 || M < 0)
+        return fail(TQ_ERR_SHAPE, "%s: n_proj=%d M=%d", fname, n_proj, M);
+    if (n_proj == 0 || M == 0)
+        return ok();
+    if (!projs)
+        return fail(TQ_ERR_NULL, "%s: projs is NULL", fname);
+    std::vector<tq::QuantStackEntry> list;
+    list.reserve(size_t(n_proj) * size_t(M));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        if (p.K < 0 || p.K % 16 != 0)
+            return fail(TQ_ERR_SHAPE, "%s: entry %d: K=%d", fname, j, p.K);
+        if (!p.x_scale || (p.K > 0 && (!p.x || !p.xq)))
+            return fail(TQ_ERR_NULL, "%s: entry %d: NULL pointer", fname, j);
+        if ((p.K > 0 && (!aligned(p.x, 16) || !aligned(p.xq, 16))) || !aligned(p.x_scale, 4) ||
+            (p.x_sum && !aligned(p.x_sum, 4)))
+            return fail(TQ_ERR_ALIGN, "%s: entry %d: misaligned pointer", fname, j);
+        if (p.K == 0) {
+            cudaError_t e = cudaMemsetAsync(p.x_scale, 0, size_t(M) * sizeof(float), stream);
+            if (e == cudaSuccess && p.x_sum)
+                e = cudaMemsetAsync(p.x_sum, 0, size_t(M) * sizeof(int32_t), stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, fname);
+            continue;
+        }
+        for (int m = 0; m < M; ++m) {
+            tq::QuantStackEntry q = {};
+            q.x = p.x + size_t(m) * size_t(p.K);
+            q.xq = p.xq + size_t(m) * size_t(p.K);
+            q.x_scale = p.x_scale + m;
+            q.x_sum = p.x_sum ? p.x_sum + m : nullptr;
+            q.K = p.K;
+            list.push_back(q);
+        }
+    }
+    tq::QuantStackParams &params = *quant_params();
+    for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
+        const size_t n = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
+        params.n = int(n);
+        std::memcpy(params.e, list.data() + base, n * sizeof(tq::QuantStackEntry));
+        cudaError_t e = tq::launch_quant_stack(params, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fname);
+    }
+    return ok();
+}
+
+tq_status gemv_stack_impl(const char *fname, const tq_proj *projs, int n_proj, int M,
+                          unsigned flags, cudaStream_t stream)
+{
+    if (n_proj < 0 || M < 0)
+        return fail(TQ_ERR_SHAPE, "%s: n_proj=%d M=%d", fname, n_proj, M);
+    const unsigned qflags = flags & (TQ_STACK_QUANTIZE | TQ_STACK_RMSNORM | TQ_STACK_RELU2_MUL);
+    if ((flags & ~(unsigned(TQ_STACK_OVERLAP_PREV) | qflags)) || (qflags & (qflags - 1)))
+        return fail(TQ_ERR_VALUE, "%s: bad flags 0x%x", fname, flags);
+    if (M > kStackMaxM)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: M=%d > %d", fname, M, kStackMaxM);
+    if (qflags && M > 1)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: quantising flags need M == 1 (M=%d)", fname, M);
+    if (n_proj == 0 || M == 0)
+        return ok();
+    if (!projs)
+        return fail(TQ_ERR_NULL, "%s: projs is NULL", fname);
+    // the launch's quantising mode: 1 absmax of bf16 x, 2 RMSNorm then absmax,
+    // 3 relu(x_f32)^2 * up, RMSNorm, absmax
+    const int mode = qflags == TQ_STACK_QUANTIZE ? 1
+                     : qflags == TQ_STACK_RMSNORM ? 2
+                     : qflags == TQ_STACK_RELU2_MUL ? 3 : 0;
+    std::vector<tq::StreamEntry> list;
+    list.reserve(size_t(n_proj));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        char fn[64];
+        snprintf(fn, sizeof fn, "%s[%d]", fname, j);
+        tq_status st =
+            check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, M, p.N, p.K);
+        if (st != TQ_OK)
+            return st;
+        const void *xin = mode == 3 ? static_cast<const void *>(p.x_f32)
+                                    : static_cast<const void *>(p.x);
+        if (mode && p.K > 0) {
+            if (!xin || (mode == 3 && !p.up) || (mode >= 2 && !p.gain))
+                return fail(TQ_ERR_NULL, "%s: x is NULL (or x_f32, up or gain for its mode)", fn);
+            if (!aligned(xin, 16) || (mode == 3 && !aligned(p.up, 16)) ||
+                (mode >= 2 && !aligned(p.gain, 4)))
+                return fail(TQ_ERR_ALIGN, "%s: x must be 16-byte aligned (x_f32, up too)", fn);
+            if (mode >= 2 && (!(p.eps >= 0.0f) || p.eps > FLT_MAX))
+                return fail(TQ_ERR_VALUE, "%s: eps must be finite and >= 0", fn);
+        }
+        if (p.N == 0 && !mode)
+            continue;
+        if (p.K == 0) {
+            // Every accumulator is 0; a quantising call also reports the
+            // empty token's scale and sum as 0.
+            cudaError_t e = cudaSuccess;
+            if (mode)
+                e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
+            if (e == cudaSuccess && mode)
+                e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, fn);
+            st = zero_outputs(p.y, p.acc_out, size_t(M) * size_t(p.N), stream);
+            if (st != TQ_OK)
+                return st;
+            continue;
+        }
+        if (p.N == 0) {
+            // Nothing to multiply, but the quantiser's outputs are owed.
+            cudaError_t e;
+            if (mode == 1) {
+                tq::QuantStackParams *qp = quant_params();
+                qp->n = 1;
+                qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
+                e = tq::launch_quant_stack(*qp, stream);
+            } else {
+                e = tq::launch_rms_quant(mode == 2 ? 0 : 2, p.x, p.x_f32, p.up, p.gain, p.eps,
+                                         p.xq, p.x_scale, p.x_sum, 1, p.K, stream);
+            }
+            if (e != cudaSuccess)
+                return cuda_fail(e, fn);
+            continue;
+        }
+        tq::StreamEntry e = {};
+        e.packed = p.packed;
+        e.xin = xin;
+        e.gain = p.gain;
+        e.up = p.up;
+        e.eps = p.eps;
+        e.xq = p.xq;
+        e.x_scale = p.x_scale;
+        e.x_sum = p.x_sum;
+        e.y = p.y;
+        e.acc_out = p.acc_out;
+        e.w_scale = p.w_scale;
+        e.N4 = p.N / 4;
+        e.K = p.K;
+        list.push_back(e);
+    }
+    if (M > tq::kStreamMaxTokens) {
+        // 5 <= M <= 32: the tensor-core batched-decode kernel's group plan
+        // (no programmatic overlap: TQ_STACK_OVERLAP_PREV has no effect).
+        std::vector<tq::GroupEntry> group;
+        group.reserve(list.size());
+        for (const tq::StreamEntry &e : list)
+            group.push_back(tq::GroupEntry{e.packed, e.w_scale, e.xq, e.x_scale, e.x_sum, e.y,
+                                           e.acc_out, 4 * e.N4, e.K});
+        cudaError_t e = tq::launch_smallm_group(group.data(), int(group.size()), M, stream);
+        return e == cudaSuccess ? ok() : cuda_fail(e, fname);
+    }
+    const bool overlap = (flags & TQ_STACK_OVERLAP_PREV) != 0;
+    for (size_t base = 0; base < list.size(); base += tq::kStreamStackMax) {
+        const int n = int(std::min(list.size() - base, size_t(tq::kStreamStackMax)));
+        cudaError_t e = tq::launch_stream_gemv(list.data() + base, n, M, overlap && base == 0,
+                                               false, mode, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fname);
+    }
+    return ok();
 }
 
 }  // namespace
@@ -285,146 +451,24 @@ tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq
 
 tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t stream)
 {
-    if (n_proj < 0)
-        return fail(TQ_ERR_SHAPE, "tq_quantize_act_stack: n_proj=%d", n_proj);
-    if (n_proj == 0)
-        return ok();
-    if (!projs)
-        return fail(TQ_ERR_NULL, "tq_quantize_act_stack: projs is NULL");
-    std::vector<tq::QuantStackEntry> list;
-    list.reserve(size_t(n_proj));
-    for (int j = 0; j < n_proj; ++j) {
-        const tq_proj &p = projs[j];
-        if (p.K < 0 || p.K % 16 != 0)
-            return fail(TQ_ERR_SHAPE, "tq_quantize_act_stack: entry %d: K=%d", j, p.K);
-        if (!p.x_scale || (p.K > 0 && (!p.x || !p.xq)))
-            return fail(TQ_ERR_NULL, "tq_quantize_act_stack: entry %d: NULL pointer", j);
-        if ((p.K > 0 && (!aligned(p.x, 16) || !aligned(p.xq, 16))) || !aligned(p.x_scale, 4) ||
-            (p.x_sum && !aligned(p.x_sum, 4)))
-            return fail(TQ_ERR_ALIGN, "tq_quantize_act_stack: entry %d: misaligned pointer", j);
-        if (p.K == 0) {
-            cudaError_t e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
-            if (e == cudaSuccess && p.x_sum)
-                e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
-            if (e != cudaSuccess)
-                return cuda_fail(e, "tq_quantize_act_stack");
-            continue;
-        }
-        tq::QuantStackEntry q = {};
-        q.x = p.x;
-        q.xq = p.xq;
-        q.x_scale = p.x_scale;
-        q.x_sum = p.x_sum;
-        q.K = p.K;
-        list.push_back(q);
-    }
-    tq::QuantStackParams &params = *quant_params();
-    for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
-        const size_t n = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
-        params.n = int(n);
-        std::memcpy(params.e, list.data() + base, n * sizeof(tq::QuantStackEntry));
-        cudaError_t e = tq::launch_quant_stack(params, stream);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "tq_quantize_act_stack");
-    }
-    return ok();
+    return quantize_stack_impl("tq_quantize_act_stack", projs, n_proj, 1, stream);
+}
+
+tq_status tq_quantize_act_stack_batch(const tq_proj *projs, int n_proj, int M,
+                                      cudaStream_t stream)
+{
+    return quantize_stack_impl("tq_quantize_act_stack_batch", projs, n_proj, M, stream);
 }
 
 tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaStream_t stream)
 {
-    if (n_proj < 0)
-        return fail(TQ_ERR_SHAPE, "tq_gemv_stack: n_proj=%d", n_proj);
-    const unsigned qflags = flags & (TQ_STACK_QUANTIZE | TQ_STACK_RMSNORM | TQ_STACK_RELU2_MUL);
-    if ((flags & ~(unsigned(TQ_STACK_OVERLAP_PREV) | qflags)) || (qflags & (qflags - 1)))
-        return fail(TQ_ERR_VALUE, "tq_gemv_stack: bad flags 0x%x", flags);
-    if (n_proj == 0)
-        return ok();
-    if (!projs)
-        return fail(TQ_ERR_NULL, "tq_gemv_stack: projs is NULL");
-    // the launch's quantising mode: 1 absmax of bf16 x, 2 RMSNorm then absmax,
-    // 3 relu(x_f32)^2 * up, RMSNorm, absmax
-    const int mode = qflags == TQ_STACK_QUANTIZE ? 1
-                     : qflags == TQ_STACK_RMSNORM ? 2
-                     : qflags == TQ_STACK_RELU2_MUL ? 3 : 0;
-    std::vector<tq::StreamEntry> list;
-    list.reserve(size_t(n_proj));
-    for (int j = 0; j < n_proj; ++j) {
-        const tq_proj &p = projs[j];
-        char fn[64];
-        snprintf(fn, sizeof fn, "tq_gemv_stack[%d]", j);
-        tq_status st =
-            check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, 1, p.N, p.K);
-        if (st != TQ_OK)
-            return st;
-        const void *xin = mode == 3 ? static_cast<const void *>(p.x_f32)
-                                    : static_cast<const void *>(p.x);
-        if (mode && p.K > 0) {
-            if (!xin || (mode == 3 && !p.up) || (mode >= 2 && !p.gain))
-                return fail(TQ_ERR_NULL, "%s: x is NULL (or x_f32, up or gain for its mode)", fn);
-            if (!aligned(xin, 16) || (mode == 3 && !aligned(p.up, 16)) ||
-                (mode >= 2 && !aligned(p.gain, 4)))
-                return fail(TQ_ERR_ALIGN, "%s: x must be 16-byte aligned (x_f32, up too)", fn);
-            if (mode >= 2 && (!(p.eps >= 0.0f) || p.eps > FLT_MAX))
-                return fail(TQ_ERR_VALUE, "%s: eps must be finite and >= 0", fn);
-        }
-        if (p.N == 0 && !mode)
-            continue;
-        if (p.K == 0) {
-            // Every accumulator is 0; a quantising call also reports the
-            // empty token's scale and sum as 0.
-            cudaError_t e = cudaSuccess;
-            if (mode)
-                e = cudaMemsetAsync(p.x_scale, 0, sizeof(float), stream);
-            if (e == cudaSuccess && mode)
-                e = cudaMemsetAsync(p.x_sum, 0, sizeof(int32_t), stream);
-            if (e != cudaSuccess)
-                return cuda_fail(e, fn);
-            st = zero_outputs(p.y, p.acc_out, size_t(p.N), stream);
-            if (st != TQ_OK)
-                return st;
-            continue;
-        }
-        if (p.N == 0) {
-            // Nothing to multiply, but the quantiser's outputs are owed.
-            cudaError_t e;
-            if (mode == 1) {
-                tq::QuantStackParams *qp = quant_params();
-                qp->n = 1;
-                qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
-                e = tq::launch_quant_stack(*qp, stream);
-            } else {
-                e = tq::launch_rms_quant(mode == 2 ? 0 : 2, p.x, p.x_f32, p.up, p.gain, p.eps,
-                                         p.xq, p.x_scale, p.x_sum, 1, p.K, stream);
-            }
-            if (e != cudaSuccess)
-                return cuda_fail(e, fn);
-            continue;
-        }
-        tq::StreamEntry e = {};
-        e.packed = p.packed;
-        e.xin = xin;
-        e.gain = p.gain;
-        e.up = p.up;
-        e.eps = p.eps;
-        e.xq = p.xq;
-        e.x_scale = p.x_scale;
-        e.x_sum = p.x_sum;
-        e.y = p.y;
-        e.acc_out = p.acc_out;
-        e.w_scale = p.w_scale;
-        e.N4 = p.N / 4;
-        e.K = p.K;
-        list.push_back(e);
-    }
-    const bool overlap = (flags & TQ_STACK_OVERLAP_PREV) != 0;
-    for (size_t base = 0; base < list.size(); base += tq::kStreamStackMax) {
-        const int n = int(std::min(list.size() - base, size_t(tq::kStreamStackMax)));
-        cudaError_t e = tq::launch_stream_gemv(list.data() + base, n, 1, overlap && base == 0,
-                                               false, mode, stream);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "tq_gemv_stack");
-    }
-    return ok();
+    return gemv_stack_impl("tq_gemv_stack", projs, n_proj, 1, flags, stream);
+}
+
+tq_status tq_gemv_stack_batch(const tq_proj *projs, int n_proj, int M, unsigned flags,
+                              cudaStream_t stream)
+{
+    return gemv_stack_impl("tq_gemv_stack_batch", projs, n_proj, M, flags, stream);
 }
 
 tq_status tq_gemv_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
@@ -537,6 +581,8 @@ tq_status tq_device_error(uint32_t *code, int reset)
     }
     if (e != cudaSuccess)
         return cuda_fail(e, "tq_device_error");
+    if (v != 0)
+        tq::group_scratch_mark_dirty();  // a kernel that gave up may have left partial sums
     *code = v;
     return ok();
 }

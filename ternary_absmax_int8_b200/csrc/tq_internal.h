@@ -121,6 +121,24 @@ size_t smallm_workspace_bytes(int N, int M);
 // (no allocation by anyone); cudaErrorInvalidValue when the shape needs more
 // than noalloc_scratch_capacity() bytes of it.
 size_t noalloc_scratch_capacity();
+
+// Group plan of the batched-decode kernel: several projections (N > 0,
+// K > 0) at 5 <= M <= 32 tokens, up to 16 per launch, one stream-K partition
+// over all of their tiles; split tiles finish through a fixed device scratch
+// that every launch leaves zeroed.
+struct GroupEntry {
+    const uint8_t *packed;
+    float w_scale;
+    const int8_t *xq;
+    const float *x_scale;
+    const int32_t *x_sum;
+    float *y;
+    int32_t *acc_out;
+    int N, K;
+};
+cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t stream);
+// After a device error was reported: the next group call refills the scratch.
+void group_scratch_mark_dirty();
 cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
                                      const float *x_scale, const int32_t *x_sum, float *y,
                                      int32_t *acc_out, int M, int N, int K, cudaStream_t stream);

@@ -157,6 +157,36 @@ def test_stack_argument_checks():
     tq.tq_quantize_act_stack([], stream=0)
 
 
+def test_stack_batch_argument_checks():
+    good = dict(packed=A, x=A, xq=A, x_scale=A, x_sum=A, y=A, w_scale=1.0, N=640, K=2560)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack_batch([tq.make_proj(**good)], 33, stream=0)     # at most 32 tokens
+    assert e.value.name == "TQ_ERR_UNSUPPORTED"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack_batch([tq.make_proj(**good)], 2, flags=tq.TQ_STACK_QUANTIZE, stream=0)
+    assert e.value.name == "TQ_ERR_UNSUPPORTED"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack_batch([tq.make_proj(**good)], -1, stream=0)
+    assert e.value.name == "TQ_ERR_SHAPE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_stack_batch([tq.make_proj(**good)], 2, flags=16, stream=0)
+    assert e.value.name == "TQ_ERR_VALUE"
+    with pytest.raises(tq.TQError) as e:                            # checks run for every entry
+        tq.tq_gemv_stack_batch([tq.make_proj(**good), tq.make_proj(**dict(good, xq=A + 4))], 3,
+                               stream=0)
+    assert e.value.name == "TQ_ERR_ALIGN" and "[1]" in str(e.value)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_quantize_act_stack_batch([tq.make_proj(**dict(good, x=None))], 2, stream=0)
+    assert e.value.name == "TQ_ERR_NULL"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_quantize_act_stack_batch([tq.make_proj(**good)], -2, stream=0)
+    assert e.value.name == "TQ_ERR_SHAPE"
+    # M == 0 and empty tables are no-ops
+    tq.tq_gemv_stack_batch([tq.make_proj(**good)], 0, stream=0)
+    tq.tq_quantize_act_stack_batch([tq.make_proj(**good)], 0, stream=0)
+    tq.tq_gemv_stack_batch([], 3, stream=0)
+
+
 def test_tq_proj_layout_matches_header():
     # 7 pointers, a float and two ints (68, padded to 72), then 3 pointers, a
     # float and an int: 72 + 24 + 8 = 104
