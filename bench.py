@@ -56,6 +56,10 @@ DESCRIPTIONS = {
                   "down ternary projections), M=1, 210 projections, 2.08e9 weights",
     "stack10_m1": "decode layer stack: 10 x BitNet-b1.58-2B-4T decoder layer, M=1 "
                   "(profiling case)",
+    "stack30_m4": "decode layer stack (30 layers, 210 projections) at M=4 tokens per "
+                  "projection: streaming kernel",
+    "stack30_m16": "decode layer stack (30 layers, 210 projections) at M=16 tokens per "
+                   "projection: tensor-core group plan, 16 projections per launch",
     "layer_m1": "one BitNet-b1.58-2B-4T decoder layer, 7 ternary projections, M=1",
     "single_640x2560_m1": "one ternary projection N=640 K=2560, M=1",
     "prefill_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120",
@@ -384,7 +388,7 @@ def run_ours(args, rank: int, world: int):
     # batches for comparison with their grouped launch): a graph of R calls of
     # one projection over the rotated weight copies, time per call.
     per_proj = []
-    if not stack:
+    if not stack and len(projs) <= 8:
         R = copies * max(1, 32 // copies)
         for j, p in enumerate(projs):
             call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
@@ -469,6 +473,8 @@ def run_ours(args, rank: int, world: int):
             "seed": args.seed,
         },
         "passes_per_s": round(whole_job_rate(world, 1.0, ms_step), 1),
+        # tokens through every projection of the workload per second
+        "token_passes_per_s": round(whole_job_rate(world, float(M), ms_step), 1),
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "us_per_projection": round(ms_step * 1e3 / len(projs), 4),
         "quant_us_per_step": round(quant_ms_step * 1e3, 3),

@@ -12,7 +12,10 @@
 // * Tile: 32 packed rows = 128 MMA rows with row r = 4 j + p holding plane p
 //   of packed row j (feature i0 + j + p N/4); BN = 16 or 32 token columns.
 //   With this order a warp's 32 tensor-memory lanes are 8 packed rows x 4
-//   planes, so each packed byte is read from shared memory once.
+//   planes, so each packed byte is read from shared memory once. A lane
+//   keeps its plane's bits in place (code c stored as c * 4^p, one AND per
+//   word): the MMA sums are 4^p times the code sums, exactly, and the
+//   epilogue shifts them back.
 // * The expansion warps unpack codes in registers and store them straight
 //   into tensor memory (tcgen05.st): the A operand never passes through shared
 //   memory, which at small N would otherwise bound the kernel (16 KB written
@@ -36,9 +39,16 @@
 //     of different shapes, one tensor map pair per projection, so that one
 //     launch balances, say, the 10-unit tiles of a 2560-wide projection
 //     against the 27-unit tiles of a 6912-wide one.
-// * Warp roles (16 warps): 0 TMA producer, 1 TMEM allocator + MMA issuer,
-//   4..11 expansion (two sets of four warps, one TMEM lane quarter each,
-//   taking alternate units), 12..15 epilogue. All mbarrier waits are bounded.
+// * Warp roles (16 warps): 0 TMA producer, 1..3 MMA issuers (1 also
+//   allocates tensor memory), 4..11 expansion (two sets of four warps, one
+//   TMEM lane quarter each, taking alternate units), 12..15 epilogue. All
+//   mbarrier waits are bounded.
+// * A thread blocks on each tcgen05.mma it issues for about 117 cycles
+//   whatever N is (measured on B200, 16 <= N <= 64), while the tensor core
+//   would finish a 128 x 16 x 32 product in a few: one issuing thread caps a
+//   CTA at 8 KB of weights per ~0.5 us. So three threads issue, taking units
+//   in turn, each into its own accumulator; the epilogue adds the partial
+//   accumulators of the issuers that had units in the segment.
 #include <algorithm>
 #include <mutex>
 #include <utility>
@@ -62,6 +72,7 @@ constexpr int kSA = 4;                 // tensor-memory A slots
 // overlaps the tensor-memory allocation); the producer warp issues the rest.
 // Few: every copy issued here delays the barrier the whole CTA waits on.
 constexpr int kEarlyUnits = 2;
+constexpr int kIssuers = 3;            // MMA-issuing warps 1..3, one accumulator each
 constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
 constexpr int kThreads = 512;
 constexpr int kExpandWarp0 = 4;        // expansion warps 4..11: two sets of four
@@ -278,8 +289,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
     using L = SmallMSmem<BN>;
     constexpr int kSP = L::kSP;
     constexpr uint32_t kIdesc = idesc_i8_u8s8(kRows, BN);
-    constexpr int kTmemCols = 512;  // kSA * kACols + 2 * BN, rounded to a power of two
-    static_assert(kSA * kACols + 2 * BN <= kTmemCols, "tensor memory plan");
+    constexpr int kTmemCols = 512;  // kSA * kACols + 2 * kIssuers * BN, rounded to a power of two
+    static_assert(kSA * kACols + 2 * kIssuers * BN <= kTmemCols, "tensor memory plan");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -370,7 +381,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         for (int s = 0; s < kSA; ++s)
             mbar_init(&a_full[s], 4);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_full[b], kIssuers);  // every issuer commits every segment
             mbar_init(&acc_empty[b], 4);
         }
         // every epilogue thread of every other CTA of the cluster arrives once
@@ -395,7 +406,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         cluster_sync_all();
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t tmem_a = tmem_base;                    // kSA slots of kACols
-    const uint32_t tmem_d = tmem_base + kSA * kACols;     // 2 x BN accumulator columns
+    // accumulators: [2 buffers][kIssuers][BN columns]
+    const uint32_t tmem_d = tmem_base + kSA * kACols;
 
     if (warp == 0) {
         // -------------------------------------------------- TMA producer
@@ -422,10 +434,12 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                 mbar_wait(&tma_full[s], uint32_t((last / kSP) & 1), p.err);
             }
         }
-    } else if (warp == 1) {
-        // -------------------------------------------------- MMA issuer
+    } else if (warp >= 1 && warp <= kIssuers) {
+        // -------------------------------------------------- MMA issuers
+        // issuer t = warp - 1 takes the CTA's units i with i % kIssuers == t
+        const int t = warp - 1;
         if (lane == 0) {
-            int i = 0;
+            int i = 0, last = -1;
             bool ok = true;
             Seg g = first_seg();
             for (int sg = 0; sg < cw.nseg && ok; ++sg, g = next_seg(g, sg)) {
@@ -433,8 +447,11 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                 if (sg >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((sg >> 1) - 1) & 1), p.err))
                     break;
                 tc_fence_after();
-                const uint32_t d = tmem_d + uint32_t(buf * BN);
+                const uint32_t d = tmem_d + uint32_t((buf * kIssuers + t) * BN);
+                bool fresh = true;  // this issuer's first unit of the segment
                 for (int k = g.k0; k < g.k1; ++k, ++i) {
+                    if (i % kIssuers != t)
+                        continue;
                     const int s = i % kSP, sa = i % kSA;
                     if (!mbar_wait(&tma_full[s], uint32_t((i / kSP) & 1), p.err) ||
                         !mbar_wait(&a_full[sa], uint32_t((i / kSA) & 1), p.err)) {
@@ -450,15 +467,17 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                         umma_i8_ts(d, ta + uint32_t(kk * 8),
                                    umma_desc_advance(db, uint32_t((kk >> 2) * (L::kBBytes / 2) +
                                                                   (kk & 3) * 32)),
-                                   kIdesc, (k == g.k0 && kk == 0) ? 0u : 1u);
+                                   kIdesc, (fresh && kk == 0) ? 0u : 1u);
                     umma_commit(&mma_done[s]);
+                    fresh = false;
+                    last = i;
                 }
                 if (ok)
                     umma_commit(&acc_full[buf]);
             }
-            if (i > 0) {
-                const int s = (i - 1) % kSP;
-                mbar_wait(&mma_done[s], uint32_t(((i - 1) / kSP) & 1), p.err);
+            if (last >= 0) {
+                const int s = last % kSP;
+                mbar_wait(&mma_done[s], uint32_t((last / kSP) & 1), p.err);
             }
         }
     } else if (warp >= kExpandWarp0 && warp < kEpiWarp0) {
@@ -484,6 +503,10 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                     break;
                 tc_fence_after();
                 const uint8_t *P = sP + s * L::kPBytes;
+                // The lane's plane bits stay in place: each byte holds c * 4^pl
+                // (at most 128, still a u8), one AND per word; the epilogue
+                // shifts the exact int32 sums back down.
+                const uint32_t mask = 0x03030303u << (2 * pl);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t v[32];
@@ -491,10 +514,10 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                     for (int c = 0; c < 8; ++c) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(P + h * (L::kPBytes / 2) +
                                                                          sw128_off(j, c));
-                        v[4 * c + 0] = (w.x >> (2 * pl)) & 0x03030303u;
-                        v[4 * c + 1] = (w.y >> (2 * pl)) & 0x03030303u;
-                        v[4 * c + 2] = (w.z >> (2 * pl)) & 0x03030303u;
-                        v[4 * c + 3] = (w.w >> (2 * pl)) & 0x03030303u;
+                        v[4 * c + 0] = w.x & mask;
+                        v[4 * c + 1] = w.y & mask;
+                        v[4 * c + 2] = w.z & mask;
+                        v[4 * c + 3] = w.w & mask;
                     }
                     tmem_st32_async(tmem_a + lane_base + uint32_t(sa * kACols + h * 32), v);
                 }
@@ -517,7 +540,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         const GroupProj self{p.N4, U, p.tiles, 0, 0, p.w_scale, p.x_scale, p.x_sum, p.y,
                              p.acc_out};
         Seg g = first_seg();
-        for (int sg = 0; sg < cw.nseg; ++sg, g = next_seg(g, sg)) {
+        int i0 = 0;  // the CTA's unit counter at the start of segment sg
+        for (int sg = 0; sg < cw.nseg; ++sg, i0 += g.k1 - g.k0, g = next_seg(g, sg)) {
             const GroupProj *pj;
             if constexpr (Group)
                 pj = &gt->g[g.proj];
@@ -533,15 +557,31 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             if (epilogue_any(!got))
                 break;
             tc_fence_after();
+            // The segment's units i0, i0 + 1, ... went to issuers i0 % kIssuers,
+            // then the next ones in turn: add the partial accumulators of the
+            // issuers that had one (warp-uniform), 16 columns at a time.
             uint32_t v[32];
-            if constexpr (BN == 32) {
-                tmem_ld32(tmem_d + lane_base + uint32_t(buf * BN), v);
-            } else {
-                uint32_t h[16];
-                tmem_ld16(tmem_d + lane_base + uint32_t(buf * BN), h);
+            {
+                const int n_u = g.k1 - g.k0, r0 = i0 % kIssuers;
+                const uint32_t dcol = tmem_d + lane_base + uint32_t(buf * kIssuers * BN);
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    v[c] = h[c];
+                for (int h = 0; h < BN / 16; ++h) {
+                    uint32_t tmp[16];
+                    tmem_ld16(dcol + uint32_t(r0 * BN + h * 16), tmp);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        v[h * 16 + c] = tmp[c];
+#pragma unroll
+                    for (int j = 1; j < kIssuers; ++j) {
+                        if (j < n_u) {
+                            const int tt = (r0 + j) % kIssuers;
+                            tmem_ld16(dcol + uint32_t(tt * BN + h * 16), tmp);
+#pragma unroll
+                            for (int c = 0; c < 16; ++c)
+                                v[h * 16 + c] += tmp[c];
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -586,7 +626,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
                     if (c < p.M && row_ok) {
-                        const int32_t acc = int32_t(v[c]) - __ldg(pj->x_sum + c);
+                        // sums of c * 4^pl * x: exact, |.| <= 128 * 127 * 32768
+                        const int32_t acc = (int32_t(v[c]) >> (2 * pl)) - __ldg(pj->x_sum + c);
                         const float t = __fmul_rn(pj->w_scale, __ldg(pj->x_scale + c));
                         const size_t o = size_t(c) * N + n;
                         pj->y[o] = __fmul_rn(__int2float_rn(acc), t);
@@ -633,7 +674,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                     for (int c = 0; c < 16; ++c) {
                         const int m = h * 16 + c;
                         if (m < p.M && row_ok) {
-                            const int32_t acc = d[c] - __ldg(pj->x_sum + m);
+                            const int32_t acc = (d[c] >> (2 * pl)) - __ldg(pj->x_sum + m);
                             const float t = __fmul_rn(pj->w_scale, __ldg(pj->x_scale + m));
                             const size_t o = size_t(m) * N + n;
                             pj->y[o] = __fmul_rn(__int2float_rn(acc), t);

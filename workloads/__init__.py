@@ -131,6 +131,9 @@ WORKLOADS = {
     # a 10-layer stack (175 MB of weights, still larger than L2): the small case
     # for profiler captures of the stack kernel
     "stack10_m1": (stack_shapes(10), 1),
+    # the same stack with several tokens per projection (small-batch decode)
+    "stack30_m4": (stack_shapes(STACK_LAYERS), 4),
+    "stack30_m16": (stack_shapes(STACK_LAYERS), 16),
 }
 for _m in SMALL_M_VALUES:
     WORKLOADS[f"ffn_m{_m}"] = (list(SMALL_M_SHAPES), _m)
