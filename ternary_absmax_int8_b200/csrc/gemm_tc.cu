@@ -7,7 +7,9 @@
 // on chip and runs an int8 contraction on the tensor cores.
 //
 //   D[n, m] = sum_k c[n, k] * xq[m, k]    (u8 codes c = w + 1 in {0,1,2},
-//                                          s8 activations, s32 in TMEM)
+//                                          s8 activations, s32 in TMEM;
+//                                          plane p's codes enter as c * 4^p,
+//                                          its sums leave shifted by 2p)
 //   acc[m, n] = D[n, m] - x_sum[m]          (since w = c - 1)
 //   y[m, n] = float(acc) * (w_scale * x_scale[m])
 //
@@ -265,13 +267,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                         const int g = j >> 5, jj = j & 31;
                         const uint4 v = *reinterpret_cast<const uint4 *>(P + sw128_off(j, c));
                         uint8_t *Ag = A + g * kAGroupBytes;
+// plane bits left in place: code c held as c * 4^pl (<= 128, a u8),
+                        // one AND per word; the epilogue shifts the sums back
 #pragma unroll
                         for (int pl = 0; pl < 4; ++pl) {
-                            uint4 o;
-                            o.x = (v.x >> (2 * pl)) & 0x03030303u;
-                            o.y = (v.y >> (2 * pl)) & 0x03030303u;
-                            o.z = (v.z >> (2 * pl)) & 0x03030303u;
-                            o.w = (v.w >> (2 * pl)) & 0x03030303u;
+                            const uint32_t m = 0x03030303u << (2 * pl);
+                            const uint4 o = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
                             *reinterpret_cast<uint4 *>(Ag + sw128_off(jj + 32 * pl, c)) = o;
                         }
                     }
@@ -313,7 +314,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     const float ts = __shfl_sync(0xffffffffu, my_t, i);
                     const int32_t xs = __shfl_sync(0xffffffffu, my_s, i);
                     if (row_ok && mbase + i < p.M)
-                        store_out(p, mbase + i, n, int32_t(v[i]), ts, xs);
+                        store_out(p, mbase + i, n, int32_t(v[i]) >> (2 * q), ts, xs);
                 }
             }
             tc_fence_before();
