@@ -1,0 +1,74 @@
+"""Host logic of bench.py, on CPU: how each workload is launched, the launch
+and byte counts its JSON line reports, and the reference arm's line (the
+oracle timed on a bounded sample)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+from workloads import WORKLOADS, algorithmic_bytes, make_projections
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _projs(name):
+    shapes, M = WORKLOADS[name]
+    return list(make_projections(shapes[:7], M=M, seed=0, with_weights=False))
+
+
+@pytest.mark.parametrize("name,mode", [
+    ("stack30_m1", "fused"), ("layer_m1", "fused"), ("ffn_m1", "fused"),
+    ("ffn_m2", "batch"), ("ffn_m4", "batch"), ("ffn_m8", "batch"), ("ffn_m24", "batch"),
+    ("stack30_m4", "batch"), ("stack30_m16", "batch"),
+    ("single_640x2560_m1", "per_projection"), ("prefill_m512", "per_projection"),
+])
+def test_step_mode(name, mode):
+    assert bench.step_mode(_projs(name)) == mode
+
+
+def test_batch_launch_counts():
+    # 512 token rows per quantiser launch; 256 projections per streaming
+    # launch, 16 per tensor-core group launch
+    assert bench.batch_launches(3, 4) == 1 + 1
+    assert bench.batch_launches(3, 16) == 1 + 1
+    assert bench.batch_launches(210, 4) == 2 + 1
+    assert bench.batch_launches(210, 16) == 7 + 14
+    assert bench.batch_launches(300, 2) == 2 + 2
+
+
+def test_step_bytes_by_mode():
+    fused = _projs("ffn_m1")
+    # one quantising launch: GEMV bytes + bf16 activations read
+    assert bench.workload_step_bytes("ffn_m1", fused) == sum(
+        algorithmic_bytes(p.N, p.K, 1) + 2 * p.K for p in fused)
+    batch = _projs("ffn_m16")
+    # quantiser (bf16 in, int8 + scale + sum out) then the GEMV
+    assert bench.workload_step_bytes("ffn_m16", batch) == sum(
+        2 * 16 * p.K + 16 * p.K + 16 * 8 + algorithmic_bytes(p.N, p.K, 16) for p in batch)
+
+
+def test_whole_job_rate_and_max_over_ranks_identity():
+    assert bench.whole_job_rate(4, 1e9, 2.0) == pytest.approx(2e12)
+    assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
+
+
+def test_reference_arm_line():
+    out = subprocess.run(
+        [sys.executable, "bench.py", "--impl", "reference", "--workload", "ffn_m4",
+         "--steps", "1", "--warmup", "3"],
+        cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads(out.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_warmup_below_three_is_rejected():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--warmup", "2"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0 and "warmup" in out.stderr
