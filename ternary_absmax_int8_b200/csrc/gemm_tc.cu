@@ -37,6 +37,7 @@
 // shared-memory stores per 4 bytes of weights, is what bounds a stage
 // otherwise). Every mbarrier wait is
 // bounded; loads never use cluster multicast.
+#include <atomic>
 #include <algorithm>
 #include <cstring>
 
@@ -344,7 +345,7 @@ cudaError_t launch_shape(const uint8_t *packed, const int8_t *xq, PrefillParams 
     prm.feat_tiles = (prm.N4 + S::kPackedRows - 1) / S::kPackedRows;
     prm.tok_tiles = (prm.M + BN - 1) / BN;
     const size_t smem = S::bytes + 1024;  // + alignment slack
-    static int configured_dev = -1;
+    static std::atomic<int> configured_dev{-1};  // set by any host thread
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {

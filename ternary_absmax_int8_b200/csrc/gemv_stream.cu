@@ -35,6 +35,7 @@
 //  * Every mbarrier wait is bounded (2 s of global time); on a timeout the
 //    kernel records an error bit and winds down, the producer first waiting
 //    (bounded) for its copies in flight.
+#include <atomic>
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
@@ -670,7 +671,7 @@ cudaError_t launch_instance(const StreamParams<MaxE> &p, int grid, size_t smem, 
                             cudaStream_t stream)
 {
     auto kern = stream_gemv_kernel<W, G, MaxE, MT, CPS>;
-    static int configured_dev = -1;  // per instantiation
+    static std::atomic<int> configured_dev{-1};  // per instantiation, any host thread
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {

@@ -49,6 +49,7 @@
 //   CTA at 8 KB of weights per ~0.5 us. So three threads issue, taking units
 //   in turn, each into its own accumulator; the epilogue adds the partial
 //   accumulators of the issuers that had units in the segment.
+#include <atomic>
 #include <algorithm>
 #include <mutex>
 #include <utility>
@@ -719,7 +720,7 @@ smallm_group_kernel(const __grid_constant__ GroupTable gt, const __grid_constant
 template <int BN>
 cudaError_t configure_bn()
 {
-    static int configured_dev = -1;
+    static std::atomic<int> configured_dev{-1};  // set by any host thread
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
@@ -1040,7 +1041,7 @@ cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const
                                      const float *x_scale, const int32_t *x_sum, float *y,
                                      int32_t *acc_out, int M, int N, int K, cudaStream_t stream)
 {
-    static void *scratch[64] = {nullptr};
+    static std::atomic<void *> scratch[64] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)

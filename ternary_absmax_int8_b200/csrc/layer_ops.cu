@@ -24,6 +24,7 @@
 // with programmatic stream serialisation and wait for the previous grid
 // before any memory access, so a following stack GEMV launched with
 // TQ_STACK_OVERLAP_PREV streams its weights while they run.
+#include <atomic>
 #include <algorithm>
 #include <cfloat>
 
@@ -242,7 +243,7 @@ cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f
     cfg.blockDim = dim3(kRowThreads);
     cfg.dynamicSmemBytes = size_t(K) * sizeof(float);
     cfg.stream = stream;
-    static int configured_dev = -1;  // the row may need more than 48 KB
+    static std::atomic<int> configured_dev{-1};  // the row may need more than 48 KB
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_dev != dev) {

@@ -1,5 +1,6 @@
 // tq_api.cu -- the C ABI of libtq (declared in include/tq.h): argument
 // checks, then kernel launches. Nothing here allocates device memory.
+#include <atomic>
 #include <cfloat>
 #include <cstdarg>
 #include <cstdio>
@@ -23,7 +24,7 @@ cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t
 
 unsigned *device_error_word()
 {
-    static unsigned *cache[64] = {nullptr};
+    static std::atomic<unsigned *> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return nullptr;
@@ -38,7 +39,7 @@ unsigned *device_error_word()
 
 int device_sm_count()
 {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return 1;
