@@ -227,3 +227,32 @@ def test_absmean_pack_argument_checks():
     with pytest.raises(tq.TQError) as e:
         tq.tq_absmean_pack(A + 4, A, A, 8, 32, stream=0)
     assert e.value.name == "TQ_ERR_ALIGN"
+
+
+def test_header_is_c_and_struct_layout_matches_binding(tmp_path):
+    # include/tq.h must compile as C (a C ABI), and the C compiler's layout of
+    # tq_proj must be the one the ctypes binding marshals.
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "tq.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(tq_proj), offsetof(tq_proj, w_scale),\n'
+        "         offsetof(tq_proj, K), offsetof(tq_proj, gain), offsetof(tq_proj, eps),\n"
+        "         offsetof(tq_proj, reserved));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(root, "include"), "-isystem", cuda_inc,
+                    str(src), "-o", str(exe)], check=True, capture_output=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    T = tq.TqProj
+    assert got == [ctypes.sizeof(T), T.w_scale.offset, T.K.offset, T.gain.offset,
+                   T.eps.offset, T.reserved.offset]
