@@ -175,3 +175,15 @@ def test_group_plan_after_a_reported_device_error(cuda_device):
     st.run()
     _check(st, refs)
     assert tq.tq_device_error(reset=True) == 0
+
+
+def test_full_stack_30_layers_m16_group_plan(cuda_device):
+    # The launch configuration bench.py times for stack30_m16: all 210
+    # projections of the 30-layer stack at 16 tokens, 14 group launches of at
+    # most 16 projections; every output against the oracle.
+    projs = list(make_projections(stack_shapes(30), M=16, seed=17))
+    st = BatchStack(projs, 16)
+    refs = parallel_map(_oracle, projs)
+    st.run(tq.TQ_STACK_OVERLAP_PREV)
+    _check(st, refs)
+    assert tq.tq_device_error(reset=True) == 0
