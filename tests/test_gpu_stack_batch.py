@@ -187,3 +187,14 @@ def test_full_stack_30_layers_m16_group_plan(cuda_device):
     st.run(tq.TQ_STACK_OVERLAP_PREV)
     _check(st, refs)
     assert tq.tq_device_error(reset=True) == 0
+
+
+def test_full_stack_30_layers_m4_streaming(cuda_device):
+    # bench.py's stack30_m4: all 210 projections at 4 tokens in one streaming
+    # launch; every output against the oracle.
+    projs = list(make_projections(stack_shapes(30), M=4, seed=18))
+    st = BatchStack(projs, 4)
+    refs = parallel_map(_oracle, projs)
+    st.run()
+    _check(st, refs)
+    assert tq.tq_device_error(reset=True) == 0
