@@ -74,11 +74,20 @@ constexpr int kSA = 4;                 // tensor-memory A slots
 // Few: every copy issued here delays the barrier the whole CTA waits on.
 constexpr int kEarlyUnits = 2;
 constexpr int kIssuers = 3;            // MMA-issuing warps 1..3, one accumulator each
+// "A slot filled" barriers, one per unit modulo lcm(kIssuers, kSA): each then
+// has a single MMA issuer and a single expansion set, so its waiter has
+// always seen the phase before the one it waits for. (With one barrier per
+// A slot, an issuer could wait for unit i's phase while unit i - kSA, which
+// another issuer consumes, was still being expanded: the parity wait then
+// matched the phase before that one and passed early.)
+constexpr int kAFull = 12;
 constexpr int kACols = kUnitK / 4;     // TMEM columns per A slot (4 bytes per column)
 constexpr int kThreads = 512;
 constexpr int kExpandWarp0 = 4;        // expansion warps 4..11: two sets of four
 constexpr int kExpandSets = 2;         // set s expands the CTA's units s, s + 2, ...
 constexpr int kEpiWarp0 = 4 + 4 * kExpandSets;  // epilogue warps 12..15
+static_assert(kAFull % kIssuers == 0 && kAFull % kSA == 0 && kAFull % kExpandSets == 0,
+              "a_full barrier ownership");
 constexpr int kMaxGrid = 512;
 
 constexpr int kPlanStreamK = 0;
@@ -186,9 +195,9 @@ struct SmallMSmem {
     static constexpr size_t slot_off = b_off + size_t(kSP) * kBBytes;
     static constexpr size_t kSlotBytes = size_t(kRows) * BN * 4;
     static constexpr size_t bar_off = slot_off + size_t(kMaxCluster - 1) * kSlotBytes;
-    // tma_full[SP], p_free[SP], mma_done[SP], a_full[SA], acc_full[2],
+    // tma_full[SP], p_free[SP], mma_done[SP], a_full[kAFull], acc_full[2],
     // acc_empty[2], red_done
-    static constexpr int kBars = 3 * kSP + kSA + 5;
+    static constexpr int kBars = 3 * kSP + kAFull + 5;
     static constexpr size_t misc_off = bar_off + kBars * 8;  // tmem slot, finisher flag
     static constexpr size_t bytes = misc_off + 16;
 };
@@ -304,7 +313,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
     uint64_t *p_free = bars + kSP;
     uint64_t *mma_done = bars + 2 * kSP;
     uint64_t *a_full = bars + 3 * kSP;
-    uint64_t *acc_full = a_full + kSA;
+    uint64_t *acc_full = a_full + kAFull;
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *red_done = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
@@ -379,7 +388,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             mbar_init(&p_free[s], 4);
             mbar_init(&mma_done[s], 1);
         }
-        for (int s = 0; s < kSA; ++s)
+        for (int s = 0; s < kAFull; ++s)
             mbar_init(&a_full[s], 4);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], kIssuers);  // every issuer commits every segment
@@ -455,7 +464,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                         continue;
                     const int s = i % kSP, sa = i % kSA;
                     if (!mbar_wait(&tma_full[s], uint32_t((i / kSP) & 1), p.err) ||
-                        !mbar_wait(&a_full[sa], uint32_t((i / kSA) & 1), p.err)) {
+                        !mbar_wait(&a_full[i % kAFull], uint32_t((i / kAFull) & 1), p.err)) {
                         ok = false;
                         break;
                     }
@@ -526,7 +535,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&a_full[sa]);
+                    mbar_arrive(&a_full[i % kAFull]);
                     mbar_arrive(&p_free[s]);
                 }
             }
@@ -542,6 +551,11 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                              p.acc_out};
         Seg g = first_seg();
         int i0 = 0;  // the CTA's unit counter at the start of segment sg
+        // Once a wait has given up (the error word is set and the outputs are
+        // void), the remaining segments skip their waits and accumulator
+        // reads but still count their split tiles in, so that every split
+        // tile's finisher still runs and leaves the scratch zeroed.
+        bool failed = false;
         for (int sg = 0; sg < cw.nseg; ++sg, i0 += g.k1 - g.k0, g = next_seg(g, sg)) {
             const GroupProj *pj;
             if constexpr (Group)
@@ -552,17 +566,21 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             const int tile = g.tile;
             const bool whole = g.k0 == 0 && g.k1 == pj->U;
             const int buf = sg & 1;
-            const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((sg >> 1) & 1), p.err);
-            // The four epilogue warps meet at named barriers below: decide
-            // together whether to go on.
-            if (epilogue_any(!got))
-                break;
-            tc_fence_after();
+            if (!failed) {
+                const bool got = mbar_wait_warp(&acc_full[buf], uint32_t((sg >> 1) & 1), p.err);
+                // The four epilogue warps meet at named barriers below: decide
+                // together.
+                failed = epilogue_any(!got);
+            }
             // The segment's units i0, i0 + 1, ... went to issuers i0 % kIssuers,
             // then the next ones in turn: add the partial accumulators of the
             // issuers that had one (warp-uniform), 16 columns at a time.
             uint32_t v[32];
-            {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+                v[c] = 0;
+            if (!failed) {
+                tc_fence_after();
                 const int n_u = g.k1 - g.k0, r0 = i0 % kIssuers;
                 const uint32_t dcol = tmem_d + lane_base + uint32_t(buf * kIssuers * BN);
 #pragma unroll
@@ -583,11 +601,11 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers now
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers now
 
             const int prow = tile * kPRows + jr;
             const bool row_ok = prow < pj->N4;
@@ -626,7 +644,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             if (whole || split_cluster) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c) {
-                    if (c < p.M && row_ok) {
+                    if (c < p.M && row_ok && !failed) {
                         // sums of c * 4^pl * x: exact, |.| <= 128 * 127 * 32768
                         const int32_t acc = (int32_t(v[c]) >> (2 * pl)) - __ldg(pj->x_sum + c);
                         const float t = __fmul_rn(pj->w_scale, __ldg(pj->x_scale + c));

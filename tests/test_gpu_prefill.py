@@ -1,8 +1,7 @@
 """GPU parity of tq_gemm_prefill (M = 512 prompt processing) against the oracle.
 
-Full outputs at M = 128 and 256 for the FFN shapes; at M = 512 on the three
-prefill shapes (including the 27B-scale 17408 x 5120) a sample of token rows,
-first and last included, is checked on all N outputs. Ragged M and N exercise
+Full outputs at M = 128 and 256 for the FFN shapes and at M = 512 on the three
+prefill shapes (including the 27B-scale 17408 x 5120). Ragged M and N exercise
 partial tiles; the shapes cover both work splits of the kernel: whole tiles per
 CTA (including CTAs that take a second tile) and K split over the CTAs of a
 thread-block cluster with a reduce-scatter of the partial sums.
@@ -10,7 +9,6 @@ thread-block cluster with a reduce-scatter of the partial sums.
 import numpy as np
 import pytest
 
-import oracle
 from tests._gpu import assert_parity, gpu_forward, host_pack, oracle_forward
 from workloads import PREFILL_M, PREFILL_SHAPES, activations_bf16, make_projections, \
     stored_weight_scale, ternary_weights
@@ -26,18 +24,14 @@ def test_prefill_full_outputs(cuda_device, M):
                       oracle_forward(p.w, p.w_scale, p.x_bf16), f"{p.name} M={M}")
 
 
-def test_prefill_m512_sampled_rows(cuda_device):
-    rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([[0, PREFILL_M - 1], rng.choice(PREFILL_M, 30, replace=False)]))
+def test_prefill_m512_full_outputs(cuda_device):
+    # The three prefill shapes at 512 tokens, every output: the oracle runs
+    # over disjoint output-row ranges on all host threads (same function,
+    # same result; 45.6 G multiply-adds on the largest shape).
     for p in make_projections(PREFILL_SHAPES, M=PREFILL_M, seed=0):
         P = host_pack(p.w)
-        q, xs, xsum, acc, y = gpu_forward(P, p.N, p.w_scale, p.x_bf16)
-        rq, rxs, rxsum = oracle.quant(p.x_bf16)
-        assert (q == rq).all() and (xs.view(np.uint32) == rxs.view(np.uint32)).all()
-        assert (xsum == rxsum).all()
-        sub = (q[rows], xs[rows], xsum[rows], acc[rows], y[rows])
-        ref = oracle_forward(p.w, p.w_scale, p.x_bf16[rows])
-        assert_parity(sub, ref, p.name)
+        assert_parity(gpu_forward(P, p.N, p.w_scale, p.x_bf16),
+                      oracle_forward(p.w, p.w_scale, p.x_bf16), f"{p.name} M={PREFILL_M}")
 
 
 @pytest.mark.parametrize("N,K,M", [(516, 272, 130), (4, 16, 129), (2048, 1024, 384),
