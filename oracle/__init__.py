@@ -53,9 +53,18 @@ def _load():
             lib.oracle_rmsnorm.argtypes = [p, i64, i64, p, ctypes.c_float, p]
             lib.oracle_relu2_mul.argtypes = [p, p, i64, p]
             lib.oracle_absmean.argtypes = [p, i64, i64, p, p]
+            lib.oracle_hadamard_rotate.argtypes = [p, i64, i64, i64, p]
+            lib.oracle_quant4.argtypes = [p, i64, i64, p, p, p]
+            lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+            lib.oracle_half_to_double.restype = ctypes.c_double
+            lib.oracle_pack_binary.argtypes = [p, p, i64, i64]
+            lib.oracle_unpack_binary.argtypes = [p, p, i64, i64]
+            lib.oracle_gemv_binary.argtypes = [p, i64, i64, p, p, i64, p, i64, i64, p, p]
             for f in (lib.oracle_pack, lib.oracle_unpack, lib.oracle_quant,
                       lib.oracle_gemv, lib.oracle_epilogue, lib.oracle_quant_f32,
-                      lib.oracle_rmsnorm, lib.oracle_relu2_mul, lib.oracle_absmean):
+                      lib.oracle_rmsnorm, lib.oracle_relu2_mul, lib.oracle_absmean,
+                      lib.oracle_hadamard_rotate, lib.oracle_quant4, lib.oracle_pack_binary,
+                      lib.oracle_unpack_binary, lib.oracle_gemv_binary):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -212,3 +221,128 @@ def absmean(W_bf16: np.ndarray):
     g = np.empty(1, np.float32)
     _check(_load().oracle_absmean(_ptr(W), N, K, _ptr(w), _ptr(g)), "absmean")
     return w, g[0]
+
+
+# ------------------------------------------------ Hadamard-rotated 4-bit route
+def hadamard_rotate(x_bf16: np.ndarray, n: int) -> np.ndarray:
+    """Blockwise normalised Sylvester-Hadamard rotation of bf16 rows [M, K]
+    (blocks of n along K) -> fp32 [M, K]."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    M, K = x.shape
+    h = np.empty((M, K), np.float32)
+    _check(_load().oracle_hadamard_rotate(_ptr(x), M, K, int(n), _ptr(h)), "hadamard_rotate")
+    return h
+
+
+def quant4(h: np.ndarray):
+    """4-bit absmax quantisation (codes -7..7, one per int8) of fp32 rows
+    h [M, K] -> (q, x_scale, x_sum)."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    M, K = h.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty(M, np.float32)
+    t = np.empty(M, np.int32)
+    _check(_load().oracle_quant4(_ptr(h), M, K, _ptr(q), _ptr(s), _ptr(t)), "quant4")
+    return q, s, t
+
+
+def hadamard_quant4(x_bf16: np.ndarray, n: int):
+    """Rotation, then the 4-bit quantiser: (q, x_scale, x_sum)."""
+    return quant4(hadamard_rotate(x_bf16, n))
+
+
+def forward_had4(P: np.ndarray, N: int, w_scale: float, x_bf16: np.ndarray, n: int,
+                 threads: int = 1):
+    """The Hadamard route for one projection: rotate, quantise to 4 bits,
+    accumulate against the ternary weights, scale. Returns (q, x_scale, x_sum,
+    acc, y)."""
+    q, xs, xsum = hadamard_quant4(x_bf16, n)
+    acc = gemv(P, N, q) if threads == 1 else gemv_threads(P, N, q, threads)
+    return q, xs, xsum, acc, epilogue(acc, w_scale, xs)
+
+
+# ------------------------------------------------------------ binary g128
+def half_to_double(h: int) -> float:
+    """fp16 bit pattern -> float, by the IEEE binary16 definition."""
+    return float(_load().oracle_half_to_double(int(h)))
+
+
+def pack_binary(w: np.ndarray) -> np.ndarray:
+    """int8 [N,K] in {-1,+1} -> uint8 [N/8,K]."""
+    w = np.ascontiguousarray(w, dtype=np.int8)
+    N, K = w.shape
+    if N % 8:
+        raise OracleError("pack_binary: bad shape")
+    B = np.empty((N // 8, K), dtype=np.uint8)
+    _check(_load().oracle_pack_binary(_ptr(w), _ptr(B), N, K), "pack_binary")
+    return B
+
+
+def unpack_binary(B: np.ndarray, N: int) -> np.ndarray:
+    """uint8 [N/8,K] -> int8 [N,K] in {-1,+1}."""
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    K = B.shape[1]
+    if B.shape[0] * 8 != N:
+        raise OracleError("unpack_binary: bad shape")
+    w = np.empty((N, K), dtype=np.int8)
+    _check(_load().oracle_unpack_binary(_ptr(B), _ptr(w), N, K), "unpack_binary")
+    return w
+
+
+def gemv_binary(B: np.ndarray, N: int, s_f16: np.ndarray, q: np.ndarray, x_scale: np.ndarray,
+                n0: int = 0, n1: int | None = None):
+    """(acc int32 [M, n1-n0], y fp64 [M, n1-n0]) for output rows n0..n1-1 of
+    the binary projection B with fp16 group scales s_f16 [N, K/128] (uint16
+    bit patterns or float16)."""
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    s = np.ascontiguousarray(np.asarray(s_f16).view(np.uint16))
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    if q.ndim == 1:
+        q = q[None, :]
+    x_scale = np.ascontiguousarray(x_scale, dtype=np.float32).reshape(-1)
+    K = B.shape[1]
+    M = q.shape[0]
+    if q.shape[1] != K or B.shape[0] * 8 != N or s.shape != (N, K // 128) or x_scale.size != M:
+        raise OracleError("gemv_binary: bad shape")
+    if n1 is None:
+        n1 = N
+    acc = np.empty((M, n1 - n0), np.int32)
+    y = np.empty((M, n1 - n0), np.float64)
+    _check(_load().oracle_gemv_binary(_ptr(B), N, K, _ptr(s), _ptr(q), M, _ptr(x_scale), n0, n1,
+                                      _ptr(acc), _ptr(y)), "gemv_binary")
+    return acc, y
+
+
+def gemv_binary_threads(B, N, s_f16, q, x_scale, threads: int | None = None):
+    """``gemv_binary`` over all rows as disjoint row ranges on several host
+    threads (same function, same result; for parity runs on large shapes)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    if q.ndim == 1:
+        q = q[None, :]
+    threads = threads or os.cpu_count() or 1
+    bounds = (np.linspace(0, N // 8, min(threads, max(1, N // 8)) + 1).astype(np.int64)) * 8
+    acc = np.empty((q.shape[0], N), np.int32)
+    y = np.empty((q.shape[0], N), np.float64)
+
+    def run(i):
+        a, b = int(bounds[i]), int(bounds[i + 1])
+        if b > a:
+            acc[:, a:b], y[:, a:b] = gemv_binary(B, N, s_f16, q, x_scale, a, b)
+
+    with ThreadPoolExecutor(len(bounds) - 1) as ex:
+        list(ex.map(run, range(len(bounds) - 1)))
+    return acc, y
+
+
+def forward_binary(B: np.ndarray, N: int, s_f16: np.ndarray, x_bf16: np.ndarray,
+                   threads: int = 1):
+    """The binary g128 path for one projection: int8 absmax quantisation, then
+    the group-scaled accumulation. Returns (q, x_scale, x_sum, acc, y)."""
+    q, xs, xsum = quant(x_bf16)
+    if threads == 1:
+        acc, y = gemv_binary(B, N, s_f16, q, xs)
+    else:
+        acc, y = gemv_binary_threads(B, N, s_f16, q, xs, threads)
+    return q, xs, xsum, acc, y

@@ -52,9 +52,14 @@
  *    gives w = 0. The packed weights then follow oracle_pack, and gamma is
  *    the stored per-tensor scale.
  *
+ * Two further paths, with their readings next to their code below: the
+ * Hadamard-rotated 4-bit activations of prompt processing and the binary
+ * g128 weight format.
+ *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared.
  * Status codes: 0 ok; 1 a value outside the domain (a weight not in
- * {-1,0,1}, or a packed code 3); 2 a bad shape.
+ * {-1,0,1} -- {-1,+1} for the binary format --, or a packed code 3); 2 a bad
+ * shape.
  */
 #include <math.h>
 #include <stdint.h>
@@ -117,8 +122,11 @@ int oracle_unpack(const uint8_t *P, int8_t *w, int64_t N, int64_t K)
     return 0;
 }
 
-/* Absmax int8 quantisation of one fp32 row (the reading above). */
-static void quant_row(const float *row, int64_t K, int8_t *q, float *x_scale, int32_t *x_sum)
+/* Absmax quantisation of one fp32 row to the symmetric levels -qb..qb (the
+ * reading above, with qb = 127 for int8 and qb = 7 for the 4-bit codes of
+ * the Hadamard route). */
+static void quant_row_levels(const float *row, int64_t K, float qb, int8_t *q, float *x_scale,
+                             int32_t *x_sum)
 {
     float amax = 0.0f;
     for (int64_t k = 0; k < K; ++k) {
@@ -132,18 +140,24 @@ static void quant_row(const float *row, int64_t K, int8_t *q, float *x_scale, in
             q[k] = 0;
         *x_scale = 0.0f;
     } else {
-        volatile float s = 127.0f / amax; /* one fp32 rounding */
+        volatile float s = qb / amax; /* one fp32 rounding */
         for (int64_t k = 0; k < K; ++k) {
             volatile float t = row[k] * s; /* one fp32 rounding */
             float r = rintf(t); /* default mode: nearest, ties to even */
-            if (r > 127.0f) r = 127.0f;
-            if (r < -127.0f) r = -127.0f;
+            if (r > qb) r = qb;
+            if (r < -qb) r = -qb;
             q[k] = (int8_t)r;
             sum += (int32_t)r;
         }
-        *x_scale = amax / 127.0f;
+        *x_scale = amax / qb;
     }
     *x_sum = sum;
+}
+
+/* Absmax int8 quantisation of one fp32 row (the reading above). */
+static void quant_row(const float *row, int64_t K, int8_t *q, float *x_scale, int32_t *x_sum)
+{
+    quant_row_levels(row, K, 127.0f, q, x_scale, x_sum);
 }
 
 /* Per-token absmax int8 quantisation of x [M,K] (bf16 bit patterns). */
@@ -267,5 +281,168 @@ int oracle_epilogue(const int32_t *acc, int64_t M, int64_t N, float w_scale,
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n)
             y[m * N + n] = (double)acc[m * N + n] * (double)w_scale * (double)x_scale[m];
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Hadamard-rotated 4-bit activations for prompt processing (1bit engine blog,
+ * "509 tokens a second of prompt: the Hadamard route ships" and "Qwen3.8-27B
+ * at 45.7 tok/s ...": 4-bit activations on the matrix units, kept accurate by
+ * a Hadamard rotation; 1bit.systems README, read-more item "Training-Runs --
+ * BitNet v2 Hadamard"). The pages print no formula. Readings taken:
+ *  - The rotation acts on each block of n consecutive entries of a token row
+ *    (n a power of two dividing K): h = H_n x / sqrt(n), with H_n the
+ *    Sylvester-Hadamard matrix, H_n[i][j] = (-1)^popcount(i & j).
+ *  - Each sum over j is accumulated in fp64. For bf16 inputs every partial
+ *    sum is then exact (the inputs are multiples of the block's smallest
+ *    unit in the last place, and n * 2^8 times the largest over that unit
+ *    stays below 2^53 unless the block's magnitudes span more than ~2^35),
+ *    so the result does not depend on the order of the additions. The sum
+ *    times fl64(1/sqrt(n)) is rounded once to fp32 (for n a power of four,
+ *    1/sqrt(n) is a power of two and that product is exact).
+ *  - 4-bit codes: the absmax quantiser above with 7 levels each side
+ *    (q in -7..7, s = 7 / amax, x_scale = amax / 7), one code per int8.
+ * ---------------------------------------------------------------------- */
+
+/* (-1)^popcount(i & j), written out bit by bit. */
+static int hadamard_sign(int64_t i, int64_t j)
+{
+    int64_t b = i & j;
+    int odd = 0;
+    while (b) {
+        odd ^= (int)(b & 1);
+        b >>= 1;
+    }
+    return odd ? -1 : 1;
+}
+
+/* h [M,K] = the blockwise normalised Hadamard rotation of x [M,K] (bf16 bit
+ * patterns), n the block size. */
+int oracle_hadamard_rotate(const uint16_t *x, int64_t M, int64_t K, int64_t n, float *h)
+{
+    if (M < 0 || K < 0 || n < 1 || (n & (n - 1)) != 0 || K % n != 0)
+        return 2;
+    const double c = 1.0 / sqrt((double)n);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t b = 0; b < K; b += n)
+            for (int64_t i = 0; i < n; ++i) {
+                double s = 0.0;
+                for (int64_t j = 0; j < n; ++j)
+                    s += (double)hadamard_sign(i, j) * (double)bf16_to_float(x[m * K + b + j]);
+                h[m * K + b + i] = (float)(s * c);
+            }
+    return 0;
+}
+
+/* Per-token 4-bit absmax quantisation of fp32 rows h [M,K]. */
+int oracle_quant4(const float *h, int64_t M, int64_t K, int8_t *q, float *x_scale, int32_t *x_sum)
+{
+    if (M < 0 || K < 0)
+        return 2;
+    for (int64_t m = 0; m < M; ++m)
+        quant_row_levels(h + m * K, K, 7.0f, q + m * K, &x_scale[m], &x_sum[m]);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Binary g128 weights (baguaai "BitNet" tag page, the Bonsai 27B item: a
+ * true 1-bit binary scheme in which 128 weights share one fp16 scale, about
+ * 1.125 bits per weight). The page gives no bit order, no group direction
+ * and no activation format. Readings taken:
+ *  - A weight is +1 or -1: bit 1 is +1, bit 0 is -1.
+ *  - Eight weights per byte in the plane layout of the ternary format: the
+ *    packed tensor of an [N, K] projection is uint8 [N/8, K], bit p of byte
+ *    (i, k) holding output row i + p*(N/8).
+ *  - Groups are 128 consecutive k of one output row (K a multiple of 128);
+ *    scale s[n, g] (fp16) belongs to row n, columns 128 g .. 128 g + 127.
+ *  - Activations: the per-token absmax int8 quantiser above.
+ *  - acc[m, n, g] = sum over the group of w * q (int32, exact);
+ *    y[m, n] = x_scale[m] * sum_g s[n, g] * acc[m, n, g], in fp64 here.
+ *    The group-free total sum_g acc[m, n, g] is also returned (int32).
+ * ---------------------------------------------------------------------- */
+
+/* fp16 bit pattern to double, by the IEEE binary16 definition. */
+double oracle_half_to_double(uint16_t h)
+{
+    const int sign = (h >> 15) & 1;
+    const int e = (h >> 10) & 0x1F;
+    const int f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24); /* subnormal: f * 2^-14 * 2^-10 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* Pack w [N,K] in {-1,+1} into B [N/8,K]. */
+int oracle_pack_binary(const int8_t *w, uint8_t *B, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || N % 8 != 0)
+        return 2;
+    const int64_t Q = N / 8;
+    for (int64_t i = 0; i < Q; ++i)
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned byte = 0;
+            for (int p = 0; p < 8; ++p) {
+                int v = w[(i + p * Q) * K + k];
+                if (v != 1 && v != -1)
+                    return 1;
+                if (v == 1)
+                    byte |= 1u << p;
+            }
+            B[i * K + k] = (uint8_t)byte;
+        }
+    return 0;
+}
+
+/* The weight of output row n at column k, read out of B by definition. */
+static int binary_weight_at(const uint8_t *B, int64_t Q, int64_t K, int64_t n, int64_t k)
+{
+    int64_t i = n % Q;    /* packed row */
+    int p = (int)(n / Q); /* bit, 0..7 */
+    return ((B[i * K + k] >> p) & 1) ? 1 : -1;
+}
+
+/* Unpack B [N/8,K] into w [N,K]. */
+int oracle_unpack_binary(const uint8_t *B, int8_t *w, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || N % 8 != 0)
+        return 2;
+    const int64_t Q = N / 8;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            w[n * K + k] = (int8_t)binary_weight_at(B, Q, K, n, k);
+    return 0;
+}
+
+/* For output rows n0 <= n < n1 and all M rows of q [M,K]: acc [M, n1-n0]
+ * (int32, sum over all K of w * q) and y [M, n1-n0] (fp64, the group-scaled
+ * sum times x_scale). s holds the fp16 scales [N, K/128] as bit patterns. */
+int oracle_gemv_binary(const uint8_t *B, int64_t N, int64_t K, const uint16_t *s,
+                       const int8_t *q, int64_t M, const float *x_scale, int64_t n0, int64_t n1,
+                       int32_t *acc, double *y)
+{
+    if (N < 0 || K < 0 || M < 0 || N % 8 != 0 || K % 128 != 0 || n0 < 0 || n1 > N || n0 > n1)
+        return 2;
+    const int64_t Q = N / 8, G = K / 128, W = n1 - n0;
+    for (int64_t m = 0; m < M; ++m) {
+        const int8_t *qm = q + m * K;
+        for (int64_t n = n0; n < n1; ++n) {
+            int32_t total = 0;
+            double sum = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                int32_t a = 0;
+                for (int64_t k = 128 * g; k < 128 * g + 128; ++k)
+                    a += binary_weight_at(B, Q, K, n, k) * (int32_t)qm[k];
+                total += a;
+                sum += (double)a * oracle_half_to_double(s[n * G + g]);
+            }
+            acc[m * W + (n - n0)] = total;
+            y[m * W + (n - n0)] = sum * (double)x_scale[m];
+        }
+    }
     return 0;
 }

@@ -123,6 +123,78 @@ def stack_shapes(layers: int = STACK_LAYERS):
     return [(f"L{l}.{name}", N, K) for l in range(layers) for (name, N, K) in DECODER_LAYER]
 
 
+# ------------------------------------------------------------ binary g128
+# Binary weights (baguaai "BitNet" tag page, Bonsai 27B item: 1 bit per weight,
+# one fp16 scale per 128 weights). The shapes are the 27B-scale FFN of the
+# prefill configuration: gate/up [17408 x 5120], down [5120 x 17408].
+BINARY_GROUP = 128
+BINARY_FFN27B = (("gate_proj", 17408, 5120), ("up_proj", 17408, 5120),
+                 ("down_proj", 5120, 17408))
+BINARY_LAYERS = 8
+# fp16 group scales are drawn uniformly from this range: the size of mean|W|
+# over 128 latent weights of N(0, 0.02^2) (0.02 * sqrt(2 / pi) = 0.016); the
+# page gives no distribution.
+BINARY_SCALE_RANGE = (0.012, 0.020)
+
+
+@dataclass
+class BinaryProjection:
+    """One synthetic binary g128 projection and M activation rows."""
+    name: str
+    N: int
+    K: int
+    M: int
+    w: np.ndarray          # int8 [N, K] in {-1, +1}
+    s_f16: np.ndarray      # uint16 [N, K/128] fp16 bit patterns (group scales)
+    x_bf16: np.ndarray     # uint16 [M, K] bf16 bit patterns
+
+
+def binary_weights(rng: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """int8 [N, K], i.i.d. -1 / +1 with probability 1/2 each."""
+    return (rng.integers(0, 2, size=(N, K), dtype=np.int8) * 2 - 1).astype(np.int8)
+
+
+def group_scales_f16(rng: np.random.Generator, N: int, K: int) -> np.ndarray:
+    """uint16 [N, K/128] fp16 bit patterns, uniform on BINARY_SCALE_RANGE."""
+    lo, hi = BINARY_SCALE_RANGE
+    s = rng.uniform(lo, hi, size=(N, K // BINARY_GROUP)).astype(np.float16)
+    return s.view(np.uint16)
+
+
+def make_binary_projections(shapes, M: int, seed: int = 0):
+    """Yield BinaryProjection objects for ``shapes`` (sequence of (name, N, K)).
+    Spawned streams as in ``make_projections``: weights (and then scales) of
+    projection j from the first child's stream j, activations from the
+    second's."""
+    shapes = list(shapes)
+    root = np.random.SeedSequence(seed)
+    w_root, x_root = root.spawn(2)
+    w_seqs = w_root.spawn(len(shapes))
+    x_seqs = x_root.spawn(len(shapes))
+    for j, (name, N, K) in enumerate(shapes):
+        rng = np.random.Generator(np.random.PCG64(w_seqs[j]))
+        w = binary_weights(rng, N, K)
+        s = group_scales_f16(rng, N, K)
+        x = activations_bf16(np.random.Generator(np.random.PCG64(x_seqs[j])), M, K)
+        yield BinaryProjection(name, N, K, M, w, s, x)
+
+
+def binary_stack_shapes(layers: int = BINARY_LAYERS):
+    """``layers`` copies of the 27B-scale FFN projections (binary weights)."""
+    return [(f"L{l}.{name}", N, K) for l in range(layers) for (name, N, K) in BINARY_FFN27B]
+
+
+def binary_bytes(N: int, K: int, M: int) -> int:
+    """Bytes one binary GEMV must move: bits (N*K/8) + fp16 scales (N*K/128*2)
+    + int8 activations + fp32 output + per-row scale (4 B)."""
+    return N * K // 8 + N * (K // BINARY_GROUP) * 2 + M * K + M * N * 4 + M * 4
+
+
+# Hadamard route: block size of the rotation. 256 is the largest power of two
+# dividing every K of the prefill shapes (2560 = 10 x 256, 6912 = 27 x 256,
+# 5120 = 20 x 256), and 1/sqrt(256) = 1/16 is exact.
+HADAMARD_BLOCK = 256
+
 # Named workloads. Each maps to (shapes, M).
 WORKLOADS = {
     "single_640x2560_m1": ([("proj", 640, 2560)], 1),
@@ -138,6 +210,10 @@ WORKLOADS = {
 for _m in SMALL_M_VALUES:
     WORKLOADS[f"ffn_m{_m}"] = (list(SMALL_M_SHAPES), _m)
 WORKLOADS["prefill_m512"] = (list(PREFILL_SHAPES), PREFILL_M)
+# the same contraction with Hadamard-rotated 4-bit activations
+WORKLOADS["prefill_had4_m512"] = (list(PREFILL_SHAPES), PREFILL_M)
+# binary g128 weights: 8 layers of the 27B-scale FFN, 301 MB per pass
+WORKLOADS["binary_ffn27b_m1"] = (binary_stack_shapes(BINARY_LAYERS), 1)
 
 
 def algorithmic_bytes(N: int, K: int, M: int) -> int:
