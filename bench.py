@@ -43,7 +43,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import (WORKLOADS, algorithmic_bytes, make_projections)  # noqa: E402
+from workloads import (HADAMARD_BLOCK, NEXT_WORKLOADS, WORKLOADS, algorithmic_bytes,  # noqa: E402
+                       binary_bytes, make_binary_projections, make_projections)
 
 METRIC = ("ternary GEMV achieved HBM GB/s (% of B200 peak) at M=1; layer-stack passes/s")
 PEAK_FALLBACK_GBS = 6650.0
@@ -63,6 +64,11 @@ DESCRIPTIONS = {
     "layer_m1": "one BitNet-b1.58-2B-4T decoder layer, 7 ternary projections, M=1",
     "single_640x2560_m1": "one ternary projection N=640 K=2560, M=1",
     "prefill_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120",
+    "prefill_had4_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120 with "
+                         "Hadamard-rotated 4-bit activations (blockwise rotation, n=256)",
+    "binary_ffn27b_m1": "binary g128 decode: 8 x 27B-scale FFN layer (gate/up 17408x5120, down "
+                        "5120x17408), 1 bit + fp16 scale per 128 weights, M=1, 24 projections, "
+                        "2.14e9 weights",
 }
 
 
@@ -592,6 +598,272 @@ def run_reference(args, rank: int, world: int):
     }
 
 
+# --------------------------------------- Hadamard prefill, binary g128 decode
+def run_next(args, rank: int, world: int):
+    """prefill_had4_m512: per projection, the fused Hadamard rotation + 4-bit
+    quantiser launch and the prefill GEMM on its codes; binary_ffn27b_m1: the
+    stack quantiser and one binary g128 GEMV launch over the 24 projections.
+    Same JSON line as the other workloads."""
+    import torch
+
+    import ternary_absmax_int8_b200 as tq
+
+    shapes, M = NEXT_WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return next_reference(args, shapes, M, rank, world)
+    dev_i = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev_i)
+    stream = torch.cuda.current_stream()
+    had = args.workload == "prefill_had4_m512"
+    if had:
+        projs = list(make_projections(shapes, M=M, seed=args.seed))
+        wbytes = sum(p.N * p.K // 4 for p in projs)
+    else:
+        projs = list(make_binary_projections(shapes, M=M, seed=args.seed))
+        wbytes = sum(p.N * p.K // 8 + p.N * p.K // 64 for p in projs)
+    copies = 1 if wbytes > 2 * L2_BYTES else -(-2 * L2_BYTES // wbytes)
+    n = len(projs)
+    x_host = torch.from_numpy(np.concatenate([p.x_bf16.view(np.int16).reshape(-1)
+                                              for p in projs])).pin_memory()
+    x_dev = x_host.cuda()
+    kx = np.concatenate([[0], np.cumsum([p.M * p.K for p in projs])]).astype(np.int64)
+    ny = np.concatenate([[0], np.cumsum([p.M * p.N for p in projs])]).astype(np.int64)
+    xq = torch.empty(int(kx[-1]), dtype=torch.int8, device="cuda")
+    xs = torch.empty(n * M, device="cuda")
+    xsum = torch.empty(n * M, dtype=torch.int32, device="cuda")
+    y_dev = torch.empty(int(ny[-1]), device="cuda")
+    y_host = torch.empty(int(ny[-1])).pin_memory()
+    if had:
+        W = []
+        for p in projs:
+            P = np.empty((p.N // 4, p.K), np.uint8)
+            tq.tq_pack_host(p.w, P, p.M, p.N, p.K)
+            W.append([torch.from_numpy(P).cuda() for _ in range(copies)])
+
+        def quant(c, s_):
+            for j, p in enumerate(projs):
+                tq.tq_hadamard_quantize_act(x_dev.data_ptr() + 2 * int(kx[j]),
+                                            xq.data_ptr() + int(kx[j]), xs.data_ptr() + 4 * j * M,
+                                            xsum.data_ptr() + 4 * j * M, p.M, p.K,
+                                            HADAMARD_BLOCK, stream=s_)
+
+        def gemv(c, s_):
+            for j, p in enumerate(projs):
+                tq.tq_gemm_prefill(W[j][c], float(p.w_scale), xq.data_ptr() + int(kx[j]),
+                                   xs.data_ptr() + 4 * j * M, xsum.data_ptr() + 4 * j * M,
+                                   y_dev.data_ptr() + 4 * int(ny[j]), None, p.M, p.N, p.K,
+                                   stream=s_)
+
+        sb = sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
+        gemv_units = sum(2.0 * p.M * p.N * p.K for p in projs)
+        launches = 2 * n
+        kernel = "prefill_tc_kernel"
+    else:
+        B = []
+        for p in projs:
+            bits = np.empty((p.N // 8, p.K), np.uint8)
+            sp = np.empty((p.N // 8, p.K // 128, 8), np.uint16)
+            tq.tq_pack_binary_host(p.w, p.s_f16, bits, sp, p.N, p.K)
+            B.append([(torch.from_numpy(bits).cuda(), torch.from_numpy(sp.view(np.int16)).cuda())
+                      for _ in range(copies)])
+        qtab = [tq.make_proj(x=x_dev.data_ptr() + 2 * int(kx[j]), xq=xq.data_ptr() + int(kx[j]),
+                             x_scale=xs.data_ptr() + 4 * j * M, x_sum=xsum.data_ptr() + 4 * j * M,
+                             N=p.N, K=p.K) for j, p in enumerate(projs)]
+        btabs = [[tq.make_binary_proj(bits=B[j][c][0], scales_packed=B[j][c][1],
+                                      xq=xq.data_ptr() + int(kx[j]),
+                                      x_scale=xs.data_ptr() + 4 * j * M,
+                                      y=y_dev.data_ptr() + 4 * int(ny[j]), N=p.N, K=p.K)
+                  for j, p in enumerate(projs)] for c in range(copies)]
+
+        def quant(c, s_):
+            tq.tq_quantize_act_stack_batch(qtab, M, stream=s_)
+
+        def gemv(c, s_):
+            tq.tq_gemv_binary_stack(btabs[c], M, stream=s_)
+
+        sb = sum(quant_bytes(p.K, p.M) + binary_bytes(p.N, p.K, p.M) for p in projs)
+        gemv_units = float(sum(binary_bytes(p.N, p.K, p.M) for p in projs))
+        launches = 2
+        kernel = "binary_gemv_kernel"
+
+    def step(c, s_):
+        quant(c, s_)
+        gemv(c, s_)
+
+    for i in range(args.warmup):
+        step(i % copies, stream)
+    torch.cuda.synchronize()
+    K_ = args.steps
+    S = copies * max(1, 8 // copies)
+    n_chunks, rem = divmod(K_, S)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=cs):
+            fn(cs)
+        return g
+
+    chunk = capture(lambda cs: [step(i % copies, cs) for i in range(S)])
+    single = [capture(lambda cs, c=c: step(c, cs)) for c in range(copies)] if rem else []
+    chunk.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev_i)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(n_chunks):
+        chunk.replay()
+    for i in range(rem):
+        single[(n_chunks * S + i) % copies].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+
+    def graph_ms(fn, reps=3):
+        g = capture(fn)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    quant_ms = graph_ms(lambda cs: [quant(i % copies, cs) for i in range(S)]) / S
+    gemv_ms = graph_ms(lambda cs: [gemv(i % copies, cs) for i in range(S)]) / S
+    e2e_steps = max(K_, int(0.5e3 / max(total_ms / K_, 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(i % copies, stream)
+        y_host.copy_(y_dev, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    time.sleep(0.3)
+    clk = clocks.stop()
+    assert tq.tq_device_error(reset=True) == 0, "a kernel reported a device error"
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device="cuda")
+    if rank != 0:
+        return None
+    ms_step = total_ms / K_
+    value = whole_job_rate(world, sb, ms_step) / 1e9
+    if had:
+        tpeak, tkind = measured_tensor_peak()
+        achieved = gemv_units / (gemv_ms * 1e9)
+        roof = {"kernel": kernel, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": tpeak, "peak_kind": tkind, "unit": "TOPS (int8)",
+                "frac": round(achieved / tpeak, 4), "traffic": None,
+                "algorithmic_ops_per_step": gemv_units}
+    else:
+        peak, peak_kind = measured_peak()
+        achieved = gemv_units / (gemv_ms * 1e6)
+        roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "algorithmic_bytes_per_launch": int(gemv_units)}
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K_, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": ("int8 codes -7..7 (bf16 in, fp64 rotation) x ternary -> int32, fp32 out"
+                  if had else "int8 x binary (1 bit) -> int32 per group, fp64 group scaling, "
+                              "fp32 out"),
+        "data": ("synthetic (seeded ternary weights P=0.3/0.4/0.3, bf16 N(0,1) activations "
+                 "with 1% x20 outliers)" if had else
+                 "synthetic (seeded binary weights P=1/2, fp16 group scales U(0.012, 0.020), "
+                 "bf16 N(0,1) activations with 1% x20 outliers)"),
+        "config": {"workload": f"{args.workload}: {DESCRIPTIONS[args.workload]}",
+                   "projections": n, "tokens_M": M, "weight_bytes": wbytes, "step_bytes": sb,
+                   "weight_copies_rotated": copies,
+                   "l2": ("inputs larger than L2 (weight stream > 126 MB), no flush"
+                          if copies == 1 else f"{copies} rotated weight copies, "
+                          f"{copies * wbytes / 2**20:.0f} MiB > L2"),
+                   "parallelism": "single GPU" if world == 1 else f"replicas x{world}",
+                   "seed": args.seed},
+        "quant_us_per_step": round(quant_ms * 1e3, 3),
+        "gemv_us_per_step": round(gemv_ms * 1e3, 3),
+        "roofline": roof,
+        "e2e": {"value": round(whole_job_rate(world, sb, e2e_ms / e2e_steps) / 1e9, 1),
+                "unit": "GB/s", "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 4),
+                "ms_per_step": round(e2e_ms / e2e_steps, 5)},
+        "gpu_launches": launches * K_,
+        "clocks": clk,
+        "impl": "ours",
+    }
+    if had:
+        out["tops"] = round(world * gemv_units / (ms_step * 1e9), 1)
+    else:
+        out["passes_per_s"] = round(whole_job_rate(world, 1.0, ms_step), 1)
+    if world == 1 and not args.no_cpu_baseline:
+        sample = dict(args.__dict__)
+        sample["impl"], sample["steps"], sample["warmup"] = "reference", 1, 0
+        ref = next_reference(argparse.Namespace(**sample), shapes, M, 0, 1)
+        out["cpu_baseline"] = dict(ref["cpu_baseline"])
+    return out
+
+
+def next_reference(args, shapes, M, rank, world):
+    """The oracle on a bounded sample per step: 16 tokens of each prefill shape
+    (Hadamard route), or one layer's three binary projections."""
+    if rank != 0:
+        return None
+    import oracle
+
+    had = args.workload == "prefill_had4_m512"
+    if had:
+        sp = list(make_projections(shapes, M=16, seed=args.seed))
+        packed = [oracle.pack(p.w) for p in sp]
+        sb = sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in sp)
+
+        def one():
+            for P, p in zip(packed, sp):
+                oracle.forward_had4(P, p.N, p.w_scale, p.x_bf16, HADAMARD_BLOCK)
+    else:
+        sp = list(make_binary_projections(shapes[:3], M=M, seed=args.seed))
+        packed = [oracle.pack_binary(p.w) for p in sp]
+        sb = sum(quant_bytes(p.K, p.M) + binary_bytes(p.N, p.K, p.M) for p in sp)
+
+        def one():
+            for B, p in zip(packed, sp):
+                oracle.forward_binary(B, p.N, p.s_f16, p.x_bf16)
+
+    for _ in range(args.warmup):
+        one()
+    n = max(1, args.steps)
+    t0 = time.perf_counter()
+    for _ in range(n):
+        one()
+    el = time.perf_counter() - t0
+    value = sb * n / el / 1e9
+    sample = (f"{len(sp)} projections, {sp[0].M} tokens each, of {args.workload} per step, one "
+              f"thread, on {os.cpu_count()} host cores")
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / n * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "oracle (int32 accumulate, fp64 scaling)", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {DESCRIPTIONS[args.workload]}",
+                   "parallelism": "host, one thread"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 # ------------------------------------------------ decoder-layer chains
 CHAIN_WORKLOADS = {
     "ffn_block30_m1": "30 x BitNet-b1.58-2B-4T FFN block, M=1, real dependencies, two launches "
@@ -875,17 +1147,57 @@ def _ref_line(args, world, value, ms, sample):
     }
 
 
+# Workloads measured after the headline in the default run, in the same
+# process, each with its own clock record: the single projection, one decoder
+# layer, the batched-decode FFN sweep, prefill, the small-batch stacks and the
+# two further paths.
+EXTRA_CONFIGS = (["single_640x2560_m1", "layer_m1"] + [f"ffn_m{m}" for m in (1, 2, 4, 8, 16, 24)]
+                 + ["prefill_m512", "stack30_m4", "stack30_m16", "prefill_had4_m512",
+                    "binary_ffn27b_m1"])
+
+
+def summarise(line):
+    """The figures of one workload's JSON line kept under "configs"."""
+    r = line["roofline"]
+    out = {"us_per_step": round(line["ms_per_step"] * 1e3, 3), "GB_s": line["value"],
+           "roofline_kernel": r["kernel"], "roofline_achieved": r["achieved"],
+           "roofline_unit": r["unit"], "frac": r["frac"], "steps": line["steps"],
+           "sm_mhz": line["clocks"].get("sm_mhz"), "reasons": line["clocks"].get("reasons")}
+    for k in ("tops", "token_passes_per_s", "passes_per_s"):
+        if k in line:
+            out[k] = line[k]
+    if "per_projection" in line:
+        out["per_projection"] = line["per_projection"]
+    return out
+
+
+def run_extra_configs(args):
+    res = {}
+    for w in EXTRA_CONFIGS:
+        heavy = w.startswith("prefill") or w.startswith("stack30") or w.startswith("binary")
+        a = argparse.Namespace(**dict(args.__dict__, workload=w, steps=50 if heavy else 200,
+                                      warmup=3, no_cpu_baseline=True))
+        if w in NEXT_WORKLOADS:
+            line = run_next(a, 0, 1)
+        else:
+            line = run_ours(a, 0, 1)
+        res[w] = summarise(line)
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CHAIN_WORKLOADS),
-                    default="stack30_m1")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(CHAIN_WORKLOADS) +
+                    sorted(NEXT_WORKLOADS), default="stack30_m1")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads measured after the default one")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -902,6 +1214,8 @@ def main():
     try:
         if args.workload in CHAIN_WORKLOADS:
             out = run_chain(args, rank, world)
+        elif args.workload in NEXT_WORKLOADS:
+            out = run_next(args, rank, world)
         elif args.impl == "ours":
             out = run_ours(args, rank, world)
         else:
@@ -910,6 +1224,9 @@ def main():
         if world > 1 and args.impl == "ours":
             import torch.distributed as dist
             dist.destroy_process_group()
+    if (out is not None and world == 1 and args.impl == "ours" and not args.no_configs
+            and args.workload == "stack30_m1"):
+        out["configs"] = run_extra_configs(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 

@@ -294,6 +294,93 @@ tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scal
                           cudaStream_t stream);
 
 /*
+ * tq_hadamard_quantize_act -- 4-bit activation codes for prompt processing by
+ * the Hadamard route (1bit engine blog, "509 tokens a second of prompt: the
+ * Hadamard route ships" and "Qwen3.8-27B at 45.7 tok/s ...": 4-bit
+ * activations on the matrix units, kept accurate by a Hadamard rotation;
+ * 1bit.systems README, read-more item "Training-Runs -- BitNet v2 Hadamard").
+ * The pages print no formula. Reading: per token row, each block of n
+ * consecutive entries is rotated, h = H_n x / sqrt(n), H_n the
+ * Sylvester-Hadamard matrix (H_n[i][j] = (-1)^popcount(i & j)); the sums are
+ * exact in fp64 (bf16 inputs) and fl64(sum * fl64(1/sqrt(n))) is rounded once
+ * to fp32. Then amax = max |h|, s = fl32(7 / amax),
+ * xq = clamp(round_half_even(fl32(h * s)), -7, 7), x_scale = fl32(amax / 7),
+ * x_sum = sum xq (an all-zero row gives zeros).
+ * The codes, one per int8, feed tq_gemm_prefill (or tq_gemv) exactly like
+ * 8-bit codes; the weights are those of the rotated basis (the rotation's
+ * transpose is folded into them when they are trained or converted).
+ *   x       device, bf16 bit patterns [M, K], 16-byte aligned
+ *   xq      device, int8 [M, K], 16-byte aligned (written; values -7..7)
+ *   x_scale device, fp32 [M] (written); x_sum device, int32 [M] (written;
+ *           may be NULL)
+ *   n       block size: 32, 64, 128, 256, 512 or 1024, dividing K
+ * 0 <= K <= 32768 (M == 0 or K == 0: no-op); TQ_ERR_SHAPE if n is not one
+ * of those or does not divide K. One CTA per token row; asynchronous.
+ */
+tq_status tq_hadamard_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
+                                   int M, int K, int n, cudaStream_t stream);
+
+/*
+ * Binary g128 weights (baguaai "BitNet" tag page, Bonsai 27B item: a true
+ * 1-bit binary scheme in which 128 weights share one fp16 scale, about 1.125
+ * bits per weight). The page gives no bit order, group direction or
+ * activation format. Readings:
+ *   - a weight is +1 or -1; bit 1 is +1, bit 0 is -1;
+ *   - bits uint8 [N/8, K]: bit p of byte (i, k) is the weight of output row
+ *     i + p*N/8 at column k (the plane layout of the ternary format);
+ *   - a group is 128 consecutive k of one output row (K % 128 == 0), with one
+ *     fp16 scale; the device keeps the scales as [N/8, K/128, 8], entry
+ *     (i, g, p) scaling row i + p*N/8 on group g;
+ *   - activations: the per-token int8 absmax codes of tq_quantize_act;
+ *   - acc[m, n] = sum_k w[n, k] xq[m, k] (int32, exact);
+ *     y[m, n] = fl32(x_scale[m] * sum_g scale[n, g] * sum_{k in g} w xq),
+ *     each product exact in fp64 and the sum in fp64.
+ *
+ * tq_pack_binary_host -- host packing, synchronous.
+ *   w             host, int8 [N, K], every value -1 or +1
+ *   scales        host, fp16 bit patterns [N, K/128] (scales[n, g] for
+ *                 columns 128 g .. 128 g + 127)
+ *   bits          host, uint8 [N/8, K] (written)
+ *   scales_packed host, fp16 bit patterns [N/8, K/128, 8] (written)
+ * N % 8 == 0, K % 128 == 0, N, K >= 0 (TQ_ERR_SHAPE). TQ_ERR_VALUE if a
+ * weight is not -1 or +1 (outputs then partly written).
+ */
+tq_status tq_pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
+                              uint16_t *scales_packed, int N, int K);
+
+/*
+ * tq_gemv_binary -- decode GEMV over binary g128 weights, 1 <= M <= 4 tokens.
+ *   bits          device, uint8 [N/8, K], 16-byte aligned
+ *   scales_packed device, fp16 bits [N/8, K/128, 8], 16-byte aligned
+ *   xq            device, int8 [M, K], 16-byte aligned
+ *   x_scale       device, fp32 [M]
+ *   y             device, fp32 [M, N] (written)
+ *   acc_out       device, int32 [M, N] (written: sum_k w xq) or NULL
+ * N % 8 == 0, K % 128 == 0, K <= 32768; M > 4 is TQ_ERR_UNSUPPORTED; M == 0,
+ * N == 0 or K == 0 (all outputs 0) handled. One persistent launch streaming
+ * the bits and scales; asynchronous on `stream`.
+ *
+ * tq_gemv_binary_stack -- the same for a table of projections (one launch per
+ * 128 of them), each with its own shapes and buffers, M tokens each.
+ */
+tq_status tq_gemv_binary(const uint8_t *bits, const uint16_t *scales_packed, const int8_t *xq,
+                         const float *x_scale, float *y, int32_t *acc_out, int M, int N, int K,
+                         cudaStream_t stream);
+
+typedef struct tq_binary_proj {
+    const uint8_t *bits;            /* device, [N/8, K] */
+    const uint16_t *scales_packed;  /* device, [N/8, K/128, 8] fp16 */
+    const int8_t *xq;               /* device, [M, K] */
+    const float *x_scale;           /* device, [M] */
+    float *y;                       /* device, [M, N] */
+    int32_t *acc_out;               /* device, [M, N] or NULL */
+    int N, K;
+} tq_binary_proj;
+
+tq_status tq_gemv_binary_stack(const tq_binary_proj *projs, int n_proj, int M,
+                               cudaStream_t stream);
+
+/*
  * tq_selftest_wait_timeout -- exercise the failure path of the kernels'
  * bounded waits without a fault: one thread waits, with the same bounded
  * wait the kernels use, on an mbarrier that nothing ever arrives on. After

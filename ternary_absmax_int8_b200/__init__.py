@@ -22,6 +22,8 @@ __all__ = [
     "tq_gemv_stack_batch", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
     "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack", "tq_selftest_wait_timeout",
+    "tq_hadamard_quantize_act", "TqBinaryProj", "tq_pack_binary_host", "tq_gemv_binary",
+    "tq_gemv_binary_stack", "make_binary_proj",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -66,6 +68,20 @@ class TqProj(ctypes.Structure):
     ]
 
 
+class TqBinaryProj(ctypes.Structure):
+    """Mirror of ``struct tq_binary_proj``."""
+    _fields_ = [
+        ("bits", ctypes.c_void_p),
+        ("scales_packed", ctypes.c_void_p),
+        ("xq", ctypes.c_void_p),
+        ("x_scale", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("acc_out", ctypes.c_void_p),
+        ("N", ctypes.c_int),
+        ("K", ctypes.c_int),
+    ]
+
+
 _SIGS = {
     "tq_pack_host": [_vp, _vp, _i, _i, _i, _vp],
     "tq_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
@@ -81,6 +97,10 @@ _SIGS = {
     "tq_relu2_mul_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
     "tq_absmean_pack": [_vp, _vp, _vp, _i, _i, _vp],
     "tq_selftest_wait_timeout": [ctypes.c_uint, _vp],
+    "tq_hadamard_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_pack_binary_host": [_vp, _vp, _vp, _vp, _i, _i],
+    "tq_gemv_binary": [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_gemv_binary_stack": [ctypes.POINTER(TqBinaryProj), _i, _i, _vp],
 }
 _lib_handle = None
 
@@ -196,6 +216,37 @@ def tq_absmean_pack(w_bf16, packed, w_scale, N: int, K: int, stream=None) -> Non
 def tq_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     """A bounded wait that nothing satisfies: sets the device error word."""
     _check(_load().tq_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def tq_hadamard_quantize_act(x, xq, x_scale, x_sum, M: int, K: int, n: int,
+                             stream=None) -> None:
+    """Blockwise Hadamard rotation (block n) then 4-bit absmax codes (-7..7 in int8)."""
+    _check(_load().tq_hadamard_quantize_act(_ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, K,
+                                         int(n), _stream(stream)))
+
+
+def tq_pack_binary_host(w, scales, bits, scales_packed, N: int, K: int) -> None:
+    """Host packing of binary g128 weights: w int8 [N,K] in {-1,+1}, fp16 scales
+    [N,K/128] -> bits uint8 [N/8,K], scales_packed fp16 [N/8,K/128,8]."""
+    _check(_load().tq_pack_binary_host(_ptr(w), _ptr(scales), _ptr(bits), _ptr(scales_packed),
+                                    int(N), int(K)))
+
+
+def tq_gemv_binary(bits, scales_packed, xq, x_scale, y, acc_out, M: int, N: int, K: int,
+                   stream=None) -> None:
+    _check(_load().tq_gemv_binary(_ptr(bits), _ptr(scales_packed), _ptr(xq), _ptr(x_scale),
+                               _ptr(y), _ptr(acc_out), M, N, K, _stream(stream)))
+
+
+def make_binary_proj(bits=None, scales_packed=None, xq=None, x_scale=None, y=None, acc_out=None,
+                     N: int = 0, K: int = 0) -> TqBinaryProj:
+    return TqBinaryProj(_ptr(bits), _ptr(scales_packed), _ptr(xq), _ptr(x_scale), _ptr(y),
+                        _ptr(acc_out), int(N), int(K))
+
+
+def tq_gemv_binary_stack(projs, M: int, stream=None) -> None:
+    arr = (TqBinaryProj * len(projs))(*projs)
+    _check(_load().tq_gemv_binary_stack(arr, len(projs), int(M), _stream(stream)))
 
 
 def make_proj(packed=None, x=None, xq=None, x_scale=None, x_sum=None, y=None, acc_out=None,

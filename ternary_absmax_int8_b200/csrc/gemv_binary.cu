@@ -1,0 +1,551 @@
+// gemv_binary.cu -- decode GEMV over binary g128 weights (M <= 4 tokens), one
+// projection or a table of projections per launch.
+//
+// The format (baguaai "BitNet" tag page, Bonsai 27B item: a true 1-bit
+// binary scheme, 128 weights sharing one fp16 scale, about 1.125 bits per
+// weight), as this library stores it:
+//   bits   uint8 [N/8, K]: bit p of byte (i, k) is the weight of output row
+//          i + p N/8 at column k, 1 meaning +1 and 0 meaning -1 (the plane
+//          layout of the ternary format, eight planes instead of four);
+//   scales fp16 [N/8, K/128, 8]: entry (i, g, p) scales row i + p N/8 on
+//          columns 128 g .. 128 g + 127.
+// With int8 activations q (per-token absmax) and x_scale:
+//   S[n, g] = sum_{k in g} b[n, k] q[k],   Q[g] = sum_{k in g} q[k],
+//   acc[n, g] = 2 S[n, g] - Q[g]  (since w = 2 b - 1; exact int32),
+//   y[n] = fl32(x_scale * sum_g scale[n, g] acc[n, g]), the products exact in
+//   fp64 (an int32 below 2^15 times an fp16) and the sum in fp64 (exact unless
+//   a row's scales span more than ~2^20), so the order of the additions does
+//   not change the result.
+//
+// The weight stream is read once per token and dominates the bytes, so the
+// kernel streams like the ternary decode kernel: persistent CTAs, one per SM;
+// tiles of R whole packed rows (their bits and their scales, two 1-D bulk
+// copies through the TMA engine, no multicast) in a ring of shared-memory
+// stages guarded by mbarriers; two groups of eight consumer warps take
+// alternate tiles; the CTA's activations are resident in shared memory.
+//
+// Consumer arithmetic. A warp item is one packed row (or one of 2^lg pieces
+// of its groups); lane (seg, sub) = (lane >> 3, lane & 7) takes 16-byte chunk
+// `sub` of groups g0 + seg, g0 + seg + 4, ... For a 32-bit word u of bits
+// (four columns, eight planes per byte), dp4a of the nested masks
+// u & 0x01.., u & 0x03.., ..., u & 0x7F.. and u itself (unsigned bytes x
+// signed int8) gives the nested sums T_j = sum_{p <= j} 2^p S_p: seven logic
+// ops and eight dp4a per word. A transposing butterfly over the segment's
+// eight lanes (seven shuffles) leaves lane `sub` holding the group's T_sub;
+// with T_{sub-1} from its neighbour, S_sub = (T_sub - T_{sub-1}) >> sub.
+// Each lane so owns plane `sub` of its row: it scales the group's acc in
+// fp64 and adds, and after the row the four segments' sums are added.
+#include <atomic>
+#include <algorithm>
+#include <vector>
+
+#include <cuda_fp16.h>
+
+#include "tq_internal.h"
+
+namespace tq {
+
+namespace {
+
+constexpr int kBinW = 8;                  // consumer warps per group
+constexpr int kBinG = 2;                  // groups (take alternate tiles)
+constexpr int kBinWC = kBinW * kBinG;     // consumer warps
+constexpr int kBinMaxStages = 8;
+constexpr int kBinMaxRows = 16;           // packed rows per tile
+constexpr int kBinSplitRows = 4;          // rows per tile when rows are cut into pieces
+constexpr int kBinTileBytes = 40960;      // bit bytes per tile, aim
+constexpr int kBinGroup = 128;
+
+struct BinStageDesc {
+    int entry, row0, rows, pad_;
+};
+
+template <int MT>
+struct BinTail {
+    static constexpr int kDesc = kBinMaxStages * int(sizeof(BinStageDesc));
+    static constexpr int kBars = 2 * kBinMaxStages + 1;
+    static constexpr int kSlots = kBinMaxStages * kBinSplitRows * MT * 8;
+    static constexpr int kCnt = kBinMaxStages * kBinSplitRows;
+    static constexpr size_t bytes()
+    {
+        return kDesc + kBars * 8 + size_t(kSlots) * 8 + size_t(kSlots) * 4 + size_t(kCnt) * 4 + 64;
+    }
+};
+
+// Eight int32 values per lane over the eight lanes of a segment: on return
+// lane `sub` holds the segment's total of value `sub` (seven shuffles).
+__device__ __forceinline__ int32_t transpose_reduce8(const int32_t (&v)[8], int sub)
+{
+    const bool b2 = sub & 4, b1 = sub & 2, b0 = sub & 1;
+    int32_t k[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int32_t keep = b2 ? v[4 + i] : v[i];
+        const int32_t send = b2 ? v[i] : v[4 + i];
+        k[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    int32_t l[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int32_t keep = b1 ? k[2 + i] : k[i];
+        const int32_t send = b1 ? k[i] : k[2 + i];
+        l[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    const int32_t keep = b0 ? l[1] : l[0];
+    const int32_t send = b0 ? l[0] : l[1];
+    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+
+// Nested-mask sums of one 16-byte chunk of bits against 16 activations.
+__device__ __forceinline__ void dot_bits16(const uint4 w, const uint4 x, int32_t (&t)[8])
+{
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        t[0] = dp4a_us(ws[j] & 0x01010101u, xs[j], t[0]);
+        t[1] = dp4a_us(ws[j] & 0x03030303u, xs[j], t[1]);
+        t[2] = dp4a_us(ws[j] & 0x07070707u, xs[j], t[2]);
+        t[3] = dp4a_us(ws[j] & 0x0F0F0F0Fu, xs[j], t[3]);
+        t[4] = dp4a_us(ws[j] & 0x1F1F1F1Fu, xs[j], t[4]);
+        t[5] = dp4a_us(ws[j] & 0x3F3F3F3Fu, xs[j], t[5]);
+        t[6] = dp4a_us(ws[j] & 0x7F7F7F7Fu, xs[j], t[6]);
+        t[7] = dp4a_us(ws[j], xs[j], t[7]);
+    }
+}
+
+template <int MaxE, int MT>
+__global__ void __launch_bounds__((kBinWC + 1) * 32, 1)
+binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int t_begin = p.cta_tile0[blockIdx.x], t_end = p.cta_tile0[blockIdx.x + 1];
+    const int e_first = p.cta_entry0[blockIdx.x];
+    const int n_ent = p.cta_nent[blockIdx.x];
+    BinEntry *tab = reinterpret_cast<BinEntry *>(smem);
+    float *xsc = reinterpret_cast<float *>(tab + n_ent);  // [n_ent][MT]
+    int *xoff = reinterpret_cast<int *>(xsc + n_ent * MT);
+    int *qoff = xoff + n_ent;
+    uint8_t *xcache = smem + p.head_bytes;
+    int32_t *qsum = reinterpret_cast<int32_t *>(xcache + p.x_slot);
+    uint8_t *ring = xcache + p.x_slot + p.q_slot;
+    BinStageDesc *desc = reinterpret_cast<BinStageDesc *>(ring + size_t(p.stages) * p.w_slot);
+    uint64_t *full = reinterpret_cast<uint64_t *>(desc + kBinMaxStages);
+    uint64_t *empty = full + kBinMaxStages;
+    uint64_t *xbar = empty + kBinMaxStages;
+    double *dpart = reinterpret_cast<double *>(xbar + 1);
+    int32_t *ipart = reinterpret_cast<int32_t *>(dpart + BinTail<MT>::kSlots);
+    int32_t *cnt = ipart + BinTail<MT>::kSlots;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    for (int i = threadIdx.x; i < BinTail<MT>::kSlots; i += blockDim.x) {
+        dpart[i] = 0.0;
+        ipart[i] = 0;
+    }
+    for (int i = threadIdx.x; i < BinTail<MT>::kCnt; i += blockDim.x)
+        cnt[i] = 0;
+    {
+        static_assert(sizeof(BinEntry) % 8 == 0, "entry size");
+        const uint64_t *src = reinterpret_cast<const uint64_t *>(&p.e[e_first]);
+        uint64_t *dst = reinterpret_cast<uint64_t *>(tab);
+        const int n64 = n_ent * int(sizeof(BinEntry) / 8);
+        for (int i = threadIdx.x; i < n64; i += blockDim.x)
+            dst[i] = src[i];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int xo = 0, qo = 0;
+        for (int j = 0; j < n_ent; ++j) {
+            xoff[j] = xo;
+            qoff[j] = qo;
+            xo += (p.M * tab[j].K + 127) & ~127;
+            qo += p.M * (tab[j].K / kBinGroup);
+        }
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kBinW);
+        }
+        mbar_init(xbar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kBinWC) {
+        // ------------------------------------------------------ producer
+        if (lane != 0)
+            return;
+        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_x = policy_evict_last();
+        if (t_end > t_begin) {
+            uint32_t total = 0;
+            for (int j = 0; j < n_ent; ++j)
+                total += uint32_t(p.M * tab[j].K);
+            mbar_arrive_expect_tx(xbar, total);
+            for (int j = 0; j < n_ent; ++j)
+                bulk_g2s(xcache + xoff[j], tab[j].xq, uint32_t(p.M * tab[j].K), xbar, pol_x);
+        } else {
+            mbar_arrive(xbar);
+        }
+        int cursor = 0, it = 0, stage = 0;
+        uint32_t phase = 0;
+        for (int t = t_begin; t < t_end; ++t, ++it) {
+            while (cursor + 1 < n_ent && tab[cursor + 1].tile_begin <= t)
+                ++cursor;
+            const BinEntry &e = tab[cursor];
+            const int K = e.K, ng = K / kBinGroup;
+            const int row0 = (t - e.tile_begin) * e.rows_per_tile;
+            const int rows = min(e.rows_per_tile, e.N8 - row0);
+            if (it >= p.stages && !mbar_wait(&empty[stage], phase ^ 1u, p.err))
+                break;
+            const uint32_t bbytes = uint32_t(rows) * uint32_t(K);
+            const uint32_t sbytes = uint32_t(rows) * uint32_t(ng) * 16u;
+            desc[stage] = BinStageDesc{cursor, row0, rows, 0};
+            uint8_t *dst = ring + size_t(stage) * p.w_slot;
+            mbar_arrive_expect_tx(&full[stage], bbytes + sbytes);
+            bulk_g2s(dst, e.bits + size_t(row0) * K, bbytes, &full[stage], pol_w);
+            bulk_g2s(dst + size_t(e.rows_per_tile) * K, e.scales + size_t(row0) * ng * 8, sbytes,
+                     &full[stage], pol_w);
+            if (++stage == p.stages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        // Do not retire while a copy this thread issued is in flight.
+        for (int s = 0; s < p.stages; ++s) {
+            if (s < stage)
+                mbar_wait(&full[s], phase, p.err);
+            else if (it >= p.stages)
+                mbar_wait(&full[s], phase ^ 1u, p.err);
+        }
+        mbar_wait(xbar, 0, p.err);
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    if (t_end > t_begin && !mbar_wait_warp(xbar, 0, p.err))
+        return;
+    // Per token and group, Q[g] = sum of the group's 128 codes.
+    for (int j = 0; j < n_ent; ++j) {
+        const int K = tab[j].K, ng = K / kBinGroup;
+        for (int i = threadIdx.x; i < p.M * ng; i += kBinWC * 32) {
+            const int m = i / ng, g = i - m * ng;
+            const uint4 *xv = reinterpret_cast<const uint4 *>(xcache + xoff[j] + m * K + g * kBinGroup);
+            int32_t s = 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = xv[c];
+                s = __dp4a(int(v.x), 0x01010101, s);
+                s = __dp4a(int(v.y), 0x01010101, s);
+                s = __dp4a(int(v.z), 0x01010101, s);
+                s = __dp4a(int(v.w), 0x01010101, s);
+            }
+            qsum[qoff[j] + i] = s;
+        }
+        for (int m = threadIdx.x; m < p.M; m += kBinWC * 32)
+            xsc[j * MT + m] = __ldg(tab[j].x_scale + m);
+    }
+    named_bar_sync(1, kBinWC * 32);
+
+    const int grp = warp / kBinW, wg = warp - grp * kBinW;
+    const int seg = lane >> 3, sub = lane & 7;
+    int stage = grp;  // stages % kBinG == 0: the group keeps to stages grp + k G
+    uint32_t phase = 0;
+    int rot = 0;
+    for (int t = t_begin + grp; t < t_end; t += kBinG) {
+        if (!mbar_wait_warp(&full[stage], phase, p.err))
+            return;
+        const BinStageDesc d = desc[stage];
+        const BinEntry &e = tab[d.entry];
+        const int K = e.K, ng = K / kBinGroup, N8 = e.N8;
+        const int lg = e.lg;
+        const uint8_t *sb = ring + size_t(stage) * p.w_slot;
+        const __half *ss = reinterpret_cast<const __half *>(sb + size_t(e.rows_per_tile) * K);
+        const uint8_t *sx = xcache + xoff[d.entry];
+        const int32_t *sq = qsum + qoff[d.entry];
+        float xs[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+            xs[m] = m < p.M ? xsc[d.entry * MT + m] : 0.0f;
+
+        const int n_items = d.rows << lg;
+        bool released = false;
+        const int first_item = (wg - rot + kBinW) % kBinW;
+        const int last_item = n_items - 1 - ((n_items - 1 - first_item) % kBinW + kBinW) % kBinW;
+        rot = (rot + n_items) % kBinW;
+        for (int item = first_item; item < n_items; item += kBinW) {
+            const int r = item >> lg, piece = item & ((1 << lg) - 1);
+            const int g0 = (piece * ng) >> lg, g1 = ((piece + 1) * ng) >> lg;
+            const uint8_t *wrow = sb + size_t(r) * K;
+            double accd[MT];
+            int32_t itot[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                accd[m] = 0.0;
+                itot[m] = 0;
+            }
+            for (int gb = g0; gb < g1; gb += 4) {
+                const int g = gb + seg;
+                const bool valid = g < g1;
+                int32_t tt[MT][8];
+#pragma unroll
+                for (int m = 0; m < MT; ++m)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        tt[m][j] = 0;
+                if (valid) {
+                    const uint4 wv =
+                        *reinterpret_cast<const uint4 *>(wrow + g * kBinGroup + sub * 16);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        if (MT == 1 || m < p.M) {
+                            const uint4 xv = *reinterpret_cast<const uint4 *>(
+                                sx + m * K + g * kBinGroup + sub * 16);
+                            dot_bits16(wv, xv, tt[m]);
+                        }
+                }
+                const float scf = valid ? __half2float(ss[(r * ng + g) * 8 + sub]) : 0.0f;
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (MT == 1 || m < p.M) {
+                        const int32_t tsub = transpose_reduce8(tt[m], sub);
+                        int32_t tprev = __shfl_up_sync(0xffffffffu, tsub, 1, 8);
+                        if (sub == 0)
+                            tprev = 0;
+                        if (valid) {
+                            const int32_t s_p = (tsub - tprev) >> sub;  // exact: a multiple of 2^sub
+                            const int32_t a = 2 * s_p - sq[m * ng + g];
+                            itot[m] += a;
+                            accd[m] = __dadd_rn(accd[m], __dmul_rn(double(a), double(scf)));
+                        }
+                    }
+                }
+            }
+            if (lg == 0 && item == last_item) {
+                // last read of the stage by this warp (split rows still
+                // read nothing more from it either, but keep their slots)
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[stage]);
+                released = true;
+            }
+            // add the four segments' sums: every lane then holds plane sub's
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (MT == 1 || m < p.M) {
+                    accd[m] = __dadd_rn(accd[m], __shfl_xor_sync(0xffffffffu, accd[m], 8));
+                    accd[m] = __dadd_rn(accd[m], __shfl_xor_sync(0xffffffffu, accd[m], 16));
+                    itot[m] += __shfl_xor_sync(0xffffffffu, itot[m], 8);
+                    itot[m] += __shfl_xor_sync(0xffffffffu, itot[m], 16);
+                }
+            }
+            const int row = d.row0 + r;
+            const size_t n_out = size_t(row) + size_t(sub) * N8;
+            if (lg == 0) {
+                if (seg == 0) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        if (MT == 1 || m < p.M) {
+                            const size_t o = size_t(m) * (8 * size_t(N8)) + n_out;
+                            e.y[o] = __double2float_rn(__dmul_rn(accd[m], double(xs[m])));
+                            if (e.acc_out)
+                                e.acc_out[o] = itot[m];
+                        }
+                    }
+                }
+            } else {
+                const int slot = (stage * kBinSplitRows + r) * MT;
+                if (seg == 0) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        if (MT == 1 || m < p.M) {
+                            atomicAdd(&dpart[(slot + m) * 8 + sub], accd[m]);
+                            atomicAdd(&ipart[(slot + m) * 8 + sub], itot[m]);
+                        }
+                }
+                __threadfence_block();  // partial sums before the count
+                __syncwarp();
+                int old = 0;
+                if (lane == 0)
+                    old = atomicAdd(&cnt[stage * kBinSplitRows + r], 1);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old == (1 << lg) - 1) {
+                    // the last piece of this row: finish it
+                    __threadfence_block();
+                    if (seg == 0) {
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+                            if (MT == 1 || m < p.M) {
+                                volatile double *dv = dpart + (slot + m) * 8 + sub;
+                                const double v = *dv;
+                                *dv = 0.0;
+                                const int32_t iv = atomicExch(&ipart[(slot + m) * 8 + sub], 0);
+                                const size_t o = size_t(m) * (8 * size_t(N8)) + n_out;
+                                e.y[o] = __double2float_rn(__dmul_rn(v, double(xs[m])));
+                                if (e.acc_out)
+                                    e.acc_out[o] = iv;
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        cnt[stage * kBinSplitRows + r] = 0;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && !released)
+            mbar_arrive(&empty[stage]);
+        stage += kBinG;
+        if (stage >= p.stages) {
+            stage -= p.stages;
+            phase ^= 1u;
+        }
+    }
+}
+
+template <int MaxE, int MT>
+cudaError_t launch_bin_instance(const BinParams<MaxE> &p, int grid, size_t smem,
+                                cudaStream_t stream)
+{
+    auto kern = binary_gemv_kernel<MaxE, MT>;
+    static std::atomic<int> configured_dev{-1};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (configured_dev != dev) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (err != cudaSuccess)
+            return err;
+        configured_dev = dev;
+    }
+    kern<<<grid, (kBinWC + 1) * 32, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int MaxE>
+cudaError_t launch_bin_sized(BinEntry *entries, int n, int M, cudaStream_t stream)
+{
+    BinParams<MaxE> p;
+    static_assert(sizeof(BinParams<MaxE>) <= 32000, "kernel parameters exceed 32 KB");
+    const int sms = std::min(device_sm_count(), kBinMaxGrid);
+    const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);
+    int total = 0;
+    size_t w_slot = 0;
+    for (int j = 0; j < n; ++j) {
+        BinEntry &e = entries[j];
+        const int K = e.K, ng = K / kBinGroup;
+        int R = kBinMaxRows;
+        while (R > 1 && R * K > kBinTileBytes)
+            R >>= 1;
+        // Cut rows into pieces of their groups when a tile has fewer rows
+        // than a group has warps (at least four groups per piece).
+        int lg = 0;
+        while ((R << lg) < kBinW && (ng >> (lg + 1)) >= 4)
+            ++lg;
+        if (lg > 0 && R > kBinSplitRows)
+            return cudaErrorInvalidValue;  // not reached: lg > 0 only when R < kBinW / 2
+        e.rows_per_tile = R;
+        e.lg = lg;
+        e.tile_begin = total;
+        total += (e.N8 + R - 1) / R;
+        w_slot = std::max(w_slot, (size_t(R) * K + 127) / 128 * 128 +
+                                      (size_t(R) * ng * 16 + 127) / 128 * 128);
+        p.e[j] = e;
+    }
+    if (total == 0)
+        return cudaSuccess;
+    p.n_entries = n;
+    p.total_tiles = total;
+    p.M = M;
+    p.w_slot = int(w_slot);
+    const int grid = std::min(total, sms);
+    // contiguous tile ranges per CTA, balanced by bytes (plus a fixed cost per tile)
+    std::vector<long long> prefix(size_t(total) + 1, 0);
+    {
+        int t = 0;
+        for (int j = 0; j < n; ++j) {
+            const BinEntry &e = p.e[j];
+            const int tiles = (e.N8 + e.rows_per_tile - 1) / e.rows_per_tile;
+            for (int i = 0; i < tiles; ++i, ++t) {
+                const int rows = std::min(e.rows_per_tile, e.N8 - i * e.rows_per_tile);
+                prefix[size_t(t) + 1] = prefix[size_t(t)] + (long long)rows * e.K * 9 / 8 + 4096;
+            }
+        }
+    }
+    p.cta_tile0[0] = 0;
+    for (int b = 1; b < grid; ++b) {
+        const long long target = prefix[size_t(total)] * b / grid;
+        int t = int(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
+        t = std::max(t, p.cta_tile0[b - 1] + 1);
+        t = std::min(t, total - (grid - b));
+        p.cta_tile0[b] = t;
+    }
+    p.cta_tile0[grid] = total;
+    int max_local = 1;
+    size_t x_max = 0, q_max = 0;
+    for (int b = 0; b < grid; ++b) {
+        auto entry_of = [&](int t) {
+            int lo = 0, hi = n - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) / 2;
+                if (p.e[mid].tile_begin <= t)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            return lo;
+        };
+        const int e0 = entry_of(p.cta_tile0[b]);
+        const int e1 = entry_of(p.cta_tile0[b + 1] - 1);
+        p.cta_entry0[b] = e0;
+        p.cta_nent[b] = e1 - e0 + 1;
+        max_local = std::max(max_local, e1 - e0 + 1);
+        size_t xb = 0, qb = 0;
+        for (int j = e0; j <= e1; ++j) {
+            xb += (size_t(M) * p.e[j].K + 127) / 128 * 128;
+            qb += size_t(M) * (p.e[j].K / kBinGroup) * 4;
+        }
+        x_max = std::max(x_max, xb);
+        q_max = std::max(q_max, qb);
+    }
+    p.x_slot = int(x_max);
+    p.q_slot = int((q_max + 127) / 128 * 128);
+    p.head_bytes = int((size_t(max_local) * (sizeof(BinEntry) + size_t(mt) * 4 + 8) + 127) / 128 * 128);
+    p.err = device_error_word();
+    if (!p.err)
+        return cudaErrorUnknown;
+    const size_t tail = mt == 1 ? BinTail<1>::bytes()
+                                : (mt == 2 ? BinTail<2>::bytes() : BinTail<4>::bytes());
+    const size_t fixed = size_t(p.head_bytes) + p.x_slot + p.q_slot + tail;
+    const size_t budget = 227 * 1024;
+    int stages = budget > fixed ? int((budget - fixed) / w_slot) : 0;
+    stages = std::min(stages, kBinMaxStages);
+    // each consumer group must see every phase of the stages it uses
+    stages -= stages % kBinG;
+    if (stages < kBinG)
+        return cudaErrorInvalidValue;
+    p.stages = stages;
+    const size_t smem = fixed + size_t(stages) * w_slot;
+    switch (mt) {
+    case 1: return launch_bin_instance<MaxE, 1>(p, grid, smem, stream);
+    case 2: return launch_bin_instance<MaxE, 2>(p, grid, smem, stream);
+    default: return launch_bin_instance<MaxE, 4>(p, grid, smem, stream);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_binary_gemv(BinEntry *entries, int n, int M, cudaStream_t stream)
+{
+    if (n <= 0)
+        return cudaSuccess;
+    if (M < 1 || M > kBinMaxTokens || n > kBinStackMax)
+        return cudaErrorInvalidValue;
+    if (n == 1)
+        return launch_bin_sized<1>(entries, n, M, stream);
+    return launch_bin_sized<kBinStackMax>(entries, n, M, stream);
+}
+
+}  // namespace tq

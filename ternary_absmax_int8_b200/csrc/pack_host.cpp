@@ -37,3 +37,41 @@ bool pack_ternary_host(const int8_t *w, uint8_t *packed, int N, int K)
 }
 
 }  // namespace tq
+
+namespace tq {
+
+// Binary g128 packing (baguaai "BitNet" tag page, Bonsai 27B item: one bit
+// per weight, 128 weights sharing one fp16 scale). Layout (not given on the
+// page): bits [N/8, K], bit p of byte (i, k) = weight of row i + p*N/8 at
+// column k, 1 for +1 and 0 for -1; the fp16 scales [N, K/128] are regrouped
+// as [N/8, K/128, 8] so that a packed row's tile carries the eight scales of
+// each of its groups in 16 contiguous bytes. Returns false if some weight is
+// not -1 or +1.
+bool pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
+                      uint16_t *scales_packed, int N, int K)
+{
+    const size_t Q = size_t(N) / 8;
+    const size_t Ks = size_t(K);
+    const size_t G = Ks / 128;
+    unsigned bad = 0;
+    for (size_t i = 0; i < Q; ++i) {
+        uint8_t *out = bits + i * Ks;
+        for (size_t k = 0; k < Ks; ++k)
+            out[k] = 0;
+        for (unsigned p = 0; p < 8; ++p) {
+            const int8_t *wr = w + (i + p * Q) * Ks;
+            for (size_t k = 0; k < Ks; ++k) {
+                const int v = wr[k];
+                bad |= unsigned(v != 1 && v != -1);
+                out[k] = uint8_t(out[k] | (unsigned(v == 1) << p));
+            }
+            for (size_t g = 0; g < G; ++g)
+                scales_packed[(i * G + g) * 8 + p] = scales[(i + p * Q) * G + g];
+        }
+        if (bad)
+            return false;
+    }
+    return true;
+}
+
+}  // namespace tq

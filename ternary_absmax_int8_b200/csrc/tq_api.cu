@@ -17,6 +17,8 @@ namespace tq {
 __device__ unsigned int g_device_error = 0;
 
 bool pack_ternary_host(const int8_t *w, uint8_t *packed, int N, int K);
+bool pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
+                      uint16_t *scales_packed, int N, int K);
 cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
                               const float *x_scale, const int32_t *x_sum, float *y,
                               int32_t *acc_out, int M, int N, int K, cudaStream_t stream,
@@ -554,6 +556,129 @@ tq_status tq_absmean_pack(const uint16_t *w_bf16, uint8_t *packed, float *w_scal
         return fail(TQ_ERR_ALIGN, "tq_absmean_pack: weights and packed bytes 16-byte aligned");
     cudaError_t e = tq::launch_absmean_pack(w_bf16, packed, w_scale, N, K, stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "tq_absmean_pack");
+}
+
+tq_status tq_hadamard_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
+                                   int M, int K, int n, cudaStream_t stream)
+{
+    const char *fn = "tq_hadamard_quantize_act";
+    if (M < 0 || K < 0)
+        return fail(TQ_ERR_SHAPE, "%s: negative size (M=%d K=%d)", fn, M, K);
+    if (n < 32 || n > 1024 || (n & (n - 1)) != 0 || K % n != 0)
+        return fail(TQ_ERR_SHAPE, "%s: block size n=%d must be a power of two in 32..1024 dividing K=%d",
+                    fn, n, K);
+    if (M == 0 || K == 0)
+        return ok();
+    if (K > tq::kStreamMaxK)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: K=%d exceeds %d", fn, K, tq::kStreamMaxK);
+    if (!x || !xq || !x_scale)
+        return fail(TQ_ERR_NULL, "%s: a required pointer is NULL", fn);
+    if (!aligned(x, 16) || !aligned(xq, 16) || !aligned(x_scale, 4) || (x_sum && !aligned(x_sum, 4)))
+        return fail(TQ_ERR_ALIGN, "%s: x and xq 16-byte aligned, vectors 4-byte aligned", fn);
+    cudaError_t e = tq::launch_hadamard_quant4(x, xq, x_scale, x_sum, M, K, n, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, fn);
+}
+
+tq_status tq_pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
+                              uint16_t *scales_packed, int N, int K)
+{
+    if (N < 0 || K < 0 || N % 8 != 0 || K % 128 != 0)
+        return fail(TQ_ERR_SHAPE, "tq_pack_binary_host: N=%d K=%d (need N %% 8 == 0, K %% 128 == 0)",
+                    N, K);
+    if (N == 0 || K == 0)
+        return ok();
+    if (!w || !scales || !bits || !scales_packed)
+        return fail(TQ_ERR_NULL, "tq_pack_binary_host: a required pointer is NULL");
+    if (!tq::pack_binary_host(w, scales, bits, scales_packed, N, K))
+        return fail(TQ_ERR_VALUE, "tq_pack_binary_host: a weight is not -1 or +1");
+    return ok();
+}
+
+namespace {
+
+tq_status check_binary_args(const char *fn, const tq_binary_proj &p, int M)
+{
+    if (M < 0 || p.N < 0 || p.K < 0)
+        return fail(TQ_ERR_SHAPE, "%s: negative size (M=%d N=%d K=%d)", fn, M, p.N, p.K);
+    if (p.N % 8 != 0 || p.K % 128 != 0)
+        return fail(TQ_ERR_SHAPE, "%s: N=%d K=%d (need N %% 8 == 0, K %% 128 == 0)", fn, p.N, p.K);
+    if (M > tq::kBinMaxTokens)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: M=%d (1..%d tokens)", fn, M, tq::kBinMaxTokens);
+    if (M == 0 || p.N == 0)
+        return TQ_OK;
+    if (!p.y || (p.K > 0 && (!p.bits || !p.scales_packed || !p.xq || !p.x_scale)))
+        return fail(TQ_ERR_NULL, "%s: a required pointer is NULL", fn);
+    if ((p.bits && !aligned(p.bits, 16)) || (p.scales_packed && !aligned(p.scales_packed, 16)) ||
+        (p.xq && !aligned(p.xq, 16)))
+        return fail(TQ_ERR_ALIGN, "%s: bits, scales and xq must be 16-byte aligned", fn);
+    if ((p.x_scale && !aligned(p.x_scale, 4)) || !aligned(p.y, 4) ||
+        (p.acc_out && !aligned(p.acc_out, 4)))
+        return fail(TQ_ERR_ALIGN, "%s: x_scale, y, acc_out must be 4-byte aligned", fn);
+    if (p.K > tq::kStreamMaxK)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: K=%d exceeds %d", fn, p.K, tq::kStreamMaxK);
+    return TQ_OK;
+}
+
+tq::BinEntry bin_entry(const tq_binary_proj &p)
+{
+    tq::BinEntry e = {};
+    e.bits = p.bits;
+    e.scales = p.scales_packed;
+    e.xq = p.xq;
+    e.x_scale = p.x_scale;
+    e.y = p.y;
+    e.acc_out = p.acc_out;
+    e.N8 = p.N / 8;
+    e.K = p.K;
+    return e;
+}
+
+}  // namespace
+
+tq_status tq_gemv_binary_stack(const tq_binary_proj *projs, int n_proj, int M, cudaStream_t stream)
+{
+    const char *fn = "tq_gemv_binary_stack";
+    if (n_proj < 0 || (n_proj > 0 && !projs))
+        return fail(TQ_ERR_NULL, "%s: projs is NULL", fn);
+    std::vector<tq::BinEntry> list;
+    list.reserve(size_t(n_proj));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_status st = check_binary_args(fn, projs[j], M);
+        if (st != TQ_OK)
+            return st;
+    }
+    if (M == 0)
+        return ok();
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_binary_proj &p = projs[j];
+        if (p.N == 0)
+            continue;
+        if (p.K == 0) {
+            const tq_status st = zero_outputs(p.y, p.acc_out, size_t(M) * p.N, stream);
+            if (st != TQ_OK)
+                return st;
+            continue;
+        }
+        list.push_back(bin_entry(p));
+    }
+    for (size_t base = 0; base < list.size(); base += tq::kBinStackMax) {
+        const int n = int(std::min(list.size() - base, size_t(tq::kBinStackMax)));
+        cudaError_t e = tq::launch_binary_gemv(list.data() + base, n, M, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fn);
+    }
+    return ok();
+}
+
+tq_status tq_gemv_binary(const uint8_t *bits, const uint16_t *scales_packed, const int8_t *xq,
+                         const float *x_scale, float *y, int32_t *acc_out, int M, int N, int K,
+                         cudaStream_t stream)
+{
+    const tq_binary_proj p = {bits, scales_packed, xq, x_scale, y, acc_out, N, K};
+    const tq_status st = check_binary_args("tq_gemv_binary", p, M);
+    if (st != TQ_OK)
+        return st;
+    return tq_gemv_binary_stack(&p, 1, M, stream);
 }
 
 tq_status tq_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream)

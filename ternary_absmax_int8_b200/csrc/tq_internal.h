@@ -151,6 +151,47 @@ cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f
 cudaError_t launch_absmean_pack(const uint16_t *w, uint8_t *packed, float *w_scale, int N, int K,
                                 cudaStream_t stream);
 
+// ------------------------------------------- Hadamard-rotated 4-bit codes
+// One CTA per token row; n (the rotation's block size) in {32, ..., 1024}
+// dividing K (cudaErrorInvalidValue otherwise).
+cudaError_t launch_hadamard_quant4(const uint16_t *x, int8_t *xq, float *x_scale,
+                                   int32_t *x_sum, int M, int K, int n, cudaStream_t stream);
+
+// --------------------------------------------- binary g128 GEMV (M <= 4)
+// One entry = one projection: bits uint8 [N8, K] (bit p of byte (i, k) = row
+// i + p N8, 1 = +1), scales fp16 [N8, K/128, 8]. Tiles of rows_per_tile whole
+// packed rows; each row is cut into 2^lg pieces of its groups.
+struct BinEntry {
+    const uint8_t *bits;
+    const uint16_t *scales;
+    const int8_t *xq;       // [M, K]
+    const float *x_scale;   // [M]
+    float *y;               // [M, 8 N8]
+    int32_t *acc_out;       // [M, 8 N8] or null: sum_k w q
+    int N8, K;
+    int rows_per_tile, lg, tile_begin, pad_;
+};
+
+constexpr int kBinMaxTokens = 4;
+constexpr int kBinStackMax = 128;   // entries per launch
+constexpr int kBinMaxGrid = 160;    // CTAs per launch
+
+template <int MaxE>
+struct BinParams {
+    int n_entries, total_tiles, M, stages;
+    int w_slot;      // bytes of a ring stage (a tile's bits, then its scales)
+    int x_slot;      // bytes of the CTA's resident activations
+    int q_slot;      // bytes of the per-token group sums of the activations
+    int head_bytes;  // shared memory for the entry table and per-entry offsets
+    unsigned *err;
+    int cta_tile0[kBinMaxGrid + 1];
+    int cta_entry0[kBinMaxGrid];
+    int cta_nent[kBinMaxGrid];
+    BinEntry e[MaxE];
+};
+
+cudaError_t launch_binary_gemv(BinEntry *entries, int n, int M, cudaStream_t stream);
+
 // Device address of the library's error word on the current device.
 unsigned *device_error_word();
 

@@ -256,3 +256,118 @@ def test_header_is_c_and_struct_layout_matches_binding(tmp_path):
     T = tq.TqProj
     assert got == [ctypes.sizeof(T), T.w_scale.offset, T.K.offset, T.gain.offset,
                    T.eps.offset, T.reserved.offset]
+
+
+# ------------------------------------------------------ binary g128, Hadamard
+@pytest.mark.parametrize("N,K", [(8, 128), (64, 256), (5120, 384)])
+def test_binary_host_packer_matches_oracle_and_scale_layout(N, K):
+    from workloads import make_binary_projections
+    p = next(make_binary_projections([("b", N, K)], M=1, seed=N + K))
+    bits = np.zeros((N // 8, K), np.uint8)
+    sp = np.zeros((N // 8, K // 128, 8), np.uint16)
+    tq.tq_pack_binary_host(p.w, p.s_f16, bits, sp, N, K)
+    assert (bits == oracle.pack_binary(p.w)).all()
+    # entry (i, g, p) is the scale of row i + p N/8 on group g
+    Q = N // 8
+    for i in (0, Q // 2, Q - 1):
+        for pl in range(8):
+            assert (sp[i, :, pl] == p.s_f16[i + pl * Q]).all()
+
+
+def test_binary_host_packer_rejects_bad_input():
+    w = np.ones((8, 128), np.int8)
+    s = np.zeros((8, 1), np.uint16)
+    bits = np.zeros((1, 128), np.uint8)
+    sp = np.zeros((1, 1, 8), np.uint16)
+    w[3, 7] = 0
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_pack_binary_host(w, s, bits, sp, 8, 128)
+    assert e.value.name == "TQ_ERR_VALUE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_pack_binary_host(w, s, bits, sp, 8, 64)  # K % 128
+    assert e.value.name == "TQ_ERR_SHAPE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_pack_binary_host(w, s, bits, sp, 4, 128)  # N % 8
+    assert e.value.name == "TQ_ERR_SHAPE"
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_pack_binary_host(w, None, bits, sp, 8, 128)
+    assert e.value.name == "TQ_ERR_NULL"
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(N=12), "TQ_ERR_SHAPE"),
+    (dict(K=192), "TQ_ERR_SHAPE"),
+    (dict(M=5), "TQ_ERR_UNSUPPORTED"),
+    (dict(K=32768 + 128), "TQ_ERR_UNSUPPORTED"),
+    (dict(bits=None), "TQ_ERR_NULL"),
+    (dict(y=None), "TQ_ERR_NULL"),
+    (dict(bits=A + 8), "TQ_ERR_ALIGN"),
+    (dict(scales_packed=A + 4), "TQ_ERR_ALIGN"),
+    (dict(y=A + 2), "TQ_ERR_ALIGN"),
+])
+def test_binary_gemv_argument_checks(kw, status):
+    args = dict(bits=A, scales_packed=A, xq=A, x_scale=A, y=A, acc_out=None, M=1, N=640, K=2560)
+    args.update(kw)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_binary(args["bits"], args["scales_packed"], args["xq"], args["x_scale"],
+                          args["y"], args["acc_out"], args["M"], args["N"], args["K"], stream=0)
+    assert e.value.name == status
+    # the stack call checks every entry the same way
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_gemv_binary_stack([tq.make_binary_proj(**{k: v for k, v in args.items()
+                                                        if k != "M"})], args["M"], stream=0)
+    assert e.value.name == status
+
+
+def test_binary_noops():
+    tq.tq_gemv_binary(None, None, None, None, None, None, 0, 640, 2560, stream=0)  # M = 0
+    tq.tq_gemv_binary(None, None, None, None, None, None, 1, 0, 2560, stream=0)    # N = 0
+    tq.tq_gemv_binary_stack([], 1, stream=0)
+
+
+def test_binary_proj_layout_matches_header(tmp_path):
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "tq.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu %zu %zu\\n", sizeof(tq_binary_proj), offsetof(tq_binary_proj, N),\n'
+        "         offsetof(tq_binary_proj, K));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), "-isystem", cuda_inc,
+                    str(src), "-o", str(exe)], check=True, capture_output=True)
+    got = [int(v) for v in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    T = tq.TqBinaryProj
+    assert got == [ctypes.sizeof(T), T.N.offset, T.K.offset] == [56, 48, 52]
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n=48), "TQ_ERR_SHAPE"),
+    (dict(n=16), "TQ_ERR_SHAPE"),
+    (dict(n=2048), "TQ_ERR_SHAPE"),
+    (dict(K=2560, n=1024), "TQ_ERR_SHAPE"),   # 1024 does not divide 2560
+    (dict(K=65536, n=256), "TQ_ERR_UNSUPPORTED"),
+    (dict(x=None), "TQ_ERR_NULL"),
+    (dict(xq=A + 8), "TQ_ERR_ALIGN"),
+    (dict(M=-1), "TQ_ERR_SHAPE"),
+])
+def test_hadamard_quantize_argument_checks(kw, status):
+    args = dict(x=A, xq=A, x_scale=A, x_sum=A, M=4, K=2560, n=256)
+    args.update(kw)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_hadamard_quantize_act(args["x"], args["xq"], args["x_scale"], args["x_sum"],
+                                    args["M"], args["K"], args["n"], stream=0)
+    assert e.value.name == status
+
+
+def test_hadamard_quantize_noops():
+    tq.tq_hadamard_quantize_act(None, None, None, None, 0, 2560, 256, stream=0)
+    tq.tq_hadamard_quantize_act(None, None, None, None, 3, 0, 256, stream=0)

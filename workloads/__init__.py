@@ -210,10 +210,14 @@ WORKLOADS = {
 for _m in SMALL_M_VALUES:
     WORKLOADS[f"ffn_m{_m}"] = (list(SMALL_M_SHAPES), _m)
 WORKLOADS["prefill_m512"] = (list(PREFILL_SHAPES), PREFILL_M)
-# the same contraction with Hadamard-rotated 4-bit activations
-WORKLOADS["prefill_had4_m512"] = (list(PREFILL_SHAPES), PREFILL_M)
-# binary g128 weights: 8 layers of the 27B-scale FFN, 301 MB per pass
-WORKLOADS["binary_ffn27b_m1"] = (binary_stack_shapes(BINARY_LAYERS), 1)
+
+# Workloads of the other two paths, (shapes, M): the prefill contraction with
+# Hadamard-rotated 4-bit activations, and binary g128 weights (8 layers of the
+# 27B-scale FFN, 302 MB of bits and scales per pass).
+NEXT_WORKLOADS = {
+    "prefill_had4_m512": (list(PREFILL_SHAPES), PREFILL_M),
+    "binary_ffn27b_m1": (binary_stack_shapes(BINARY_LAYERS), 1),
+}
 
 
 def algorithmic_bytes(N: int, K: int, M: int) -> int:
