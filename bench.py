@@ -194,9 +194,17 @@ def measured_tensor_peak():
 
 
 def stack_kernel_sha() -> str:
+    """Hash of the stack kernel's sources: its file, the headers it uses and
+    the streaming section of the launch-parameter header (other kernels'
+    declarations there do not change it)."""
+    d = os.path.dirname(STACK_KERNEL_SRC)
     h = hashlib.sha256()
-    for name in ("gemv_stream.cu", "quant_core.cuh", "tq_device.cuh", "tq_internal.h"):
-        h.update(open(os.path.join(os.path.dirname(STACK_KERNEL_SRC), name), "rb").read())
+    for name in ("gemv_stream.cu", "quant_core.cuh", "tq_device.cuh"):
+        h.update(open(os.path.join(d, name), "rb").read())
+    text = open(os.path.join(d, "tq_internal.h"), "rb").read()
+    start = text.index(b"// ------------------------------------------------- streaming GEMV")
+    end = text.index(b"\n// ------", start + 1)
+    h.update(text[start:end])
     return h.hexdigest()[:16]
 
 

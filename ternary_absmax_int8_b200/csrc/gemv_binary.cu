@@ -25,16 +25,17 @@
 // alternate tiles; the CTA's activations are resident in shared memory.
 //
 // Consumer arithmetic. A warp item is one packed row (or one of 2^lg pieces
-// of its groups); lane (seg, sub) = (lane >> 3, lane & 7) takes 16-byte chunk
-// `sub` of groups g0 + seg, g0 + seg + 4, ... For a 32-bit word u of bits
-// (four columns, eight planes per byte), dp4a of the nested masks
-// u & 0x01.., u & 0x03.., ..., u & 0x7F.. and u itself (unsigned bytes x
-// signed int8) gives the nested sums T_j = sum_{p <= j} 2^p S_p: seven logic
-// ops and eight dp4a per word. A transposing butterfly over the segment's
-// eight lanes (seven shuffles) leaves lane `sub` holding the group's T_sub;
-// with T_{sub-1} from its neighbour, S_sub = (T_sub - T_{sub-1}) >> sub.
-// Each lane so owns plane `sub` of its row: it scales the group's acc in
-// fp64 and adds, and after the row the four segments' sums are added.
+// of its groups); lane (seg, sub) = (lane >> 2, lane & 3) takes two of the
+// eight 16-byte chunks of groups g0 + seg, g0 + seg + 8, ... For a 32-bit
+// word u of bits (four columns, eight planes per byte), dp4a of the nested
+// masks u & 0x01.., u & 0x03.., ..., u & 0x7F.. and u itself (unsigned bytes
+// x signed int8) gives the nested sums T_j = sum_{p <= j} 2^p S_p: seven
+// logic ops and eight dp4a per word. A transposing butterfly over the
+// segment's four lanes (six shuffles) leaves lane `sub` holding the group's
+// T_{2 sub} and T_{2 sub + 1}; with T_{2 sub - 1} from its neighbour,
+// S_p = (T_p - T_{p-1}) >> p. Each lane so owns planes 2 sub and 2 sub + 1
+// of its row: it scales the group's acc in fp64 and adds, and after the row
+// the eight segments' sums are added.
 #include <atomic>
 #include <algorithm>
 #include <vector>
@@ -72,28 +73,27 @@ struct BinTail {
     }
 };
 
-// Eight int32 values per lane over the eight lanes of a segment: on return
-// lane `sub` holds the segment's total of value `sub` (seven shuffles).
-__device__ __forceinline__ int32_t transpose_reduce8(const int32_t (&v)[8], int sub)
+// Eight int32 values per lane over the four lanes of a segment: on return
+// lane `sub` holds the segment's totals of values 2 sub and 2 sub + 1 (six
+// shuffles).
+__device__ __forceinline__ int2 transpose_reduce8x4(const int32_t (&v)[8], int sub)
 {
-    const bool b2 = sub & 4, b1 = sub & 2, b0 = sub & 1;
+    const bool b1 = sub & 2, b0 = sub & 1;
     int32_t k[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int32_t keep = b2 ? v[4 + i] : v[i];
-        const int32_t send = b2 ? v[i] : v[4 + i];
-        k[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        const int32_t keep = b1 ? v[4 + i] : v[i];
+        const int32_t send = b1 ? v[i] : v[4 + i];
+        k[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
     }
     int32_t l[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const int32_t keep = b1 ? k[2 + i] : k[i];
-        const int32_t send = b1 ? k[i] : k[2 + i];
-        l[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        const int32_t keep = b0 ? k[2 + i] : k[i];
+        const int32_t send = b0 ? k[i] : k[2 + i];
+        l[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
     }
-    const int32_t keep = b0 ? l[1] : l[0];
-    const int32_t send = b0 ? l[0] : l[1];
-    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    return make_int2(l[0], l[1]);
 }
 
 // Nested-mask sums of one 16-byte chunk of bits against 16 activations.
@@ -248,7 +248,7 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
     named_bar_sync(1, kBinWC * 32);
 
     const int grp = warp / kBinW, wg = warp - grp * kBinW;
-    const int seg = lane >> 3, sub = lane & 7;
+    const int seg = lane >> 2, sub = lane & 3;
     int stage = grp;  // stages % kBinG == 0: the group keeps to stages grp + k G
     uint32_t phase = 0;
     int rot = 0;
@@ -277,14 +277,19 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
             const int r = item >> lg, piece = item & ((1 << lg) - 1);
             const int g0 = (piece * ng) >> lg, g1 = ((piece + 1) * ng) >> lg;
             const uint8_t *wrow = sb + size_t(r) * K;
-            double accd[MT];
-            int32_t itot[MT];
+            // planes 2 sub and 2 sub + 1 of this lane's segment groups
+            double accd[MT][2];
+            int32_t itot[MT][2];
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-                accd[m] = 0.0;
-                itot[m] = 0;
+                accd[m][0] = accd[m][1] = 0.0;
+                itot[m][0] = itot[m][1] = 0;
             }
-            for (int gb = g0; gb < g1; gb += 4) {
+            // The lane's two chunks of a group, rotated by segment so that a
+            // warp's 16-byte reads hit each bank slot four times (the
+            // minimum of four wavefronts per 512 bytes).
+            const int c0 = (2 * sub + seg) & 7, c1 = c0 ^ 1;
+            for (int gb = g0; gb < g1; gb += 8) {
                 const int g = gb + seg;
                 const bool valid = g < g1;
                 int32_t tt[MT][8];
@@ -294,29 +299,39 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
                     for (int j = 0; j < 8; ++j)
                         tt[m][j] = 0;
                 if (valid) {
-                    const uint4 wv =
-                        *reinterpret_cast<const uint4 *>(wrow + g * kBinGroup + sub * 16);
+                    const uint8_t *wg = wrow + g * kBinGroup;
+                    const uint4 w0 = *reinterpret_cast<const uint4 *>(wg + c0 * 16);
+                    const uint4 w1 = *reinterpret_cast<const uint4 *>(wg + c1 * 16);
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
                         if (MT == 1 || m < p.M) {
-                            const uint4 xv = *reinterpret_cast<const uint4 *>(
-                                sx + m * K + g * kBinGroup + sub * 16);
-                            dot_bits16(wv, xv, tt[m]);
+                            const uint8_t *xg = sx + m * K + g * kBinGroup;
+                            dot_bits16(w0, *reinterpret_cast<const uint4 *>(xg + c0 * 16), tt[m]);
+                            dot_bits16(w1, *reinterpret_cast<const uint4 *>(xg + c1 * 16), tt[m]);
                         }
                 }
-                const float scf = valid ? __half2float(ss[(r * ng + g) * 8 + sub]) : 0.0f;
+                // the fp16 scales of planes 2 sub, 2 sub + 1 (one 32-bit word)
+                const __half2 sc2 = valid ? *reinterpret_cast<const __half2 *>(
+                                                ss + (r * ng + g) * 8 + 2 * sub)
+                                          : __float2half2_rn(0.0f);
+                const float2 scf = __half22float2(sc2);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     if (MT == 1 || m < p.M) {
-                        const int32_t tsub = transpose_reduce8(tt[m], sub);
-                        int32_t tprev = __shfl_up_sync(0xffffffffu, tsub, 1, 8);
+                        const int2 t = transpose_reduce8x4(tt[m], sub);  // T_{2sub}, T_{2sub+1}
+                        int32_t tprev = __shfl_up_sync(0xffffffffu, t.y, 1, 4);  // T_{2sub-1}
                         if (sub == 0)
                             tprev = 0;
                         if (valid) {
-                            const int32_t s_p = (tsub - tprev) >> sub;  // exact: a multiple of 2^sub
-                            const int32_t a = 2 * s_p - sq[m * ng + g];
-                            itot[m] += a;
-                            accd[m] = __dadd_rn(accd[m], __dmul_rn(double(a), double(scf)));
+                            // exact: each difference is a multiple of 2^plane
+                            const int32_t s_lo = (t.x - tprev) >> (2 * sub);
+                            const int32_t s_hi = (t.y - t.x) >> (2 * sub + 1);
+                            const int32_t q = sq[m * ng + g];
+                            const int32_t a_lo = 2 * s_lo - q, a_hi = 2 * s_hi - q;
+                            itot[m][0] += a_lo;
+                            itot[m][1] += a_hi;
+                            accd[m][0] = __dadd_rn(accd[m][0], __dmul_rn(double(a_lo), double(scf.x)));
+                            accd[m][1] = __dadd_rn(accd[m][1], __dmul_rn(double(a_hi), double(scf.y)));
                         }
                     }
                 }
@@ -329,27 +344,36 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
                     mbar_arrive(&empty[stage]);
                 released = true;
             }
-            // add the four segments' sums: every lane then holds plane sub's
+            // add the eight segments' sums: lane sub of every segment then
+            // holds planes 2 sub and 2 sub + 1 of the row
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (MT == 1 || m < p.M) {
-                    accd[m] = __dadd_rn(accd[m], __shfl_xor_sync(0xffffffffu, accd[m], 8));
-                    accd[m] = __dadd_rn(accd[m], __shfl_xor_sync(0xffffffffu, accd[m], 16));
-                    itot[m] += __shfl_xor_sync(0xffffffffu, itot[m], 8);
-                    itot[m] += __shfl_xor_sync(0xffffffffu, itot[m], 16);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                        for (int o = 4; o < 32; o <<= 1) {
+                            accd[m][h] = __dadd_rn(accd[m][h],
+                                                   __shfl_xor_sync(0xffffffffu, accd[m][h], o));
+                            itot[m][h] += __shfl_xor_sync(0xffffffffu, itot[m][h], o);
+                        }
+                    }
                 }
             }
             const int row = d.row0 + r;
-            const size_t n_out = size_t(row) + size_t(sub) * N8;
             if (lg == 0) {
                 if (seg == 0) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         if (MT == 1 || m < p.M) {
-                            const size_t o = size_t(m) * (8 * size_t(N8)) + n_out;
-                            e.y[o] = __double2float_rn(__dmul_rn(accd[m], double(xs[m])));
-                            if (e.acc_out)
-                                e.acc_out[o] = itot[m];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const size_t o = size_t(m) * (8 * size_t(N8)) + size_t(row) +
+                                                 size_t(2 * sub + h) * N8;
+                                e.y[o] = __double2float_rn(__dmul_rn(accd[m][h], double(xs[m])));
+                                if (e.acc_out)
+                                    e.acc_out[o] = itot[m][h];
+                            }
                         }
                     }
                 }
@@ -358,10 +382,12 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
                 if (seg == 0) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
-                        if (MT == 1 || m < p.M) {
-                            atomicAdd(&dpart[(slot + m) * 8 + sub], accd[m]);
-                            atomicAdd(&ipart[(slot + m) * 8 + sub], itot[m]);
-                        }
+                        if (MT == 1 || m < p.M)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                atomicAdd(&dpart[(slot + m) * 8 + 2 * sub + h], accd[m][h]);
+                                atomicAdd(&ipart[(slot + m) * 8 + 2 * sub + h], itot[m][h]);
+                            }
                 }
                 __threadfence_block();  // partial sums before the count
                 __syncwarp();
@@ -372,15 +398,16 @@ binary_gemv_kernel(const __grid_constant__ BinParams<MaxE> p)
                 if (old == (1 << lg) - 1) {
                     // the last piece of this row: finish it
                     __threadfence_block();
-                    if (seg == 0) {
+                    if (lane < 8) {  // lane = plane
 #pragma unroll
                         for (int m = 0; m < MT; ++m) {
                             if (MT == 1 || m < p.M) {
-                                volatile double *dv = dpart + (slot + m) * 8 + sub;
+                                volatile double *dv = dpart + (slot + m) * 8 + lane;
                                 const double v = *dv;
                                 *dv = 0.0;
-                                const int32_t iv = atomicExch(&ipart[(slot + m) * 8 + sub], 0);
-                                const size_t o = size_t(m) * (8 * size_t(N8)) + n_out;
+                                const int32_t iv = atomicExch(&ipart[(slot + m) * 8 + lane], 0);
+                                const size_t o = size_t(m) * (8 * size_t(N8)) + size_t(row) +
+                                                 size_t(lane) * N8;
                                 e.y[o] = __double2float_rn(__dmul_rn(v, double(xs[m])));
                                 if (e.acc_out)
                                     e.acc_out[o] = iv;

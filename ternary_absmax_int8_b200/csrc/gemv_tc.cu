@@ -93,7 +93,7 @@ constexpr int kMaxGrid = 512;
 constexpr int kPlanStreamK = 0;
 constexpr int kPlanCluster = 1;
 constexpr int kMaxCluster = 8;
-constexpr int kMaxGroup = 16;          // projections per group launch
+constexpr int kMaxGroup = 64;          // projections per group launch
 
 struct SmallMParams {
     int N4, K, M;
@@ -363,21 +363,33 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             return cw.seg(p, sg);
     };
 
-    // The producer's copies, unit by unit in the CTA's order.
-    auto issue = [&](int issued, const Seg &g, int k) {
+    // The producer's copies, unit by unit in the CTA's order: the packed
+    // weights (which no earlier kernel writes) and the activations (which
+    // the previous kernel on the stream may still be writing: copied only
+    // after griddepcontrol.wait).
+    auto issue_w = [&](int issued, const Seg &g, int k) {
         const int s = issued % kSP;
         const int k0 = k * kUnitK;
         mbar_arrive_expect_tx(&tma_full[s], L::kPBytes + L::kBBytes);
         uint8_t *P = sP + s * L::kPBytes;
-        uint8_t *B = sB + s * L::kBBytes;
-        const CUtensorMap *mp = maps_p + g.proj, *mx = maps_x + g.proj;
+        const CUtensorMap *mp = maps_p + g.proj;
         tma_load_2d(P, mp, k0, g.tile * kPRows, &tma_full[s]);
         tma_load_2d(P + L::kPBytes / 2, mp, k0 + 128, g.tile * kPRows, &tma_full[s]);
+    };
+    auto issue_x = [&](int issued, const Seg &g, int k) {
+        const int s = issued % kSP;
+        const int k0 = k * kUnitK;
+        uint8_t *B = sB + s * L::kBBytes;
+        const CUtensorMap *mx = maps_x + g.proj;
         tma_load_2d(B, mx, k0, 0, &tma_full[s]);
         tma_load_2d(B + L::kBBytes / 2, mx, k0 + 128, 0, &tma_full[s]);
     };
-    int early = 0;  // copies thread 0 issued before the CTA barrier
+    int early = 0;  // weight copies thread 0 issued before the CTA barrier
     if (threadIdx.x == 0) {
+        // A following kernel launched with programmatic serialisation may
+        // start its own set-up and weight copies as SMs free up; it touches
+        // nothing this grid reads or writes before its griddepcontrol.wait.
+        pdl_launch_dependents();
         {
             const int j0 = cw.nseg > 0 ? first_seg().proj : 0;
             prefetch_tensormap(maps_p + j0);
@@ -402,7 +414,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         Seg g = first_seg();
         for (int sg = 0; sg < cw.nseg && early < kEarlyUnits; ++sg, g = next_seg(g, sg)) {
             for (int k = g.k0; k < g.k1 && early < kEarlyUnits; ++k)
-                issue(early++, g, k);
+                issue_w(early++, g, k);
         }
     }
     if (warp == 1)
@@ -424,11 +436,14 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         if (lane == 0) {
             int issued = 0;
             bool ok = true;
+            pdl_wait();  // activations of the previous kernel on the stream
             Seg g = first_seg();
             for (int sg = 0; sg < cw.nseg && ok; ++sg, g = next_seg(g, sg)) {
                 for (int k = g.k0; k < g.k1; ++k, ++issued) {
-                    if (issued < early)
-                        continue;  // issued before the CTA barrier
+                    if (issued < early) {
+                        issue_x(issued, g, k);  // its weights went before the CTA barrier
+                        continue;
+                    }
                     const int s = issued % kSP;
                     const uint32_t use = uint32_t(issued / kSP);
                     if (use > 0 && (!mbar_wait(&p_free[s], (use - 1) & 1, p.err) ||
@@ -436,7 +451,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                         ok = false;
                         break;
                     }
-                    issue(issued, g, k);
+                    issue_w(issued, g, k);
+                    issue_x(issued, g, k);
                 }
             }
             for (int s = 0; s < kSP && s < issued; ++s) {
@@ -549,6 +565,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
         // the single projection of a plain launch, in the group's form
         const GroupProj self{p.N4, U, p.tiles, 0, 0, p.w_scale, p.x_scale, p.x_sum, p.y,
                              p.acc_out};
+        pdl_wait();  // x_scale, x_sum, the outputs and the scratch
         Seg g = first_seg();
         int i0 = 0;  // the CTA's unit counter at the start of segment sg
         // Once a wait has given up (the error word is set and the outputs are
@@ -659,9 +676,16 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             // Stream-K partial tile: add into the workspace, then count this
             // CTA in. (Tiles and units of a group launch are numbered across
             // its projections.)
+            // Scratch slot: the tile's index for a single projection; in a
+            // group launch the index of the CTA holding the tile's first unit
+            // (each CTA's range ends in at most one split tile, so the
+            // slots are unique and the scratch is sized by the grid, not by
+            // the tiles).
             const int wtile = pj->tile0 + tile;
             const int wunit = pj->unit0 + tile * pj->U;
-            int32_t *wt = p.ws + size_t(wtile) * BN * kRows;
+            const int first = cta_of_unit(wunit, p.total_units, p.grid);
+            const int slot = Group ? first : wtile;
+            int32_t *wt = p.ws + size_t(slot) * BN * kRows;
 #pragma unroll
             for (int c = 0; c < BN; ++c)
                 if (c < p.M)
@@ -670,9 +694,8 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
             // issued its adds (the barrier orders them before its release).
             named_bar_sync(2, 128);
             if (threadIdx.x == kEpiWarp0 * 32) {
-                const int first = cta_of_unit(wunit, p.total_units, p.grid);
                 const int last = cta_of_unit(wunit + pj->U - 1, p.total_units, p.grid);
-                const int old = atom_add_acq_rel_gpu(p.cnt + wtile, 1);
+                const int old = atom_add_acq_rel_gpu(p.cnt + slot, 1);
                 *fin_flag = (old == last - first) ? 1 : 0;
             }
             named_bar_sync(2, 128);
@@ -703,7 +726,7 @@ __device__ __forceinline__ void smallm_body(const CUtensorMap *maps_p, const CUt
                     }
                 }
                 if (threadIdx.x == kEpiWarp0 * 32)
-                    p.cnt[wtile] = 0;
+                    p.cnt[slot] = 0;
             }
             named_bar_sync(2, 128);  // fin_flag is reused by the next segment
         }
@@ -884,13 +907,15 @@ cudaError_t launch_smallm_streamk(const uint8_t *packed, float w_scale, const in
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / sizeof(int32_t)];
 
-// Fixed scratch of the group plan. Unlike tq_gemv_noalloc's it is not
-// zero-filled before every call: every launch leaves the parts it used zero
-// (the CTA that completes a split tile zeroes its partial sums and counter),
-// so only the first call on a device, and the first one after a device error
-// was reported (a kernel that gave up a wait may have left sums behind), fill
-// it.
-constexpr size_t kGroupScratchBytes = size_t(8) << 20;
+// Fixed scratch of the group plan: one slot of partial sums (BN = 32 at most)
+// and one counter per CTA of the largest grid. Unlike tq_gemv_noalloc's it
+// is not zero-filled before every call: every launch leaves the parts it
+// used zero (the CTA that completes a split tile zeroes its partial sums and
+// counter, also after a wait gave up), so only the first call on a device,
+// and the first one after a device error was reported, fill it.
+constexpr size_t kGroupSlotBytes = size_t(32) * kRows * 4;
+constexpr size_t kGroupScratchBytes =
+    (size_t(kMaxGrid) * (kGroupSlotBytes + 4) + 255) / 256 * 256;
 static __device__ __align__(256) int32_t g_group_scratch[kGroupScratchBytes / sizeof(int32_t)];
 
 struct GroupScratch {
@@ -912,8 +937,15 @@ GroupTable *group_table()
     return &t;
 }
 
+static_assert(sizeof(GroupTable) + sizeof(SmallMParams) <= 32000, "kernel parameters exceed 32 KB");
+
+// With `pdl` the launch may begin (set-up, tensor memory, weight copies)
+// while the previous kernel on the stream drains; the kernel reads
+// activations and scales and touches outputs and scratch only after
+// griddepcontrol.wait.
 template <int BN>
-cudaError_t launch_group_bn(const GroupTable &gt, const SmallMParams &prm, cudaStream_t stream)
+cudaError_t launch_group_bn(const GroupTable &gt, const SmallMParams &prm, bool pdl,
+                            cudaStream_t stream)
 {
     cudaError_t e = configure_bn<BN>();
     if (e != cudaSuccess)
@@ -923,6 +955,11 @@ cudaError_t launch_group_bn(const GroupTable &gt, const SmallMParams &prm, cudaS
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = SmallMSmem<BN>::bytes + 1024;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, smallm_group_kernel<BN>, gt, prm);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -965,7 +1002,8 @@ void group_scratch_mark_dirty()
         c = false;
 }
 
-cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t stream)
+cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, bool overlap_prev,
+                                cudaStream_t stream)
 {
     if (M < 5 || M > 32 || n < 0)
         return cudaErrorInvalidValue;
@@ -978,6 +1016,7 @@ cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t 
         return err;
     if (dev < 0 || dev >= 64)
         return cudaErrorInvalidDevice;
+    const int sms = device_sm_count();
     int32_t *scratch = nullptr;
     {
         GroupScratch &gs = group_scratch();
@@ -995,29 +1034,17 @@ cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t 
         }
         scratch = static_cast<int32_t *>(gs.ptr[dev]);
     }
-    // tiles whose partial sums (and counter) the scratch holds at once
-    const int cap_tiles = int(kGroupScratchBytes / (size_t(BN) * kRows * 4 + 4));
-    const int sms = device_sm_count();
     int i = 0;
+    bool first = true;
     while (i < n) {
-        const int tiles_i = (e[i].N / 4 + kPRows - 1) / kPRows;
-        if (tiles_i > cap_tiles) {
-            // too large for the scratch: this projection alone, cluster plan
-            err = launch_smallm_tc(e[i].packed, e[i].w_scale, e[i].xq, e[i].x_scale, e[i].x_sum,
-                                   e[i].y, e[i].acc_out, M, e[i].N, e[i].K, stream);
-            if (err != cudaSuccess)
-                return err;
-            ++i;
-            continue;
-        }
         GroupTable &gt = *group_table();
         int j = 0, tiles = 0, units = 0;
         while (i < n && j < kMaxGroup) {
             const GroupEntry &x = e[i];
             const int t = (x.N / 4 + kPRows - 1) / kPRows;
-            if (tiles + t > cap_tiles)
-                break;
             const int U = (x.K + kUnitK - 1) / kUnitK;
+            if ((long long)units + (long long)t * U > (1 << 30))
+                break;
             if (!make_map(&gt.map_p[j], x.packed, x.K, x.N / 4, kPRows) ||
                 !make_map(&gt.map_x[j], x.xq, x.K, M, BN))
                 return cudaErrorInvalidValue;
@@ -1028,6 +1055,8 @@ cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t 
             ++j;
             ++i;
         }
+        if (j == 0)
+            return cudaErrorInvalidValue;
         gt.n = j;
         SmallMParams prm = {};
         prm.M = M;
@@ -1038,14 +1067,22 @@ cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t 
         prm.units_per_tile = 1;  // unused by the group plan
         prm.total_units = units;
         prm.grid = std::min({units, sms, kMaxGrid});
+        // slots of partial sums, one per CTA, then one counter per CTA
+        if (size_t(prm.grid) * (size_t(BN) * kRows * 4 + 4) > kGroupScratchBytes)
+            return cudaErrorInvalidValue;
         prm.ws = scratch;
-        prm.cnt = scratch + size_t(tiles) * BN * kRows;
+        prm.cnt = scratch + size_t(prm.grid) * BN * kRows;
         prm.err = device_error_word();
         if (!prm.err)
             return cudaErrorUnknown;
-        err = BN == 16 ? launch_group_bn<16>(gt, prm, stream) : launch_group_bn<32>(gt, prm, stream);
+        // consecutive group launches of one call may overlap; the first one
+        // overlaps the previous kernel only if the caller allows it
+        const bool pdl = first ? overlap_prev : true;
+        err = BN == 16 ? launch_group_bn<16>(gt, prm, pdl, stream)
+                       : launch_group_bn<32>(gt, prm, pdl, stream);
         if (err != cudaSuccess)
             return err;
+        first = false;
     }
     return cudaSuccess;
 }

@@ -324,13 +324,15 @@ tq_status gemv_stack_impl(const char *fname, const tq_proj *projs, int n_proj, i
     }
     if (M > tq::kStreamMaxTokens) {
         // 5 <= M <= 32: the tensor-core batched-decode kernel's group plan
-        // (no programmatic overlap: TQ_STACK_OVERLAP_PREV has no effect).
+        // (TQ_STACK_OVERLAP_PREV: its first launch may start while the
+        // previous kernel drains).
         std::vector<tq::GroupEntry> group;
         group.reserve(list.size());
         for (const tq::StreamEntry &e : list)
             group.push_back(tq::GroupEntry{e.packed, e.w_scale, e.xq, e.x_scale, e.x_sum, e.y,
                                            e.acc_out, 4 * e.N4, e.K});
-        cudaError_t e = tq::launch_smallm_group(group.data(), int(group.size()), M, stream);
+        cudaError_t e = tq::launch_smallm_group(group.data(), int(group.size()), M,
+                                                (flags & TQ_STACK_OVERLAP_PREV) != 0, stream);
         return e == cudaSuccess ? ok() : cuda_fail(e, fname);
     }
     const bool overlap = (flags & TQ_STACK_OVERLAP_PREV) != 0;

@@ -123,9 +123,11 @@ size_t smallm_workspace_bytes(int N, int M);
 size_t noalloc_scratch_capacity();
 
 // Group plan of the batched-decode kernel: several projections (N > 0,
-// K > 0) at 5 <= M <= 32 tokens, up to 16 per launch, one stream-K partition
+// K > 0) at 5 <= M <= 32 tokens, up to 64 per launch, one stream-K partition
 // over all of their tiles; split tiles finish through a fixed device scratch
-// that every launch leaves zeroed.
+// (one slot per CTA) that every launch leaves zeroed. With overlap_prev the
+// first launch may start while the previous kernel on the stream drains
+// (programmatic dependent launch); later launches of the call always may.
 struct GroupEntry {
     const uint8_t *packed;
     float w_scale;
@@ -136,7 +138,8 @@ struct GroupEntry {
     int32_t *acc_out;
     int N, K;
 };
-cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, cudaStream_t stream);
+cudaError_t launch_smallm_group(const GroupEntry *e, int n, int M, bool overlap_prev,
+                                cudaStream_t stream);
 // After a device error was reported: the next group call refills the scratch.
 void group_scratch_mark_dirty();
 cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const int8_t *xq,
