@@ -57,10 +57,13 @@ DESCRIPTIONS = {
                   "down ternary projections), M=1, 210 projections, 2.08e9 weights",
     "stack10_m1": "decode layer stack: 10 x BitNet-b1.58-2B-4T decoder layer, M=1 "
                   "(profiling case)",
-    "stack30_m4": "decode layer stack (30 layers, 210 projections) at M=4 tokens per "
-                  "projection: streaming kernel",
+    "stack30_m2": "decode layer stack (30 layers, 210 projections) at M=2 tokens per projection",
+    "stack30_m4": "decode layer stack (30 layers, 210 projections) at M=4 tokens per projection",
+    "stack30_m8": "decode layer stack (30 layers, 210 projections) at M=8 tokens per projection",
     "stack30_m16": "decode layer stack (30 layers, 210 projections) at M=16 tokens per "
-                   "projection: tensor-core group plan, 16 projections per launch",
+                   "projection",
+    "stack30_m24": "decode layer stack (30 layers, 210 projections) at M=24 tokens per "
+                   "projection",
     "layer_m1": "one BitNet-b1.58-2B-4T decoder layer, 7 ternary projections, M=1",
     "single_640x2560_m1": "one ternary projection N=640 K=2560, M=1",
     "prefill_m512": "prefill M=512 through ternary 6912x2560, 2560x6912, 17408x5120",
@@ -98,8 +101,10 @@ def step_mode(projs) -> str:
 def batch_launches(n: int, M: int) -> int:
     """Kernel launches of tq_quantize_act_stack_batch + tq_gemv_stack_batch
     over n projections of M tokens: 512 token rows per quantiser launch; 256
-    projections per streaming launch (M <= 4), 16 per tensor-core group launch."""
-    return -(-n * M // 512) + (-(-n // 256) if M <= 4 else -(-n // 16))
+    projections per streaming or warp-MMA launch, 64 per tensor-core group
+    launch."""
+    per = 64 if batch_kernel_name(M, "batch") == "smallm_group_kernel" else 256
+    return -(-n * M // 512) + -(-n // per)
 
 
 def workload_step_bytes(workload: str, projs) -> int:
@@ -448,8 +453,7 @@ def run_ours(args, rank: int, world: int):
                 "algorithmic_ops_per_step": flops}
     else:
         roof = {
-            "kernel": "stream_gemv_kernel" if M <= 4 else
-                      ("smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"),
+            "kernel": batch_kernel_name(M, mode),
             "bound": "hbm",
             "achieved": round(achieved, 1),
             "peak": peak,
@@ -518,6 +522,19 @@ def run_ours(args, rank: int, world: int):
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(projs, args, budget_s=args.cpu_seconds)
     return out
+
+
+def batch_kernel_name(M: int, mode: str) -> str:
+    """The kernel the library runs for M tokens per projection (its default
+    choice by M, or the one TQ_BATCH_KERNEL forces)."""
+    forced = os.environ.get("TQ_BATCH_KERNEL", "")
+    if M == 1:
+        return "stream_gemv_kernel"
+    if forced == "stream" and M <= 4 or forced == "" and M <= 2:
+        return "stream_gemv_kernel"
+    if forced == "mma" or forced == "" and M <= 16:
+        return "mma_gemv_kernel"
+    return "smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"
 
 
 def gemv_launches(M: int) -> int:

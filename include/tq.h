@@ -102,6 +102,12 @@ tq_status tq_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t
  *   acc_out device, int32 [M, N], written when not NULL (the exact
  *           accumulator; for checking), else untouched.
  * TQ_ERR_UNSUPPORTED for M > 24 (use tq_gemm_prefill) or K > 32768.
+ * Kernels (chosen by M from B200 measurements; many concurrent users make
+ * decode a small batch: 1bit engine blog, "One GPU, many users"): M <= 2 the
+ * streaming dp4a kernel; 3 <= M <= 16 the warp-MMA kernel (mma.sync int8 on
+ * the masked packed bytes); 17 <= M the tensor-core (tcgen05) batched-decode
+ * kernel. The environment variable TQ_BATCH_KERNEL=stream|mma|tc forces one
+ * where it applies (for measurement).
  */
 tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq,
                   const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
@@ -200,18 +206,23 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
  * 0 <= M <= 32 (TQ_ERR_UNSUPPORTED above); M == 0 is a no-op and M == 1 is
  * tq_gemv_stack. The quantising flags need M == 1 (TQ_ERR_UNSUPPORTED
  * otherwise); TQ_STACK_OVERLAP_PREV is accepted at every M.
- *   M <= 4: the streaming kernel, one launch per 256 projections.
- *   5 <= M <= 32: the tensor-core batched-decode kernel, one launch per 16
+ *   M <= 2: the streaming kernel, one launch per 256 projections.
+ *   3 <= M <= 16: the warp-MMA kernel, one launch per 256 projections (16-row
+ *   tiles of all projections balanced over the SMs); no scratch memory.
+ *   17 <= M <= 32: the tensor-core batched-decode kernel, one launch per 64
  *   projections, its K work split evenly over the SMs across projection
- *   boundaries (TQ_STACK_OVERLAP_PREV has no effect there). Tiles split between
- *   CTAs finish through a fixed 8 MiB device array compiled into the library,
- *   which every launch leaves zeroed; the first call on a device (make it
- *   before any stream capture) and the first call after tq_device_error
- *   reported a nonzero code zero-fill it on `stream` first. Calls whose work
- *   overlaps on the GPU (two streams) race on that array and must be
- *   serialised by the caller. A projection too large for the array
- *   (N > 130,944 at M <= 16, N > 65,408 at M > 16) runs alone as tq_gemv
- *   would run it.
+ *   boundaries. Tiles split between CTAs finish through a fixed device array
+ *   compiled into the library (one slot per CTA), which every launch leaves
+ *   zeroed, also one whose bounded wait gave up; the first call on a device
+ *   (make it before any stream capture) and the first call after
+ *   tq_device_error reported a nonzero code zero-fill it on `stream` first.
+ *   Calls whose work overlaps on the GPU (two streams) race on that array and
+ *   must be serialised by the caller.
+ * TQ_STACK_OVERLAP_PREV lets the first launch start while the previous
+ * kernel on the stream drains (programmatic dependent launch: weights may be
+ * streamed early, activations, scales and outputs are touched only after
+ * the previous kernel completes); later launches of the call always may.
+ * TQ_BATCH_KERNEL (see tq_gemv) applies here too.
  */
 tq_status tq_quantize_act_stack_batch(const tq_proj *projs, int n_proj, int M,
                                       cudaStream_t stream);

@@ -4,6 +4,7 @@
 #include <cfloat>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <algorithm>
 #include <mutex>
@@ -131,6 +132,40 @@ tq_status zero_outputs(float *y, int32_t *acc_out, size_t count, cudaStream_t s)
     return e == cudaSuccess ? ok() : cuda_fail(e, "zero outputs");
 }
 
+// Which kernel runs a group of M-token projections: the streaming dp4a kernel
+// (M <= 4 per launch), the warp-MMA kernel (2 <= M <= 32) or the tensor-core
+// group plan (5 <= M <= 32). The choice by M follows B200 measurements of the
+// 30-layer stack and the FFN projections; TQ_BATCH_KERNEL=stream|mma|tc
+// forces one where it applies (for measurement).
+enum class BatchKernel { kStream, kWarpMma, kTensor };
+
+BatchKernel batch_kernel(int M)
+{
+    static const int forced = [] {
+        const char *v = getenv("TQ_BATCH_KERNEL");
+        if (!v)
+            return -1;
+        if (!strcmp(v, "stream"))
+            return 0;
+        if (!strcmp(v, "mma"))
+            return 1;
+        if (!strcmp(v, "tc"))
+            return 2;
+        return -1;
+    }();
+    if (M <= 1)
+        return BatchKernel::kStream;
+    if (forced == 0 && M <= tq::kStreamMaxTokens)
+        return BatchKernel::kStream;
+    if (forced == 1)
+        return BatchKernel::kWarpMma;
+    if (forced == 2 && M >= 5)
+        return BatchKernel::kTensor;
+    if (M <= 2)
+        return BatchKernel::kStream;
+    return M <= 16 ? BatchKernel::kWarpMma : BatchKernel::kTensor;
+}
+
 // Tokens in groups of up to four, one streaming launch per group.
 tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
                         const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
@@ -156,13 +191,26 @@ tq_status stream_groups(const uint8_t *packed, float w_scale, const int8_t *xq,
     return ok();
 }
 
-// 5 <= M <= 32: the tensor-core batched-decode kernel.
-tq_status smallm_tc(const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
-                    const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K,
-                    cudaStream_t stream, const char *fn)
+// One projection at 1 <= M <= 32 tokens, by the kernel batch_kernel(M)
+// picks: streaming (tokens in groups of four), warp MMA, or the tensor-core
+// batched-decode kernel (thread-block clusters split K when tiles are few).
+tq_status small_batch(const uint8_t *packed, float w_scale, const int8_t *xq, const float *x_scale,
+                      const int32_t *x_sum, float *y, int32_t *acc_out, int M, int N, int K,
+                      cudaStream_t stream, const char *fn)
 {
-    cudaError_t err = tq::launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N,
-                                           K, stream);
+    cudaError_t err;
+    switch (batch_kernel(M)) {
+    case BatchKernel::kStream:
+        return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream, fn);
+    case BatchKernel::kWarpMma: {
+        const tq::MmaEntry e{packed, xq, x_scale, x_sum, y, acc_out, w_scale, N / 4, K, 0};
+        err = tq::launch_mma_gemv(&e, 1, M, false, stream);
+        break;
+    }
+    default:
+        err = tq::launch_smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
+                                   stream);
+    }
     return err == cudaSuccess ? ok() : cuda_fail(err, fn);
 }
 
@@ -322,10 +370,11 @@ tq_status gemv_stack_impl(const char *fname, const tq_proj *projs, int n_proj, i
         e.K = p.K;
         list.push_back(e);
     }
-    if (M > tq::kStreamMaxTokens) {
-        // 5 <= M <= 32: the tensor-core batched-decode kernel's group plan
-        // (TQ_STACK_OVERLAP_PREV: its first launch may start while the
-        // previous kernel drains).
+    const BatchKernel bk = batch_kernel(M);
+    if (bk == BatchKernel::kTensor) {
+        // the tensor-core batched-decode kernel's group plan, up to 64
+        // projections per launch (TQ_STACK_OVERLAP_PREV: its first launch
+        // may start while the previous kernel drains)
         std::vector<tq::GroupEntry> group;
         group.reserve(list.size());
         for (const tq::StreamEntry &e : list)
@@ -333,6 +382,19 @@ tq_status gemv_stack_impl(const char *fname, const tq_proj *projs, int n_proj, i
                                            e.acc_out, 4 * e.N4, e.K});
         cudaError_t e = tq::launch_smallm_group(group.data(), int(group.size()), M,
                                                 (flags & TQ_STACK_OVERLAP_PREV) != 0, stream);
+        return e == cudaSuccess ? ok() : cuda_fail(e, fname);
+    }
+    if (bk == BatchKernel::kWarpMma) {
+        // the warp-MMA small-batch kernel, one launch per 256 projections
+        // (TQ_STACK_OVERLAP_PREV: the first launch may start while the
+        // previous kernel drains)
+        std::vector<tq::MmaEntry> mma;
+        mma.reserve(list.size());
+        for (const tq::StreamEntry &e : list)
+            mma.push_back(tq::MmaEntry{e.packed, e.xq, e.x_scale, e.x_sum, e.y, e.acc_out,
+                                       e.w_scale, e.N4, e.K, 0});
+        cudaError_t e = tq::launch_mma_gemv(mma.data(), int(mma.size()), M,
+                                            (flags & TQ_STACK_OVERLAP_PREV) != 0, stream);
         return e == cudaSuccess ? ok() : cuda_fail(e, fname);
     }
     const bool overlap = (flags & TQ_STACK_OVERLAP_PREV) != 0;
@@ -421,11 +483,8 @@ tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq, const 
         return ok();
     if (K == 0)
         return zero_outputs(y, acc_out, size_t(M) * N, stream);
-    if (M > tq::kStreamMaxTokens)
-        return smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
-                         "tq_gemv");
-    return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
-                         "tq_gemv");
+    return small_batch(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                       "tq_gemv");
 }
 
 tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq,
@@ -440,9 +499,9 @@ tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq
         return ok();
     if (K == 0)
         return zero_outputs(y, acc_out, size_t(M) * N, stream);
-    if (M > tq::kStreamMaxTokens && M <= 32)
-        return smallm_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
-                         "tq_gemm_prefill");
+    if (M <= 32)
+        return small_batch(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
+                           "tq_gemm_prefill");
     bool handled = false;
     cudaError_t e = tq::launch_prefill_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
                                           stream, &handled);

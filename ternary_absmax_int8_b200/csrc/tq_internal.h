@@ -146,6 +146,38 @@ cudaError_t launch_smallm_tc_noalloc(const uint8_t *packed, float w_scale, const
                                      const float *x_scale, const int32_t *x_sum, float *y,
                                      int32_t *acc_out, int M, int N, int K, cudaStream_t stream);
 
+// ------------------------------- small-batch decode on the warp MMA (M <= 32)
+// One entry = one projection (packed [N4, K], activations [M, K], outputs
+// [M, 4 N4]); tile_begin is filled by the launcher.
+struct MmaEntry {
+    const uint8_t *packed;
+    const int8_t *xq;
+    const float *x_scale;
+    const int32_t *x_sum;
+    float *y;
+    int32_t *acc_out;
+    float w_scale;
+    int N4, K;
+    int tile_begin;
+};
+
+constexpr int kMmaMaxTokens = 32;
+constexpr int kMmaStackMax = 256;  // entries per launch
+constexpr int kMmaMaxGrid = 320;   // CTAs per launch
+
+struct MmaParams {
+    int n_entries, M;
+    int lgP;  // log2 of the warps per team (each tile's K is split over a team)
+    int cta_tile0[kMmaMaxGrid + 1];
+    MmaEntry e[kMmaStackMax];
+};
+
+// One launch per 256 projections; with overlap_prev the first may start
+// while the previous kernel on the stream drains (its weights are not being
+// written), later ones always may.
+cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_prev,
+                            cudaStream_t stream);
+
 // ------------------------------------------ decoder-layer neighbours, absmean
 // input: 0 = bf16 x, 1 = fp32 x, 2 = relu(x_f32)^2 * up. One CTA per row.
 cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f32,

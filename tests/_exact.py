@@ -41,3 +41,52 @@ def bf16(v: float) -> int:
     u = int(f.view(np.uint32)[0])
     assert u & 0xFFFF == 0, f"{v} is not exactly representable in bf16"
     return u >> 16
+
+
+# ------------------------------------------------ order-free fp64 statistics
+# The RMSNorm factor and the absmean scale are fp64 sums rounded to fp32
+# after a few more fp64 operations. The GPU adds in a tree order, the oracle
+# left to right; both results lie within (n - 1) u S of the exact sum S of
+# the n non-negative terms (u = 2^-53; each term x^2 of an fp32 x, or |x| of a
+# bf16 x, is exact in fp64). The operations after the sum are the same IEEE
+# operations on both sides and are monotone in the sum, so if both ends of
+# that interval give the same fp32 result, every order of the additions does.
+
+U64 = 2.0 ** -53
+
+
+def rms_factor(S: float, K: int, eps32: float) -> np.float32:
+    """fl32(1 / sqrt(S / K + eps)) with the fp64 operations of the oracle."""
+    return np.float32(1.0 / math.sqrt(S / K + eps32))
+
+
+def rms_interval_ok(S: float, K: int, eps32: float) -> bool:
+    """True if every sum within the order-error band around S (K terms)
+    gives the same fp32 factor."""
+    d = K * U64 * S * 1.0000001                       # (n - 1) u S, and the rounding of S
+    return rms_factor(max(S - d, 0.0), K, eps32) == rms_factor(S + d, K, eps32)
+
+
+def rms_order_free(v: np.ndarray, eps: float) -> np.ndarray:
+    """Per row of fp32 v [M, K]: True if every fp64 summation order of the
+    squares gives the same fp32 RMSNorm factor."""
+    v = np.asarray(v, np.float32)
+    eps32 = float(np.float32(eps))
+    M, K = v.shape
+    out = np.empty(M, bool)
+    for m in range(M):
+        sq = (v[m].astype(np.float64)) ** 2           # exact squares
+        out[m] = rms_interval_ok(math.fsum(sq.tolist()), K, eps32)  # exactly rounded sum
+    return out
+
+
+def absmean_order_free(w_bits: np.ndarray) -> bool:
+    """True if every fp64 summation order of |W| (bf16 bit patterns) gives
+    the same fp32 scale fl32(S / n)."""
+    a = np.abs((w_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)).ravel()
+    n = a.size
+    if n == 0:
+        return True
+    S = math.fsum(a.tolist())
+    d = n * U64 * S * 1.0000001
+    return np.float32(max(S - d, 0.0) / n) == np.float32((S + d) / n)

@@ -9,6 +9,7 @@ import torch
 
 import oracle
 import ternary_absmax_int8_b200 as tq
+from tests._exact import absmean_order_free, rms_order_free
 from tests._gpu import assert_y_close, dev, host_pack
 from workloads import activations_bf16, make_projections
 
@@ -18,6 +19,15 @@ EPS = 1e-5
 
 def f32_of_bf16(b):
     return (np.asarray(b, dtype=np.uint32) << 16).view(np.float32)
+
+
+def rms_ref(v, g, eps):
+    """The oracle's RMSNorm, after checking that no row's normalising factor
+    depends on the order of the fp64 sum of squares: the GPU adds in a tree
+    order, the oracle left to right, and the bit-exact comparison below is
+    only justified when every order gives the same fp32 factor."""
+    assert rms_order_free(v, eps).all(), "an RMSNorm factor depends on the summation order"
+    return oracle.rmsnorm(v, g, eps)
 
 
 def gains(rng, K):
@@ -51,7 +61,7 @@ def test_rmsnorm_quantize_bf16(cuda_device, M, K):
     rng = np.random.default_rng(M * 7 + K)
     xb = activations_bf16(rng, M, K)
     g = gains(rng, K)
-    ref = oracle.quant_f32(oracle.rmsnorm(f32_of_bf16(xb), g, EPS))
+    ref = oracle.quant_f32(rms_ref(f32_of_bf16(xb), g, EPS))
     assert_same(run_rms(M, K, g, EPS, x_bf16=xb), ref, f"bf16 M={M} K={K}")
 
 
@@ -60,7 +70,7 @@ def test_rmsnorm_quantize_f32(cuda_device, M, K):
     rng = np.random.default_rng(100 + M + K)
     x = (rng.standard_normal((M, K)) * 3).astype(np.float32)
     g = gains(rng, K)
-    ref = oracle.quant_f32(oracle.rmsnorm(x, g, EPS))
+    ref = oracle.quant_f32(rms_ref(x, g, EPS))
     assert_same(run_rms(M, K, g, EPS, x_f32=x), ref, f"f32 M={M} K={K}")
 
 
@@ -70,7 +80,7 @@ def test_relu2_mul_rmsnorm_quantize(cuda_device, M, K):
     gate = (rng.standard_normal((M, K)) * 2).astype(np.float32)
     up = (rng.standard_normal((M, K)) * 2).astype(np.float32)
     g = gains(rng, K)
-    ref = oracle.quant_f32(oracle.rmsnorm(oracle.relu2_mul(gate, up), g, EPS))
+    ref = oracle.quant_f32(rms_ref(oracle.relu2_mul(gate, up), g, EPS))
     assert_same(run_rms(M, K, g, EPS, gate=gate, up=up), ref, f"relu2 M={M} K={K}")
 
 
@@ -86,13 +96,13 @@ def test_rms_degenerate_rows(cuda_device):
     for eps in (0.0, 1.0):
         if eps == 0.0:
             xx = x[[0, 2, 3]]       # eps = 0 with a zero row would divide by 0
-            ref = oracle.quant_f32(oracle.rmsnorm(xx, g, eps))
+            ref = oracle.quant_f32(rms_ref(xx, g, eps))
             assert_same(run_rms(3, K, g, eps, x_f32=xx), ref, "f32 eps=0")
         else:
-            ref = oracle.quant_f32(oracle.rmsnorm(x, g, eps))
+            ref = oracle.quant_f32(rms_ref(x, g, eps))
             assert_same(run_rms(4, K, g, eps, x_f32=x), ref, "f32 eps=1")
             up = np.ones_like(gate)
-            ref = oracle.quant_f32(oracle.rmsnorm(oracle.relu2_mul(gate, up), g, eps))
+            ref = oracle.quant_f32(rms_ref(oracle.relu2_mul(gate, up), g, eps))
             assert_same(run_rms(4, K, g, eps, gate=gate, up=up), ref, "relu2 eps=1")
 
 
@@ -147,11 +157,11 @@ def test_ffn_block_chain(cuda_device, M, overlap):
     torch.cuda.synchronize()
 
     # ---- oracle, the same chain
-    q, s, t = oracle.quant_f32(oracle.rmsnorm(f32_of_bf16(xb), g_in, EPS))
+    q, s, t = oracle.quant_f32(rms_ref(f32_of_bf16(xb), g_in, EPS))
     acc_g = oracle.gemv_threads(oracle.pack(gate_p.w), I, q)
     acc_u = oracle.gemv_threads(oracle.pack(up_p.w), I, q)
     h = oracle.relu2_mul(y32(acc_g, gate_p.w_scale, s), y32(acc_u, up_p.w_scale, s))
-    q2, s2, t2 = oracle.quant_f32(oracle.rmsnorm(h, g_ffn, EPS))
+    q2, s2, t2 = oracle.quant_f32(rms_ref(h, g_ffn, EPS))
     acc_d = oracle.gemv_threads(oracle.pack(down_p.w), H, q2)
     y_d = oracle.epilogue(acc_d, down_p.w_scale, s2)
 
@@ -175,6 +185,9 @@ def test_absmean_pack_latent_weights(cuda_device, N, K):
     rng = np.random.default_rng(N + K)
     W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
     Wb = torch.from_numpy(W).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    # the fp64 sum of |W| (GPU tree order, oracle left to right) rounds to the
+    # same fp32 scale in every order for this input
+    assert absmean_order_free(Wb)
     w, g = oracle.absmean(Wb)
     packed, ws = run_absmean(Wb)
     assert np.float32(ws).view(np.uint32) == np.float32(g).view(np.uint32)
@@ -245,14 +258,14 @@ def test_ffn_block_fused_two_launches(cuda_device, layers):
     for l in range(layers):
         gp, upp, dp = projs[3 * l:3 * l + 3]
         xq, xq_b, xs, xsum, xq2, xs2, xsum2, yd, accd = out[l]
-        q, s, t = oracle.quant_f32(oracle.rmsnorm(f32_of_bf16(gp.x_bf16), gin[l], EPS))
+        q, s, t = oracle.quant_f32(rms_ref(f32_of_bf16(gp.x_bf16), gin[l], EPS))
         for qq, j in ((xq, 0), (xq_b, 1)):
             assert_same((qq.cpu().numpy()[None], xs.cpu().numpy()[j:j + 1],
                          xsum.cpu().numpy()[j:j + 1]), (q, s, t), f"layer {l} input codes")
         acc_g = oracle.gemv_threads(oracle.pack(gp.w), I, q)
         acc_u = oracle.gemv_threads(oracle.pack(upp.w), I, q)
         h = oracle.relu2_mul(y32(acc_g, gp.w_scale, s), y32(acc_u, upp.w_scale, s))
-        q2, s2, t2 = oracle.quant_f32(oracle.rmsnorm(h, gff[l], EPS))
+        q2, s2, t2 = oracle.quant_f32(rms_ref(h, gff[l], EPS))
         assert_same((xq2.cpu().numpy()[None], xs2.cpu().numpy(), xsum2.cpu().numpy()),
                     (q2, s2, t2), f"layer {l} down codes")
         acc_d = oracle.gemv_threads(oracle.pack(dp.w), H, q2)

@@ -204,8 +204,11 @@ WORKLOADS = {
     # for profiler captures of the stack kernel
     "stack10_m1": (stack_shapes(10), 1),
     # the same stack with several tokens per projection (small-batch decode)
+    "stack30_m2": (stack_shapes(STACK_LAYERS), 2),
     "stack30_m4": (stack_shapes(STACK_LAYERS), 4),
+    "stack30_m8": (stack_shapes(STACK_LAYERS), 8),
     "stack30_m16": (stack_shapes(STACK_LAYERS), 16),
+    "stack30_m24": (stack_shapes(STACK_LAYERS), 24),
 }
 for _m in SMALL_M_VALUES:
     WORKLOADS[f"ffn_m{_m}"] = (list(SMALL_M_SHAPES), _m)
