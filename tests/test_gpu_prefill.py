@@ -58,3 +58,31 @@ def test_prefill_second_tile_per_cta(cuda_device):
     rows = np.array([0, 255, 256, 300, 511, 512, 700, 767, 768, 1000, 1023])
     sub = (q[rows], xs[rows], xsum[rows], acc[rows], y[rows])
     assert_parity(sub, oracle_forward(w, ws, xb[rows]), "17408x512 M=1024")
+
+
+def test_prefill_repeated_and_after_error(cuda_device):
+    # Repeated calls give identical bytes and match the oracle, also after a
+    # device error has been reported in between.
+    import torch
+
+    import ternary_absmax_int8_b200 as tq
+    from tests._gpu import dev, gpu_quant
+    p = next(make_projections([("ffn_2560x6912", 2560, 6912)], M=PREFILL_M, seed=11))
+    P = dev(host_pack(p.w))
+    xq, xs, xsum = gpu_quant(p.x_bf16)
+    ref = oracle_forward(p.w, p.w_scale, p.x_bf16)
+    outs = []
+    for i in range(3):
+        if i == 2:
+            tq.tq_selftest_wait_timeout(100)
+            assert tq.tq_device_error(reset=True) != 0
+        y = torch.full((p.M, p.N), float("nan"), device="cuda")
+        acc = torch.full((p.M, p.N), -(2 ** 31), dtype=torch.int32, device="cuda")
+        tq.tq_gemm_prefill(P, float(p.w_scale), xq, xs, xsum, y, acc, p.M, p.N, p.K)
+        torch.cuda.synchronize()
+        got = (xq.cpu().numpy(), xs.cpu().numpy(), xsum.cpu().numpy(), acc.cpu().numpy(),
+               y.cpu().numpy())
+        assert_parity(got, ref, f"call {i}")
+        outs.append(got[4])
+    assert all(np.array_equal(o.view(np.uint32), outs[0].view(np.uint32)) for o in outs)
+    assert tq.tq_device_error(reset=True) == 0
