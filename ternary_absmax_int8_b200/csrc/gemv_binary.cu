@@ -37,11 +37,14 @@
 // of its row: it scales the group's acc in fp64 and adds, and after the row
 // the eight segments' sums are added.
 #include <atomic>
+#include <cstdlib>
+#include <cstring>
 #include <algorithm>
 #include <vector>
 
 #include <cuda_fp16.h>
 
+#include "mma_common.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -562,6 +565,357 @@ cudaError_t launch_bin_sized(BinEntry *entries, int n, int M, cudaStream_t strea
     }
 }
 
+// ------------------------------------------------------------------------
+// One token (M = 1) on the warp-level integer MMA. A byte of bits holds the
+// eight planes of one column, so with the nested masks 0x01.., 0x03.., ...,
+// 0x7F.. and 0xFF.. (unsigned bytes) an m16n8k32 MMA on 16 packed rows x 32
+// columns gives D_j = sum_{p <= j} 2^p S_p for all 16 rows at once: eight
+// MMAs and 28 logic ops per 32-column block, against 64 dp4a per lane. A
+// lane's A fragment comes from 16 contiguous bytes of each of its rows (the
+// column permutation of the ternary warp-MMA kernel, shared with the
+// activations), streamed by cp.async into per-warp rings together with the
+// 16 rows' fp16 scales of the group (so that their HBM latency is hidden as
+// deep as the bits').
+// A step is one 128-column group: each mask's chain of four MMAs starts from
+// zero, and every column of the B fragment carries the token's codes, so the
+// accumulators of all four lanes of a quad hold the group's nested sums T_j
+// of rows g and g + 8. Lane t takes planes 2t and 2t + 1 -- all four lanes
+// share the per-group scaling --: S_p = (T_p - T_{p-1}) >> p,
+// acc = 2 S - Q_g, and the lane adds acc times the plane's fp16 scale in fp64
+// (exact).
+// Tiles of 16 packed rows (128 outputs) x the full K, contiguous ranges per
+// CTA (16 warps, one per SM); teams of P warps split a tile's groups when
+// tiles are few and add their fp64 and int32 partials in shared memory (exact,
+// order-free).
+constexpr int kBmW = 20;                      // warps per CTA (96 registers each)
+constexpr int kBmThreads = kBmW * 32;
+constexpr int kBmRing = 4;                    // stages per warp (a power of two)
+constexpr int kBmBits = 2 * 2 * 32 * 16;      // [2 rows][2 halves][32 lanes][16 B]
+constexpr int kBmScales = 16 * 16;            // then the scales: [16 rows][8 planes] fp16
+constexpr int kBmStage = kBmBits + kBmScales + kBinGroup;  // then the group's 128 codes
+constexpr int kBmRows = 16;
+
+struct BmCursor {
+    int tile, entry, step, step_end;
+    int K, G;
+    const uint8_t *row;  // the lane's row g at column 16 t
+    const uint16_t *sc;  // scales of the lane's row g (t = 0) or g + 8 (t = 1): [group][8]
+    const int8_t *xq;    // the token's codes at column 16 g (lanes t = 2)
+    bool ok0, ok1;
+};
+
+struct BmWalk {
+    const BinMmaEntry *tab;
+    int n_ent, t_end, teams, piece, lgP, g, t;
+
+    __device__ void start(BmCursor &c, int tl) const
+    {
+        c.tile = tl;
+        while (c.entry + 1 < n_ent && tab[c.entry + 1].tile_begin <= tl)
+            ++c.entry;
+        const BinMmaEntry &e = tab[c.entry];
+        c.K = e.K;
+        c.G = e.K / kBinGroup;
+        c.step = (c.G * piece) >> lgP;
+        c.step_end = (c.G * (piece + 1)) >> lgP;
+        const int r = (tl - e.tile_begin) * kBmRows + g;
+        c.ok0 = r < e.N8;
+        c.ok1 = r + 8 < e.N8;
+        c.row = e.bits + size_t(c.ok0 ? r : 0) * e.K + 16 * t;
+        const int rs = t == 1 && c.ok1 ? r + 8 : (c.ok0 ? r : 0);
+        c.sc = e.scales + size_t(rs) * c.G * 8;
+        c.xq = e.xq + 16 * g;
+    }
+    __device__ void settle(BmCursor &c) const
+    {
+        while (c.tile < t_end && c.step >= c.step_end) {
+            if (c.tile + teams >= t_end) {
+                c.tile = t_end;
+                break;
+            }
+            start(c, c.tile + teams);
+        }
+    }
+};
+
+__global__ void __launch_bounds__(kBmThreads, 1)
+binary_mma_kernel(const __grid_constant__ BinMmaParams p)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int kRingBytes = kBmRing * kBmStage;
+    double *dslot = reinterpret_cast<double *>(smem + kBmW * kRingBytes);  // [W][16 rows][8]
+    int32_t *islot = reinterpret_cast<int32_t *>(dslot + kBmW * 16 * 8);   // [W][16][8]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const uint8_t *ring = smem + warp * kRingBytes + lane * 16;
+    const uint32_t ring_s = smem_u32(ring);
+
+    const int t_begin = p.cta_tile0[blockIdx.x], t_end = p.cta_tile0[blockIdx.x + 1];
+    const int lgP = p.lgP, P = 1 << lgP, teams = kBmW >> lgP;
+    // teams of P warps; warps past the last whole team (kBmW not a multiple
+    // of P) stay idle
+    const int team = warp >> lgP, piece = warp & (P - 1);
+    const int first = team < teams ? t_begin + team : t_end;
+    const BmWalk wk{p.e, p.n_entries, t_end, teams, piece, lgP, g, t};
+
+    BmCursor lc{t_end, 0, 0, 0, 0, 0, nullptr, nullptr, nullptr, false, false};
+    if (first < t_end) {
+        wk.start(lc, first);
+        wk.settle(lc);
+    }
+    int issued = 0;
+    // this lane's copy target past the bits: a scale row (t < 2) or 16 codes (t = 2)
+    const uint32_t sc_s = smem_u32(smem + warp * kRingBytes + kBmBits) +
+                          uint32_t(t < 2 ? (g + 8 * t) * 16 : kBmScales + 16 * g);
+    auto issue = [&]() {
+        const uint32_t dst = ring_s + uint32_t(issued & (kBmRing - 1)) * kBmStage;
+        __syncwarp();  // the slot's scales were last read by other lanes
+        if (lc.tile < t_end) {
+            const uint8_t *src = lc.row + size_t(lc.step) * kBinGroup;
+            // row g + 8 past the end: a zero-size copy from row g's address
+            const uint8_t *src8 = lc.ok1 ? src + size_t(8) * lc.K : src;
+            cp_async16(dst, src, lc.ok0);
+            cp_async16(dst + 512, src + 64, lc.ok0);
+            cp_async16(dst + 1024, src8, lc.ok1);
+            cp_async16(dst + 1536, src8 + 64, lc.ok1);
+            if (t < 2)  // lanes t = 0, 1: the 8 scales of row g + 8 t at this group
+                cp_async16(sc_s + uint32_t(issued & (kBmRing - 1)) * kBmStage,
+                           lc.sc + size_t(lc.step) * 8, t == 0 ? lc.ok0 : lc.ok1);
+            else if (t == 2)  // lanes t = 2: codes 16 g .. 16 g + 15 of the group
+                cp_async16(sc_s + uint32_t(issued & (kBmRing - 1)) * kBmStage,
+                           lc.xq + size_t(lc.step) * kBinGroup, true);
+            ++lc.step;
+            wk.settle(lc);
+        }
+        cp_async_commit();
+        ++issued;
+    };
+#pragma unroll
+    for (int i = 0; i < kBmRing - 1; ++i)
+        issue();
+
+
+    double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};  // [row g / g + 8][plane 2t / 2t + 1]
+    int32_t tot[2][2] = {{0, 0}, {0, 0}};
+    int consumed = 0;
+    int fent = 0;
+    while (fent + 1 < p.n_entries && p.e[fent + 1].tile_begin <= t_begin)
+        ++fent;
+
+    // One 128-column group from a ring stage into the lane's accumulators.
+    auto group = [&](const uint8_t *stage) {
+        // the token's codes for the lane's 16 + 16 columns of the group; every
+        // B column carries them (lane (g, t) supplies column g), so that all
+        // four lanes of a quad receive the row's sums
+        const uint4 q0 = *reinterpret_cast<const uint4 *>(stage + kBmBits + kBmScales + 16 * t);
+        const uint4 q1 =
+            *reinterpret_cast<const uint4 *>(stage + kBmBits + kBmScales + 64 + 16 * t);
+        // the group's code sum
+        int32_t qs = 0;
+        qs = __dp4a(int(q0.x), 0x01010101, qs);
+        qs = __dp4a(int(q0.y), 0x01010101, qs);
+        qs = __dp4a(int(q0.z), 0x01010101, qs);
+        qs = __dp4a(int(q0.w), 0x01010101, qs);
+        qs = __dp4a(int(q1.x), 0x01010101, qs);
+        qs = __dp4a(int(q1.y), 0x01010101, qs);
+        qs = __dp4a(int(q1.z), 0x01010101, qs);
+        qs = __dp4a(int(q1.w), 0x01010101, qs);
+        qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+        const int32_t Q = qs + __shfl_xor_sync(0xffffffffu, qs, 2);
+
+        const uint8_t *src = stage + lane * 16;
+        // planes 2 t, 2 t + 1 of rows g and g + 8 (zero past the end)
+        const uint8_t *ssc = stage + kBmBits + g * 16 + 4 * t;
+        const float2 s0 = __half22float2(*reinterpret_cast<const __half2 *>(ssc));
+        const float2 s1 = __half22float2(*reinterpret_cast<const __half2 *>(ssc + 128));
+        int32_t d[8][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 lo4 = *reinterpret_cast<const uint4 *>(src + h * 512);         // row g
+            const uint4 hi4 = *reinterpret_cast<const uint4 *>(src + 1024 + h * 512);  // row g + 8
+            const uint4 qq = h == 0 ? q0 : q1;
+            const uint32_t al[4] = {lo4.x, lo4.y, lo4.z, lo4.w};
+            const uint32_t ah[4] = {hi4.x, hi4.y, hi4.z, hi4.w};
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t a0 = al[2 * b], a2 = al[2 * b + 1];
+                const uint32_t a1 = ah[2 * b], a3 = ah[2 * b + 1];
+                const uint32_t b0 = b == 0 ? qq.x : qq.z, b1 = b == 0 ? qq.y : qq.w;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    // j = 6: the raw bytes as signed, T_6 - 128 S_7 (with the
+                    // unsigned T_6 + 128 S_7 of j = 7 it gives T_6, no mask)
+                    const uint32_t mk = j >= 6 ? 0xFFFFFFFFu : 0x01010101u * ((2u << j) - 1u);
+                    if (j == 6) {
+                        if (h == 0 && b == 0)
+                            mma_s8s8_z(d[j], a0, a1, a2, a3, b0, b1);
+                        else
+                            mma_s8s8(d[j], a0, a1, a2, a3, b0, b1);
+                    } else if (h == 0 && b == 0) {
+                        mma_u8s8_z(d[j], a0 & mk, a1 & mk, a2 & mk, a3 & mk, b0, b1);
+                    } else {
+                        mma_u8s8(d[j], a0 & mk, a1 & mk, a2 & mk, a3 & mk, b0, b1);
+                    }
+                }
+            }
+        }
+        // the group's nested sums of rows g (fragment word 0) and g + 8
+        // (word 2), the same in every lane of the quad: lane t takes
+        // T_{2t-1}, T_{2t}, T_{2t+1}
+        const bool b1 = t & 2, b0 = t & 1;
+#pragma unroll
+        for (int rs = 0; rs < 2; ++rs) {
+            const int w = 2 * rs;
+            const int32_t t6 = (d[7][w] + d[6][w]) >> 1;
+            const int32_t t_lo = b1 ? (b0 ? t6 : d[4][w]) : (b0 ? d[2][w] : d[0][w]);
+            const int32_t t_hi = b1 ? (b0 ? d[7][w] : d[5][w]) : (b0 ? d[3][w] : d[1][w]);
+            const int32_t t_pr = b1 ? (b0 ? d[5][w] : d[3][w]) : (b0 ? d[1][w] : 0);
+            const int32_t a_lo = 2 * ((t_lo - t_pr) >> (2 * t)) - Q;
+            const int32_t a_hi = 2 * ((t_hi - t_lo) >> (2 * t + 1)) - Q;
+            const float2 sc = rs == 0 ? s0 : s1;
+            acc[rs][0] = __dadd_rn(acc[rs][0], __dmul_rn(double(a_lo), double(sc.x)));
+            acc[rs][1] = __dadd_rn(acc[rs][1], __dmul_rn(double(a_hi), double(sc.y)));
+            tot[rs][0] += a_lo;
+            tot[rs][1] += a_hi;
+        }
+    };
+
+    for (int tile = first; tile < t_end; tile += teams) {
+        while (fent + 1 < p.n_entries && p.e[fent + 1].tile_begin <= tile)
+            ++fent;
+        const BinMmaEntry &e = p.e[fent];
+        // this warp's share of the tile's groups (a contiguous piece, possibly empty)
+        const int G = e.K / kBinGroup;
+        const int n_steps = ((G * (piece + 1)) >> lgP) - ((G * piece) >> lgP);
+        for (int st = 0; st < n_steps; ++st) {
+            issue();
+            cp_async_wait<kBmRing - 1>();
+            __syncwarp();
+            group(smem + warp * kRingBytes + (consumed & (kBmRing - 1)) * kBmStage);
+            ++consumed;
+        }
+        const int r0 = (tile - e.tile_begin) * kBmRows;
+        const float xs = __ldg(e.x_scale);
+        if (P == 1) {
+#pragma unroll
+            for (int rs = 0; rs < 2; ++rs) {
+                const int row = r0 + g + 8 * rs;
+                if (row < e.N8) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const size_t o = size_t(row) + size_t(2 * t + h) * e.N8;
+                        e.y[o] = __double2float_rn(__dmul_rn(acc[rs][h], double(xs)));
+                        if (e.acc_out)
+                            e.acc_out[o] = tot[rs][h];
+                    }
+                }
+            }
+        } else {
+            // the team adds its partials: slot [warp][row][plane]
+            double *dm = dslot + warp * 128;
+            int32_t *im = islot + warp * 128;
+#pragma unroll
+            for (int rs = 0; rs < 2; ++rs)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    dm[(g + 8 * rs) * 8 + 2 * t + h] = acc[rs][h];
+                    im[(g + 8 * rs) * 8 + 2 * t + h] = tot[rs][h];
+                }
+            named_bar_sync(1 + team, 32 * P);
+            const double *td = dslot + team * P * 128;
+            const int32_t *ti = islot + team * P * 128;
+            for (int o = piece * 32 + lane; o < 128; o += 32 * P) {
+                const int row = r0 + (o >> 3), pl = o & 7;
+                double a = 0.0;
+                int32_t s = 0;
+                for (int w = 0; w < P; ++w) {
+                    a = __dadd_rn(a, td[w * 128 + o]);
+                    s += ti[w * 128 + o];
+                }
+                if (row < e.N8) {
+                    const size_t out = size_t(row) + size_t(pl) * e.N8;
+                    e.y[out] = __double2float_rn(__dmul_rn(a, double(xs)));
+                    if (e.acc_out)
+                        e.acc_out[out] = s;
+                }
+            }
+            named_bar_sync(1 + team, 32 * P);  // the slots are rewritten by the next tile
+        }
+#pragma unroll
+        for (int rs = 0; rs < 2; ++rs)
+            acc[rs][0] = acc[rs][1] = 0.0, tot[rs][0] = tot[rs][1] = 0;
+    }
+    cp_async_wait<0>();
+}
+
+BinMmaParams *bin_mma_params()
+{
+    static thread_local BinMmaParams p;
+    return &p;
+}
+
+cudaError_t launch_binary_mma(const BinEntry *entries, int n, cudaStream_t stream)
+{
+    const int sms = device_sm_count();
+    constexpr size_t smem = size_t(kBmW) * kBmRing * kBmStage + size_t(kBmW) * 128 * (8 + 4);
+    static std::atomic<int> configured_dev{-1};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (configured_dev != dev) {
+        err = cudaFuncSetAttribute(binary_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(smem));
+        if (err != cudaSuccess)
+            return err;
+        configured_dev = dev;
+    }
+    for (int base = 0; base < n; base += kBinStackMax) {
+        const int cnt = std::min(n - base, kBinStackMax);
+        BinMmaParams &p = *bin_mma_params();
+        p.n_entries = cnt;
+        int total = 0;
+        for (int j = 0; j < cnt; ++j) {
+            const BinEntry &b = entries[base + j];
+            p.e[j] = BinMmaEntry{b.bits, b.scales, b.xq, b.x_scale, b.y, b.acc_out, b.N8, b.K,
+                                 total, 0};
+            total += (b.N8 + kBmRows - 1) / kBmRows;
+        }
+        if (total == 0)
+            continue;
+        const int grid = std::min({total, sms, kMmaMaxGrid});
+        int lgP = 0;
+        while ((2 << lgP) <= kBmW && (long long)total << lgP < 2LL * kBmW * grid)
+            ++lgP;
+        p.lgP = lgP;
+        std::vector<long long> prefix(size_t(total) + 1, 0);
+        {
+            int tt = 0;
+            for (int j = 0; j < cnt; ++j) {
+                const BinMmaEntry &e = p.e[j];
+                const int tiles = (e.N8 + kBmRows - 1) / kBmRows;
+                for (int i = 0; i < tiles; ++i, ++tt)
+                    prefix[size_t(tt) + 1] =
+                        prefix[size_t(tt)] + (long long)kBmRows * e.K * 9 / 8 + 2048;
+            }
+        }
+        p.cta_tile0[0] = 0;
+        for (int b = 1; b < grid; ++b) {
+            const long long target = prefix[size_t(total)] * b / grid;
+            int tt = int(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
+            tt = std::max(tt, p.cta_tile0[b - 1] + 1);
+            tt = std::min(tt, total - (grid - b));
+            p.cta_tile0[b] = tt;
+        }
+        p.cta_tile0[grid] = total;
+        binary_mma_kernel<<<grid, kBmThreads, smem, stream>>>(p);
+        err = cudaGetLastError();
+        if (err != cudaSuccess)
+            return err;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t launch_binary_gemv(BinEntry *entries, int n, int M, cudaStream_t stream)
@@ -570,6 +924,13 @@ cudaError_t launch_binary_gemv(BinEntry *entries, int n, int M, cudaStream_t str
         return cudaSuccess;
     if (M < 1 || M > kBinMaxTokens || n > kBinStackMax)
         return cudaErrorInvalidValue;
+    // TQ_BINARY_KERNEL=dp4a runs one token on the dp4a kernel too (for measurement)
+    static const bool force_dp4a = [] {
+        const char *v = getenv("TQ_BINARY_KERNEL");
+        return v && !strcmp(v, "dp4a");
+    }();
+    if (M == 1 && !force_dp4a)
+        return launch_binary_mma(entries, n, stream);
     if (n == 1)
         return launch_bin_sized<1>(entries, n, M, stream);
     return launch_bin_sized<kBinStackMax>(entries, n, M, stream);

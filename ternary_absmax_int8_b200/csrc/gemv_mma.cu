@@ -40,6 +40,7 @@
 #include <algorithm>
 #include <vector>
 
+#include "mma_common.cuh"
 #include "tq_internal.h"
 
 namespace tq {
@@ -60,26 +61,6 @@ template <int NT>
 constexpr int kStep = 64 * kHalves<NT>;
 template <int NT>
 constexpr int kStageBytes = 2 * kHalves<NT> * 32 * 16;
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
-{
-    const int n = valid ? 16 : 0;  // 0: fill with zeros, read nothing
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ void mma_u8s8(int32_t (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // A warp's walk over the (tile, step) pairs it computes: the tiles of its
 // team (t_begin + team, + teams, ...) and, in each, its piece

@@ -225,6 +225,26 @@ struct BinParams {
     BinEntry e[MaxE];
 };
 
+// The one-token (M = 1) form on the warp-level MMA: 16-row tiles over all
+// projections, per-CTA ranges balanced by bytes, teams of 2^lgP warps.
+struct BinMmaEntry {
+    const uint8_t *bits;
+    const uint16_t *scales;
+    const int8_t *xq;
+    const float *x_scale;
+    float *y;
+    int32_t *acc_out;
+    int N8, K;
+    int tile_begin, pad_;
+};
+
+struct BinMmaParams {
+    int n_entries, lgP;
+    int cta_tile0[kBinMaxGrid * 2 + 1];
+    BinMmaEntry e[kBinStackMax];
+};
+
+// M == 1: the warp-MMA kernel; M = 2..4: the dp4a kernel.
 cudaError_t launch_binary_gemv(BinEntry *entries, int n, int M, cudaStream_t stream);
 
 // Device address of the library's error word on the current device.

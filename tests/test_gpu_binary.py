@@ -89,3 +89,31 @@ def test_stack_of_8_layers_one_launch(cuda_device):
     for d in ds:
         d.check(threads=THREADS)
     assert tq.tq_device_error(reset=True) == 0
+
+
+def test_one_token_mixed_stack(cuda_device):
+    # one token: a table of ragged projections (tiles of 16 packed rows that
+    # end mid-tile, single-group rows, long rows) in one launch
+    shapes = [("a", 8, 128), ("b", 24, 256), ("c", 4104, 384), ("d", 640, 2560),
+              ("e", 136, 1152), ("f", 2048, 32768), ("g", 8, 30720)]
+    projs = list(make_binary_projections(shapes, M=1, seed=91))
+    ds = [BinDev(p) for p in projs]
+    tq.tq_gemv_binary_stack([d.proj() for d in ds], 1)
+    torch.cuda.synchronize()
+    for d in ds:
+        d.check(threads=THREADS)
+
+
+def test_one_token_degenerate(cuda_device):
+    ps = list(make_binary_projections([("a", 640, 1280), ("b", 264, 1280)], M=1, seed=92))
+    ps[0].w[:] = 1                      # all +1: acc = x_sum
+    ps[1].x_bf16[0] = 0                 # a zero token: x_scale 0, acc 0, y 0
+    for p in ps:
+        d = BinDev(p)
+        tq.tq_gemv_binary(d.bits, d.sp, d.xq, d.xs, d.y, d.acc, 1, p.N, p.K)
+        torch.cuda.synchronize()
+        d.check()
+        if p.name == "a":
+            assert (d.acc.cpu().numpy() == d.xsum.cpu().numpy()[:, None]).all()
+        else:
+            assert not d.acc.cpu().numpy().any() and not d.y.cpu().numpy().any()
