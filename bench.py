@@ -88,13 +88,17 @@ def step_bytes(projs) -> int:
 def step_mode(projs) -> str:
     """How a step launches: "fused" -- one quantising stack launch for every
     projection (M = 1); "batch" -- the stack quantiser, then
-    tq_gemv_stack_batch (M = 2..32); "per_projection" -- a quantiser launch
-    and a GEMV launch per projection (a single projection, or prefill)."""
+    tq_gemv_stack_batch (M = 2..32); "prefill" -- the stack quantiser, then
+    tq_gemm_prefill_stack (M >= 33, several projections); "per_projection" --
+    a quantiser launch and a GEMV launch per projection (a single
+    projection)."""
     M = projs[0].M
     if len(projs) > 1 and M == 1:
         return "fused"
     if len(projs) > 1 and M <= 32:
         return "batch"
+    if len(projs) > 1:
+        return "prefill"
     return "per_projection"
 
 
@@ -105,6 +109,14 @@ def batch_launches(n: int, M: int) -> int:
     launch."""
     per = 64 if batch_kernel_name(M, "batch") == "smallm_group_kernel" else 256
     return -(-n * M // 512) + -(-n // per)
+
+
+def prefill_launches(n: int, M: int) -> int:
+    """Kernel launches of tq_quantize_act_stack_batch + tq_gemm_prefill_stack
+    over n projections of M >= 33 tokens: 512 token rows per quantiser launch,
+    16 projections per prefill launch (up to 4096 tiles each, which every
+    measured shape stays within)."""
+    return -(-n * M // 512) + -(-n // 16)
 
 
 def workload_step_bytes(workload: str, projs) -> int:
@@ -284,7 +296,7 @@ def run_ours(args, rank: int, world: int):
     def quant(c, s):
         if stack:
             return  # quantised inside the stack launch
-        if mode == "batch":
+        if mode in ("batch", "prefill"):
             tq.tq_quantize_act_stack_batch(tables[c], M, stream=s)
             return
         for j, p in enumerate(projs):
@@ -303,6 +315,9 @@ def run_ours(args, rank: int, world: int):
             # weights may stream while the quantiser drains
             tq.tq_gemv_stack_batch(tables[c], M, flags=tq.TQ_STACK_OVERLAP_PREV, stream=s)
             return
+        if mode == "prefill":
+            tq.tq_gemm_prefill_stack(tables[c], M, stream=s)
+            return
         for j, p in enumerate(projs):
             t = tables[c][j]
             call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill
@@ -312,7 +327,8 @@ def run_ours(args, rank: int, world: int):
         quant(c, s)
         gemv(c, s, first)
 
-    launches_per_step = {"fused": 1, "batch": batch_launches(len(projs), M)}.get(
+    launches_per_step = {"fused": 1, "batch": batch_launches(len(projs), M),
+                         "prefill": prefill_launches(len(projs), M)}.get(
         mode, sum(1 + gemv_launches(p.M) for p in projs))
 
     def barrier():
@@ -498,10 +514,12 @@ def run_ours(args, rank: int, world: int):
         "quant_us_per_step": round(quant_ms_step * 1e3, 3),
         "gemv_us_per_step": round(gemv_avg * 1e3, 3),
         "quantiser": {"fused": "fused into the stack launch",
-                      "batch": "one stack quantiser launch for all projections"}.get(
+                      "batch": "one stack quantiser launch for all projections",
+                      "prefill": "one stack quantiser launch for all projections"}.get(
                           mode, "separate launch per projection"),
         "launch_form": {"fused": "one quantising tq_gemv_stack launch",
-                        "batch": "tq_quantize_act_stack_batch + tq_gemv_stack_batch"}
+                        "batch": "tq_quantize_act_stack_batch + tq_gemv_stack_batch",
+                        "prefill": "tq_quantize_act_stack_batch + tq_gemm_prefill_stack"}
         .get(mode, "tq_quantize_act + tq_gemv / tq_gemm_prefill per projection"),
         "roofline": roof,
         "e2e": {
@@ -535,6 +553,14 @@ def batch_kernel_name(M: int, mode: str) -> str:
     if forced == "mma" or forced == "" and M <= 16:
         return "mma_gemv_kernel"
     return "smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"
+
+
+def binary_kernel_name(M: int) -> str:
+    """The binary g128 kernel the library runs for M tokens (the warp-MMA
+    kernel for one token unless TQ_BINARY_KERNEL=dp4a forces the dp4a one)."""
+    if M == 1 and os.environ.get("TQ_BINARY_KERNEL", "") != "dp4a":
+        return "binary_mma_kernel"
+    return "binary_gemv_kernel"
 
 
 def gemv_launches(M: int) -> int:
@@ -672,16 +698,18 @@ def run_next(args, rank: int, world: int):
                                             xsum.data_ptr() + 4 * j * M, p.M, p.K,
                                             HADAMARD_BLOCK, stream=s_)
 
+        ptabs = [[tq.make_proj(packed=W[j][c], xq=xq.data_ptr() + int(kx[j]),
+                               x_scale=xs.data_ptr() + 4 * j * M,
+                               x_sum=xsum.data_ptr() + 4 * j * M,
+                               y=y_dev.data_ptr() + 4 * int(ny[j]), w_scale=float(p.w_scale),
+                               N=p.N, K=p.K) for j, p in enumerate(projs)] for c in range(copies)]
+
         def gemv(c, s_):
-            for j, p in enumerate(projs):
-                tq.tq_gemm_prefill(W[j][c], float(p.w_scale), xq.data_ptr() + int(kx[j]),
-                                   xs.data_ptr() + 4 * j * M, xsum.data_ptr() + 4 * j * M,
-                                   y_dev.data_ptr() + 4 * int(ny[j]), None, p.M, p.N, p.K,
-                                   stream=s_)
+            tq.tq_gemm_prefill_stack(ptabs[c], M, stream=s_)
 
         sb = sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
         gemv_units = sum(2.0 * p.M * p.N * p.K for p in projs)
-        launches = 2 * n
+        launches = n + -(-n // 16)
         kernel = "prefill_tc_kernel"
     else:
         B = []
@@ -709,7 +737,7 @@ def run_next(args, rank: int, world: int):
         sb = sum(quant_bytes(p.K, p.M) + binary_bytes(p.N, p.K, p.M) for p in projs)
         gemv_units = float(sum(binary_bytes(p.N, p.K, p.M) for p in projs))
         launches = 2
-        kernel = "binary_gemv_kernel"
+        kernel = binary_kernel_name(M)
 
     def step(c, s_):
         quant(c, s_)

@@ -115,9 +115,12 @@ tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq,
 
 /*
  * tq_gemm_prefill -- the same contract as tq_gemv for any M >= 1 (prompt
- * processing). M >= 128 runs on the tensor cores (tcgen05, int8 in, int32
- * accumulators in tensor memory, the 2-bit codes expanded in shared memory);
- * smaller M runs tq_gemv's kernels. TQ_ERR_UNSUPPORTED for K > 32768.
+ * processing; prefill is set by the matrix units: 1bit engine blog, "Qwen3.8-27B
+ * at 45.7 tok/s ..."). M >= 33 runs on the tensor cores (tcgen05, int8 in,
+ * int32 accumulators in tensor memory, the 2-bit codes expanded in shared
+ * memory, 128-feature x 256-token tiles, 128-token tiles for M <= 128);
+ * smaller M runs tq_gemv's kernels. TQ_ERR_UNSUPPORTED for K > 32768,
+ * N > 2^21 or M > 2^22.
  */
 tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq,
                           const float *x_scale, const int32_t *x_sum, float *y,
@@ -226,6 +229,24 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
  */
 tq_status tq_quantize_act_stack_batch(const tq_proj *projs, int n_proj, int M,
                                       cudaStream_t stream);
+
+/*
+ * tq_gemm_prefill_stack -- tq_gemm_prefill for several independent
+ * projections at the same M (the rows of a prompt through, say, the gate
+ * and up projections of a layer, or through several layers' projections
+ * whose inputs are ready), each with the [M, K] / [M] / [M, N] shapes of the
+ * _batch calls above. projs is a HOST array read during the call only; x,
+ * flags-only fields and `reserved` are ignored. For M >= 33 one launch takes
+ * up to 16 projections: the 128-feature tiles of all of them are dealt to
+ * persistent CTAs longest first (by K), so that projections too small to
+ * fill the GPU alone fill it together, and each CTA's accumulator is
+ * double-buffered in tensor memory so that its output stores overlap the
+ * next tile's MMAs. M <= 32 runs tq_gemv_stack_batch. Results are those of
+ * tq_gemm_prefill on each projection, bit for bit. Projections are
+ * independent: no output may be another's input and no buffer may be shared.
+ * Errors: those of tq_gemm_prefill for any entry (nothing is launched).
+ */
+tq_status tq_gemm_prefill_stack(const tq_proj *projs, int n_proj, int M, cudaStream_t stream);
 tq_status tq_gemv_stack_batch(const tq_proj *projs, int n_proj, int M, unsigned flags,
                               cudaStream_t stream);
 

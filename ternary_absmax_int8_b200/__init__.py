@@ -19,7 +19,7 @@ __all__ = [
     "TQ_STACK_RELU2_MUL", "TqProj", "lib_path",
     "tq_pack_host", "tq_quantize_act", "tq_gemv", "tq_gemm_prefill",
     "tq_quantize_act_stack", "tq_gemv_stack", "tq_quantize_act_stack_batch",
-    "tq_gemv_stack_batch", "tq_device_error", "tq_gemv_noalloc",
+    "tq_gemv_stack_batch", "tq_gemm_prefill_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
     "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack", "tq_selftest_wait_timeout",
     "tq_hadamard_quantize_act", "TqBinaryProj", "tq_pack_binary_host", "tq_gemv_binary",
@@ -92,6 +92,7 @@ _SIGS = {
     "tq_gemv_stack": [ctypes.POINTER(TqProj), _i, ctypes.c_uint, _vp],
     "tq_quantize_act_stack_batch": [ctypes.POINTER(TqProj), _i, _i, _vp],
     "tq_gemv_stack_batch": [ctypes.POINTER(TqProj), _i, _i, ctypes.c_uint, _vp],
+    "tq_gemm_prefill_stack": [ctypes.POINTER(TqProj), _i, _i, _vp],
     "tq_device_error": [ctypes.POINTER(ctypes.c_uint32), _i],
     "tq_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
     "tq_relu2_mul_rmsnorm_quantize": [_vp, _vp, _vp, _f, _vp, _vp, _vp, _i, _i, _vp],
@@ -280,6 +281,11 @@ def tq_quantize_act_stack_batch(projs, M: int, stream=None) -> None:
 def tq_gemv_stack_batch(projs, M: int, flags: int = 0, stream=None) -> None:
     arr, n = _proj_array(projs)
     _check(_load().tq_gemv_stack_batch(arr, n, int(M), int(flags), _stream(stream)))
+
+
+def tq_gemm_prefill_stack(projs, M: int, stream=None) -> None:
+    arr, n = _proj_array(projs)
+    _check(_load().tq_gemm_prefill_stack(arr, n, int(M), _stream(stream)))
 
 
 def tq_device_error(reset: bool = False) -> int:

@@ -1,5 +1,6 @@
 // gemm_tc.cu -- prompt-processing (M >= 33 tokens) ternary GEMM on the
-// 5th-generation tensor cores (tcgen05, int8, accumulators in tensor memory).
+// 5th-generation tensor cores (tcgen05, int8, accumulators in tensor memory),
+// one projection or a group of projections per launch.
 //
 // Prompt processing is bound by the GPU's matrix units rather than by bytes
 // (1bit engine blog, "Qwen3.8-27B at 45.7 tok/s ..."): at M = 512 every
@@ -13,33 +14,31 @@
 //   acc[m, n] = D[n, m] - x_sum[m]          (since w = c - 1)
 //   y[m, n] = float(acc) * (w_scale * x_scale[m])
 //
-// Tile: G x 128 output features x BN tokens, K in stages of 128 bytes; G (1
-// or 2) MMA groups of 128 rows share each activation stage, so the
-// activation operand is read from L2 once per G x 128 features. In group g,
-// MMA row r = 32 p + j is feature i0 + 32 g + j + p N/4: one TMA tile of
-// G x 32 packed rows (128B-swizzled) expands into the G A operands of 16 KB.
-// The host picks (G, BN) in {(2,256), (1,256), (1,128)} for the least
-// estimated time (waves of tiles over the SMs x cycles per K stage;
-// larger tiles on ties), since a 512-token prompt through a 2560-feature
-// projection makes only 20 tiles of the largest shape.
+// Tile: 128 output features x BN tokens (BN = 256, or 128 for M <= 128), K in
+// stages of 128 bytes. MMA row r = 32 p + j is feature i0 + j + p N/4: one
+// TMA tile of 32 packed rows (128B-swizzled) expands into the 16 KB A
+// operand of the stage. A launch takes the tiles of all its projections
+// (shapes and K may differ) and deals them to persistent CTAs by a static
+// longest-first schedule computed on the host, so that projections too
+// small to fill the GPU alone fill it together.
 //
-// Warp roles (14 warps, one CTA per SM, persistent over tiles):
+// Warp roles (18 warps, one CTA per SM):
 //   warp 0       TMA producer: packed tile + activation tile per K stage
 //   warp 1       TMEM allocator; lane 0 issues the MMAs and commits
-//   warps 2..13  expand the codes into the A stage (canonical K-major, 128B
+//   warps 2..9   expand the codes into the A stage (canonical K-major, 128B
 //                swizzle), fence to the async proxy, signal the MMA
-//   warps 6..13  then run the tile's epilogue: warp w reads TMEM lane
-//                quarter w % 4 of its group (G = 2) or of its half of the
-//                columns (G = 1), subtracts x_sum, scales, stores y
-// The accumulator (G x BN columns) is single-buffered: a CTA's next tile
-// starts its MMAs once the epilogue has drained it, so the epilogue warps
-// are free to expand codes during the main loop (expansion, 16 bytes of
-// shared-memory stores per 4 bytes of weights, is what bounds a stage
-// otherwise). Every mbarrier wait is
-// bounded; loads never use cluster multicast.
+//   warps 10..17 epilogue: warp w reads TMEM lane quarter w % 4 (the plane)
+//                over half of the tile's columns, subtracts x_sum, scales and
+//                stores y
+// The accumulator is double-buffered in tensor memory (2 x BN columns): the
+// MMAs of a CTA's next tile run while the epilogue warps drain the previous
+// one, so the output stores (4 bytes per element, as many bytes as the
+// weights many times over at M = 512) overlap the contraction. Every mbarrier
+// wait is bounded; loads never use cluster multicast.
 #include <atomic>
 #include <algorithm>
 #include <cstring>
+#include <vector>
 
 #include "tc_common.cuh"
 
@@ -47,72 +46,110 @@ namespace tq {
 
 namespace {
 
-constexpr int kGM = 128;                // MMA M: rows of one group
-constexpr int kBK = 128;                // bytes of K per stage
-constexpr int kAGroupBytes = kGM * kBK; // 16 KB
-constexpr int kThreads = 448;
-constexpr int kExpWarp0 = 2;             // warps 2..13 expand codes
-constexpr int kExpWarps = 12;
-constexpr int kEpiWarp0 = 6;             // warps 6..13 also run the epilogue
-constexpr int kEpiWarps = 8;
+constexpr int kGM = 128;                 // MMA M: rows of a tile
+constexpr int kBK = 128;                 // bytes of K per stage
+constexpr int kABytes = kGM * kBK;       // 16 KB
+constexpr int kPackedRows = 32;          // packed rows per tile
+constexpr int kPBytes = kPackedRows * kBK;
+constexpr int kExpWarp0 = 2, kExpWarps = 8;
+constexpr int kEpiWarp0 = kExpWarp0 + kExpWarps, kEpiWarps = 8;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;  // 576
 constexpr size_t kSmemLimit = 227 * 1024;
 
-struct PrefillParams {
-    int N4, K, M;
-    int feat_tiles, tok_tiles, k_stages;
+// A tile of a group launch: projection (4 bits), token tile (14 bits),
+// feature tile (14 bits).
+__host__ __device__ constexpr uint32_t tile_code(int e, int tt, int ft)
+{
+    return (uint32_t(e) << 28) | (uint32_t(tt) << 14) | uint32_t(ft);
+}
+constexpr int kTileField = 1 << 14;
+
+struct PrefillProj {
+    int N4, KS;  // packed rows, K stages
+    int vec;     // outputs written four features per 16-byte store (N4 % 4 == 0, aligned)
     float w_scale;
     const float *x_scale;
     const int32_t *x_sum;
     float *y;
     int32_t *acc_out;
-    unsigned *err;
 };
 
-template <int G, int BN>
+// The launch's table (a kernel parameter; tensor maps 64-byte aligned).
+struct PrefillTable {
+    CUtensorMap map_p[kPrefillMaxGroup];
+    CUtensorMap map_x[kPrefillMaxGroup];
+    PrefillProj e[kPrefillMaxGroup];
+    int n, M;
+    unsigned *err;
+    int cta0[kPrefillMaxGrid + 1];  // CTA b works through tile[cta0[b] .. cta0[b + 1] - 1]
+    uint32_t tile[kPrefillMaxTiles];
+};
+static_assert(sizeof(PrefillTable) <= 32000, "kernel parameters");
+
+template <int BN>
 struct PrefillShape {
-    static constexpr int kPackedRows = 32 * G;          // packed rows per tile
-    static constexpr int kABytes = G * kAGroupBytes;
     static constexpr int kBBytes = BN * kBK;
-    static constexpr int kPBytes = kPackedRows * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
-    static constexpr int kBarCount_(int s) { return 4 * s + 2; }
+    static constexpr int kBarCount_(int s) { return 4 * s + 4; }
     // as many stages as fit next to the barriers and the 1 KB alignment slack
     static constexpr int kStages =
-        int((kSmemLimit - 1024 - 256) / size_t(kStageBytes)) > 6
+        int((kSmemLimit - 1024 - 512) / size_t(kStageBytes)) > 6
             ? 6
-            : int((kSmemLimit - 1024 - 256) / size_t(kStageBytes));
-    static constexpr int kAccCols = G * BN;
-    static constexpr int kTmemCols = kAccCols < 32 ? 32 : kAccCols;  // a power of two here
+            : int((kSmemLimit - 1024 - 512) / size_t(kStageBytes));
+    static constexpr int kTmemCols = 2 * BN;  // two accumulators
     // 1024-byte aligned operand stages (the 128B swizzle atom is 1 KB)
     static constexpr size_t a_off = 0;
     static constexpr size_t b_off = a_off + size_t(kStages) * kABytes;
     static constexpr size_t p_off = b_off + size_t(kStages) * kBBytes;
     static constexpr size_t bar_off = p_off + size_t(kStages) * kPBytes;
-    // barriers: tma_full, a_full, mma_done, p_free per stage; acc_full, acc_empty
+    // barriers: tma_full, a_full, mma_done, p_free per stage; acc_full[2], acc_empty[2]
     static constexpr size_t tmem_slot_off = bar_off + size_t(kBarCount_(kStages)) * 8;
     static constexpr size_t bytes = tmem_slot_off + 16;
-    static_assert(kStages >= 2, "two stages at least");
+    static_assert(kStages >= 3, "three stages at least");
     static_assert(bytes + 1024 <= kSmemLimit, "shared memory");
     static_assert((kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512, "tensor memory");
 };
 
-// One output element: y (and the exact accumulator when asked).
-__device__ __forceinline__ void store_out(const PrefillParams &p, int m, int n, int32_t d,
+// One output element: y (and the exact accumulator when asked); streaming
+// stores (the outputs are not read again by this kernel).
+__device__ __forceinline__ void store_out(const PrefillProj &e, int N, int m, int n, int32_t d,
                                           float t, int32_t xs)
 {
     const int32_t acc = d - xs;
-    const size_t o = size_t(m) * (4 * size_t(p.N4)) + n;
-    p.y[o] = __fmul_rn(__int2float_rn(acc), t);
-    if (p.acc_out)
-        p.acc_out[o] = acc;
+    const size_t o = size_t(m) * size_t(N) + n;
+    __stcs(e.y + o, __fmul_rn(__int2float_rn(acc), t));
+    if (e.acc_out)
+        __stcs(e.acc_out + o, acc);
 }
 
-template <int G, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_x,
-                  const __grid_constant__ PrefillParams p)
+// 4 x 4 transpose within each quad of lanes: lane 4a + i holds m[k] = the
+// value of feature 4a + i at token k (k = 0..3); on return f[j] = the value
+// of feature 4a + j at token i (two rounds of exchanges, lanes i ^ 2 then i ^ 1).
+__device__ __forceinline__ void quad_transpose(const int32_t (&m)[4], int32_t (&f)[4], int i)
 {
-    using S = PrefillShape<G, BN>;
+    const bool b1 = i & 2, b0 = i & 1;
+    // round 1: keep the tokens whose bit 1 equals ours, trade the others
+    const int32_t r0 = __shfl_xor_sync(0xffffffffu, b1 ? m[0] : m[2], 2);
+    const int32_t r1 = __shfl_xor_sync(0xffffffffu, b1 ? m[1] : m[3], 2);
+    const int32_t k0 = b1 ? m[2] : m[0], k1 = b1 ? m[3] : m[1];
+    // w[rb][kb]: rb = bit 1 of the feature, kb = bit 0 of the token
+    const int32_t w00 = b1 ? r0 : k0, w01 = b1 ? r1 : k1;
+    const int32_t w10 = b1 ? k0 : r0, w11 = b1 ? k1 : r1;
+    // round 2: keep kb == bit 0 of ours, trade the other
+    const int32_t u0 = __shfl_xor_sync(0xffffffffu, b0 ? w00 : w01, 1);
+    const int32_t u1 = __shfl_xor_sync(0xffffffffu, b0 ? w10 : w11, 1);
+    const int32_t c0 = b0 ? w01 : w00, c1 = b0 ? w11 : w10;
+    f[0] = b0 ? u0 : c0;
+    f[1] = b0 ? c0 : u0;
+    f[2] = b0 ? u1 : c1;
+    f[3] = b0 ? c1 : u1;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
+{
+    using S = PrefillShape<BN>;
     constexpr int kStages = S::kStages;
     constexpr uint32_t kIdesc = idesc_i8_u8s8(kGM, BN);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -127,25 +164,29 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
     uint64_t *a_full = bars + kStages;
     uint64_t *mma_done = bars + 2 * kStages;
     uint64_t *p_free = bars + 3 * kStages;
-    uint64_t *acc_full = bars + 4 * kStages;
-    uint64_t *acc_empty = acc_full + 1;
+    uint64_t *acc_full = bars + 4 * kStages;  // [2]
+    uint64_t *acc_empty = acc_full + 2;       // [2]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = p.feat_tiles * p.tok_tiles;
-    const int KS = p.k_stages;
+    const int t_begin = tab.cta0[blockIdx.x], t_end = tab.cta0[blockIdx.x + 1];
+    unsigned *err = tab.err;
 
     if (threadIdx.x == 0) {
-        prefetch_tensormap(&map_p);
-        prefetch_tensormap(&map_x);
+        for (int j = 0; j < tab.n; ++j) {
+            prefetch_tensormap(&tab.map_p[j]);
+            prefetch_tensormap(&tab.map_x[j]);
+        }
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&tma_full[s], 1);
             mbar_init(&a_full[s], kExpWarps);
             mbar_init(&mma_done[s], 1);
             mbar_init(&p_free[s], kExpWarps);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kEpiWarps);
+        }
         fence_mbar_init();
     }
     if (warp == 1)
@@ -162,20 +203,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-                const int ft = t / p.tok_tiles, tt = t - ft * p.tok_tiles;
+            for (int i = t_begin; i < t_end && ok; ++i) {
+                const uint32_t code = tab.tile[i];
+                const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
+                          ft = int(code & (kTileField - 1));
+                const int KS = tab.e[e].KS;
                 for (int ks = 0; ks < KS; ++ks) {
                     if (issued >= kStages) {
-                        if (!mbar_wait(&mma_done[stage], phase ^ 1u, p.err) ||
-                            !mbar_wait(&p_free[stage], phase ^ 1u, p.err)) {
+                        if (!mbar_wait(&mma_done[stage], phase ^ 1u, err) ||
+                            !mbar_wait(&p_free[stage], phase ^ 1u, err)) {
                             ok = false;
                             break;
                         }
                     }
-                    mbar_arrive_expect_tx(&tma_full[stage], S::kPBytes + S::kBBytes);
-                    tma_load_2d(sP + stage * S::kPBytes, &map_p, ks * kBK, ft * S::kPackedRows,
+                    mbar_arrive_expect_tx(&tma_full[stage], kPBytes + S::kBBytes);
+                    tma_load_2d(sP + stage * kPBytes, &tab.map_p[e], ks * kBK, ft * kPackedRows,
                                 &tma_full[stage]);
-                    tma_load_2d(sB + stage * S::kBBytes, &map_x, ks * kBK, tt * BN, &tma_full[stage]);
+                    tma_load_2d(sB + stage * S::kBBytes, &tab.map_x[e], ks * kBK, tt * BN,
+                                &tma_full[stage]);
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -186,7 +231,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
             // wait for the copies still in flight before the CTA may retire
             for (int s = 0; s < kStages && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % kStages);  // last use of stage s
-                mbar_wait(&tma_full[s], uint32_t((last / kStages) & 1), p.err);
+                mbar_wait(&tma_full[s], uint32_t((last / kStages) & 1), err);
             }
         }
     } else if (warp == 1) {
@@ -194,31 +239,31 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int local = 0;
             bool ok = true;
             int issued = 0;
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
-                if (local >= 1 && !mbar_wait(acc_empty, uint32_t((local - 1) & 1), p.err))
+            for (int i = t_begin, local = 0; i < t_end && ok; ++i, ++local) {
+                const int buf = local & 1;
+                // the epilogue has drained this accumulator's previous tile
+                if (local >= 2 && !mbar_wait(&acc_empty[buf], uint32_t(((local - 2) >> 1) & 1), err))
                     break;
                 tc_fence_after();
+                const uint32_t d_tmem = tmem_base + uint32_t(buf * BN);
+                const int KS = tab.e[tab.tile[i] >> 28].KS;
                 for (int ks = 0; ks < KS; ++ks) {
-                    if (!mbar_wait(&tma_full[stage], phase, p.err) ||
-                        !mbar_wait(&a_full[stage], phase, p.err)) {
+                    if (!mbar_wait(&tma_full[stage], phase, err) ||
+                        !mbar_wait(&a_full[stage], phase, err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     // one descriptor per operand and stage, advanced by adds
-                    const uint64_t da = umma_desc_sw128(smem_u32(sA + stage * S::kABytes));
+                    const uint64_t da = umma_desc_sw128(smem_u32(sA + stage * kABytes));
                     const uint64_t db = umma_desc_sw128(smem_u32(sB + stage * S::kBBytes));
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int kk = 0; kk < kBK / 32; ++kk)
-                            umma_i8(tmem_base + uint32_t(g * BN),
-                                    umma_desc_advance(da, uint32_t(g * kAGroupBytes + kk * 32)),
-                                    umma_desc_advance(db, uint32_t(kk * 32)), kIdesc,
-                                    (ks > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        umma_i8(d_tmem, umma_desc_advance(da, uint32_t(kk * 32)),
+                                umma_desc_advance(db, uint32_t(kk * 32)), kIdesc,
+                                (ks > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&mma_done[stage]);
                     ++issued;
                     if (++stage == kStages) {
@@ -227,56 +272,44 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     }
                 }
                 if (ok)
-                    umma_commit(acc_full);
+                    umma_commit(&acc_full[buf]);
             }
             // the last commit tracks every MMA this thread issued
             if (issued > 0) {
                 const int s = (issued - 1) % kStages;
-                mbar_wait(&mma_done[s], uint32_t(((issued - 1) / kStages) & 1), p.err);
+                mbar_wait(&mma_done[s], uint32_t(((issued - 1) / kStages) & 1), err);
             }
         }
-    } else {
-        // -------------------------- code expansion, then (warps 6..13) epilogue
-        const int et = threadIdx.x - kExpWarp0 * 32;  // 0..383
-        const bool epi = warp >= kEpiWarp0;
-        const int q = warp & 3;                  // TMEM lane quarter = plane
-        const int sub = (warp - kEpiWarp0) >> 2;
-        const int eg = G == 2 ? sub : 0;         // MMA group of this epilogue warp
-        const int cb = G == 2 ? 0 : sub * (BN / 2);  // its columns: [cb, cb + ncol)
-        constexpr int ncol = G == 2 ? BN : BN / 2;
-        constexpr int kUnits = S::kPackedRows * 8;   // 16-byte chunks of packed bytes per stage
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------ code expansion
+        // thread et expands 16-byte chunk et of the stage's packed tile:
+        // packed row j = et / 8, chunk c = et % 8
+        const int et = threadIdx.x - kExpWarp0 * 32;  // 0..255
+        const int j = et >> 3, c = et & 7;
+        static_assert(kExpWarps * 32 == kPackedRows * 8, "one chunk per expansion thread");
         int stage = 0;
         uint32_t phase = 0;
         int seen = 0;
-        int local = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++local) {
+        for (int i = t_begin; i < t_end && ok; ++i) {
+            const int KS = tab.e[tab.tile[i] >> 28].KS;
             for (int ks = 0; ks < KS; ++ks) {
-                bool w1 = mbar_wait_warp(&tma_full[stage], phase, p.err);
-                bool w2 = w1 && (seen < kStages || mbar_wait_warp(&mma_done[stage], phase ^ 1u, p.err));
+                const bool w1 = mbar_wait_warp(&tma_full[stage], phase, err);
+                const bool w2 =
+                    w1 && (seen < kStages || mbar_wait_warp(&mma_done[stage], phase ^ 1u, err));
                 if (!w2) {
                     ok = false;
                     break;
                 }
-                const uint8_t *P = sP + stage * S::kPBytes;
-                uint8_t *A = sA + stage * S::kABytes;
+                const uint4 v = *reinterpret_cast<const uint4 *>(sP + stage * kPBytes + sw128_off(j, c));
+                uint8_t *A = sA + stage * kABytes;
+                // plane bits left in place: code c held as c * 4^pl (<= 128, a
+                // u8), one AND per word; the epilogue shifts the sums back
 #pragma unroll
-                for (int h = 0; h < (kUnits + kExpWarps * 32 - 1) / (kExpWarps * 32); ++h) {
-                    const int idx = et + h * kExpWarps * 32;  // (packed row j of the tile, chunk c)
-                    if (idx < kUnits) {
-                        const int j = idx >> 3, c = idx & 7;
-                        const int g = j >> 5, jj = j & 31;
-                        const uint4 v = *reinterpret_cast<const uint4 *>(P + sw128_off(j, c));
-                        uint8_t *Ag = A + g * kAGroupBytes;
-// plane bits left in place: code c held as c * 4^pl (<= 128, a u8),
-                        // one AND per word; the epilogue shifts the sums back
-#pragma unroll
-                        for (int pl = 0; pl < 4; ++pl) {
-                            const uint32_t m = 0x03030303u << (2 * pl);
-                            const uint4 o = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
-                            *reinterpret_cast<uint4 *>(Ag + sw128_off(jj + 32 * pl, c)) = o;
-                        }
-                    }
+                for (int pl = 0; pl < 4; ++pl) {
+                    const uint32_t m = 0x03030303u << (2 * pl);
+                    const uint4 o = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
+                    *reinterpret_cast<uint4 *>(A + sw128_off(j + 32 * pl, c)) = o;
                 }
                 fence_proxy_async_smem();  // make the codes visible to the tensor cores
                 __syncwarp();
@@ -290,38 +323,79 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
                     phase ^= 1u;
                 }
             }
-            if (!epi || !ok)
-                continue;
-            // ---- epilogue of tile t
-            const int ft = t / p.tok_tiles, tt = t - ft * p.tok_tiles;
-            if (!mbar_wait_warp(acc_full, uint32_t(local & 1), p.err))
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;                           // TMEM lane quarter = plane
+        const int half = (warp - kEpiWarp0) >> 2;         // its half of the columns
+        constexpr int ncol = BN / 2;
+        const int cb = half * ncol;
+        for (int i = t_begin, local = 0; i < t_end; ++i, ++local) {
+            const uint32_t code = tab.tile[i];
+            const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
+                      ft = int(code & (kTileField - 1));
+            const PrefillProj &pe = tab.e[e];
+            const int buf = local & 1;
+            if (!mbar_wait_warp(&acc_full[buf], uint32_t((local >> 1) & 1), err))
                 break;
             tc_fence_after();
-            const int prow = ft * S::kPackedRows + eg * 32 + lane;  // packed row of this lane
-            const bool row_ok = prow < p.N4;
-            const int n = prow + q * p.N4;
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(eg * BN + cb);
+            const int N4 = pe.N4, N = 4 * N4;
+            const int prow = ft * kPackedRows + lane;  // packed row of this lane
+            const bool row_ok = prow < N4;
+            const int n = prow + q * N4;
+            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN + cb);
             for (int c0 = 0; c0 < ncol; c0 += 32) {
                 const int mbase = tt * BN + cb + c0;
-                if (mbase >= p.M)
+                if (mbase >= tab.M)
                     break;
                 uint32_t v[32];
                 tmem_ld32(tbase + uint32_t(c0), v);
                 const int my_m = mbase + lane;
-                const float my_t = my_m < p.M ? __fmul_rn(p.w_scale, __ldg(p.x_scale + my_m)) : 0.0f;
-                const int32_t my_s = my_m < p.M ? __ldg(p.x_sum + my_m) : 0;
+                const float my_t =
+                    my_m < tab.M ? __fmul_rn(pe.w_scale, __ldg(pe.x_scale + my_m)) : 0.0f;
+                const int32_t my_s = my_m < tab.M ? __ldg(pe.x_sum + my_m) : 0;
+                if (pe.vec) {
+                    // quads of lanes trade values so that each lane writes four
+                    // consecutive features of one token: a 16-byte store
+                    const int i4 = lane & 3;
+                    const int f0 = ft * kPackedRows + (lane & ~3);  // first feature of the quad
+                    const size_t n0 = size_t(f0) + size_t(q) * N4;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float ts = __shfl_sync(0xffffffffu, my_t, i);
-                    const int32_t xs = __shfl_sync(0xffffffffu, my_s, i);
-                    if (row_ok && mbase + i < p.M)
-                        store_out(p, mbase + i, n, int32_t(v[i]) >> (2 * q), ts, xs);
+                    for (int k0 = 0; k0 < 32; k0 += 4) {
+                        const int32_t m4[4] = {int32_t(v[k0]) >> (2 * q), int32_t(v[k0 + 1]) >> (2 * q),
+                                               int32_t(v[k0 + 2]) >> (2 * q),
+                                               int32_t(v[k0 + 3]) >> (2 * q)};
+                        int32_t f4[4];
+                        quad_transpose(m4, f4, i4);
+                        const int tk = k0 + i4;  // this lane's token in the chunk
+                        const float ts = __shfl_sync(0xffffffffu, my_t, tk);
+                        const int32_t xs = __shfl_sync(0xffffffffu, my_s, tk);
+                        if (f0 < N4 && mbase + tk < tab.M) {
+                            const size_t o = size_t(mbase + tk) * size_t(N) + n0;
+                            const int4 a4 = make_int4(f4[0] - xs, f4[1] - xs, f4[2] - xs, f4[3] - xs);
+                            __stcs(reinterpret_cast<float4 *>(pe.y + o),
+                                   make_float4(__fmul_rn(__int2float_rn(a4.x), ts),
+                                               __fmul_rn(__int2float_rn(a4.y), ts),
+                                               __fmul_rn(__int2float_rn(a4.z), ts),
+                                               __fmul_rn(__int2float_rn(a4.w), ts)));
+                            if (pe.acc_out)
+                                __stcs(reinterpret_cast<int4 *>(pe.acc_out + o), a4);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const float ts = __shfl_sync(0xffffffffu, my_t, k);
+                        const int32_t xs = __shfl_sync(0xffffffffu, my_s, k);
+                        if (row_ok && mbase + k < tab.M)
+                            store_out(pe, N, mbase + k, n, int32_t(v[k]) >> (2 * q), ts, xs);
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(acc_empty);
+                mbar_arrive(&acc_empty[buf]);
         }
     }
 
@@ -333,89 +407,142 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_consta
         tmem_dealloc(tmem_base, S::kTmemCols);
 }
 
-template <int G, int BN>
-cudaError_t launch_shape(const uint8_t *packed, const int8_t *xq, PrefillParams prm,
-                         cudaStream_t stream)
+// Deal the tiles [0, n) (costs cost[i]) to `grid` CTAs, longest first, each
+// to the least-loaded CTA; fill order[] CTA by CTA and cta0[].
+void schedule_lpt(const std::vector<int> &cost, int grid, std::vector<int> &order, int *cta0)
 {
-    using S = PrefillShape<G, BN>;
-    CUtensorMap map_p, map_x;
-    if (!make_map(&map_p, packed, prm.K, prm.N4, S::kPackedRows) ||
-        !make_map(&map_x, xq, prm.K, prm.M, BN))
-        return cudaErrorInvalidValue;
-    prm.feat_tiles = (prm.N4 + S::kPackedRows - 1) / S::kPackedRows;
-    prm.tok_tiles = (prm.M + BN - 1) / BN;
+    const int n = int(cost.size());
+    std::vector<int> idx(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i)
+        idx[size_t(i)] = i;
+    std::stable_sort(idx.begin(), idx.end(),
+                     [&](int a, int b) { return cost[size_t(a)] > cost[size_t(b)]; });
+    std::vector<long long> load(static_cast<size_t>(grid), 0);
+    std::vector<int> owner(static_cast<size_t>(n));
+    for (int i : idx) {
+        int best = 0;
+        for (int b = 1; b < grid; ++b)
+            if (load[size_t(b)] < load[size_t(best)])
+                best = b;
+        owner[size_t(i)] = best;
+        load[size_t(best)] += cost[size_t(i)];
+    }
+    std::vector<int> count(static_cast<size_t>(grid), 0);
+    for (int i = 0; i < n; ++i)
+        ++count[size_t(owner[size_t(i)])];
+    cta0[0] = 0;
+    for (int b = 0; b < grid; ++b)
+        cta0[b + 1] = cta0[b] + count[size_t(b)];
+    std::vector<int> fill(cta0, cta0 + grid);
+    order.assign(size_t(n), 0);
+    for (int i : idx)  // longest first within each CTA too
+        order[size_t(fill[size_t(owner[size_t(i)])]++)] = i;
+}
+
+PrefillTable *prefill_table()
+{
+    static thread_local PrefillTable t;
+    return &t;
+}
+
+template <int BN>
+cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
+{
+    using S = PrefillShape<BN>;
     const size_t smem = S::bytes + 1024;  // + alignment slack
     static std::atomic<int> configured_dev{-1};  // set by any host thread
     int dev = 0;
-    cudaGetDevice(&dev);
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
     if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<G, BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess)
-            return e;
+        err = cudaFuncSetAttribute(prefill_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(smem));
+        if (err != cudaSuccess)
+            return err;
         configured_dev = dev;
     }
-    const int tiles = prm.feat_tiles * prm.tok_tiles;
-    const int grid = std::min(tiles, device_sm_count());
-    prefill_tc_kernel<G, BN><<<grid, kThreads, smem, stream>>>(map_p, map_x, prm);
-    return cudaGetLastError();
+    unsigned *err_word = device_error_word();
+    if (!err_word)
+        return cudaErrorUnknown;
+    const int tok_tiles = (M + BN - 1) / BN;
+    // every tile of every projection, in projection order
+    std::vector<uint32_t> codes;
+    std::vector<int> cost;
+    for (int j = 0; j < n; ++j) {
+        const int ft_tiles = (in[j].N / 4 + kPackedRows - 1) / kPackedRows;
+        const int KS = (in[j].K + kBK - 1) / kBK;
+        for (int ft = 0; ft < ft_tiles; ++ft)
+            for (int tt = 0; tt < tok_tiles; ++tt) {
+                codes.push_back(tile_code(j, tt, ft));
+                cost.push_back(KS);
+            }
+    }
+    PrefillTable &tab = *prefill_table();
+    std::memset(static_cast<void *>(&tab), 0, sizeof(tab));
+    tab.n = n;
+    tab.M = M;
+    tab.err = err_word;
+    for (int j = 0; j < n; ++j) {
+        if (!make_map(&tab.map_p[j], in[j].packed, in[j].K, in[j].N / 4, kPackedRows) ||
+            !make_map(&tab.map_x[j], in[j].xq, in[j].K, M, BN))
+            return cudaErrorInvalidValue;
+        const bool vec = (in[j].N / 4) % 4 == 0 && reinterpret_cast<uintptr_t>(in[j].y) % 16 == 0 &&
+                         reinterpret_cast<uintptr_t>(in[j].acc_out) % 16 == 0;
+        tab.e[j] = PrefillProj{in[j].N / 4, (in[j].K + kBK - 1) / kBK, vec ? 1 : 0, in[j].w_scale,
+                               in[j].x_scale, in[j].x_sum, in[j].y, in[j].acc_out};
+    }
+    // launches of up to kPrefillMaxTiles tiles each (any subset of tiles is a
+    // valid launch); one launch for every shape this library is measured on
+    const int sms = device_sm_count();
+    const int total = int(codes.size());
+    for (int base = 0; base < total; base += kPrefillMaxTiles) {
+        const int cnt = std::min(total - base, kPrefillMaxTiles);
+        const int grid = std::min({cnt, sms, kPrefillMaxGrid});
+        std::vector<int> sub(cost.begin() + base, cost.begin() + base + cnt), order;
+        schedule_lpt(sub, grid, order, tab.cta0);
+        for (int i = 0; i < cnt; ++i)
+            tab.tile[i] = codes[size_t(base + order[size_t(i)])];
+        prefill_tc_kernel<BN><<<grid, kThreads, smem, stream>>>(tab);
+        err = cudaGetLastError();
+        if (err != cudaSuccess)
+            return err;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
 
 constexpr int kPrefillMinM = 33;
 
+cudaError_t launch_prefill_group(const PrefillEntry *e, int n, int M, cudaStream_t stream,
+                                 bool *handled)
+{
+    *handled = false;
+    if (M < kPrefillMinM || n <= 0)
+        return cudaSuccess;
+    if (n > kPrefillMaxGroup)
+        return cudaErrorInvalidValue;
+    for (int j = 0; j < n; ++j)
+        if ((e[j].N / 4 + kPackedRows - 1) / kPackedRows > kTileField)
+            return cudaErrorInvalidValue;
+    // 128-token tiles while they waste less of the MMA than 256-token ones
+    const bool narrow = M <= 128;
+    if ((M + (narrow ? 127 : 255)) / (narrow ? 128 : 256) > kTileField)
+        return cudaErrorInvalidValue;
+    const cudaError_t err = narrow ? launch_bn<128>(e, n, M, stream) : launch_bn<256>(e, n, M, stream);
+    if (err == cudaSuccess)
+        *handled = true;
+    return err;
+}
+
 cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
                               const float *x_scale, const int32_t *x_sum, float *y,
                               int32_t *acc_out, int M, int N, int K, cudaStream_t stream,
                               bool *handled)
 {
-    *handled = false;
-    if (M < kPrefillMinM)
-        return cudaSuccess;
-    PrefillParams prm = {};
-    prm.N4 = N / 4;
-    prm.K = K;
-    prm.M = M;
-    prm.k_stages = (K + kBK - 1) / kBK;
-    prm.w_scale = w_scale;
-    prm.x_scale = x_scale;
-    prm.x_sum = x_sum;
-    prm.y = y;
-    prm.acc_out = acc_out;
-    prm.err = device_error_word();
-    if (!prm.err)
-        return cudaErrorUnknown;
-    // Tile shape: the least estimated time = waves of tiles over the SMs x
-    // cycles per K stage of one tile. A stage is 4 G MMAs of K = 32, each
-    // costing its execution (BN / 2 cycles at the int8 rate) or its issue by
-    // the single MMA thread (~100 cycles, measured), whichever is longer,
-    // plus ~100 cycles of pipeline overhead. The larger tile wins ties (fewer
-    // operand re-reads from L2).
-    const int sms = device_sm_count();
-    const int shapes[3][2] = {{2, 256}, {1, 256}, {1, 128}};
-    int best = 0;
-    long long best_cost = -1;
-    for (int i = 0; i < 3; ++i) {
-        const int G = shapes[i][0], BN = shapes[i][1];
-        const long long tiles =
-            (long long)((prm.N4 + 32 * G - 1) / (32 * G)) * ((M + BN - 1) / BN);
-        const long long stage = 4LL * G * std::max(BN / 2, 100) + 100;
-        const long long cost = (tiles + sms - 1) / sms * stage;
-        if (best_cost < 0 || cost < best_cost) {
-            best = i;
-            best_cost = cost;
-        }
-    }
-    cudaError_t e;
-    switch (best) {
-    case 0: e = launch_shape<2, 256>(packed, xq, prm, stream); break;
-    case 1: e = launch_shape<1, 256>(packed, xq, prm, stream); break;
-    default: e = launch_shape<1, 128>(packed, xq, prm, stream); break;
-    }
-    if (e == cudaSuccess)
-        *handled = true;
-    return e;
+    const PrefillEntry e{packed, w_scale, xq, x_scale, x_sum, y, acc_out, N, K};
+    return launch_prefill_group(&e, 1, M, stream, handled);
 }
 
 }  // namespace tq

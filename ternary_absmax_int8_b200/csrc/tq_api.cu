@@ -20,11 +20,6 @@ __device__ unsigned int g_device_error = 0;
 bool pack_ternary_host(const int8_t *w, uint8_t *packed, int N, int K);
 bool pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
                       uint16_t *scales_packed, int N, int K);
-cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
-                              const float *x_scale, const int32_t *x_sum, float *y,
-                              int32_t *acc_out, int M, int N, int K, cudaStream_t stream,
-                              bool *handled);
-
 unsigned *device_error_word()
 {
     static std::atomic<unsigned *> cache[64] = {};
@@ -505,12 +500,60 @@ tq_status tq_gemm_prefill(const uint8_t *packed, float w_scale, const int8_t *xq
     bool handled = false;
     cudaError_t e = tq::launch_prefill_tc(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K,
                                           stream, &handled);
+    if (e == cudaErrorInvalidValue && !handled)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_gemm_prefill: N=%d or M=%d exceeds the tile fields",
+                    N, M);
     if (e != cudaSuccess)
         return cuda_fail(e, "tq_gemm_prefill");
     if (handled)
         return ok();
     return stream_groups(packed, w_scale, xq, x_scale, x_sum, y, acc_out, M, N, K, stream,
                          "tq_gemm_prefill");
+}
+
+tq_status tq_gemm_prefill_stack(const tq_proj *projs, int n_proj, int M, cudaStream_t stream)
+{
+    const char *fn = "tq_gemm_prefill_stack";
+    if (n_proj < 0 || (n_proj > 0 && !projs))
+        return fail(TQ_ERR_NULL, "%s: projs is NULL", fn);
+    if (M < 0)
+        return fail(TQ_ERR_SHAPE, "%s: negative M=%d", fn, M);
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        const tq_status st =
+            check_gemv_args(fn, p.packed, p.xq, p.x_scale, p.x_sum, p.y, p.acc_out, M, p.N, p.K);
+        if (st != TQ_OK)
+            return st;
+    }
+    if (M == 0 || n_proj == 0)
+        return ok();
+    if (M <= 32)  // small batches: the decode kernels
+        return gemv_stack_impl(fn, projs, n_proj, M, 0, stream);
+    std::vector<tq::PrefillEntry> list;
+    list.reserve(size_t(n_proj));
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        if (p.N == 0)
+            continue;
+        if (p.K == 0) {
+            const tq_status st = zero_outputs(p.y, p.acc_out, size_t(M) * p.N, stream);
+            if (st != TQ_OK)
+                return st;
+            continue;
+        }
+        list.push_back(tq::PrefillEntry{p.packed, p.w_scale, p.xq, p.x_scale, p.x_sum, p.y,
+                                        p.acc_out, p.N, p.K});
+    }
+    for (size_t base = 0; base < list.size(); base += tq::kPrefillMaxGroup) {
+        const int n = int(std::min(list.size() - base, size_t(tq::kPrefillMaxGroup)));
+        bool handled = false;
+        const cudaError_t e = tq::launch_prefill_group(list.data() + base, n, M, stream, &handled);
+        if (e == cudaErrorInvalidValue && !handled)
+            return fail(TQ_ERR_UNSUPPORTED, "%s: a shape exceeds the prefill tile fields", fn);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fn);
+    }
+    return ok();
 }
 
 tq_status tq_quantize_act_stack(const tq_proj *projs, int n_proj, cudaStream_t stream)

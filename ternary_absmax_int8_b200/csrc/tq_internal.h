@@ -178,6 +178,35 @@ struct MmaParams {
 cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_prev,
                             cudaStream_t stream);
 
+// ----------------------------------------- prompt processing (M >= 33)
+// One projection of a prefill launch: packed [N/4, K], activations [M, K],
+// outputs [M, N]. A launch takes up to kPrefillMaxGroup projections; their
+// 128-feature x BN-token tiles are dealt to persistent CTAs longest first.
+struct PrefillEntry {
+    const uint8_t *packed;
+    float w_scale;
+    const int8_t *xq;
+    const float *x_scale;
+    const int32_t *x_sum;
+    float *y;
+    int32_t *acc_out;
+    int N, K;
+};
+
+constexpr int kPrefillMaxGroup = 16;    // projections per call
+constexpr int kPrefillMaxTiles = 4096;  // tiles per launch (more: several launches)
+constexpr int kPrefillMaxGrid = 160;    // CTAs per launch
+
+// *handled = false (and nothing launched) for M < 33; cudaErrorInvalidValue
+// for more than kPrefillMaxGroup projections or shapes beyond the tile
+// fields (N > 2^21 or M > 2^22).
+cudaError_t launch_prefill_group(const PrefillEntry *e, int n, int M, cudaStream_t stream,
+                                 bool *handled);
+cudaError_t launch_prefill_tc(const uint8_t *packed, float w_scale, const int8_t *xq,
+                              const float *x_scale, const int32_t *x_sum, float *y,
+                              int32_t *acc_out, int M, int N, int K, cudaStream_t stream,
+                              bool *handled);
+
 // ------------------------------------------ decoder-layer neighbours, absmean
 // input: 0 = bf16 x, 1 = fp32 x, 2 = relu(x_f32)^2 * up. One CTA per row.
 cudaError_t launch_rms_quant(int input, const uint16_t *x_bf16, const float *x_f32,

@@ -23,7 +23,7 @@ def _projs(name):
     ("stack30_m1", "fused"), ("layer_m1", "fused"), ("ffn_m1", "fused"),
     ("ffn_m2", "batch"), ("ffn_m4", "batch"), ("ffn_m8", "batch"), ("ffn_m24", "batch"),
     ("stack30_m4", "batch"), ("stack30_m16", "batch"),
-    ("single_640x2560_m1", "per_projection"), ("prefill_m512", "per_projection"),
+    ("single_640x2560_m1", "per_projection"), ("prefill_m512", "prefill"),
 ])
 def test_step_mode(name, mode):
     assert bench.step_mode(_projs(name)) == mode
@@ -38,6 +38,21 @@ def test_batch_launch_counts():
     assert bench.batch_launches(210, 16) == 7 + 1
     assert bench.batch_launches(210, 24) == 10 + 4
     assert bench.batch_launches(300, 2) == 2 + 2
+
+
+def test_prefill_launch_counts():
+    # 512 token rows per quantiser launch, 16 projections per grouped prefill launch
+    assert bench.prefill_launches(3, 512) == 3 + 1
+    assert bench.prefill_launches(16, 64) == 2 + 1
+    assert bench.prefill_launches(17, 512) == 17 + 2
+
+
+def test_binary_kernel_name(monkeypatch):
+    monkeypatch.delenv("TQ_BINARY_KERNEL", raising=False)
+    assert [bench.binary_kernel_name(m) for m in (1, 2, 4)] == [
+        "binary_mma_kernel", "binary_gemv_kernel", "binary_gemv_kernel"]
+    monkeypatch.setenv("TQ_BINARY_KERNEL", "dp4a")
+    assert bench.binary_kernel_name(1) == "binary_gemv_kernel"
 
 
 def test_kernel_names_follow_the_choice_by_m(monkeypatch):

@@ -2,9 +2,8 @@
 
 Full outputs at M = 128 and 256 for the FFN shapes and at M = 512 on the three
 prefill shapes (including the 27B-scale 17408 x 5120). Ragged M and N exercise
-partial tiles; the shapes cover both work splits of the kernel: whole tiles per
-CTA (including CTAs that take a second tile) and K split over the CTAs of a
-thread-block cluster with a reduce-scatter of the partial sums.
+partial tiles (128- and 256-token tiles); CTAs that take several tiles drain
+and refill both tensor-memory accumulators.
 """
 import numpy as np
 import pytest
@@ -46,9 +45,9 @@ def test_prefill_ragged(cuda_device, N, K, M):
 
 
 def test_prefill_second_tile_per_cta(cuda_device):
-    # 68 x 4 = 272 tiles of 256 features x 256 tokens on 148 SMs: most CTAs
-    # take two tiles, so the accumulator is drained and refilled; sampled
-    # token rows from every token tile, all N outputs.
+    # 136 x 4 = 544 tiles of 128 features x 256 tokens on 148 SMs: every CTA
+    # takes three or four tiles, so both accumulators are drained and
+    # refilled; sampled token rows from every token tile, all N outputs.
     N, K, M = 17408, 512, 1024
     rng = np.random.default_rng(5)
     w = ternary_weights(rng, N, K)
