@@ -51,6 +51,7 @@ PEAK_FALLBACK_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 STACK_KERNEL_SRC = os.path.join(ROOT, "ternary_absmax_int8_b200", "csrc", "gemv_stream.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+TRAFFIC_BINARY_FILE = os.path.join(ROOT, "profiles", "traffic_binary.json")
 
 DESCRIPTIONS = {
     "stack30_m1": "decode layer stack: 30 x BitNet-b1.58-2B-4T decoder layer (q,k,v,o,gate,up,"
@@ -223,6 +224,33 @@ def stack_kernel_sha() -> str:
     end = text.index(b"\n// ------", start + 1)
     h.update(text[start:end])
     return h.hexdigest()[:16]
+
+
+def binary_kernel_sha() -> str:
+    """Hash of the binary g128 kernels' sources (their file, the headers they
+    use and the binary section of the launch-parameter header)."""
+    d = os.path.dirname(STACK_KERNEL_SRC)
+    h = hashlib.sha256()
+    for name in ("gemv_binary.cu", "mma_common.cuh", "tq_device.cuh"):
+        h.update(open(os.path.join(d, name), "rb").read())
+    text = open(os.path.join(d, "tq_internal.h"), "rb").read()
+    start = text.index(b"// --------------------------------------------- binary g128 GEMV")
+    end = text.index(b"\n// Device address of the library's error word", start + 1)
+    h.update(text[start:end])
+    return h.hexdigest()[:16]
+
+
+def recorded_binary_traffic(workload: str, kernel: str):
+    """DRAM bytes of one binary GEMV launch from a committed ncu summary of
+    the same kernel version and workload; None otherwise."""
+    try:
+        d = json.load(open(TRAFFIC_BINARY_FILE))
+    except (OSError, ValueError):
+        return None
+    if (d.get("kernel_sha") != binary_kernel_sha() or d.get("workload") != workload
+            or d.get("kernel") != kernel):
+        return None
+    return float(d["dram_bytes_read"] + d["dram_bytes_write"])
 
 
 def recorded_traffic(workload: str):
@@ -822,7 +850,8 @@ def run_next(args, rank: int, world: int):
         achieved = gemv_units / (gemv_ms * 1e6)
         roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs copy bandwidth)",
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": recorded_binary_traffic(args.workload, kernel),
                 "algorithmic_bytes_per_launch": int(gemv_units)}
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,

@@ -98,3 +98,10 @@ def test_warmup_below_three_is_rejected():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--warmup", "2"],
                          cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_recorded_binary_traffic_needs_the_same_kernel_and_workload():
+    # a record is used only for the kernel version, kernel and workload it was taken on
+    assert bench.recorded_binary_traffic("binary_ffn27b_m1", "binary_gemv_kernel") is None
+    assert bench.recorded_binary_traffic("prefill_m512", "binary_mma_kernel") is None
+    assert len(bench.binary_kernel_sha()) == 16
