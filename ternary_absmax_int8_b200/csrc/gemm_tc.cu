@@ -29,7 +29,11 @@
 //                swizzle), fence to the async proxy, signal the MMA
 //   warps 10..17 epilogue: warp w reads TMEM lane quarter w % 4 (the plane)
 //                over half of the tile's columns, subtracts x_sum, scales and
-//                stores y
+//                stores y; of a CTA's last tile the expansion warps, idle by
+//                then, drain half of the columns
+// Launched with programmatic serialisation: the set-up (barriers, tensor
+// memory, tensor-map prefetch) overlaps the previous grid's tail, and every
+// access to global memory waits for that grid (griddepcontrol.wait).
 // The accumulator is double-buffered in tensor memory (2 x BN columns): the
 // MMAs of a CTA's next tile run while the epilogue warps drain the previous
 // one, so the output stores (4 bytes per element, as many bytes as the
@@ -145,6 +149,70 @@ __device__ __forceinline__ void quad_transpose(const int32_t (&m)[4], int32_t (&
     f[3] = b0 ? c1 : u1;
 }
 
+// Epilogue of columns [c_begin, c_end) (tokens tt * BN + c) of one tile's
+// accumulator, by one warp of TMEM lane quarter q (plane q): lane = packed
+// row ft * 32 + lane, feature n = that row + q N/4.
+template <int BN>
+__device__ __forceinline__ void drain_columns(const PrefillTable &tab, uint32_t code,
+                                              uint32_t tmem_acc, int q, int c_begin, int c_end,
+                                              int lane)
+{
+    const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
+              ft = int(code & (kTileField - 1));
+    const PrefillProj &pe = tab.e[e];
+    const int N4 = pe.N4, N = 4 * N4;
+    const int prow = ft * kPackedRows + lane;  // packed row of this lane
+    const bool row_ok = prow < N4;
+    const int n = prow + q * N4;
+    const uint32_t tbase = tmem_acc + (uint32_t(q * 32) << 16);
+    for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+        const int mbase = tt * BN + c0;
+        if (mbase >= tab.M)
+            break;
+        uint32_t v[32];
+        tmem_ld32(tbase + uint32_t(c0), v);
+        const int my_m = mbase + lane;
+        const float my_t = my_m < tab.M ? __fmul_rn(pe.w_scale, __ldg(pe.x_scale + my_m)) : 0.0f;
+        const int32_t my_s = my_m < tab.M ? __ldg(pe.x_sum + my_m) : 0;
+        if (pe.vec) {
+            // quads of lanes trade values so that each lane writes four
+            // consecutive features of one token: a 16-byte store
+            const int i4 = lane & 3;
+            const int f0 = ft * kPackedRows + (lane & ~3);  // first feature of the quad
+            const size_t n0 = size_t(f0) + size_t(q) * N4;
+#pragma unroll
+            for (int k0 = 0; k0 < 32; k0 += 4) {
+                const int32_t m4[4] = {int32_t(v[k0]) >> (2 * q), int32_t(v[k0 + 1]) >> (2 * q),
+                                       int32_t(v[k0 + 2]) >> (2 * q), int32_t(v[k0 + 3]) >> (2 * q)};
+                int32_t f4[4];
+                quad_transpose(m4, f4, i4);
+                const int tk = k0 + i4;  // this lane's token in the chunk
+                const float ts = __shfl_sync(0xffffffffu, my_t, tk);
+                const int32_t xs = __shfl_sync(0xffffffffu, my_s, tk);
+                if (f0 < N4 && mbase + tk < tab.M) {
+                    const size_t o = size_t(mbase + tk) * size_t(N) + n0;
+                    const int4 a4 = make_int4(f4[0] - xs, f4[1] - xs, f4[2] - xs, f4[3] - xs);
+                    __stcs(reinterpret_cast<float4 *>(pe.y + o),
+                           make_float4(__fmul_rn(__int2float_rn(a4.x), ts),
+                                       __fmul_rn(__int2float_rn(a4.y), ts),
+                                       __fmul_rn(__int2float_rn(a4.z), ts),
+                                       __fmul_rn(__int2float_rn(a4.w), ts)));
+                    if (pe.acc_out)
+                        __stcs(reinterpret_cast<int4 *>(pe.acc_out + o), a4);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float ts = __shfl_sync(0xffffffffu, my_t, k);
+                const int32_t xs = __shfl_sync(0xffffffffu, my_s, k);
+                if (row_ok && mbase + k < tab.M)
+                    store_out(pe, N, mbase + k, n, int32_t(v[k]) >> (2 * q), ts, xs);
+            }
+        }
+    }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
@@ -171,6 +239,9 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t_begin = tab.cta0[blockIdx.x], t_end = tab.cta0[blockIdx.x + 1];
     unsigned *err = tab.err;
+    // The next grid on the stream may start its set-up now; it waits for this
+    // one before it touches memory.
+    pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int j = 0; j < tab.n; ++j) {
@@ -199,6 +270,9 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            // every global operand may still be written by the previous grid
+            // on the stream (launched with programmatic serialisation)
+            pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -324,74 +398,38 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
                 }
             }
         }
+        // the last tile's columns [BN/2, BN): expansion warp w drains lane
+        // quarter w % 4 over one quarter of the columns
+        const int local_last = t_end - 1 - t_begin;
+        if (ok && local_last >= 0) {
+            pdl_wait();
+            const int buf = local_last & 1;
+            if (mbar_wait_warp(&acc_full[buf], uint32_t((local_last >> 1) & 1), err)) {
+                tc_fence_after();
+                const int c_begin = BN / 2 + ((warp - kExpWarp0) >> 2) * (BN / 4);
+                drain_columns<BN>(tab, tab.tile[t_end - 1], tmem_base + uint32_t(buf * BN),
+                                  warp & 3, c_begin, c_begin + BN / 4, lane);
+                tc_fence_before();
+            }
+        }
     } else {
         // ------------------------------------------------ epilogue
-        const int q = warp & 3;                           // TMEM lane quarter = plane
-        const int half = (warp - kEpiWarp0) >> 2;         // its half of the columns
-        constexpr int ncol = BN / 2;
-        const int cb = half * ncol;
+        // warp w drains lane quarter w % 4 over its half of the columns; of the
+        // CTA's last tile it drains a quarter (the expansion warps, idle by
+        // then, drain the other half)
+        const int q = warp & 3;                    // TMEM lane quarter = plane
+        const int half = (warp - kEpiWarp0) >> 2;
+        pdl_wait();  // outputs and scales belong to the previous grid until it completes
         for (int i = t_begin, local = 0; i < t_end; ++i, ++local) {
-            const uint32_t code = tab.tile[i];
-            const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
-                      ft = int(code & (kTileField - 1));
-            const PrefillProj &pe = tab.e[e];
             const int buf = local & 1;
             if (!mbar_wait_warp(&acc_full[buf], uint32_t((local >> 1) & 1), err))
                 break;
             tc_fence_after();
-            const int N4 = pe.N4, N = 4 * N4;
-            const int prow = ft * kPackedRows + lane;  // packed row of this lane
-            const bool row_ok = prow < N4;
-            const int n = prow + q * N4;
-            const uint32_t tbase = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * BN + cb);
-            for (int c0 = 0; c0 < ncol; c0 += 32) {
-                const int mbase = tt * BN + cb + c0;
-                if (mbase >= tab.M)
-                    break;
-                uint32_t v[32];
-                tmem_ld32(tbase + uint32_t(c0), v);
-                const int my_m = mbase + lane;
-                const float my_t =
-                    my_m < tab.M ? __fmul_rn(pe.w_scale, __ldg(pe.x_scale + my_m)) : 0.0f;
-                const int32_t my_s = my_m < tab.M ? __ldg(pe.x_sum + my_m) : 0;
-                if (pe.vec) {
-                    // quads of lanes trade values so that each lane writes four
-                    // consecutive features of one token: a 16-byte store
-                    const int i4 = lane & 3;
-                    const int f0 = ft * kPackedRows + (lane & ~3);  // first feature of the quad
-                    const size_t n0 = size_t(f0) + size_t(q) * N4;
-#pragma unroll
-                    for (int k0 = 0; k0 < 32; k0 += 4) {
-                        const int32_t m4[4] = {int32_t(v[k0]) >> (2 * q), int32_t(v[k0 + 1]) >> (2 * q),
-                                               int32_t(v[k0 + 2]) >> (2 * q),
-                                               int32_t(v[k0 + 3]) >> (2 * q)};
-                        int32_t f4[4];
-                        quad_transpose(m4, f4, i4);
-                        const int tk = k0 + i4;  // this lane's token in the chunk
-                        const float ts = __shfl_sync(0xffffffffu, my_t, tk);
-                        const int32_t xs = __shfl_sync(0xffffffffu, my_s, tk);
-                        if (f0 < N4 && mbase + tk < tab.M) {
-                            const size_t o = size_t(mbase + tk) * size_t(N) + n0;
-                            const int4 a4 = make_int4(f4[0] - xs, f4[1] - xs, f4[2] - xs, f4[3] - xs);
-                            __stcs(reinterpret_cast<float4 *>(pe.y + o),
-                                   make_float4(__fmul_rn(__int2float_rn(a4.x), ts),
-                                               __fmul_rn(__int2float_rn(a4.y), ts),
-                                               __fmul_rn(__int2float_rn(a4.z), ts),
-                                               __fmul_rn(__int2float_rn(a4.w), ts)));
-                            if (pe.acc_out)
-                                __stcs(reinterpret_cast<int4 *>(pe.acc_out + o), a4);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const float ts = __shfl_sync(0xffffffffu, my_t, k);
-                        const int32_t xs = __shfl_sync(0xffffffffu, my_s, k);
-                        if (row_ok && mbase + k < tab.M)
-                            store_out(pe, N, mbase + k, n, int32_t(v[k]) >> (2 * q), ts, xs);
-                    }
-                }
-            }
+            const bool last = i + 1 == t_end;
+            const int c_begin = last ? half * (BN / 4) : half * (BN / 2);
+            const int c_end = c_begin + (last ? BN / 4 : BN / 2);
+            drain_columns<BN>(tab, tab.tile[i], tmem_base + uint32_t(buf * BN), q, c_begin, c_end,
+                              lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -503,8 +541,19 @@ cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
         schedule_lpt(sub, grid, order, tab.cta0);
         for (int i = 0; i < cnt; ++i)
             tab.tile[i] = codes[size_t(base + order[size_t(i)])];
-        prefill_tc_kernel<BN><<<grid, kThreads, smem, stream>>>(tab);
-        err = cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<BN>, tab);
+        if (err == cudaSuccess)
+            err = cudaGetLastError();
         if (err != cudaSuccess)
             return err;
     }
