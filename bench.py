@@ -105,19 +105,19 @@ def step_mode(projs) -> str:
 
 def batch_launches(n: int, M: int) -> int:
     """Kernel launches of tq_quantize_act_stack_batch + tq_gemv_stack_batch
-    over n projections of M tokens: 512 token rows per quantiser launch; 256
+    over n projections of M tokens: 512 projections per quantiser launch; 256
     projections per streaming or warp-MMA launch, 64 per tensor-core group
     launch."""
     per = 64 if batch_kernel_name(M, "batch") == "smallm_group_kernel" else 256
-    return -(-n * M // 512) + -(-n // per)
+    return -(-n // 512) + -(-n // per)
 
 
 def prefill_launches(n: int, M: int) -> int:
     """Kernel launches of tq_quantize_act_stack_batch + tq_gemm_prefill_stack
-    over n projections of M >= 33 tokens: 512 token rows per quantiser launch,
-    16 projections per prefill launch (up to 4096 tiles each, which every
-    measured shape stays within)."""
-    return -(-n * M // 512) + -(-n // 16)
+    over n projections of M >= 33 tokens: 512 projections per quantiser
+    launch, 16 projections per prefill launch (up to 4096 tiles each, which
+    every measured shape stays within)."""
+    return -(-n // 512) + -(-n // 16)
 
 
 def workload_step_bytes(workload: str, projs) -> int:

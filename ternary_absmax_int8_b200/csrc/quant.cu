@@ -7,9 +7,13 @@
 //   amax = max_k |x|, s = fl32(127/amax), q = clamp(rne(fl32(x*s)), -127, 127),
 //   x_scale = fl32(amax/127), x_sum = sum q; amax == 0 gives zeros.
 //
-// One CTA per token row. Pass 1 reads the row as 16-byte vectors and reduces
-// |x| to amax; pass 2 re-reads it (an L1/L2 hit), converts and writes 8 codes
-// per vector, and reduces the code sum. HBM traffic: 2K bytes in, K + 8 out.
+// A row is read twice as 16-byte vectors: pass 1 reduces |x| to amax, pass
+// 2 (an L1/L2 hit) converts and writes 8 codes per vector and reduces the code
+// sum. HBM traffic: 2K bytes in, K + 8 out. One CTA per row (block-wide
+// reductions) while rows are few; one warp per row (shuffle reductions only)
+// once there are enough rows to give every SM eight.
+#include <algorithm>
+
 #include "quant_core.cuh"
 #include "tq_internal.h"
 
@@ -86,14 +90,83 @@ quant_rows_kernel(const uint16_t *__restrict__ x, int8_t *__restrict__ xq,
     quant_row(x + m * K, xq + m * K, x_scale + m, x_sum ? x_sum + m : nullptr, K);
 }
 
+// The entry holding launch row r (entries' rows are consecutive).
+__device__ __forceinline__ int entry_of_row(const QuantStackParams &p, int r)
+{
+    int lo = 0, hi = p.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.e[mid].row0 <= r)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(kQuantThreads)
 quant_stack_kernel(const __grid_constant__ QuantStackParams p)
 {
     // Let a dependent grid (the stack GEMV) launch now: it streams weights,
     // which do not depend on this grid, and waits for it before reading xq.
     pdl_launch_dependents();
-    const QuantStackEntry &e = p.e[blockIdx.x];
-    quant_row(e.x, e.xq, e.x_scale, e.x_sum, e.K);
+    const int r = blockIdx.x;
+    const QuantStackEntry &e = p.e[entry_of_row(p, r)];
+    const size_t m = size_t(r - e.row0);
+    quant_row(e.x + m * e.K, e.xq + m * e.K, e.x_scale + m, e.x_sum ? e.x_sum + m : nullptr, e.K);
+}
+
+// One warp per row, rows strided over all warps of the grid.
+__global__ void __launch_bounds__(kQuantThreads)
+quant_stack_warp_kernel(const __grid_constant__ QuantStackParams p)
+{
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int nwarps = int(gridDim.x) * (kQuantThreads / 32);
+    for (int r = int(blockIdx.x) * (kQuantThreads / 32) + int(threadIdx.x >> 5); r < p.rows;
+         r += nwarps) {
+        const QuantStackEntry &e = p.e[entry_of_row(p, r)];
+        const size_t m = size_t(r - e.row0);
+        const uint4 *xv = reinterpret_cast<const uint4 *>(e.x + m * e.K);
+        const int nvec = e.K >> 3;
+        // eight 16-byte loads per lane in flight before any is used (a warp
+        // has few rows' worth of neighbours on its SM to hide latency with)
+        constexpr int kB = 8;
+        float amax = 0.0f;
+        for (int v0 = lane; v0 < nvec; v0 += 32 * kB) {
+            uint4 u[kB];
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+                u[b] = v0 + 32 * b < nvec ? __ldg(xv + v0 + 32 * b) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+                amax = fmaxf(amax, absmax8(u[b]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = quant_inv_scale(amax);
+        int sum = 0;
+        uint2 *qv = reinterpret_cast<uint2 *>(e.xq + m * e.K);
+        for (int v0 = lane; v0 < nvec; v0 += 32 * kB) {
+            uint4 u[kB];
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+                u[b] = v0 + 32 * b < nvec ? __ldg(xv + v0 + 32 * b) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+                if (v0 + 32 * b < nvec)
+                    qv[v0 + 32 * b] = quant8(u[b], s, &sum);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+            e.x_scale[m] = quant_scale(amax);
+            if (e.x_sum)
+                e.x_sum[m] = sum;
+        }
+    }
 }
 
 }  // namespace
@@ -107,7 +180,16 @@ cudaError_t launch_quant_rows(const uint16_t *x, int8_t *xq, float *x_scale, int
 
 cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream)
 {
-    quant_stack_kernel<<<p.n, kQuantThreads, 0, stream>>>(p);
+    if (p.rows <= 0)
+        return cudaSuccess;
+    constexpr int kWarps = kQuantThreads / 32;
+    const int sms = device_sm_count();
+    if (p.rows < sms * kWarps) {
+        quant_stack_kernel<<<p.rows, kQuantThreads, 0, stream>>>(p);
+    } else {
+        const int grid = std::min((p.rows + kWarps - 1) / kWarps, sms * 8);  // 8 CTAs of 8 warps per SM
+        quant_stack_warp_kernel<<<grid, kQuantThreads, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 

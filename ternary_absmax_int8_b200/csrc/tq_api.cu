@@ -4,6 +4,7 @@
 #include <cfloat>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdint>
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
@@ -223,7 +224,7 @@ __global__ void wait_selftest_kernel(unsigned *err, unsigned long long limit_ns)
 }
 
 // The quantiser over M token rows of each projection: one entry of the stack
-// quantiser per row, all in one launch per kMaxQuantStack rows.
+// quantiser per projection, one launch per kMaxQuantStack projections.
 tq_status quantize_stack_impl(const char *fname, const tq_proj *projs, int n_proj, int M,
                               cudaStream_t stream)
 {
@@ -234,7 +235,7 @@ tq_status quantize_stack_impl(const char *fname, const tq_proj *projs, int n_pro
     if (!projs)
         return fail(TQ_ERR_NULL, "%s: projs is NULL", fname);
     std::vector<tq::QuantStackEntry> list;
-    list.reserve(size_t(n_proj) * size_t(M));
+    list.reserve(size_t(n_proj));
     for (int j = 0; j < n_proj; ++j) {
         const tq_proj &p = projs[j];
         if (p.K < 0 || p.K % 16 != 0)
@@ -244,6 +245,9 @@ tq_status quantize_stack_impl(const char *fname, const tq_proj *projs, int n_pro
         if ((p.K > 0 && (!aligned(p.x, 16) || !aligned(p.xq, 16))) || !aligned(p.x_scale, 4) ||
             (p.x_sum && !aligned(p.x_sum, 4)))
             return fail(TQ_ERR_ALIGN, "%s: entry %d: misaligned pointer", fname, j);
+    }
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
         if (p.K == 0) {
             cudaError_t e = cudaMemsetAsync(p.x_scale, 0, size_t(M) * sizeof(float), stream);
             if (e == cudaSuccess && p.x_sum)
@@ -252,21 +256,21 @@ tq_status quantize_stack_impl(const char *fname, const tq_proj *projs, int n_pro
                 return cuda_fail(e, fname);
             continue;
         }
-        for (int m = 0; m < M; ++m) {
-            tq::QuantStackEntry q = {};
-            q.x = p.x + size_t(m) * size_t(p.K);
-            q.xq = p.xq + size_t(m) * size_t(p.K);
-            q.x_scale = p.x_scale + m;
-            q.x_sum = p.x_sum ? p.x_sum + m : nullptr;
-            q.K = p.K;
-            list.push_back(q);
-        }
+        list.push_back(tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, M, 0, 0});
     }
     tq::QuantStackParams &params = *quant_params();
     for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
         const size_t n = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
         params.n = int(n);
-        std::memcpy(params.e, list.data() + base, n * sizeof(tq::QuantStackEntry));
+        long long rows = 0;
+        for (size_t i = 0; i < n; ++i) {
+            params.e[i] = list[base + i];
+            params.e[i].row0 = int(rows);
+            rows += M;
+        }
+        if (rows > INT32_MAX)
+            return fail(TQ_ERR_UNSUPPORTED, "%s: %lld rows in one call", fname, rows);
+        params.rows = int(rows);
         cudaError_t e = tq::launch_quant_stack(params, stream);
         if (e != cudaSuccess)
             return cuda_fail(e, fname);
@@ -339,7 +343,8 @@ tq_status gemv_stack_impl(const char *fname, const tq_proj *projs, int n_proj, i
             if (mode == 1) {
                 tq::QuantStackParams *qp = quant_params();
                 qp->n = 1;
-                qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 0};
+                qp->rows = 1;
+                qp->e[0] = tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, 1, 0, 0};
                 e = tq::launch_quant_stack(*qp, stream);
             } else {
                 e = tq::launch_rms_quant(mode == 2 ? 0 : 2, p.x, p.x_f32, p.up, p.gain, p.eps,

@@ -10,25 +10,28 @@
 namespace tq {
 
 // ---------------------------------------------------------------- quantise
-constexpr int kMaxQuantStack = 512;
+constexpr int kMaxQuantStack = 512;  // projections per stack quantiser launch
 
+// One projection's M token rows ([M, K] bf16 in, [M, K] codes and [M] scales
+// and sums out); row0 = the launch's index of its first row.
 struct QuantStackEntry {
     const uint16_t *x;
     int8_t *xq;
     float *x_scale;
     int32_t *x_sum;
-    int K;
-    int pad_;
+    int K, M;
+    int row0, pad_;
 };
 
 struct QuantStackParams {
-    int n;
-    int pad_;
+    int n;     // entries
+    int rows;  // sum of their M
     QuantStackEntry e[kMaxQuantStack];
 };
 
 cudaError_t launch_quant_rows(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
                               int M, int K, cudaStream_t stream);
+// One CTA per row while rows are few, one warp per row from 8 rows per SM.
 cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream);
 
 // ------------------------------------------------- streaming GEMV (M <= 4)

@@ -30,21 +30,22 @@ def test_step_mode(name, mode):
 
 
 def test_batch_launch_counts():
-    # 512 token rows per quantiser launch; 256 projections per streaming
+    # 512 projections per quantiser launch; 256 projections per streaming
     # (M <= 2) or warp-MMA (3..16) launch, 64 per tensor-core group launch
     assert bench.batch_launches(3, 4) == 1 + 1
     assert bench.batch_launches(3, 16) == 1 + 1
-    assert bench.batch_launches(210, 4) == 2 + 1
-    assert bench.batch_launches(210, 16) == 7 + 1
-    assert bench.batch_launches(210, 24) == 10 + 4
-    assert bench.batch_launches(300, 2) == 2 + 2
+    assert bench.batch_launches(210, 4) == 1 + 1
+    assert bench.batch_launches(210, 16) == 1 + 1
+    assert bench.batch_launches(210, 24) == 1 + 4
+    assert bench.batch_launches(300, 2) == 1 + 2
+    assert bench.batch_launches(600, 2) == 2 + 3
 
 
 def test_prefill_launch_counts():
-    # 512 token rows per quantiser launch, 16 projections per grouped prefill launch
-    assert bench.prefill_launches(3, 512) == 3 + 1
-    assert bench.prefill_launches(16, 64) == 2 + 1
-    assert bench.prefill_launches(17, 512) == 17 + 2
+    # 512 projections per quantiser launch, 16 per grouped prefill launch
+    assert bench.prefill_launches(3, 512) == 1 + 1
+    assert bench.prefill_launches(16, 64) == 1 + 1
+    assert bench.prefill_launches(17, 512) == 1 + 2
 
 
 def test_binary_kernel_name(monkeypatch):

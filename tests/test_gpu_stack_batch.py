@@ -92,8 +92,8 @@ def test_batch_of_one_is_the_stack(cuda_device):
 
 
 def test_mixed_stack_batched_more_than_one_launch(cuda_device):
-    # 300 projections of assorted shapes at M = 3: two GEMV launches and, with
-    # 900 token rows, two quantiser launches.
+    # 300 projections of assorted shapes at M = 3: two GEMV launches; 900
+    # token rows in one quantiser launch (a CTA per row).
     shapes = [(f"p{j}", 4 * (1 + (j * 37) % 97), 16 * (1 + (j * 11) % 40)) for j in range(300)]
     projs = list(make_projections(shapes, M=3, seed=12))
     st = BatchStack(projs, 3)
@@ -198,3 +198,28 @@ def test_full_stack_30_layers_m4_streaming(cuda_device):
     st.run()
     _check(st, refs)
     assert tq.tq_device_error(reset=True) == 0
+
+
+def test_stack_quantiser_warp_rows_and_two_launches(cuda_device):
+    # 600 projections x 4 rows of assorted K: the first launch (512
+    # projections, 2048 rows) takes a warp per row, the second (88
+    # projections, 352 rows) a CTA per row; every code, scale and sum against
+    # the oracle's quantiser.
+    M = 4
+    rng = np.random.default_rng(44)
+    from workloads import activations_bf16
+    xs_in = [activations_bf16(rng, M, 16 * (1 + (j * 13) % 64)) for j in range(600)]
+    xd = [dev(x.view(np.int16)) for x in xs_in]
+    xq = [torch.full((M, x.shape[1]), -128, dtype=torch.int8, device="cuda") for x in xs_in]
+    xs = [torch.full((M,), float("nan"), device="cuda") for _ in xs_in]
+    xsum = [torch.full((M,), -(2 ** 31), dtype=torch.int32, device="cuda") for _ in xs_in]
+    table = [tq.make_proj(x=xd[j], xq=xq[j], x_scale=xs[j], x_sum=xsum[j], N=0, K=x.shape[1])
+             for j, x in enumerate(xs_in)]
+    tq.tq_quantize_act_stack_batch(table, M)
+    torch.cuda.synchronize()
+    for j, x in enumerate(xs_in):
+        rq, rxs, rxsum = oracle.quant(x)
+        assert np.array_equal(xq[j].cpu().numpy(), rq), j
+        assert np.array_equal(xs[j].cpu().numpy().view(np.uint32), rxs.view(np.uint32)), j
+        assert np.array_equal(xsum[j].cpu().numpy(), rxsum), j
+
