@@ -41,6 +41,7 @@
 // wait is bounded; loads never use cluster multicast.
 #include <atomic>
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
@@ -151,17 +152,16 @@ __device__ __forceinline__ void quad_transpose(const int32_t (&m)[4], int32_t (&
 
 // Epilogue of columns [c_begin, c_end) (tokens tt * BN + c) of one tile's
 // accumulator, by one warp of TMEM lane quarter q (plane q): lane = packed
-// row ft * 32 + lane, feature n = that row + q N/4.
+// row prow0 + lane, feature n = that row + q N/4.
 template <int BN>
-__device__ __forceinline__ void drain_columns(const PrefillTable &tab, uint32_t code,
+__device__ __forceinline__ void drain_columns(const PrefillTable &tab, uint32_t code, int prow0,
                                               uint32_t tmem_acc, int q, int c_begin, int c_end,
                                               int lane)
 {
-    const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
-              ft = int(code & (kTileField - 1));
+    const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1));
     const PrefillProj &pe = tab.e[e];
     const int N4 = pe.N4, N = 4 * N4;
-    const int prow = ft * kPackedRows + lane;  // packed row of this lane
+    const int prow = prow0 + lane;  // packed row of this lane
     const bool row_ok = prow < N4;
     const int n = prow + q * N4;
     const uint32_t tbase = tmem_acc + (uint32_t(q * 32) << 16);
@@ -178,7 +178,7 @@ __device__ __forceinline__ void drain_columns(const PrefillTable &tab, uint32_t 
             // quads of lanes trade values so that each lane writes four
             // consecutive features of one token: a 16-byte store
             const int i4 = lane & 3;
-            const int f0 = ft * kPackedRows + (lane & ~3);  // first feature of the quad
+            const int f0 = prow0 + (lane & ~3);  // first feature of the quad
             const size_t n0 = size_t(f0) + size_t(q) * N4;
 #pragma unroll
             for (int k0 = 0; k0 < 32; k0 += 4) {
@@ -407,8 +407,10 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
             if (mbar_wait_warp(&acc_full[buf], uint32_t((local_last >> 1) & 1), err)) {
                 tc_fence_after();
                 const int c_begin = BN / 2 + ((warp - kExpWarp0) >> 2) * (BN / 4);
-                drain_columns<BN>(tab, tab.tile[t_end - 1], tmem_base + uint32_t(buf * BN),
-                                  warp & 3, c_begin, c_begin + BN / 4, lane);
+                const uint32_t code = tab.tile[t_end - 1];
+                drain_columns<BN>(tab, code, int(code & (kTileField - 1)) * kPackedRows,
+                                  tmem_base + uint32_t(buf * BN), warp & 3, c_begin,
+                                  c_begin + BN / 4, lane);
                 tc_fence_before();
             }
         }
@@ -428,8 +430,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
             const bool last = i + 1 == t_end;
             const int c_begin = last ? half * (BN / 4) : half * (BN / 2);
             const int c_end = c_begin + (last ? BN / 4 : BN / 2);
-            drain_columns<BN>(tab, tab.tile[i], tmem_base + uint32_t(buf * BN), q, c_begin, c_end,
-                              lane);
+            drain_columns<BN>(tab, tab.tile[i], int(tab.tile[i] & (kTileField - 1)) * kPackedRows,
+                              tmem_base + uint32_t(buf * BN), q, c_begin, c_end, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -443,6 +445,281 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
     tc_fence_after();
     if (warp == 1)
         tmem_dealloc(tmem_base, S::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// The pair form: the two CTAs of a cluster run 256-row MMAs
+// (tcgen05.mma.cta_group::2) on a tile of 256 features (64 packed rows: the
+// even CTA expands rows 0..31, the odd one rows 32..63) x 256 tokens (each
+// CTA holds 128 of them in shared memory). A K stage per CTA is 16 KB of
+// codes + 16 KB of activations + 4 KB of packed bytes, so six stages fit;
+// each CTA keeps its 128 rows of both accumulators in its own tensor memory.
+// Barriers: the even CTA's full (the activation halves of both CTAs) and
+// a_full (its own 8 expansion warps arrive; the odd CTA's 8 each complete 4
+// transaction bytes with an asynchronous remote store, st.async, whose
+// completion releases at cluster scope without stalling the warp -- a
+// remote arrive with cluster-scope release stalls its thread ~1,000 cycles,
+// too much per stage), each CTA's own pfull (its packed tile) and p_free,
+// and empty / acc_full committed to both CTAs by the even CTA's MMA thread;
+// acc_empty on the even CTA (both CTAs' epilogue warps).
+constexpr int kPairBN = 256;              // tokens per tile
+constexpr int kPairBHalf = (kPairBN / 2) * kBK;  // 16 KB: a CTA's activation rows
+constexpr int kPairStage = kABytes + kPairBHalf + kPBytes;
+constexpr int kPairStages =
+    int((kSmemLimit - 1024 - 512) / size_t(kPairStage)) > 6 ? 6
+                                                          : int((kSmemLimit - 1024 - 512) / size_t(kPairStage));
+struct PairSmem {
+    static constexpr size_t a_off = 0;
+    static constexpr size_t b_off = a_off + size_t(kPairStages) * kABytes;
+    static constexpr size_t p_off = b_off + size_t(kPairStages) * kPairBHalf;
+    static constexpr size_t bar_off = p_off + size_t(kPairStages) * kPBytes;
+    // full, pfull, a_full, empty, p_free per stage; acc_full[2], acc_empty[2]
+    static constexpr size_t sig_off = bar_off + size_t(5 * kPairStages + 4) * 8;
+    static constexpr size_t tmem_slot_off = sig_off + 64;  // 8 words written by st.async
+    static constexpr size_t bytes = tmem_slot_off + 16;
+    static_assert(kPairStages >= 4, "four stages at least");
+    static_assert(bytes + 1024 <= kSmemLimit, "shared memory");
+};
+constexpr int kPairTmemCols = 2 * kPairBN;  // two accumulators
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_pair_kernel(const __grid_constant__ PrefillTable tab)
+{
+    using S = PairSmem;
+    constexpr int kStages = kPairStages;
+    constexpr uint32_t kIdesc = idesc_i8_u8s8(2 * kGM, kPairBN);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem + S::a_off;
+    uint8_t *sB = smem + S::b_off;
+    uint8_t *sP = smem + S::p_off;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::bar_off);
+    uint64_t *full = bars;                     // even CTA: activations of both CTAs
+    uint64_t *pfull = bars + kStages;          // own packed tile
+    uint64_t *a_full = bars + 2 * kStages;     // even CTA: 2 x 8 expansion warps
+    uint64_t *empty = bars + 3 * kStages;      // MMAs of the stage done (committed to both)
+    uint64_t *p_free = bars + 4 * kStages;     // own packed tile read
+    uint64_t *acc_full = bars + 5 * kStages;   // [2], committed to both
+    uint64_t *acc_empty = acc_full + 2;        // [2], even CTA: 2 x 8 epilogue warps
+    uint32_t *sig = reinterpret_cast<uint32_t *>(smem + S::sig_off);  // st.async targets
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + S::tmem_slot_off);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = int(blockIdx.x >> 1);
+    const int t_begin = tab.cta0[pair], t_end = tab.cta0[pair + 1];
+    unsigned *err = tab.err;
+    pdl_launch_dependents();
+
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < tab.n; ++j) {
+            prefetch_tensormap(&tab.map_p[j]);
+            prefetch_tensormap(&tab.map_x[j]);
+        }
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&pfull[s], 1);
+            mbar_init(&a_full[s], kExpWarps);  // own warps; the odd CTA's by bytes
+            mbar_init(&empty[s], 1);
+            mbar_init(&p_free[s], kExpWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2 * kEpiWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1)
+        tmem_alloc_pair(tmem_slot, kPairTmemCols);
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers exist before either arrives remotely
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // the even CTA's barriers, as cluster addresses
+    auto lead = [&](uint64_t *b) { return map_to_rank(smem_u32(b), 0); };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            pdl_wait();
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int i = t_begin; i < t_end && ok; ++i) {
+                const uint32_t code = tab.tile[i];
+                const int e = int(code >> 28), tt = int((code >> 14) & (kTileField - 1)),
+                          ft = int(code & (kTileField - 1));
+                const int KS = tab.e[e].KS;
+                for (int ks = 0; ks < KS; ++ks) {
+                    if (issued >= kStages) {
+                        if (!mbar_wait(&empty[stage], phase ^ 1u, err) ||
+                            !mbar_wait(&p_free[stage], phase ^ 1u, err)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[stage], 2 * kPairBHalf);
+                    tma_load_2d_pair(sB + stage * kPairBHalf, &tab.map_x[e], ks * kBK,
+                                     tt * kPairBN + int(rank) * (kPairBN / 2), lead(&full[stage]));
+                    mbar_arrive_expect_tx(&pfull[stage], kPBytes);
+                    tma_load_2d(sP + stage * kPBytes, &tab.map_p[e], ks * kBK,
+                                ft * (2 * kPackedRows) + int(rank) * kPackedRows, &pfull[stage]);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the packed tiles still in flight land before the CTA may retire
+            // (the activation halves are waited for by the even CTA's MMA
+            // thread, and the CTAs retire together)
+            for (int s = 0; s < kStages && s < issued; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % kStages);
+                mbar_wait(&pfull[s], uint32_t((last / kStages) & 1), err);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int issued = 0;
+            for (int i = t_begin, local = 0; i < t_end && ok; ++i, ++local) {
+                const int buf = local & 1;
+                if (local >= 2 &&
+                    !mbar_wait_cluster(&acc_empty[buf], uint32_t(((local - 2) >> 1) & 1), err))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + uint32_t(buf * kPairBN);
+                const int KS = tab.e[tab.tile[i] >> 28].KS;
+                for (int ks = 0; ks < KS; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, err) ||
+                        !mbar_wait_cluster(&a_full[stage], phase, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = umma_desc_sw128(smem_u32(sA + stage * kABytes));
+                    const uint64_t db = umma_desc_sw128(smem_u32(sB + stage * kPairBHalf));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        umma_i8_pair(d_tmem, umma_desc_advance(da, uint32_t(kk * 32)),
+                                     umma_desc_advance(db, uint32_t(kk * 32)), kIdesc,
+                                     (ks > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair(&empty[stage]);
+                    ++issued;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok)
+                    umma_commit_pair(&acc_full[buf]);
+            }
+            if (issued > 0) {
+                const int s = (issued - 1) % kStages;
+                mbar_wait(&empty[s], uint32_t(((issued - 1) / kStages) & 1), err);
+            }
+        }
+    } else if (warp < kEpiWarp0) {
+        // ------------------------------------------------ code expansion (both CTAs)
+        const int et = threadIdx.x - kExpWarp0 * 32;  // 0..255
+        const int j = et >> 3, c = et & 7;
+        int stage = 0;
+        uint32_t phase = 0;
+        int seen = 0;
+        bool ok = true;
+        for (int i = t_begin; i < t_end && ok; ++i) {
+            const int KS = tab.e[tab.tile[i] >> 28].KS;
+            for (int ks = 0; ks < KS; ++ks) {
+                const bool w1 = mbar_wait_warp(&pfull[stage], phase, err);
+                const bool w2 =
+                    w1 && (seen < kStages || mbar_wait_warp(&empty[stage], phase ^ 1u, err));
+                if (!w2) {
+                    ok = false;
+                    break;
+                }
+                const uint4 v = *reinterpret_cast<const uint4 *>(sP + stage * kPBytes + sw128_off(j, c));
+                uint8_t *A = sA + stage * kABytes;
+#pragma unroll
+                for (int pl = 0; pl < 4; ++pl) {
+                    const uint32_t m = 0x03030303u << (2 * pl);
+                    const uint4 o = make_uint4(v.x & m, v.y & m, v.z & m, v.w & m);
+                    *reinterpret_cast<uint4 *>(A + sw128_off(j + 32 * pl, c)) = o;
+                }
+                fence_proxy_async_smem();  // the codes are read by the tensor cores
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&p_free[stage]);
+                    const int ew = warp - kExpWarp0;
+                    if (!leader)
+                        st_async_signal(map_to_rank(smem_u32(&sig[ew]), 0), 1u, lead(&a_full[stage]));
+                    else if (ew == 0)  // the odd CTA's 8 x 4 bytes
+                        mbar_arrive_expect_tx(&a_full[stage], 4 * kExpWarps);
+                    else
+                        mbar_arrive(&a_full[stage]);
+                }
+                ++seen;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // the last tile's columns [128, 256) of this CTA's rows
+        const int local_last = t_end - 1 - t_begin;
+        if (ok && local_last >= 0) {
+            pdl_wait();
+            const int buf = local_last & 1;
+            if (mbar_wait_warp(&acc_full[buf], uint32_t((local_last >> 1) & 1), err)) {
+                tc_fence_after();
+                const uint32_t code = tab.tile[t_end - 1];
+                const int c_begin = kPairBN / 2 + ((warp - kExpWarp0) >> 2) * (kPairBN / 4);
+                drain_columns<kPairBN>(tab, code,
+                                       int(code & (kTileField - 1)) * (2 * kPackedRows) +
+                                           int(rank) * kPackedRows,
+                                       tmem_base + uint32_t(buf * kPairBN), warp & 3, c_begin,
+                                       c_begin + kPairBN / 4, lane);
+                tc_fence_before();
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int half = (warp - kEpiWarp0) >> 2;
+        pdl_wait();
+        for (int i = t_begin, local = 0; i < t_end; ++i, ++local) {
+            const int buf = local & 1;
+            if (!mbar_wait_warp(&acc_full[buf], uint32_t((local >> 1) & 1), err))
+                break;
+            tc_fence_after();
+            const bool last = i + 1 == t_end;
+            const int c_begin = last ? half * (kPairBN / 4) : half * (kPairBN / 2);
+            const int c_end = c_begin + (last ? kPairBN / 4 : kPairBN / 2);
+            const uint32_t code = tab.tile[i];
+            drain_columns<kPairBN>(tab, code,
+                                   int(code & (kTileField - 1)) * (2 * kPackedRows) +
+                                       int(rank) * kPackedRows,
+                                   tmem_base + uint32_t(buf * kPairBN), q, c_begin, c_end, lane);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote(lead(&acc_empty[buf]));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // no remote arrive or MMA operand read outlives either CTA
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc_pair(tmem_base, kPairTmemCols);
 }
 
 // Deal the tiles [0, n) (costs cost[i]) to `grid` CTAs, longest first, each
@@ -483,32 +760,42 @@ PrefillTable *prefill_table()
     return &t;
 }
 
-template <int BN>
-cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
+// How a launch tiles the work: tokens per tile, packed rows per tile (32 per
+// CTA), the activation box each CTA loads, CTAs per tile.
+struct TileForm {
+    int tok, prows, xbox, ctas;
+    void (*kernel)(PrefillTable);
+    size_t smem;
+};
+
+cudaError_t configure(const TileForm &f, std::atomic<int> &configured_dev)
 {
-    using S = PrefillShape<BN>;
-    const size_t smem = S::bytes + 1024;  // + alignment slack
-    static std::atomic<int> configured_dev{-1};  // set by any host thread
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess)
         return err;
     if (configured_dev != dev) {
-        err = cudaFuncSetAttribute(prefill_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(smem));
+        err = cudaFuncSetAttribute(f.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(f.smem));
         if (err != cudaSuccess)
             return err;
         configured_dev = dev;
     }
+    return cudaSuccess;
+}
+
+cudaError_t launch_tiles(const TileForm &f, const PrefillEntry *in, int n, int M,
+                         cudaStream_t stream)
+{
     unsigned *err_word = device_error_word();
     if (!err_word)
         return cudaErrorUnknown;
-    const int tok_tiles = (M + BN - 1) / BN;
+    const int tok_tiles = (M + f.tok - 1) / f.tok;
     // every tile of every projection, in projection order
     std::vector<uint32_t> codes;
     std::vector<int> cost;
     for (int j = 0; j < n; ++j) {
-        const int ft_tiles = (in[j].N / 4 + kPackedRows - 1) / kPackedRows;
+        const int ft_tiles = (in[j].N / 4 + f.prows - 1) / f.prows;
         const int KS = (in[j].K + kBK - 1) / kBK;
         for (int ft = 0; ft < ft_tiles; ++ft)
             for (int tt = 0; tt < tok_tiles; ++tt) {
@@ -523,7 +810,7 @@ cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
     tab.err = err_word;
     for (int j = 0; j < n; ++j) {
         if (!make_map(&tab.map_p[j], in[j].packed, in[j].K, in[j].N / 4, kPackedRows) ||
-            !make_map(&tab.map_x[j], in[j].xq, in[j].K, M, BN))
+            !make_map(&tab.map_x[j], in[j].xq, in[j].K, M, f.xbox))
             return cudaErrorInvalidValue;
         const bool vec = (in[j].N / 4) % 4 == 0 && reinterpret_cast<uintptr_t>(in[j].y) % 16 == 0 &&
                          reinterpret_cast<uintptr_t>(in[j].acc_out) % 16 == 0;
@@ -532,32 +819,54 @@ cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
     }
     // launches of up to kPrefillMaxTiles tiles each (any subset of tiles is a
     // valid launch); one launch for every shape this library is measured on
-    const int sms = device_sm_count();
+    const int units = std::min(device_sm_count(), kPrefillMaxGrid) / f.ctas;
     const int total = int(codes.size());
     for (int base = 0; base < total; base += kPrefillMaxTiles) {
         const int cnt = std::min(total - base, kPrefillMaxTiles);
-        const int grid = std::min({cnt, sms, kPrefillMaxGrid});
+        const int grid = std::min(cnt, units);  // CTAs (or CTA pairs) dealt tiles
         std::vector<int> sub(cost.begin() + base, cost.begin() + base + cnt), order;
         schedule_lpt(sub, grid, order, tab.cta0);
         for (int i = 0; i < cnt; ++i)
             tab.tile[i] = codes[size_t(base + order[size_t(i)])];
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid);
+        cfg.gridDim = dim3(unsigned(grid * f.ctas));
         cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = f.smem;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = unsigned(f.ctas);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, prefill_tc_kernel<BN>, tab);
+        cfg.numAttrs = f.ctas > 1 ? 2 : 1;
+        cudaError_t err = cudaLaunchKernelEx(&cfg, f.kernel, tab);
         if (err == cudaSuccess)
             err = cudaGetLastError();
         if (err != cudaSuccess)
             return err;
     }
     return cudaSuccess;
+}
+
+template <int BN>
+cudaError_t launch_bn(const PrefillEntry *in, int n, int M, cudaStream_t stream)
+{
+    static std::atomic<int> configured_dev{-1};  // set by any host thread
+    const TileForm f{BN, kPackedRows, BN, 1, prefill_tc_kernel<BN>, PrefillShape<BN>::bytes + 1024};
+    const cudaError_t err = configure(f, configured_dev);
+    return err != cudaSuccess ? err : launch_tiles(f, in, n, M, stream);
+}
+
+cudaError_t launch_pair(const PrefillEntry *in, int n, int M, cudaStream_t stream)
+{
+    static std::atomic<int> configured_dev{-1};
+    const TileForm f{kPairBN, 2 * kPackedRows, kPairBN / 2, 2, prefill_pair_kernel,
+                     PairSmem::bytes + 1024};
+    const cudaError_t err = configure(f, configured_dev);
+    return err != cudaSuccess ? err : launch_tiles(f, in, n, M, stream);
 }
 
 }  // namespace
@@ -575,11 +884,19 @@ cudaError_t launch_prefill_group(const PrefillEntry *e, int n, int M, cudaStream
     for (int j = 0; j < n; ++j)
         if ((e[j].N / 4 + kPackedRows - 1) / kPackedRows > kTileField)
             return cudaErrorInvalidValue;
-    // 128-token tiles while they waste less of the MMA than 256-token ones
+    // 128-token tiles while they waste less of the MMA than 256-token ones;
+    // from 129 tokens CTA pairs on 256 x 256 tiles (TQ_PREFILL_PAIR=0 keeps
+    // single CTAs on 128 x 256 tiles, for measurement)
     const bool narrow = M <= 128;
     if ((M + (narrow ? 127 : 255)) / (narrow ? 128 : 256) > kTileField)
         return cudaErrorInvalidValue;
-    const cudaError_t err = narrow ? launch_bn<128>(e, n, M, stream) : launch_bn<256>(e, n, M, stream);
+    static const bool pairs = [] {
+        const char *v = getenv("TQ_PREFILL_PAIR");
+        return !(v && !strcmp(v, "0"));
+    }();
+    const cudaError_t err = narrow  ? launch_bn<128>(e, n, M, stream)
+                            : pairs ? launch_pair(e, n, M, stream)
+                                    : launch_bn<256>(e, n, M, stream);
     if (err == cudaSuccess)
         *handled = true;
     return err;

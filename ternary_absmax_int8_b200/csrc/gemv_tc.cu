@@ -202,49 +202,6 @@ struct SmallMSmem {
     static constexpr size_t bytes = misc_off + 16;
 };
 
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// mbar_wait_warp with cluster-scope acquire (the arrivals come from other
-// CTAs of the cluster, after their red operations on this CTA's memory).
-__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
-                                                       unsigned *err)
-{
-    bool done = mbar_try_wait_cluster(bar, parity);
-    if (__all_sync(0xffffffffu, done))
-        return true;
-    const unsigned long long t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        done = done || mbar_try_wait_cluster(bar, parity);
-        if (__all_sync(0xffffffffu, done))
-            return true;
-        if ((i & 255u) == 0) {
-            const bool late = global_ns() - t0 > kWaitLimitNs;
-            if (__any_sync(0xffffffffu, late)) {
-                if ((threadIdx.x & 31) == 0)
-                    atomicOr(err, kErrWaitTimeout);
-                return false;
-            }
-        }
-    }
-}
-
 // Unit u of the whole call belongs to CTA b with U(b) <= u < U(b+1).
 __device__ __forceinline__ int unit_start(int b, int total, int grid)
 {

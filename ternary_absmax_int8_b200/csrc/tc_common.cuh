@@ -216,6 +216,135 @@ __device__ __forceinline__ void red_add_cluster(uint32_t raddr, int32_t v)
                  : "memory");
 }
 
+// ------------------------------------------------- cluster-scope mbarriers
+// Arrive on an mbarrier of another CTA of the cluster (address from mapa).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait with cluster-scope acquire, one thread (arrivals from other CTAs
+// of the cluster).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, unsigned *err)
+{
+    if (mbar_try_wait_cluster(bar, parity))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cluster(bar, parity))
+            return true;
+        if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, kErrWaitTimeout);
+            return false;
+        }
+    }
+}
+
+// mbar_wait_warp with cluster-scope acquire (the arrivals come from other
+// CTAs of the cluster, after their operations on this CTA's memory).
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t *bar, uint32_t parity,
+                                                       unsigned *err)
+{
+    bool done = mbar_try_wait_cluster(bar, parity);
+    if (__all_sync(0xffffffffu, done))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        done = done || mbar_try_wait_cluster(bar, parity);
+        if (__all_sync(0xffffffffu, done))
+            return true;
+        if ((i & 255u) == 0) {
+            const bool late = global_ns() - t0 > kWaitLimitNs;
+            if (__any_sync(0xffffffffu, late)) {
+                if ((threadIdx.x & 31) == 0)
+                    atomicOr(err, kErrWaitTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Asynchronous 4-byte store to another CTA's shared memory that completes 4
+// transaction bytes on that CTA's mbarrier (both cluster addresses); the
+// issuing thread does not wait for it.
+__device__ __forceinline__ void st_async_signal(uint32_t raddr, uint32_t value, uint32_t rbar)
+{
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(raddr),
+        "r"(value), "r"(rbar)
+        : "memory");
+}
+
+// ---------------------------------------------- CTA pairs (cta_group::2)
+// The two CTAs of a cluster of two run one MMA of 256 rows: each holds 128
+// rows of A and half of B's columns in its shared memory, and its 128 rows of
+// D in its own tensor memory. Only the even CTA issues the MMAs and commits.
+
+// Tensor memory of both CTAs of the pair: issued by the same warp in each.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(slot)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols)
+                 : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T over the pair, int8 kind.
+__device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at the same offset in both CTAs of the pair once
+// the MMAs this thread issued complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(uint16_t(3))
+        : "memory");
+}
+
+// 2-D TMA load into this CTA's shared memory whose completion is counted on
+// the even CTA's mbarrier at cluster address `bar_cluster` (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+
 // ---------------------------------------------------------------- host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
