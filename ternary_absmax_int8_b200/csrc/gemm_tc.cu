@@ -461,7 +461,8 @@ prefill_tc_kernel(const __grid_constant__ PrefillTable tab)
 // remote arrive with cluster-scope release stalls its thread ~1,000 cycles,
 // too much per stage), each CTA's own pfull (its packed tile) and p_free,
 // and empty / acc_full committed to both CTAs by the even CTA's MMA thread;
-// acc_empty on the even CTA (both CTAs' epilogue warps).
+// acc_empty on the even CTA (its epilogue warps arrive, the odd CTA's
+// complete bytes the same way).
 constexpr int kPairBN = 256;              // tokens per tile
 constexpr int kPairBHalf = (kPairBN / 2) * kBK;  // 16 KB: a CTA's activation rows
 constexpr int kPairStage = kABytes + kPairBHalf + kPBytes;
@@ -475,7 +476,7 @@ struct PairSmem {
     static constexpr size_t bar_off = p_off + size_t(kPairStages) * kPBytes;
     // full, pfull, a_full, empty, p_free per stage; acc_full[2], acc_empty[2]
     static constexpr size_t sig_off = bar_off + size_t(5 * kPairStages + 4) * 8;
-    static constexpr size_t tmem_slot_off = sig_off + 64;  // 8 words written by st.async
+    static constexpr size_t tmem_slot_off = sig_off + 64;  // 16 words written by st.async
     static constexpr size_t bytes = tmem_slot_off + 16;
     static_assert(kPairStages >= 4, "four stages at least");
     static_assert(bytes + 1024 <= kSmemLimit, "shared memory");
@@ -527,7 +528,7 @@ prefill_pair_kernel(const __grid_constant__ PrefillTable tab)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 2 * kEpiWarps);
+            mbar_init(&acc_empty[b], kEpiWarps);  // own warps; the odd CTA's by bytes
         }
         fence_mbar_init();
     }
@@ -709,8 +710,16 @@ prefill_pair_kernel(const __grid_constant__ PrefillTable tab)
                                    tmem_base + uint32_t(buf * kPairBN), q, c_begin, c_end, lane);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive_remote(lead(&acc_empty[buf]));
+            if (lane == 0) {  // the accumulator's loads have completed (tcgen05.wait::ld)
+                const int ew = warp - kEpiWarp0;
+                if (!leader)
+                    st_async_signal(map_to_rank(smem_u32(&sig[kExpWarps + ew]), 0), 1u,
+                                    lead(&acc_empty[buf]));
+                else if (ew == 0)  // the odd CTA's 8 x 4 bytes
+                    mbar_arrive_expect_tx(&acc_empty[buf], 4 * kEpiWarps);
+                else
+                    mbar_arrive(&acc_empty[buf]);
+            }
         }
     }
 
