@@ -490,7 +490,7 @@ def run_ours(args, rank: int, world: int):
         # int8 contraction: tensor-bound. Peak = measured dense bf16 x the
         # nominal int8 : bf16 ratio (4.5 : 2.25 PFLOP/s).
         tpeak, tkind = measured_tensor_peak()
-        roof = {"kernel": "prefill_tc_kernel", "bound": "tensor",
+        roof = {"kernel": prefill_kernel_name(M), "bound": "tensor",
                 "achieved": round(flops / (gemv_avg * 1e9), 1), "peak": tpeak,
                 "peak_kind": tkind, "unit": "TOPS (int8)",
                 "frac": round(flops / (gemv_avg * 1e9) / tpeak, 4), "traffic": None,
@@ -581,6 +581,14 @@ def batch_kernel_name(M: int, mode: str) -> str:
     if forced == "mma" or forced == "" and M <= 16:
         return "mma_gemv_kernel"
     return "smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"
+
+
+def prefill_kernel_name(M: int) -> str:
+    """The prefill GEMM kernel the library runs for M tokens: CTA pairs from
+    129 tokens unless TQ_PREFILL_PAIR=0, single CTAs otherwise."""
+    if M > 128 and os.environ.get("TQ_PREFILL_PAIR", "") != "0":
+        return "prefill_pair_kernel"
+    return "prefill_tc_kernel"
 
 
 def binary_kernel_name(M: int) -> str:
@@ -738,7 +746,7 @@ def run_next(args, rank: int, world: int):
         sb = sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
         gemv_units = sum(2.0 * p.M * p.N * p.K for p in projs)
         launches = n + -(-n // 16)
-        kernel = "prefill_tc_kernel"
+        kernel = prefill_kernel_name(M)
     else:
         B = []
         for p in projs:

@@ -106,3 +106,12 @@ def test_recorded_binary_traffic_needs_the_same_kernel_and_workload():
     assert bench.recorded_binary_traffic("binary_ffn27b_m1", "binary_gemv_kernel") is None
     assert bench.recorded_binary_traffic("prefill_m512", "binary_mma_kernel") is None
     assert len(bench.binary_kernel_sha()) == 16
+
+
+def test_prefill_kernel_name(monkeypatch):
+    monkeypatch.delenv("TQ_PREFILL_PAIR", raising=False)
+    assert [bench.prefill_kernel_name(m) for m in (33, 128, 129, 512)] == [
+        "prefill_tc_kernel", "prefill_tc_kernel", "prefill_pair_kernel", "prefill_pair_kernel"]
+    monkeypatch.setenv("TQ_PREFILL_PAIR", "0")
+    assert bench.prefill_kernel_name(512) == "prefill_tc_kernel"
+
