@@ -27,7 +27,7 @@
 // loaded), and the activations with 16-byte loads from L1/L2.
 //
 // Work split. Tiles of 16 packed rows (64 outputs) x the full K, numbered
-// across the projections of a launch; each CTA (one per SM, 16 warps) takes a
+// across the projections of a launch; each CTA (one per SM, 16 or 20 warps) takes a
 // contiguous, byte-balanced range of tiles. Its warps form teams of P that
 // take the range's tiles in turn; the P warps of a team split a tile's
 // 64-column steps. With many tiles P = 1: a warp owns whole tiles and
@@ -47,16 +47,20 @@ namespace tq {
 
 namespace {
 
-constexpr int kMmaW = 16;         // warps per CTA
-constexpr int kMmaThreads = kMmaW * 32;
+// Warps per CTA: 12 for up to 8 tokens (256-column steps), 16 beyond.
+template <int NT>
+constexpr int kMmaW = NT == 1 ? 12 : 16;
 constexpr int kMmaRing = 4;       // cp.async stages per warp (a power of two)
 constexpr int kMmaRows = 16;      // packed rows per tile
-// A step is H halves of 64 columns (H = 2 for up to 16 tokens, 1 beyond,
-// where the accumulators and the prefetched activations take more registers
-// and the accumulator slots more shared memory); a stage holds [2 rows][H
-// halves][32 lanes][16 bytes].
+// A step is H pieces of 64 columns (H = 4 for up to 8 tokens, 2 for up to 16,
+// 1 beyond, where the accumulators and the prefetched activations take more
+// registers and the accumulator slots more shared memory); a stage holds
+// [2 rows][H pieces][32 lanes][16 bytes]. Wide steps keep the number of
+// separate row streams per SM low: 16-row tiles read as 256-byte row pieces
+// by 12 warps move ~6.1 TB/s in a copy-only test, 128-byte pieces by 16 or
+// 20 warps 5.1 or 4.2 TB/s (DRAM page locality).
 template <int NT>
-constexpr int kHalves = NT <= 2 ? 2 : 1;
+constexpr int kHalves = NT == 1 ? 4 : (NT <= 2 ? 2 : 1);
 template <int NT>
 constexpr int kStep = 64 * kHalves<NT>;
 template <int NT>
@@ -125,7 +129,7 @@ __device__ __forceinline__ void store_out(const MmaEntry &e, int M, int row, int
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kMmaThreads, 1)
+__global__ void __launch_bounds__(kMmaW<NT> * 32, 1)
 mma_gemv_kernel(const __grid_constant__ MmaParams p)
 {
     // per-warp rings: [W][kMmaRing] stages of [2 rows][H halves][32 lanes][16
@@ -135,15 +139,19 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     constexpr int H = kHalves<NT>, STEP = kStep<NT>, SB = kStageBytes<NT>;
     constexpr int kRingBytes = kMmaRing * SB;
     constexpr int kCols = 8 * NT;
-    int32_t *slots = reinterpret_cast<int32_t *>(smem + kMmaW * kRingBytes);
+    constexpr int W = kMmaW<NT>;
+    int32_t *slots = reinterpret_cast<int32_t *>(smem + W * kRingBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const uint8_t *ring = smem + warp * kRingBytes + lane * 16;
     const uint32_t ring_s = smem_u32(ring);
 
     const int t_begin = p.cta_tile0[blockIdx.x], t_end = p.cta_tile0[blockIdx.x + 1];
-    const int lgP = p.lgP, P = 1 << lgP, teams = kMmaW >> lgP;
+    const int lgP = p.lgP, P = 1 << lgP, teams = W >> lgP;
+    // teams of P warps; warps past the last whole team (W not a multiple of
+    // P) stay idle
     const int team = warp >> lgP, piece = warp & (P - 1);
+    const int first = team < teams ? t_begin + team : t_end;
     const Walk<STEP> wk{p.e, p.n_entries, t_end, teams, piece, lgP, 16 * t};
 
     if (threadIdx.x == 0)
@@ -151,8 +159,8 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
 
     // the load cursor runs kMmaRing - 1 steps ahead of the compute cursor
     Cursor lc{t_end, 0, 0, 0, 0, nullptr, false, false};
-    if (t_begin + team < t_end) {
-        wk.start(lc, t_begin + team, g);
+    if (first < t_end) {
+        wk.start(lc, first, g);
         wk.settle(lc, g);
     }
     int issued = 0;
@@ -193,8 +201,8 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     zero_acc();
     int consumed = 0;
     Cursor cc{t_end, 0, 0, 0, 0, nullptr, false, false};
-    if (t_begin + team < t_end) {
-        wk.start(cc, t_begin + team, g);
+    if (first < t_end) {
+        wk.start(cc, first, g);
         wk.settle(cc, g);
     }
 
@@ -223,7 +231,7 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     };
     load_q(cc);
 
-    for (int tile = t_begin + team; tile < t_end; tile += teams) {
+    for (int tile = first; tile < t_end; tile += teams) {
         while (fent + 1 < p.n_entries && p.e[fent + 1].tile_begin <= tile)
             ++fent;
         const MmaEntry &e = p.e[fent];
@@ -326,7 +334,8 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
 template <int NT>
 cudaError_t launch_nt(const MmaParams &p, int grid, cudaStream_t stream, bool pdl)
 {
-    constexpr size_t smem = size_t(kMmaW) * kMmaRing * kStageBytes<NT> + size_t(kMmaW) * 4 * 16 * 8 * NT * 4;
+    constexpr int W = kMmaW<NT>;
+    constexpr size_t smem = size_t(W) * kMmaRing * kStageBytes<NT> + size_t(W) * 4 * 16 * 8 * NT * 4;
     static_assert(smem <= 227 * 1024, "shared memory");
     static std::atomic<int> configured_dev{-1};
     int dev = 0;
@@ -342,7 +351,7 @@ cudaError_t launch_nt(const MmaParams &p, int grid, cudaStream_t stream, bool pd
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kMmaThreads);
+    cfg.blockDim = dim3(W * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -389,8 +398,9 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
         // teams of P: P = 1 (whole tiles per warp, no barrier) when there
         // are enough tiles to give every warp two, more when there are fewer
         const int grid = std::min({total, sms, kMmaMaxGrid});
+        const int W = M <= 8 ? kMmaW<1> : kMmaW<2>;
         int lgP = 0;
-        while ((1 << lgP) < kMmaW && (long long)total << lgP < 2LL * kMmaW * grid)
+        while ((2 << lgP) <= W && (long long)total << lgP < 2LL * W * grid)
             ++lgP;
         p.lgP = lgP;
         std::vector<long long> prefix(size_t(total) + 1, 0);
