@@ -47,20 +47,24 @@ namespace tq {
 
 namespace {
 
-// Warps per CTA: 12 for up to 8 tokens (256-column steps), 16 beyond.
+// Warps per CTA: 12 up to 16 tokens (256-column steps; up to 170 registers
+// a thread), 16 beyond.
 template <int NT>
-constexpr int kMmaW = NT == 1 ? 12 : 16;
-constexpr int kMmaRing = 4;       // cp.async stages per warp (a power of two)
+constexpr int kMmaW = NT <= 2 ? 12 : 16;
+// cp.async stages per warp (3 where two token groups' accumulator slots
+// leave no room for a fourth)
+template <int NT>
+constexpr int kRing = NT == 2 ? 3 : 4;
 constexpr int kMmaRows = 16;      // packed rows per tile
-// A step is H pieces of 64 columns (H = 4 for up to 8 tokens, 2 for up to 16,
-// 1 beyond, where the accumulators and the prefetched activations take more
-// registers and the accumulator slots more shared memory); a stage holds
+// A step is H pieces of 64 columns (H = 4 up to 16 tokens, 1 beyond, where
+// the accumulators and the prefetched activations take more registers and
+// the accumulator slots more shared memory); a stage holds
 // [2 rows][H pieces][32 lanes][16 bytes]. Wide steps keep the number of
 // separate row streams per SM low: 16-row tiles read as 256-byte row pieces
 // by 12 warps move ~6.1 TB/s in a copy-only test, 128-byte pieces by 16 or
 // 20 warps 5.1 or 4.2 TB/s (DRAM page locality).
 template <int NT>
-constexpr int kHalves = NT == 1 ? 4 : (NT <= 2 ? 2 : 1);
+constexpr int kHalves = NT <= 2 ? 4 : 1;
 template <int NT>
 constexpr int kStep = 64 * kHalves<NT>;
 template <int NT>
@@ -132,12 +136,12 @@ template <int NT>
 __global__ void __launch_bounds__(kMmaW<NT> * 32, 1)
 mma_gemv_kernel(const __grid_constant__ MmaParams p)
 {
-    // per-warp rings: [W][kMmaRing] stages of [2 rows][H halves][32 lanes][16
+    // per-warp rings: [W][RING] stages of [2 rows][H pieces][32 lanes][16
     // bytes] (16-byte lane slots keep the reads free of bank conflicts),
     // then the teams' accumulator slots [W][4 masks][16 rows][8 NT tokens]
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int H = kHalves<NT>, STEP = kStep<NT>, SB = kStageBytes<NT>;
-    constexpr int kRingBytes = kMmaRing * SB;
+    constexpr int H = kHalves<NT>, STEP = kStep<NT>, SB = kStageBytes<NT>, RING = kRing<NT>;
+    constexpr int kRingBytes = RING * SB;
     constexpr int kCols = 8 * NT;
     constexpr int W = kMmaW<NT>;
     int32_t *slots = reinterpret_cast<int32_t *>(smem + W * kRingBytes);
@@ -157,15 +161,15 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     if (threadIdx.x == 0)
         pdl_launch_dependents();
 
-    // the load cursor runs kMmaRing - 1 steps ahead of the compute cursor
+    // the load cursor runs RING - 1 steps ahead of the compute cursor
     Cursor lc{t_end, 0, 0, 0, 0, nullptr, false, false};
     if (first < t_end) {
         wk.start(lc, first, g);
         wk.settle(lc, g);
     }
-    int issued = 0;
+    int issued = 0;  // ring slot of the next copy
     auto issue = [&]() {
-        const uint32_t dst = ring_s + uint32_t(issued & (kMmaRing - 1)) * SB;
+        const uint32_t dst = ring_s + uint32_t(issued) * SB;
         if (lc.tile < t_end) {
             const int k = lc.step * STEP;  // + 16 t already in lc.row
             const uint8_t *src = lc.row + k;
@@ -180,10 +184,10 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
             wk.settle(lc, g);
         }
         cp_async_commit();  // (possibly empty) group per step keeps the count uniform
-        ++issued;
+        issued = issued + 1 == RING ? 0 : issued + 1;
     };
 #pragma unroll
-    for (int i = 0; i < kMmaRing - 1; ++i)
+    for (int i = 0; i < RING - 1; ++i)
         issue();
 
     pdl_wait();  // activations, scales, outputs of the previous kernel
@@ -199,7 +203,7 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
                     d[j][n][r] = 0;
     };
     zero_acc();
-    int consumed = 0;
+    int consumed = 0;  // ring slot of the next step to compute
     Cursor cc{t_end, 0, 0, 0, 0, nullptr, false, false};
     if (first < t_end) {
         wk.start(cc, first, g);
@@ -246,9 +250,9 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
             ++cc.step;
             wk.settle(cc, g);
             load_q(cc);  // the next step's activations
-            cp_async_wait<kMmaRing - 1>();
+            cp_async_wait<RING - 1>();
             __syncwarp();
-            const uint8_t *src = ring + (consumed & (kMmaRing - 1)) * SB;
+            const uint8_t *src = ring + consumed * SB;
 #pragma unroll
             for (int h = 0; h < H; ++h) {
                 const uint4 lo4 = *reinterpret_cast<const uint4 *>(src + h * 512);        // row g
@@ -273,7 +277,7 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
                     }
                 }
             }
-            ++consumed;
+            consumed = consumed + 1 == RING ? 0 : consumed + 1;
         }
         const int r0 = (tile - e.tile_begin) * kMmaRows;
         if (P == 1) {
@@ -335,7 +339,7 @@ template <int NT>
 cudaError_t launch_nt(const MmaParams &p, int grid, cudaStream_t stream, bool pdl)
 {
     constexpr int W = kMmaW<NT>;
-    constexpr size_t smem = size_t(W) * kMmaRing * kStageBytes<NT> + size_t(W) * 4 * 16 * 8 * NT * 4;
+    constexpr size_t smem = size_t(W) * kRing<NT> * kStageBytes<NT> + size_t(W) * 4 * 16 * 8 * NT * 4;
     static_assert(smem <= 227 * 1024, "shared memory");
     static std::atomic<int> configured_dev{-1};
     int dev = 0;
@@ -398,7 +402,7 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
         // teams of P: P = 1 (whole tiles per warp, no barrier) when there
         // are enough tiles to give every warp two, more when there are fewer
         const int grid = std::min({total, sms, kMmaMaxGrid});
-        const int W = M <= 8 ? kMmaW<1> : kMmaW<2>;
+        const int W = M <= 8 ? kMmaW<1> : (M <= 16 ? kMmaW<2> : kMmaW<4>);
         int lgP = 0;
         while ((2 << lgP) <= W && (long long)total << lgP < 2LL * W * grid)
             ++lgP;
