@@ -735,8 +735,8 @@ def run_reference(args, rank: int, world: int):
 
 # --------------------------------------- Hadamard prefill, binary g128 decode
 def run_next(args, rank: int, world: int):
-    """prefill_had4_m512: per projection, the fused Hadamard rotation + 4-bit
-    quantiser launch and the prefill GEMM on its codes; binary_ffn27b_m1: the
+    """prefill_had4_m512: the grouped Hadamard rotation + 4-bit quantiser
+    launch and the grouped prefill GEMM on its codes; binary_ffn27b_m1: the
     stack quantiser and one binary g128 GEMV launch over the 24 projections.
     Same JSON line as the other workloads."""
     import torch
@@ -775,12 +775,12 @@ def run_next(args, rank: int, world: int):
             tq.tq_pack_host(p.w, P, p.M, p.N, p.K)
             W.append([torch.from_numpy(P).cuda() for _ in range(copies)])
 
+        htab = [tq.make_proj(x=x_dev.data_ptr() + 2 * int(kx[j]), xq=xq.data_ptr() + int(kx[j]),
+                             x_scale=xs.data_ptr() + 4 * j * M, x_sum=xsum.data_ptr() + 4 * j * M,
+                             K=p.K) for j, p in enumerate(projs)]
+
         def quant(c, s_):
-            for j, p in enumerate(projs):
-                tq.tq_hadamard_quantize_act(x_dev.data_ptr() + 2 * int(kx[j]),
-                                            xq.data_ptr() + int(kx[j]), xs.data_ptr() + 4 * j * M,
-                                            xsum.data_ptr() + 4 * j * M, p.M, p.K,
-                                            HADAMARD_BLOCK, stream=s_)
+            tq.tq_hadamard_quantize_act_stack(htab, M, HADAMARD_BLOCK, stream=s_)
 
         ptabs = [[tq.make_proj(packed=W[j][c], xq=xq.data_ptr() + int(kx[j]),
                                x_scale=xs.data_ptr() + 4 * j * M,
@@ -793,7 +793,7 @@ def run_next(args, rank: int, world: int):
 
         sb = sum(quant_bytes(p.K, p.M) + algorithmic_bytes(p.N, p.K, p.M) for p in projs)
         gemv_units = sum(2.0 * p.M * p.N * p.K for p in projs)
-        launches = n + -(-n // 16)
+        launches = -(-n // 512) + -(-n // 16)
         kernel = prefill_kernel_name(M)
     else:
         B = []

@@ -353,6 +353,18 @@ tq_status tq_hadamard_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale
                                    int M, int K, int n, cudaStream_t stream);
 
 /*
+ * tq_hadamard_quantize_act_stack -- tq_hadamard_quantize_act for M token rows
+ * of each of n_proj projections (tq_proj's x, xq, x_scale, x_sum and K, with
+ * the [M, K] / [M] shapes of the _batch calls; other fields ignored) in one
+ * launch per 512 projections, every K a multiple of n. Results are those of
+ * tq_hadamard_quantize_act on each projection, byte for byte. projs is a HOST
+ * array read during the call only. Errors as tq_hadamard_quantize_act's, for
+ * any entry (nothing is launched).
+ */
+tq_status tq_hadamard_quantize_act_stack(const tq_proj *projs, int n_proj, int M, int n,
+                                         cudaStream_t stream);
+
+/*
  * Binary g128 weights (baguaai "BitNet" tag page, Bonsai 27B item: a true
  * 1-bit binary scheme in which 128 weights share one fp16 scale, about 1.125
  * bits per weight). The page gives no bit order, group direction or

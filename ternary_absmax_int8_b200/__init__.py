@@ -22,7 +22,8 @@ __all__ = [
     "tq_gemv_stack_batch", "tq_gemm_prefill_stack", "tq_device_error", "tq_gemv_noalloc",
     "tq_status_string", "tq_last_error", "make_proj", "tq_rmsnorm_quantize",
     "tq_relu2_mul_rmsnorm_quantize", "tq_absmean_pack", "tq_selftest_wait_timeout",
-    "tq_hadamard_quantize_act", "TqBinaryProj", "tq_pack_binary_host", "tq_gemv_binary",
+    "tq_hadamard_quantize_act", "tq_hadamard_quantize_act_stack", "TqBinaryProj",
+    "tq_pack_binary_host", "tq_gemv_binary",
     "tq_gemv_binary_stack", "make_binary_proj",
 ]
 
@@ -99,6 +100,7 @@ _SIGS = {
     "tq_absmean_pack": [_vp, _vp, _vp, _i, _i, _vp],
     "tq_selftest_wait_timeout": [ctypes.c_uint, _vp],
     "tq_hadamard_quantize_act": [_vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "tq_hadamard_quantize_act_stack": [ctypes.POINTER(TqProj), _i, _i, _i, _vp],
     "tq_pack_binary_host": [_vp, _vp, _vp, _vp, _i, _i],
     "tq_gemv_binary": [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "tq_gemv_binary_stack": [ctypes.POINTER(TqBinaryProj), _i, _i, _vp],
@@ -224,6 +226,11 @@ def tq_hadamard_quantize_act(x, xq, x_scale, x_sum, M: int, K: int, n: int,
     """Blockwise Hadamard rotation (block n) then 4-bit absmax codes (-7..7 in int8)."""
     _check(_load().tq_hadamard_quantize_act(_ptr(x), _ptr(xq), _ptr(x_scale), _ptr(x_sum), M, K,
                                          int(n), _stream(stream)))
+
+
+def tq_hadamard_quantize_act_stack(projs, M: int, n: int, stream=None) -> None:
+    arr, cnt = _proj_array(projs)
+    _check(_load().tq_hadamard_quantize_act_stack(arr, cnt, int(M), int(n), _stream(stream)))
 
 
 def tq_pack_binary_host(w, scales, bits, scales_packed, N: int, K: int) -> None:

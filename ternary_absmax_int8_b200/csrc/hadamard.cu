@@ -18,7 +18,8 @@
 // is exact, so the butterfly's order gives the same value as the plain
 // matrix-vector sum; fl64(sum * fl64(1/sqrt(n))) is then rounded once to fp32.
 //
-// One CTA of 256 threads per token row. Warp w rotates blocks w, w + 8, ...:
+// One CTA of 256 threads per token row (one launch per call, or per table of
+// projections in the stack form). Warp w rotates blocks w, w + 8, ...:
 // lane l holds entries l*E .. l*E + E - 1 of a block (E = n / 32) in fp64
 // registers; butterfly stages with a stride below E stay in the lane, the
 // others pair lane l with lane l ^ (stride / E) through shuffles. The fp32
@@ -66,19 +67,17 @@ __device__ __forceinline__ int code4(float h, float s)
     return min(max(r, -7), 7);
 }
 
-// E entries per lane (block size n = 32 E).
+// One token row (the whole CTA): E entries per lane (block size n = 32 E).
 template <int E>
-__global__ void __launch_bounds__(kHadThreads)
-hadamard_quant4_kernel(const uint16_t *__restrict__ x, int8_t *__restrict__ xq,
-                       float *__restrict__ x_scale, int32_t *__restrict__ x_sum, int K, double c)
+__device__ __forceinline__ void hadamard_row(const uint16_t *__restrict__ row,
+                                             int8_t *__restrict__ qrow, float *__restrict__ x_scale,
+                                             int32_t *__restrict__ x_sum, int K, double c)
 {
     extern __shared__ __align__(16) float hs[];  // [K] rotated row, fp32
     __shared__ float red_f[kHadWarps];
     __shared__ int red_i[kHadWarps];
     constexpr int n = 32 * E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t m = blockIdx.x;
-    const uint16_t *row = x + m * size_t(K);
 
     float amax = 0.0f;
     for (int b = warp; b < K / n; b += kHadWarps) {
@@ -135,7 +134,7 @@ hadamard_quant4_kernel(const uint16_t *__restrict__ x, int8_t *__restrict__ xq,
 
     const float s = amax > 0.0f ? __fdiv_rn(7.0f, amax) : 0.0f;
     int sum = 0;
-    uint32_t *qw = reinterpret_cast<uint32_t *>(xq + m * size_t(K));
+    uint32_t *qw = reinterpret_cast<uint32_t *>(qrow);
     for (int k4 = threadIdx.x; k4 < K / 4; k4 += kHadThreads) {
         const float4 h = reinterpret_cast<const float4 *>(hs)[k4];
         const int a = code4(h.x, s), b = code4(h.y, s), cc = code4(h.z, s), d = code4(h.w, s);
@@ -145,10 +144,41 @@ hadamard_quant4_kernel(const uint16_t *__restrict__ x, int8_t *__restrict__ xq,
     }
     sum = block_reduce_had(sum, HAdd(), red_i);
     if (threadIdx.x == 0) {
-        x_scale[m] = amax > 0.0f ? __fdiv_rn(amax, 7.0f) : 0.0f;
+        *x_scale = amax > 0.0f ? __fdiv_rn(amax, 7.0f) : 0.0f;
         if (x_sum)
-            x_sum[m] = sum;
+            *x_sum = sum;
     }
+}
+
+template <int E>
+__global__ void __launch_bounds__(kHadThreads)
+hadamard_quant4_kernel(const uint16_t *__restrict__ x, int8_t *__restrict__ xq,
+                       float *__restrict__ x_scale, int32_t *__restrict__ x_sum, int K, double c)
+{
+    const size_t m = blockIdx.x;
+    hadamard_row<E>(x + m * size_t(K), xq + m * size_t(K), x_scale + m, x_sum ? x_sum + m : nullptr,
+                    K, c);
+}
+
+// The rows of a table of projections, one CTA per row (row r belongs to the
+// entry with the largest row0 <= r).
+template <int E>
+__global__ void __launch_bounds__(kHadThreads)
+hadamard_quant4_stack_kernel(const __grid_constant__ QuantStackParams p, double c)
+{
+    const int r = blockIdx.x;
+    int lo = 0, hi = p.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.e[mid].row0 <= r)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const QuantStackEntry &e = p.e[lo];
+    const size_t m = size_t(r - e.row0);
+    hadamard_row<E>(e.x + m * e.K, e.xq + m * e.K, e.x_scale + m, e.x_sum ? e.x_sum + m : nullptr,
+                    e.K, c);
 }
 
 template <int E>
@@ -177,7 +207,44 @@ cudaError_t launch_e(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_s
     return cudaGetLastError();
 }
 
+template <int E>
+cudaError_t launch_stack_e(const QuantStackParams &p, int max_k, cudaStream_t stream)
+{
+    static std::atomic<int> configured_dev{-1};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (configured_dev != dev) {
+        e = cudaFuncSetAttribute(hadamard_quant4_stack_kernel<E>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(kStreamMaxK * sizeof(float)));
+        if (e != cudaSuccess)
+            return e;
+        configured_dev = dev;
+    }
+    const double c = 1.0 / sqrt(double(32 * E));  // IEEE sqrt and divide: the oracle's constant
+    hadamard_quant4_stack_kernel<E><<<p.rows, kHadThreads, size_t(max_k) * sizeof(float), stream>>>(p, c);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_hadamard_quant4_stack(const QuantStackParams &p, int max_k, int n,
+                                         cudaStream_t stream)
+{
+    if (p.rows <= 0)
+        return cudaSuccess;
+    switch (n) {
+    case 32: return launch_stack_e<1>(p, max_k, stream);
+    case 64: return launch_stack_e<2>(p, max_k, stream);
+    case 128: return launch_stack_e<4>(p, max_k, stream);
+    case 256: return launch_stack_e<8>(p, max_k, stream);
+    case 512: return launch_stack_e<16>(p, max_k, stream);
+    case 1024: return launch_stack_e<32>(p, max_k, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_hadamard_quant4(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
                                    int M, int K, int n, cudaStream_t stream)

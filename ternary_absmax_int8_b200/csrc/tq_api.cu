@@ -688,6 +688,66 @@ tq_status tq_hadamard_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale
     return e == cudaSuccess ? ok() : cuda_fail(e, fn);
 }
 
+tq_status tq_hadamard_quantize_act_stack(const tq_proj *projs, int n_proj, int M, int n,
+                                         cudaStream_t stream)
+{
+    const char *fn = "tq_hadamard_quantize_act_stack";
+    if (n_proj < 0 || M < 0)
+        return fail(TQ_ERR_SHAPE, "%s: n_proj=%d M=%d", fn, n_proj, M);
+    if (n < 32 || n > 1024 || (n & (n - 1)) != 0)
+        return fail(TQ_ERR_SHAPE, "%s: block size n=%d must be a power of two in 32..1024", fn, n);
+    if (n_proj == 0 || M == 0)
+        return ok();
+    if (!projs)
+        return fail(TQ_ERR_NULL, "%s: projs is NULL", fn);
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        if (p.K < 0 || p.K % n != 0)
+            return fail(TQ_ERR_SHAPE, "%s: entry %d: K=%d is not a multiple of n=%d", fn, j, p.K, n);
+        if (p.K > tq::kStreamMaxK)
+            return fail(TQ_ERR_UNSUPPORTED, "%s: entry %d: K=%d exceeds %d", fn, j, p.K,
+                        tq::kStreamMaxK);
+        if (!p.x_scale || (p.K > 0 && (!p.x || !p.xq)))
+            return fail(TQ_ERR_NULL, "%s: entry %d: NULL pointer", fn, j);
+        if ((p.K > 0 && (!aligned(p.x, 16) || !aligned(p.xq, 16))) || !aligned(p.x_scale, 4) ||
+            (p.x_sum && !aligned(p.x_sum, 4)))
+            return fail(TQ_ERR_ALIGN, "%s: entry %d: misaligned pointer", fn, j);
+    }
+    std::vector<tq::QuantStackEntry> list;
+    int max_k = 0;
+    for (int j = 0; j < n_proj; ++j) {
+        const tq_proj &p = projs[j];
+        if (p.K == 0) {  // no entries: zero scale and sum, as tq_quantize_act_stack
+            cudaError_t e = cudaMemsetAsync(p.x_scale, 0, size_t(M) * sizeof(float), stream);
+            if (e == cudaSuccess && p.x_sum)
+                e = cudaMemsetAsync(p.x_sum, 0, size_t(M) * sizeof(int32_t), stream);
+            if (e != cudaSuccess)
+                return cuda_fail(e, fn);
+            continue;
+        }
+        list.push_back(tq::QuantStackEntry{p.x, p.xq, p.x_scale, p.x_sum, p.K, M, 0, 0});
+        max_k = std::max(max_k, p.K);
+    }
+    tq::QuantStackParams &params = *quant_params();
+    for (size_t base = 0; base < list.size(); base += tq::kMaxQuantStack) {
+        const size_t cnt = std::min(list.size() - base, size_t(tq::kMaxQuantStack));
+        params.n = int(cnt);
+        long long rows = 0;
+        for (size_t i = 0; i < cnt; ++i) {
+            params.e[i] = list[base + i];
+            params.e[i].row0 = int(rows);
+            rows += M;
+        }
+        if (rows > INT32_MAX)
+            return fail(TQ_ERR_UNSUPPORTED, "%s: %lld rows in one call", fn, rows);
+        params.rows = int(rows);
+        const cudaError_t e = tq::launch_hadamard_quant4_stack(params, max_k, n, stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fn);
+    }
+    return ok();
+}
+
 tq_status tq_pack_binary_host(const int8_t *w, const uint16_t *scales, uint8_t *bits,
                               uint16_t *scales_packed, int N, int K)
 {

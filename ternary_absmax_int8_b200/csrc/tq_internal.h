@@ -223,6 +223,10 @@ cudaError_t launch_absmean_pack(const uint16_t *w, uint8_t *packed, float *w_sca
 // dividing K (cudaErrorInvalidValue otherwise).
 cudaError_t launch_hadamard_quant4(const uint16_t *x, int8_t *xq, float *x_scale,
                                    int32_t *x_sum, int M, int K, int n, cudaStream_t stream);
+// The same over a table of projections' rows in one launch (entries as the
+// stack quantiser's; every K a multiple of n, max_k their largest K).
+cudaError_t launch_hadamard_quant4_stack(const QuantStackParams &p, int max_k, int n,
+                                         cudaStream_t stream);
 
 // --------------------------------------------- binary g128 GEMV (M <= 4)
 // One entry = one projection: bits uint8 [N8, K] (bit p of byte (i, k) = row

@@ -371,3 +371,29 @@ def test_hadamard_quantize_argument_checks(kw, status):
 def test_hadamard_quantize_noops():
     tq.tq_hadamard_quantize_act(None, None, None, None, 0, 2560, 256, stream=0)
     tq.tq_hadamard_quantize_act(None, None, None, None, 3, 0, 256, stream=0)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n=48), "TQ_ERR_SHAPE"),
+    (dict(K=2560, n=1024), "TQ_ERR_SHAPE"),
+    (dict(K=65536, n=256), "TQ_ERR_UNSUPPORTED"),
+    (dict(x=None), "TQ_ERR_NULL"),
+    (dict(xq=A + 8), "TQ_ERR_ALIGN"),
+    (dict(M=-1), "TQ_ERR_SHAPE"),
+])
+def test_hadamard_quantize_stack_argument_checks(kw, status):
+    args = dict(x=A, xq=A, x_scale=A, x_sum=A, M=4, K=2560, n=256)
+    args.update(kw)
+    good = tq.make_proj(x=A, xq=A, x_scale=A, x_sum=A, K=2560)
+    bad = tq.make_proj(x=args["x"], xq=args["xq"], x_scale=args["x_scale"], x_sum=args["x_sum"],
+                       K=args["K"])
+    with pytest.raises(tq.TQError) as e:
+        # the faulty entry second: nothing may have been launched for the first
+        tq.tq_hadamard_quantize_act_stack([good, bad], args["M"], args["n"], stream=0)
+    assert e.value.name == status
+
+
+def test_hadamard_quantize_stack_noops():
+    good = tq.make_proj(x=A, xq=A, x_scale=A, x_sum=A, K=2560)
+    tq.tq_hadamard_quantize_act_stack([], 4, 256, stream=0)
+    tq.tq_hadamard_quantize_act_stack([good], 0, 256, stream=0)

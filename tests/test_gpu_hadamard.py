@@ -88,3 +88,25 @@ def test_had4_codes_through_every_contraction_path(cuda_device, M):
                y.cpu().numpy())
         ref = oracle.forward_had4(oracle.pack(p.w), p.N, p.w_scale, p.x_bf16, HADAMARD_BLOCK)
         assert_parity(got, ref, f"had4 M={M}")
+
+
+@pytest.mark.parametrize("n", [256, 1024])
+def test_stack_form_matches_the_oracle(cuda_device, n):
+    # the grouped form over projections of different K (one launch): every
+    # code, scale and sum against the oracle
+    M = 7
+    rng = np.random.default_rng(n)
+    xs_in = [activations_bf16(rng, M, n * k) for k in (1, 3, 10, 27)]
+    xd = [dev(x.view(np.int16)) for x in xs_in]
+    xq = [torch.full((M, x.shape[1]), 99, dtype=torch.int8, device="cuda") for x in xs_in]
+    xs = [torch.full((M,), float("nan"), device="cuda") for _ in xs_in]
+    xsum = [torch.full((M,), -(2 ** 31), dtype=torch.int32, device="cuda") for _ in xs_in]
+    table = [tq.make_proj(x=xd[j], xq=xq[j], x_scale=xs[j], x_sum=xsum[j], K=x.shape[1])
+             for j, x in enumerate(xs_in)]
+    tq.tq_hadamard_quantize_act_stack(table, M, n)
+    torch.cuda.synchronize()
+    for j, x in enumerate(xs_in):
+        rq, rxs, rxsum = oracle.hadamard_quant4(x, n)
+        assert np.array_equal(xq[j].cpu().numpy(), rq), j
+        assert np.array_equal(xs[j].cpu().numpy().view(np.uint32), rxs.view(np.uint32)), j
+        assert np.array_equal(xsum[j].cpu().numpy(), rxsum), j
