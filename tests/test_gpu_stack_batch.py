@@ -1,9 +1,10 @@
 """GPU parity of the small-batch grouped decode calls (tq_quantize_act_stack_batch
 then tq_gemv_stack_batch, M = 2..32 tokens per projection: the streaming
-kernel up to 4 tokens, the tensor-core group plan from 5) against the oracle
-on every output: per-token codes, scales and sums, int32 accumulators
-bit-exact and fp32 outputs within the parity bar. Each projection's M rows
-are independent tokens (1bit engine blog, "One GPU, many users")."""
+kernel up to 2 tokens, the warp-MMA kernel for 3..16, the tensor-core group
+plan from 17) against the oracle on every output: per-token codes, scales and
+sums, int32 accumulators bit-exact and fp32 outputs within the parity bar.
+Each projection's M rows are independent tokens (1bit engine blog, "One GPU,
+many users")."""
 import numpy as np
 import pytest
 import torch
@@ -117,11 +118,12 @@ def test_batched_degenerate_rows(cuda_device):
     _check(st, refs)
 
 
-# ------------------------------------------ 5 <= M <= 32: the group plan
+# ------------------- 5 <= M <= 16: warp MMA; 17 <= M <= 32: the group plan
 @pytest.mark.parametrize("M", [5, 8, 16, 17, 24, 32])
-def test_ffn_projections_group_plan(cuda_device, M):
-    # gate/up and down in one tensor-core launch: tiles of 10 and 27 K units
-    # share one stream-K partition, so some tiles are split between CTAs.
+def test_ffn_projections_warp_mma_and_group_plan(cuda_device, M):
+    # gate/up and down in one launch; from 17 tokens the tensor-core group
+    # plan, whose tiles of 10 and 27 K units share one stream-K partition, so
+    # some tiles are split between CTAs.
     projs = list(make_projections(SMALL_M_SHAPES, M=M, seed=40 + M))
     st = BatchStack(projs, M)
     refs = parallel_map(_oracle, projs)
@@ -136,10 +138,9 @@ def test_ffn_projections_group_plan(cuda_device, M):
     assert tq.tq_device_error(reset=True) == 0
 
 
-def test_group_plan_many_launches_mixed_shapes(cuda_device):
-    # 40 projections (three launches of at most 16), assorted N and K including
-    # K of one unit and ragged tiles, at M = 8 and then M = 20 (the other
-    # column width) on the same scratch.
+def test_many_launches_mixed_shapes(cuda_device):
+    # 40 projections, assorted N and K including K of one unit and ragged
+    # tiles, at M = 8 (warp MMA) and then M = 20 (group plan).
     shapes = [(f"p{j}", 4 * (1 + (j * 53) % 700), 16 * (1 + (j * 29) % 300)) for j in range(40)]
     shapes[3] = ("k16", 512, 16)
     shapes[7] = ("n4", 4, 2560)
@@ -151,14 +152,17 @@ def test_group_plan_many_launches_mixed_shapes(cuda_device):
         _check(st, refs)
 
 
-def test_group_plan_degenerate_rows(cuda_device):
+@pytest.mark.parametrize("M", [12, 20])
+def test_degenerate_rows(cuda_device, M):
+    # a zero token, a token of alternating +-10, all-+1 and all-zero weight
+    # blocks; warp MMA (12 tokens) and group plan (20)
     projs = list(make_projections([("a", 640, 2560), ("b", 2560, 6912), ("c", 64, 512)],
-                                  M=12, seed=15))
+                                  M=M, seed=15 + M))
     projs[0].x_bf16[3] = 0
     projs[1].x_bf16[11] = np.where(np.arange(6912) % 2 == 0, 0x4120, 0xC120).astype(np.uint16)
     projs[2].w[:] = 1
     projs[0].w[: 320] = 0
-    st = BatchStack(projs, 12)
+    st = BatchStack(projs, M)
     refs = parallel_map(_oracle, projs)
     st.run()
     _check(st, refs)
@@ -166,21 +170,21 @@ def test_group_plan_degenerate_rows(cuda_device):
 
 def test_group_plan_after_a_reported_device_error(cuda_device):
     # A bounded wait that gives up sets the device error word; reading it
-    # makes the next group call zero-fill its scratch first.
+    # makes the next group call (20 tokens) zero-fill its scratch first.
     tq.tq_selftest_wait_timeout(200)
     assert tq.tq_device_error(reset=True) != 0
-    projs = list(make_projections(SMALL_M_SHAPES, M=9, seed=16))
-    st = BatchStack(projs, 9)
+    projs = list(make_projections(SMALL_M_SHAPES, M=20, seed=16))
+    st = BatchStack(projs, 20)
     refs = parallel_map(_oracle, projs)
     st.run()
     _check(st, refs)
     assert tq.tq_device_error(reset=True) == 0
 
 
-def test_full_stack_30_layers_m16_group_plan(cuda_device):
+def test_full_stack_30_layers_m16_warp_mma(cuda_device):
     # The launch configuration bench.py times for stack30_m16: all 210
-    # projections of the 30-layer stack at 16 tokens, 14 group launches of at
-    # most 16 projections; every output against the oracle.
+    # projections of the 30-layer stack at 16 tokens in one warp-MMA launch;
+    # every output against the oracle.
     projs = list(make_projections(stack_shapes(30), M=16, seed=17))
     st = BatchStack(projs, 16)
     refs = parallel_map(_oracle, projs)
@@ -189,13 +193,24 @@ def test_full_stack_30_layers_m16_group_plan(cuda_device):
     assert tq.tq_device_error(reset=True) == 0
 
 
-def test_full_stack_30_layers_m4_streaming(cuda_device):
-    # bench.py's stack30_m4: all 210 projections at 4 tokens in one streaming
+def test_full_stack_30_layers_m4_warp_mma(cuda_device):
+    # bench.py's stack30_m4: all 210 projections at 4 tokens in one warp-MMA
     # launch; every output against the oracle.
     projs = list(make_projections(stack_shapes(30), M=4, seed=18))
     st = BatchStack(projs, 4)
     refs = parallel_map(_oracle, projs)
     st.run()
+    _check(st, refs)
+    assert tq.tq_device_error(reset=True) == 0
+
+
+def test_full_stack_30_layers_m24_group_plan(cuda_device):
+    # all 210 projections at 24 tokens: four tensor-core group launches of up
+    # to 64 projections over one stream-K partition each; every output
+    projs = list(make_projections(stack_shapes(30), M=24, seed=19))
+    st = BatchStack(projs, 24)
+    refs = parallel_map(_oracle, projs)
+    st.run(tq.TQ_STACK_OVERLAP_PREV)
     _check(st, refs)
     assert tq.tq_device_error(reset=True) == 0
 
