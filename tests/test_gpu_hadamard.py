@@ -74,9 +74,10 @@ def test_prefill_m512_had4_every_output(cuda_device):
     assert tq.tq_device_error(reset=True) == 0
 
 
-@pytest.mark.parametrize("M", [1, 8, 40])
+@pytest.mark.parametrize("M", [1, 8, 24, 40, 300])
 def test_had4_codes_through_every_contraction_path(cuda_device, M):
-    # decode streaming (M <= 4), batched decode (5..32), prefill GEMM (>= 33)
+    # streaming (1 token), warp MMA (8), tensor-core batched decode (24),
+    # prefill GEMM on single CTAs (40) and on CTA pairs (300)
     for p in make_projections([("ffn", 2560, 6912)], M=M, seed=30 + M):
         xq, xs, xsum = gpu_had4(p.x_bf16, HADAMARD_BLOCK)
         Pd = dev(host_pack(p.w))
@@ -86,7 +87,8 @@ def test_had4_codes_through_every_contraction_path(cuda_device, M):
         torch.cuda.synchronize()
         got = (xq.cpu().numpy(), xs.cpu().numpy(), xsum.cpu().numpy(), acc.cpu().numpy(),
                y.cpu().numpy())
-        ref = oracle.forward_had4(oracle.pack(p.w), p.N, p.w_scale, p.x_bf16, HADAMARD_BLOCK)
+        ref = oracle.forward_had4(oracle.pack(p.w), p.N, p.w_scale, p.x_bf16, HADAMARD_BLOCK,
+                                  threads=THREADS)
         assert_parity(got, ref, f"had4 M={M}")
 
 
