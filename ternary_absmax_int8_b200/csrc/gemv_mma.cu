@@ -47,14 +47,14 @@ namespace tq {
 
 namespace {
 
-// Warps per CTA: 12 up to 16 tokens (256-column steps; up to 170 registers
-// a thread), 16 beyond.
+// Warps per CTA: 16 up to 8 tokens, 12 for 9..16 (up to 170 registers a
+// thread for two token groups), 16 beyond; three ring stages of 256-column
+// steps up to 16 tokens (what fits next to the warps' accumulator slots).
 template <int NT>
-constexpr int kMmaW = NT <= 2 ? 12 : 16;
-// cp.async stages per warp (3 where two token groups' accumulator slots
-// leave no room for a fourth)
+constexpr int kMmaW = NT == 1 ? 16 : (NT == 2 ? 12 : 16);
+// cp.async stages per warp
 template <int NT>
-constexpr int kRing = NT == 2 ? 3 : 4;
+constexpr int kRing = NT <= 2 ? 3 : 4;
 constexpr int kMmaRows = 16;      // packed rows per tile
 // A step is H pieces of 64 columns (H = 4 up to 16 tokens, 1 beyond, where
 // the accumulators and the prefetched activations take more registers and
