@@ -265,25 +265,20 @@ def recorded_traffic(workload: str):
     return float(d["bytes_per_packed_byte"]) * d["full_packed_bytes"]
 
 
-def pipelined_e2e(steps: int, stream, h2d, compute, d2h) -> float:
-    """Device time (ms) of `steps` end-to-end steps on two buffer sets: step
-    i's host-to-device copy (h2d(i, b) on an upload stream) overlaps step
-    i - 1's compute (compute(i, b, stream)), and its device-to-host copy
-    (d2h(i, b) on a download stream) overlaps step i + 1's compute; buffer b
-    = i % 2 is reused only after step i - 2's compute and download are done.
-    Every step's inputs are uploaded and its outputs read back inside the
-    timed region."""
+def pipelined_steps(steps: int, stream, up, down, h2d, compute, d2h):
+    """Enqueue `steps` end-to-end steps on two buffer sets: step i's
+    host-to-device copy (h2d(i, b) on stream `up`) overlaps step i - 1's
+    compute (compute(i, b, stream)), and its device-to-host copy (d2h(i, b)
+    on stream `down`) overlaps step i + 1's compute; buffer b = i % 2 is
+    reused only after step i - 2's compute and download are done. Every
+    step's inputs are uploaded and its outputs read back."""
     import torch
 
-    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     computed = [torch.cuda.Event(), torch.cuda.Event()]
     uploaded = [torch.cuda.Event(), torch.cuda.Event()]
     downloaded = [torch.cuda.Event(), torch.cuda.Event()]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    up.wait_event(e0)
-    down.wait_event(e0)
+    up.wait_stream(stream)
+    down.wait_stream(stream)
     for i in range(steps):
         b = i % 2
         with torch.cuda.stream(up):
@@ -302,8 +297,32 @@ def pipelined_e2e(steps: int, stream, h2d, compute, d2h) -> float:
             downloaded[b].record(down)
     stream.wait_stream(up)
     stream.wait_stream(down)
+
+
+def pipelined_e2e(steps: int, stream, h2d, compute, d2h, chunk: int = 16) -> float:
+    """Device time (ms) of `steps` (a multiple of `chunk`) end-to-end steps:
+    pipelined_steps over `chunk` steps captured once in a CUDA graph (the
+    copies from and to pinned host memory, the library calls and the
+    cross-stream events), replayed steps / chunk times."""
+    import torch
+
+    cs, up, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    cs.wait_stream(stream)
+    with torch.cuda.stream(cs):
+        pipelined_steps(2, cs, up, down, h2d, compute, d2h)  # eager warm-up
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        pipelined_steps(chunk, cs, up, down, h2d, compute, d2h)
+    stream.wait_stream(cs)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps // chunk):
+        g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    del g
     return e0.elapsed_time(e1)
 
 
@@ -477,19 +496,20 @@ def run_ours(args, rank: int, world: int):
         quant_ms_step = graph_ms(lambda cs: [quant(i % copies, cs) for i in range(S)]) / S
         gemv_ms_step = graph_ms(lambda cs: [gemv(i % copies, cs) for i in range(S)]) / S
 
-    # End to end through the library calls themselves (no graph): host
-    # activations in, host outputs out, every step, double-buffered so that
-    # step i + 1's upload and step i - 1's download overlap step i. At least
-    # half a second of it, so that the clock samples see the GPU under load.
-    e2e_steps = max(K, int(0.5e3 / max(total_ms / K, 1e-3)))
+    # End to end through the library calls themselves: host activations in,
+    # host outputs out, every step, double-buffered so that step i + 1's
+    # upload and step i - 1's download overlap step i, replayed from a CUDA
+    # graph of 16 such steps. At least half a second of it, so that the clock
+    # samples see the GPU under load.
+    chunk = 16
+    e2e_steps = -(-max(K, int(0.5e3 / max(total_ms / K, 1e-3))) // chunk) * chunk
     xb, yb, yh = (x_dev, x_dev_b), (y_dev, y_dev_b), (y_host, y_host_b)
     tb = (tables, tables_b)
     io = dict(h2d=lambda i, b: xb[b].copy_(x_host, non_blocking=True),
               compute=lambda i, b, s: step(i % copies, s, tabs=tb[b]),
               d2h=lambda i, b: yh[b].copy_(yb[b], non_blocking=True))
-    pipelined_e2e(3, stream, **io)  # warm-up
     barrier()
-    e2e_ms = pipelined_e2e(e2e_steps, stream, **io)
+    e2e_ms = pipelined_e2e(e2e_steps, stream, chunk=chunk, **io)
     barrier()
     # both buffer sets carry the same step (same inputs, copies of the same
     # weights): equal host outputs show that the pipeline kept its order
