@@ -79,8 +79,8 @@ struct Cursor {
     int entry;     // its projection
     int step, step_end;
     int K;
-    const uint8_t *row;  // this lane's row g at column 16 t (row g + 8 is 8 K further)
-    bool ok0, ok1;       // rows g, g + 8 exist
+    const uint8_t *row, *row8;  // this lane's rows g and g + 8 at column 16 t
+    bool ok0, ok1;              // rows g, g + 8 exist
 };
 
 template <int STEP>
@@ -103,6 +103,7 @@ struct Walk {
         c.ok0 = r < e.N4;
         c.ok1 = r + 8 < e.N4;
         c.row = e.packed + size_t(r) * e.K + t16;
+        c.row8 = c.row + size_t(8) * e.K;
     }
     // from c's current step on, the next pair with a step to compute
     __device__ void settle(Cursor &c, int g) const
@@ -162,7 +163,7 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
         pdl_launch_dependents();
 
     // the load cursor runs RING - 1 steps ahead of the compute cursor
-    Cursor lc{t_end, 0, 0, 0, 0, nullptr, false, false};
+    Cursor lc{t_end, 0, 0, 0, 0, nullptr, nullptr, false, false};
     if (first < t_end) {
         wk.start(lc, first, g);
         wk.settle(lc, g);
@@ -171,14 +172,21 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     auto issue = [&]() {
         const uint32_t dst = ring_s + uint32_t(issued) * SB;
         if (lc.tile < t_end) {
-            const int k = lc.step * STEP;  // + 16 t already in lc.row
-            const uint8_t *src = lc.row + k;
-            const size_t r8 = size_t(8) * lc.K;
+            const int k = lc.step * STEP;  // + 16 t already in the row pointers
+            const uint8_t *s0 = lc.row + k, *s1 = lc.row8 + k;
+            if (k + STEP <= lc.K) {  // a whole step (warp-uniform)
 #pragma unroll
-            for (int h = 0; h < H; ++h) {
-                const bool kin = k + 64 * h + 16 * t < lc.K;
-                cp_async16(dst + h * 512, src + 64 * h, lc.ok0 && kin);
-                cp_async16(dst + (H + h) * 512, src + r8 + 64 * h, lc.ok1 && kin);
+                for (int h = 0; h < H; ++h) {
+                    cp_async16(dst + h * 512, s0 + 64 * h, lc.ok0);
+                    cp_async16(dst + (H + h) * 512, s1 + 64 * h, lc.ok1);
+                }
+            } else {
+#pragma unroll
+                for (int h = 0; h < H; ++h) {
+                    const bool kin = k + 64 * h + 16 * t < lc.K;
+                    cp_async16(dst + h * 512, s0 + 64 * h, lc.ok0 && kin);
+                    cp_async16(dst + (H + h) * 512, s1 + 64 * h, lc.ok1 && kin);
+                }
             }
             ++lc.step;
             wk.settle(lc, g);
@@ -204,7 +212,7 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     };
     zero_acc();
     int consumed = 0;  // ring slot of the next step to compute
-    Cursor cc{t_end, 0, 0, 0, 0, nullptr, false, false};
+    Cursor cc{t_end, 0, 0, 0, 0, nullptr, nullptr, false, false};
     if (first < t_end) {
         wk.start(cc, first, g);
         wk.settle(cc, g);
@@ -215,22 +223,38 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
         ++fent;
     // The activations of a step (token n 8 + g, the lane's 16 columns of each
     // half), loaded one step ahead so their latency overlaps the MMAs of the
-    // step before.
+    // step before. A lane whose token n 8 + g is past M reads token M - 1
+    // instead: its MMA column only feeds outputs that are never stored.
+    // Columns past K read the row's first 16 columns instead (K >= 16): the
+    // weights there are zero-filled, so the products vanish.
     uint4 qn[H][NT];
+    const int8_t *xrow[NT];  // the lane's token rows at column 16 t, for entry xent
+    int xent = -1;
     auto load_q = [&](const Cursor &c) {
         if (c.tile >= t_end)
             return;
-        const MmaEntry &ce = p.e[c.entry];
-        const int k = c.step * STEP + 16 * t;
+        if (c.entry != xent) {
+            xent = c.entry;
+            const MmaEntry &ce = p.e[xent];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const bool ok = n * 8 + g < p.M;
-            const int8_t *xr = ce.xq + size_t(ok ? n * 8 + g : 0) * c.K + k;
+            for (int n = 0; n < NT; ++n)
+                xrow[n] = ce.xq + size_t(min(n * 8 + g, p.M - 1)) * ce.K + 16 * t;
+        }
+        const int k = c.step * STEP;
+        if (k + STEP <= c.K) {
 #pragma unroll
-            for (int h = 0; h < H; ++h)
-                qn[h][n] = (ok && k + 64 * h < c.K)
-                               ? __ldg(reinterpret_cast<const uint4 *>(xr + 64 * h))
-                               : make_uint4(0, 0, 0, 0);
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int h = 0; h < H; ++h)
+                    qn[h][n] = __ldg(reinterpret_cast<const uint4 *>(xrow[n] + k + 64 * h));
+        } else {
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int h = 0; h < H; ++h) {
+                    const int kk = k + 64 * h + 16 * t < c.K ? k + 64 * h : -16 * t;
+                    qn[h][n] = __ldg(reinterpret_cast<const uint4 *>(xrow[n] + kk));
+                }
         }
     };
     load_q(cc);
@@ -281,15 +305,33 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
         }
         const int r0 = (tile - e.tile_begin) * kMmaRows;
         if (P == 1) {
-            // the warp holds the whole tile: epilogue from registers
+            // the warp holds the whole tile: epilogue from registers, the
+            // token's scale and sum loaded once for its eight outputs
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
-                    const int row = r0 + g + (hh >> 1) * 8, m = n * 8 + 2 * t + (hh & 1);
+                for (int par = 0; par < 2; ++par) {
+                    const int m = n * 8 + 2 * t + par;
+                    if (m >= p.M)
+                        continue;
+                    const int32_t xs = __ldg(e.x_sum + m);
+                    const float sc = __fmul_rn(e.w_scale, __ldg(e.x_scale + m));
+                    const size_t ob = size_t(m) * (4 * size_t(e.N4));
 #pragma unroll
-                    for (int pl = 0; pl < 4; ++pl)
-                        store_out(e, p.M, row, m, pl, d[pl][n][hh], pl > 0 ? d[pl - 1][n][hh] : 0);
+                    for (int half = 0; half < 2; ++half) {
+                        const int row = r0 + g + 8 * half, hh = 2 * half + par;
+                        if (row >= e.N4)
+                            continue;
+#pragma unroll
+                        for (int pl = 0; pl < 4; ++pl) {
+                            const int32_t lo = pl > 0 ? d[pl - 1][n][hh] : 0;
+                            const int32_t acc = ((d[pl][n][hh] - lo) >> (2 * pl)) - xs;
+                            const size_t out = ob + size_t(row) + size_t(pl) * e.N4;
+                            e.y[out] = __fmul_rn(__int2float_rn(acc), sc);
+                            if (e.acc_out)
+                                e.acc_out[out] = acc;
+                        }
+                    }
                 }
             zero_acc();
             continue;
