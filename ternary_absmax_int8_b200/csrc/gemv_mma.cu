@@ -86,7 +86,7 @@ struct Cursor {
 template <int STEP>
 struct Walk {
     const MmaEntry *tab;
-    int n_ent, t_end, teams, piece, lgP;
+    int n_ent, t_end, teams, piece, P;
     int t16;  // 16 t: the lane's column offset
 
     __device__ void start(Cursor &c, int tl, int g) const
@@ -97,8 +97,8 @@ struct Walk {
         const MmaEntry &e = tab[c.entry];
         c.K = e.K;
         const int S = (e.K + STEP - 1) / STEP;
-        c.step = (S * piece) >> lgP;
-        c.step_end = (S * (piece + 1)) >> lgP;
+        c.step = S * piece / P;
+        c.step_end = S * (piece + 1) / P;
         const int r = (tl - e.tile_begin) * kMmaRows + g;
         c.ok0 = r < e.N4;
         c.ok1 = r + 8 < e.N4;
@@ -152,12 +152,12 @@ mma_gemv_kernel(const __grid_constant__ MmaParams p)
     const uint32_t ring_s = smem_u32(ring);
 
     const int t_begin = p.cta_tile0[blockIdx.x], t_end = p.cta_tile0[blockIdx.x + 1];
-    const int lgP = p.lgP, P = 1 << lgP, teams = W >> lgP;
+    const int P = p.P, teams = W / P;
     // teams of P warps; warps past the last whole team (W not a multiple of
     // P) stay idle
-    const int team = warp >> lgP, piece = warp & (P - 1);
+    const int team = warp / P, piece = warp - team * P;
     const int first = team < teams ? t_begin + team : t_end;
-    const Walk<STEP> wk{p.e, p.n_entries, t_end, teams, piece, lgP, 16 * t};
+    const Walk<STEP> wk{p.e, p.n_entries, t_end, teams, piece, P, 16 * t};
 
     if (threadIdx.x == 0)
         pdl_launch_dependents();
@@ -440,15 +440,9 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
         if (total == 0)
             continue;
         // contiguous tile ranges per CTA, balanced by bytes (plus a fixed
-        // cost per tile), one CTA per SM; the warps of a CTA split tiles in
-        // teams of P: P = 1 (whole tiles per warp, no barrier) when there
-        // are enough tiles to give every warp two, more when there are fewer
+        // cost per tile), one CTA per SM
         const int grid = std::min({total, sms, kMmaMaxGrid});
         const int W = M <= 8 ? kMmaW<1> : (M <= 16 ? kMmaW<2> : kMmaW<4>);
-        int lgP = 0;
-        while ((2 << lgP) <= W && (long long)total << lgP < 2LL * W * grid)
-            ++lgP;
-        p.lgP = lgP;
         std::vector<long long> prefix(size_t(total) + 1, 0);
         {
             int tt = 0;
@@ -460,14 +454,28 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
             }
         }
         p.cta_tile0[0] = 0;
-        for (int b = 1; b < grid; ++b) {
-            const long long target = prefix[size_t(total)] * b / grid;
-            int tt = int(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
-            tt = std::max(tt, p.cta_tile0[b - 1] + 1);
-            tt = std::min(tt, total - (grid - b));
+        int max_tiles = 0;
+        for (int b = 1; b <= grid; ++b) {
+            int tt = total;
+            if (b < grid) {
+                const long long target = prefix[size_t(total)] * b / grid;
+                tt = int(std::lower_bound(prefix.begin(), prefix.end(), target) - prefix.begin());
+                tt = std::max(tt, p.cta_tile0[b - 1] + 1);
+                tt = std::min(tt, total - (grid - b));
+            }
             p.cta_tile0[b] = tt;
+            max_tiles = std::max(max_tiles, tt - p.cta_tile0[b - 1]);
         }
-        p.cta_tile0[grid] = total;
+        // The warps of a CTA form teams of P that take the range's tiles in
+        // turn, splitting each tile's steps. Teams: up to 8 tokens, one per
+        // two tiles of the longest range (a team's next tile loads while it
+        // finishes the current one); beyond, one per tile, whose steps carry
+        // twice the MMAs. With many tiles P = 1 (whole tiles per warp). B200,
+        // the FFN projections at 4, 8 and 16 tokens: 2 teams of 8 warps
+        // 6.7 / 7.3 us against 8.2 / 8.5 us for one team of 16, 3 teams of
+        // 4 warps 9.6 us against 13.0 for one of 8 (12 warps).
+        const int teams = std::min(W, M <= 8 ? (max_tiles + 1) / 2 : max_tiles);
+        p.P = W / std::max(teams, 1);
         const bool pdl = first ? overlap_prev : true;
         cudaError_t e;
         if (M <= 8)

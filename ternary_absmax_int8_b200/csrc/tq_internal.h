@@ -170,7 +170,7 @@ constexpr int kMmaMaxGrid = 320;   // CTAs per launch
 
 struct MmaParams {
     int n_entries, M;
-    int lgP;  // log2 of the warps per team (each tile's K is split over a team)
+    int P;  // warps per team (each tile's K is split over a team)
     int cta_tile0[kMmaMaxGrid + 1];
     MmaEntry e[kMmaStackMax];
 };
