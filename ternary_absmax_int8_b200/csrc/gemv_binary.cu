@@ -598,10 +598,12 @@ constexpr int kBmRows = 16;
 struct BmCursor {
     int tile, entry, step, step_end;
     int K, G;
-    const uint8_t *row;  // the lane's row g at column 16 t
-    const uint16_t *sc;  // scales of the lane's row g (t = 0) or g + 8 (t = 1): [group][8]
-    const int8_t *xq;    // the token's codes at column 16 g (lanes t = 2)
-    bool ok0, ok1;
+    const uint8_t *row, *row8;  // the lane's rows g and g + 8 at column 16 t
+    // lanes t = 0, 1: the scales of row g + 8 t ([group][8] fp16); t = 2: the
+    // token's codes at column 16 g; advanced by `aux_step` bytes per group
+    const uint8_t *aux;
+    int aux_step;
+    bool ok0, ok1, aux_ok;
 };
 
 struct BmWalk {
@@ -622,9 +624,18 @@ struct BmWalk {
         c.ok0 = r < e.N8;
         c.ok1 = r + 8 < e.N8;
         c.row = e.bits + size_t(c.ok0 ? r : 0) * e.K + 16 * t;
+        // row g + 8 past the end: zero-size copies from row g's address
+        c.row8 = c.ok1 ? c.row + size_t(8) * e.K : c.row;
         const int rs = t == 1 && c.ok1 ? r + 8 : (c.ok0 ? r : 0);
-        c.sc = e.scales + size_t(rs) * c.G * 8;
-        c.xq = e.xq + 16 * g;
+        if (t < 2) {
+            c.aux = reinterpret_cast<const uint8_t *>(e.scales + size_t(rs) * c.G * 8);
+            c.aux_step = 16;
+            c.aux_ok = t == 0 ? c.ok0 : c.ok1;
+        } else {
+            c.aux = reinterpret_cast<const uint8_t *>(e.xq) + 16 * g;
+            c.aux_step = kBinGroup;
+            c.aux_ok = true;
+        }
     }
     __device__ void settle(BmCursor &c) const
     {
@@ -658,7 +669,7 @@ binary_mma_kernel(const __grid_constant__ BinMmaParams p)
     const int first = team < teams ? t_begin + team : t_end;
     const BmWalk wk{p.e, p.n_entries, t_end, teams, piece, lgP, g, t};
 
-    BmCursor lc{t_end, 0, 0, 0, 0, 0, nullptr, nullptr, nullptr, false, false};
+    BmCursor lc{t_end, 0, 0, 0, 0, 0, nullptr, nullptr, nullptr, 0, false, false, false};
     if (first < t_end) {
         wk.start(lc, first);
         wk.settle(lc);
@@ -671,19 +682,16 @@ binary_mma_kernel(const __grid_constant__ BinMmaParams p)
         const uint32_t dst = ring_s + uint32_t(issued & (kBmRing - 1)) * kBmStage;
         __syncwarp();  // the slot's scales were last read by other lanes
         if (lc.tile < t_end) {
-            const uint8_t *src = lc.row + size_t(lc.step) * kBinGroup;
-            // row g + 8 past the end: a zero-size copy from row g's address
-            const uint8_t *src8 = lc.ok1 ? src + size_t(8) * lc.K : src;
-            cp_async16(dst, src, lc.ok0);
-            cp_async16(dst + 512, src + 64, lc.ok0);
-            cp_async16(dst + 1024, src8, lc.ok1);
-            cp_async16(dst + 1536, src8 + 64, lc.ok1);
-            if (t < 2)  // lanes t = 0, 1: the 8 scales of row g + 8 t at this group
+            const int k = lc.step * kBinGroup;
+            cp_async16(dst, lc.row + k, lc.ok0);
+            cp_async16(dst + 512, lc.row + k + 64, lc.ok0);
+            cp_async16(dst + 1024, lc.row8 + k, lc.ok1);
+            cp_async16(dst + 1536, lc.row8 + k + 64, lc.ok1);
+            // lanes t = 0, 1: the 8 scales of row g + 8 t at this group;
+            // lanes t = 2: codes 16 g .. 16 g + 15 of the group
+            if (t < 3)
                 cp_async16(sc_s + uint32_t(issued & (kBmRing - 1)) * kBmStage,
-                           lc.sc + size_t(lc.step) * 8, t == 0 ? lc.ok0 : lc.ok1);
-            else if (t == 2)  // lanes t = 2: codes 16 g .. 16 g + 15 of the group
-                cp_async16(sc_s + uint32_t(issued & (kBmRing - 1)) * kBmStage,
-                           lc.xq + size_t(lc.step) * kBinGroup, true);
+                           lc.aux + lc.step * lc.aux_step, lc.aux_ok);
             ++lc.step;
             wk.settle(lc);
         }
@@ -773,8 +781,10 @@ binary_mma_kernel(const __grid_constant__ BinMmaParams p)
             const int32_t a_lo = 2 * ((t_lo - t_pr) >> (2 * t)) - Q;
             const int32_t a_hi = 2 * ((t_hi - t_lo) >> (2 * t + 1)) - Q;
             const float2 sc = rs == 0 ? s0 : s1;
-            acc[rs][0] = __dadd_rn(acc[rs][0], __dmul_rn(double(a_lo), double(sc.x)));
-            acc[rs][1] = __dadd_rn(acc[rs][1], __dmul_rn(double(a_hi), double(sc.y)));
+            // the products are exact in fp64 (15-bit integer x 11-bit
+            // significand), so one fused multiply-add rounds as the add alone
+            acc[rs][0] = __fma_rn(double(a_lo), double(sc.x), acc[rs][0]);
+            acc[rs][1] = __fma_rn(double(a_hi), double(sc.y), acc[rs][1]);
             tot[rs][0] += a_lo;
             tot[rs][1] += a_hi;
         }
