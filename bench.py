@@ -9,7 +9,8 @@ persistent launch (tq_gemv_stack with TQ_STACK_QUANTIZE). The weight stream is
 larger than L2, so no flush is needed between steps. Other workloads of several
 projections group them the same way: one quantising stack launch at M = 1, the
 stack quantiser plus tq_gemv_stack_batch at M = 2..32 (the streaming kernel up
-to 4 tokens, the tensor-core group plan from 5); single projections and
+to 2 tokens, the warp-MMA kernel for 3..24, the tensor-core group plan from
+25); single projections and
 prefill run one quantiser launch and one GEMV launch per projection.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -646,7 +647,7 @@ def batch_kernel_name(M: int, mode: str) -> str:
         return "stream_gemv_kernel"
     if forced == "stream" and M <= 4 or forced == "" and M <= 2:
         return "stream_gemv_kernel"
-    if forced == "mma" or forced == "" and M <= 16:
+    if forced == "mma" or forced == "" and M <= 24:
         return "mma_gemv_kernel"
     return "smallm_group_kernel" if mode == "batch" else "smallm_tc_kernel"
 

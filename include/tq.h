@@ -104,10 +104,11 @@ tq_status tq_quantize_act(const uint16_t *x, int8_t *xq, float *x_scale, int32_t
  * TQ_ERR_UNSUPPORTED for M > 24 (use tq_gemm_prefill) or K > 32768.
  * Kernels (chosen by M from B200 measurements; many concurrent users make
  * decode a small batch: 1bit engine blog, "One GPU, many users"): M <= 2 the
- * streaming dp4a kernel; 3 <= M <= 16 the warp-MMA kernel (mma.sync int8 on
- * the masked packed bytes); 17 <= M the tensor-core (tcgen05) batched-decode
- * kernel. The environment variable TQ_BATCH_KERNEL=stream|mma|tc forces one
- * where it applies (for measurement).
+ * streaming dp4a kernel; 3 <= M <= 24 the warp-MMA kernel (mma.sync int8 on
+ * the masked packed bytes). The tensor-core (tcgen05) batched-decode kernel
+ * runs the grouped calls from 25 tokens and tq_gemv_noalloc. The environment
+ * variable TQ_BATCH_KERNEL=stream|mma|tc forces one where it applies (for
+ * measurement).
  */
 tq_status tq_gemv(const uint8_t *packed, float w_scale, const int8_t *xq,
                   const float *x_scale, const int32_t *x_sum, float *y, int32_t *acc_out,
@@ -210,9 +211,9 @@ tq_status tq_gemv_stack(const tq_proj *projs, int n_proj, unsigned flags, cudaSt
  * tq_gemv_stack. The quantising flags need M == 1 (TQ_ERR_UNSUPPORTED
  * otherwise); TQ_STACK_OVERLAP_PREV is accepted at every M.
  *   M <= 2: the streaming kernel, one launch per 256 projections.
- *   3 <= M <= 16: the warp-MMA kernel, one launch per 256 projections (16-row
+ *   3 <= M <= 24: the warp-MMA kernel, one launch per 256 projections (16-row
  *   tiles of all projections balanced over the SMs); no scratch memory.
- *   17 <= M <= 32: the tensor-core batched-decode kernel, one launch per 64
+ *   25 <= M <= 32: the tensor-core batched-decode kernel, one launch per 64
  *   projections, its K work split evenly over the SMs across projection
  *   boundaries. Tiles split between CTAs finish through a fixed device array
  *   compiled into the library (one slot per CTA), which every launch leaves

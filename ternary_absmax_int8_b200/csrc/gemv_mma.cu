@@ -47,24 +47,25 @@ namespace tq {
 
 namespace {
 
-// Warps per CTA: 16 up to 8 tokens, 12 for 9..16 (up to 170 registers a
-// thread for two token groups), 16 beyond; three ring stages of 256-column
-// steps up to 16 tokens (what fits next to the warps' accumulator slots).
+// Warps per CTA: 16 up to 8 tokens, 12 for 9..24 (up to 170 registers a
+// thread for two or three token groups), 16 beyond; three ring stages of
+// 256-column steps up to 16 tokens (what fits next to the warps' accumulator
+// slots), four beyond.
 template <int NT>
-constexpr int kMmaW = NT == 1 ? 16 : (NT == 2 ? 12 : 16);
+constexpr int kMmaW = NT == 1 ? 16 : (NT <= 3 ? 12 : 16);
 // cp.async stages per warp
 template <int NT>
 constexpr int kRing = NT <= 2 ? 3 : 4;
 constexpr int kMmaRows = 16;      // packed rows per tile
-// A step is H pieces of 64 columns (H = 4 up to 16 tokens, 1 beyond, where
-// the accumulators and the prefetched activations take more registers and
-// the accumulator slots more shared memory); a stage holds
+// A step is H pieces of 64 columns (H = 4 up to 16 tokens, 2 for 17..24, 1
+// beyond, where the accumulators and the prefetched activations take more
+// registers and the accumulator slots more shared memory); a stage holds
 // [2 rows][H pieces][32 lanes][16 bytes]. Wide steps keep the number of
 // separate row streams per SM low: 16-row tiles read as 256-byte row pieces
 // by 12 warps move ~6.1 TB/s in a copy-only test, 128-byte pieces by 16 or
 // 20 warps 5.1 or 4.2 TB/s (DRAM page locality).
 template <int NT>
-constexpr int kHalves = NT <= 2 ? 4 : 1;
+constexpr int kHalves = NT <= 2 ? 4 : (NT == 3 ? 2 : 1);
 template <int NT>
 constexpr int kStep = 64 * kHalves<NT>;
 template <int NT>
@@ -442,7 +443,7 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
         // contiguous tile ranges per CTA, balanced by bytes (plus a fixed
         // cost per tile), one CTA per SM
         const int grid = std::min({total, sms, kMmaMaxGrid});
-        const int W = M <= 8 ? kMmaW<1> : (M <= 16 ? kMmaW<2> : kMmaW<4>);
+        const int W = M <= 8 ? kMmaW<1> : (M <= 16 ? kMmaW<2> : (M <= 24 ? kMmaW<3> : kMmaW<4>));
         std::vector<long long> prefix(size_t(total) + 1, 0);
         {
             int tt = 0;
@@ -482,6 +483,8 @@ cudaError_t launch_mma_gemv(const MmaEntry *entries, int n, int M, bool overlap_
             e = launch_nt<1>(p, grid, stream, pdl);
         else if (M <= 16)
             e = launch_nt<2>(p, grid, stream, pdl);
+        else if (M <= 24)
+            e = launch_nt<3>(p, grid, stream, pdl);
         else
             e = launch_nt<4>(p, grid, stream, pdl);
         if (e != cudaSuccess)

@@ -131,8 +131,9 @@ tq_status zero_outputs(float *y, int32_t *acc_out, size_t count, cudaStream_t s)
 // Which kernel runs a group of M-token projections: the streaming dp4a kernel
 // (M <= 4 per launch), the warp-MMA kernel (2 <= M <= 32) or the tensor-core
 // group plan (5 <= M <= 32). The choice by M follows B200 measurements of the
-// 30-layer stack and the FFN projections; TQ_BATCH_KERNEL=stream|mma|tc
-// forces one where it applies (for measurement).
+// 30-layer stack and the FFN projections (streaming up to 2 tokens, warp MMA
+// for 3..24, the group plan for 25..32); TQ_BATCH_KERNEL=stream|mma|tc forces
+// one where it applies (for measurement).
 enum class BatchKernel { kStream, kWarpMma, kTensor };
 
 BatchKernel batch_kernel(int M)
@@ -159,7 +160,7 @@ BatchKernel batch_kernel(int M)
         return BatchKernel::kTensor;
     if (M <= 2)
         return BatchKernel::kStream;
-    return M <= 16 ? BatchKernel::kWarpMma : BatchKernel::kTensor;
+    return M <= 24 ? BatchKernel::kWarpMma : BatchKernel::kTensor;
 }
 
 // Tokens in groups of up to four, one streaming launch per group.

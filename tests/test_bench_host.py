@@ -31,12 +31,13 @@ def test_step_mode(name, mode):
 
 def test_batch_launch_counts():
     # 512 projections per quantiser launch; 256 projections per streaming
-    # (M <= 2) or warp-MMA (3..16) launch, 64 per tensor-core group launch
+    # (M <= 2) or warp-MMA (3..24) launch, 64 per tensor-core group launch
     assert bench.batch_launches(3, 4) == 1 + 1
     assert bench.batch_launches(3, 16) == 1 + 1
     assert bench.batch_launches(210, 4) == 1 + 1
     assert bench.batch_launches(210, 16) == 1 + 1
-    assert bench.batch_launches(210, 24) == 1 + 4
+    assert bench.batch_launches(210, 24) == 1 + 1
+    assert bench.batch_launches(210, 32) == 1 + 4
     assert bench.batch_launches(300, 2) == 1 + 2
     assert bench.batch_launches(600, 2) == 2 + 3
 
@@ -58,10 +59,11 @@ def test_binary_kernel_name(monkeypatch):
 
 def test_kernel_names_follow_the_choice_by_m(monkeypatch):
     monkeypatch.delenv("TQ_BATCH_KERNEL", raising=False)
-    assert [bench.batch_kernel_name(m, "batch") for m in (1, 2, 3, 16, 17, 32)] == [
+    assert [bench.batch_kernel_name(m, "batch") for m in (1, 2, 3, 16, 17, 24, 25, 32)] == [
         "stream_gemv_kernel", "stream_gemv_kernel", "mma_gemv_kernel", "mma_gemv_kernel",
-        "smallm_group_kernel", "smallm_group_kernel"]
-    assert bench.batch_kernel_name(24, "per_projection") == "smallm_tc_kernel"
+        "mma_gemv_kernel", "mma_gemv_kernel", "smallm_group_kernel", "smallm_group_kernel"]
+    assert bench.batch_kernel_name(24, "per_projection") == "mma_gemv_kernel"
+    assert bench.batch_kernel_name(28, "per_projection") == "smallm_tc_kernel"
     monkeypatch.setenv("TQ_BATCH_KERNEL", "tc")
     assert bench.batch_kernel_name(8, "batch") == "smallm_group_kernel"
 

@@ -4,7 +4,8 @@ Covers the single 640x2560 projection, one full decoder layer's seven
 projections, the batched-decode FFN shapes at every M of that workload, and
 edge cases: tiny and ragged shapes (packed row counts that leave partial
 tiles), the K limit, all-zero / all-one weights, zero activation rows,
-repeat-run byte identity.
+repeat-run byte identity. From 25 tokens the single-projection path is the
+tensor-core kernel's cluster plan (through tq_gemm_prefill).
 """
 import numpy as np
 import pytest
@@ -43,7 +44,8 @@ def test_batched_decode(cuda_device, M):
 
 @pytest.mark.parametrize("N,K,M", [(4, 16, 1), (8, 32, 2), (12, 48, 3), (60, 112, 4),
                                    (6916, 2560, 1), (2564, 6928, 5), (100, 32768, 1),
-                                   (36, 32768, 4), (1024, 16, 24), (400, 4096, 13)])
+                                   (36, 32768, 4), (1024, 16, 24), (400, 4096, 13),
+                                   (520, 2560, 20), (2564, 6928, 28), (1024, 16, 32)])
 def test_edge_shapes(cuda_device, N, K, M):
     rng = np.random.default_rng(N * 7 + K * 3 + M)
     w = ternary_weights(rng, N, K)

@@ -1,7 +1,7 @@
 """GPU parity of the small-batch grouped decode calls (tq_quantize_act_stack_batch
 then tq_gemv_stack_batch, M = 2..32 tokens per projection: the streaming
-kernel up to 2 tokens, the warp-MMA kernel for 3..16, the tensor-core group
-plan from 17) against the oracle on every output: per-token codes, scales and
+kernel up to 2 tokens, the warp-MMA kernel for 3..24, the tensor-core group
+plan from 25) against the oracle on every output: per-token codes, scales and
 sums, int32 accumulators bit-exact and fp32 outputs within the parity bar.
 Each projection's M rows are independent tokens (1bit engine blog, "One GPU,
 many users")."""
@@ -118,12 +118,13 @@ def test_batched_degenerate_rows(cuda_device):
     _check(st, refs)
 
 
-# ------------------- 5 <= M <= 16: warp MMA; 17 <= M <= 32: the group plan
-@pytest.mark.parametrize("M", [5, 8, 16, 17, 24, 32])
+# ------------------- 5 <= M <= 24: warp MMA; 25 <= M <= 32: the group plan
+@pytest.mark.parametrize("M", [5, 8, 16, 17, 24, 25, 32])
 def test_ffn_projections_warp_mma_and_group_plan(cuda_device, M):
-    # gate/up and down in one launch; from 17 tokens the tensor-core group
-    # plan, whose tiles of 10 and 27 K units share one stream-K partition, so
-    # some tiles are split between CTAs.
+    # gate/up and down in one launch; up to 24 tokens the warp-MMA kernel
+    # (one, two or three token groups), from 25 the tensor-core group plan,
+    # whose tiles of 10 and 27 K units share one stream-K partition, so some
+    # tiles are split between CTAs.
     projs = list(make_projections(SMALL_M_SHAPES, M=M, seed=40 + M))
     st = BatchStack(projs, M)
     refs = parallel_map(_oracle, projs)
@@ -140,11 +141,11 @@ def test_ffn_projections_warp_mma_and_group_plan(cuda_device, M):
 
 def test_many_launches_mixed_shapes(cuda_device):
     # 40 projections, assorted N and K including K of one unit and ragged
-    # tiles, at M = 8 (warp MMA) and then M = 20 (group plan).
+    # tiles, at M = 8 and M = 20 (warp MMA) and then M = 28 (group plan).
     shapes = [(f"p{j}", 4 * (1 + (j * 53) % 700), 16 * (1 + (j * 29) % 300)) for j in range(40)]
     shapes[3] = ("k16", 512, 16)
     shapes[7] = ("n4", 4, 2560)
-    for M, seed in ((8, 13), (20, 14)):
+    for M, seed in ((8, 13), (20, 14), (28, 12)):
         projs = list(make_projections(shapes, M=M, seed=seed))
         st = BatchStack(projs, M)
         refs = parallel_map(_oracle, projs)
@@ -152,10 +153,10 @@ def test_many_launches_mixed_shapes(cuda_device):
         _check(st, refs)
 
 
-@pytest.mark.parametrize("M", [12, 20])
+@pytest.mark.parametrize("M", [12, 20, 28])
 def test_degenerate_rows(cuda_device, M):
     # a zero token, a token of alternating +-10, all-+1 and all-zero weight
-    # blocks; warp MMA (12 tokens) and group plan (20)
+    # blocks; warp MMA (12 and 20 tokens) and group plan (28)
     projs = list(make_projections([("a", 640, 2560), ("b", 2560, 6912), ("c", 64, 512)],
                                   M=M, seed=15 + M))
     projs[0].x_bf16[3] = 0
@@ -170,11 +171,11 @@ def test_degenerate_rows(cuda_device, M):
 
 def test_group_plan_after_a_reported_device_error(cuda_device):
     # A bounded wait that gives up sets the device error word; reading it
-    # makes the next group call (20 tokens) zero-fill its scratch first.
+    # makes the next group call (28 tokens) zero-fill its scratch first.
     tq.tq_selftest_wait_timeout(200)
     assert tq.tq_device_error(reset=True) != 0
-    projs = list(make_projections(SMALL_M_SHAPES, M=20, seed=16))
-    st = BatchStack(projs, 20)
+    projs = list(make_projections(SMALL_M_SHAPES, M=28, seed=16))
+    st = BatchStack(projs, 28)
     refs = parallel_map(_oracle, projs)
     st.run()
     _check(st, refs)
@@ -204,11 +205,22 @@ def test_full_stack_30_layers_m4_warp_mma(cuda_device):
     assert tq.tq_device_error(reset=True) == 0
 
 
-def test_full_stack_30_layers_m24_group_plan(cuda_device):
-    # all 210 projections at 24 tokens: four tensor-core group launches of up
-    # to 64 projections over one stream-K partition each; every output
+def test_full_stack_30_layers_m24_warp_mma(cuda_device):
+    # bench.py's stack30_m24: all 210 projections at 24 tokens in one
+    # warp-MMA launch (three token groups); every output against the oracle.
     projs = list(make_projections(stack_shapes(30), M=24, seed=19))
     st = BatchStack(projs, 24)
+    refs = parallel_map(_oracle, projs)
+    st.run(tq.TQ_STACK_OVERLAP_PREV)
+    _check(st, refs)
+    assert tq.tq_device_error(reset=True) == 0
+
+
+def test_stack_10_layers_m32_group_plan(cuda_device):
+    # 70 projections at 32 tokens: two tensor-core group launches (64 + 6
+    # projections), each over one stream-K partition; every output.
+    projs = list(make_projections(stack_shapes(10), M=32, seed=20))
+    st = BatchStack(projs, 32)
     refs = parallel_map(_oracle, projs)
     st.run(tq.TQ_STACK_OVERLAP_PREV)
     _check(st, refs)
