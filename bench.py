@@ -300,7 +300,7 @@ def pipelined_steps(steps: int, stream, up, down, h2d, compute, d2h):
     stream.wait_stream(down)
 
 
-def pipelined_e2e(steps: int, stream, h2d, compute, d2h, chunk: int = 16) -> float:
+def pipelined_e2e(steps: int, stream, h2d, compute, d2h, chunk: int = 64) -> float:
     """Device time (ms) of `steps` (a multiple of `chunk`) end-to-end steps:
     pipelined_steps over `chunk` steps captured once in a CUDA graph (the
     copies from and to pinned host memory, the library calls and the
@@ -500,9 +500,10 @@ def run_ours(args, rank: int, world: int):
     # End to end through the library calls themselves: host activations in,
     # host outputs out, every step, double-buffered so that step i + 1's
     # upload and step i - 1's download overlap step i, replayed from a CUDA
-    # graph of 16 such steps. At least half a second of it, so that the clock
-    # samples see the GPU under load.
-    chunk = 16
+    # graph of 64 such steps (replays run one after another, so each costs
+    # one upload and one download that overlap no compute). At least half a
+    # second of it, so that the clock samples see the GPU under load.
+    chunk = 64
     e2e_steps = -(-max(K, int(0.5e3 / max(total_ms / K, 1e-3))) // chunk) * chunk
     xb, yb, yh = (x_dev, x_dev_b), (y_dev, y_dev_b), (y_host, y_host_b)
     tb = (tables, tables_b)
@@ -906,7 +907,7 @@ def run_next(args, rank: int, world: int):
     gemv_ms = graph_ms(lambda cs: [gemv(i % copies, cs) for i in range(S)]) / S
     # end to end: uploads, library calls and downloads, double-buffered and
     # replayed from a CUDA graph of 16 steps (pipelined_e2e)
-    chunk = 16
+    chunk = 64
     e2e_steps = -(-max(K_, int(0.5e3 / max(total_ms / K_, 1e-3))) // chunk) * chunk
     e2e_ms = pipelined_e2e(
         e2e_steps, stream, chunk=chunk,

@@ -182,6 +182,19 @@ def test_group_plan_after_a_reported_device_error(cuda_device):
     assert tq.tq_device_error(reset=True) == 0
 
 
+@pytest.mark.parametrize("layers,M", [(1, 12), (2, 4), (3, 8), (4, 4), (2, 12), (2, 20)])
+def test_layer_stacks_team_sizes(cuda_device, layers, M):
+    # 1 to 4 decoder layers (356 to 1424 tiles, up to 3 to 12 per CTA) give
+    # the warp-MMA kernel teams of 4 (of 12 warps), 5 and 3 (of 16: one warp
+    # idle), 2 and 2 (three token groups); every output against the oracle.
+    projs = list(make_projections(stack_shapes(layers), M=M, seed=60 + 7 * layers + M))
+    st = BatchStack(projs, M)
+    refs = parallel_map(_oracle, projs)
+    st.run()
+    _check(st, refs)
+    assert tq.tq_device_error(reset=True) == 0
+
+
 def test_full_stack_30_layers_m16_warp_mma(cuda_device):
     # The launch configuration bench.py times for stack30_m16: all 210
     # projections of the 30-layer stack at 16 tokens in one warp-MMA launch;
