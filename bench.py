@@ -89,13 +89,13 @@ def step_bytes(projs) -> int:
 
 def step_mode(projs) -> str:
     """How a step launches: "fused" -- one quantising stack launch for every
-    projection (M = 1); "batch" -- the stack quantiser, then
-    tq_gemv_stack_batch (M = 2..32); "prefill" -- the stack quantiser, then
-    tq_gemm_prefill_stack (M >= 33, several projections); "per_projection" --
-    a quantiser launch and a GEMV launch per projection (a single
-    projection)."""
+    projection (M = 1, also a single projection); "batch" -- the stack
+    quantiser, then tq_gemv_stack_batch (M = 2..32); "prefill" -- the stack
+    quantiser, then tq_gemm_prefill_stack (M >= 33, several projections);
+    "per_projection" -- a quantiser launch and a GEMV launch per projection
+    (a single projection of several tokens)."""
     M = projs[0].M
-    if len(projs) > 1 and M == 1:
+    if M == 1:
         return "fused"
     if len(projs) > 1 and M <= 32:
         return "batch"
@@ -521,7 +521,7 @@ def run_ours(args, rank: int, world: int):
     # batches for comparison with their grouped launch): a graph of R calls of
     # one projection over the rotated weight copies, time per call.
     per_proj = []
-    if not stack and len(projs) <= 8:
+    if (not stack or len(projs) == 1) and len(projs) <= 8:
         R = copies * max(1, 32 // copies)
         for j, p in enumerate(projs):
             call = tq.tq_gemv if p.M <= 24 else tq.tq_gemm_prefill

@@ -23,7 +23,7 @@ def _projs(name):
     ("stack30_m1", "fused"), ("layer_m1", "fused"), ("ffn_m1", "fused"),
     ("ffn_m2", "batch"), ("ffn_m4", "batch"), ("ffn_m8", "batch"), ("ffn_m24", "batch"),
     ("stack30_m4", "batch"), ("stack30_m16", "batch"),
-    ("single_640x2560_m1", "per_projection"), ("prefill_m512", "prefill"),
+    ("single_640x2560_m1", "fused"), ("prefill_m512", "prefill"),
 ])
 def test_step_mode(name, mode):
     assert bench.step_mode(_projs(name)) == mode
