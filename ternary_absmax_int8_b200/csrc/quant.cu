@@ -10,10 +10,15 @@
 // A row is read twice as 16-byte vectors: pass 1 reduces |x| to amax, pass
 // 2 (an L1/L2 hit) converts and writes 8 codes per vector and reduces the code
 // sum. HBM traffic: 2K bytes in, K + 8 out. One CTA per row (block-wide
-// reductions) while rows are few; one warp per row (shuffle reductions only)
-// once there are enough rows to give every SM eight.
+// reductions) while rows are few; once there are enough rows to give every
+// SM eight, one warp per row (shuffle reductions only), its row copied whole
+// into shared memory with every 16-byte copy in flight at once (one memory
+// latency per row instead of one per batch of loads and pass), or, for rows
+// too long for that, read twice from global memory.
 #include <algorithm>
+#include <atomic>
 
+#include "mma_common.cuh"
 #include "quant_core.cuh"
 #include "tq_internal.h"
 
@@ -169,6 +174,52 @@ quant_stack_warp_kernel(const __grid_constant__ QuantStackParams p)
     }
 }
 
+// One warp per row, the row staged in shared memory: [warps][row_bytes].
+constexpr int kQsWarps = 4;
+constexpr int kQsMaxRowBytes = 48 * 1024;  // K <= 24576 on this path
+
+__global__ void __launch_bounds__(kQsWarps * 32)
+quant_stack_smem_kernel(const __grid_constant__ QuantStackParams p, int row_bytes)
+{
+    extern __shared__ __align__(16) uint8_t qs_buf[];
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint4 *sv = reinterpret_cast<const uint4 *>(qs_buf + size_t(warp) * row_bytes);
+    const uint32_t sv_s = smem_u32(sv);
+    const int nwarps = int(gridDim.x) * kQsWarps;
+    for (int r = int(blockIdx.x) * kQsWarps + warp; r < p.rows; r += nwarps) {
+        const QuantStackEntry &e = p.e[entry_of_row(p, r)];
+        const size_t m = size_t(r - e.row0);
+        const uint4 *xv = reinterpret_cast<const uint4 *>(e.x + m * e.K);
+        const int nvec = e.K >> 3;
+        __syncwarp();  // every lane is done reading the previous row
+        for (int v = lane; v < nvec; v += 32)
+            cp_async16(sv_s + uint32_t(v) * 16u, xv + v, true);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        float amax = 0.0f;
+        for (int v = lane; v < nvec; v += 32)
+            amax = fmaxf(amax, absmax8(sv[v]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = quant_inv_scale(amax);
+        int sum = 0;
+        uint2 *qv = reinterpret_cast<uint2 *>(e.xq + m * e.K);
+        for (int v = lane; v < nvec; v += 32)
+            qv[v] = quant8(sv[v], s, &sum);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) {
+            e.x_scale[m] = quant_scale(amax);
+            if (e.x_sum)
+                e.x_sum[m] = sum;
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_rows(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum,
@@ -186,10 +237,36 @@ cudaError_t launch_quant_stack(const QuantStackParams &p, cudaStream_t stream)
     const int sms = device_sm_count();
     if (p.rows < sms * kWarps) {
         quant_stack_kernel<<<p.rows, kQuantThreads, 0, stream>>>(p);
-    } else {
+        return cudaGetLastError();
+    }
+    int max_k = 0;
+    for (int j = 0; j < p.n; ++j)
+        max_k = std::max(max_k, p.e[j].K);
+    const int row_bytes = 2 * max_k;
+    if (row_bytes == 0 || row_bytes > kQsMaxRowBytes) {
         const int grid = std::min((p.rows + kWarps - 1) / kWarps, sms * 8);  // 8 CTAs of 8 warps per SM
         quant_stack_warp_kernel<<<grid, kQuantThreads, 0, stream>>>(p);
+        return cudaGetLastError();
     }
+    static std::atomic<int> configured_dev{-1};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (configured_dev != dev) {
+        err = cudaFuncSetAttribute(quant_stack_smem_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   kQsWarps * kQsMaxRowBytes);
+        if (err != cudaSuccess)
+            return err;
+        configured_dev = dev;
+    }
+    const size_t smem = size_t(kQsWarps) * row_bytes;
+    // CTAs per SM that the row buffers allow (227 KB per SM, 1 KB of it
+    // reserved per CTA; up to 8 CTAs of 4 warps)
+    const int per_sm = std::max(1, std::min(8, int((227 * 1024) / (smem + 1024))));
+    const int grid = std::min((p.rows + kQsWarps - 1) / kQsWarps, sms * per_sm);
+    quant_stack_smem_kernel<<<grid, kQsWarps * 32, smem, stream>>>(p, row_bytes);
     return cudaGetLastError();
 }
 
