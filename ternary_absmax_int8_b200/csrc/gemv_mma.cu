@@ -27,15 +27,15 @@
 // loaded), and the activations with 16-byte loads from L1/L2.
 //
 // Work split. Tiles of 16 packed rows (64 outputs) x the full K, numbered
-// across the projections of a launch; each CTA (one per SM, 16 or 20 warps) takes a
-// contiguous, byte-balanced range of tiles. Its warps form teams of P that
-// take the range's tiles in turn; the P warps of a team split a tile's
-// 64-column steps. With many tiles P = 1: a warp owns whole tiles and
-// applies the epilogue y = float(acc) * (w_scale * x_scale) from its
-// registers, no barrier. With few tiles (a single projection), P up to 16:
-// the team adds its accumulators in shared memory (integer adds, exact in any
-// order) behind a named barrier. A warp's loads for its next tile are in
-// flight while it finishes the current one.
+// across the projections of a launch; each CTA (one per SM, 12 or 16 warps)
+// takes a contiguous, byte-balanced range of tiles. Its warps form teams of
+// P (any P up to the warp count) that take the range's tiles in turn; the P
+// warps of a team split a tile's steps. With many tiles P = 1: a warp owns
+// whole tiles and applies the epilogue y = float(acc) * (w_scale * x_scale)
+// from its registers, no barrier. With few tiles (one projection, one FFN)
+// the team adds its accumulators in shared memory (integer adds, exact in
+// any order) behind a named barrier. A warp's loads for its next tile are
+// in flight while it finishes the current one.
 #include <atomic>
 #include <algorithm>
 #include <vector>
