@@ -266,6 +266,29 @@ def recorded_traffic(workload: str):
     return float(d["bytes_per_packed_byte"]) * d["full_packed_bytes"]
 
 
+def step_spread(marks, steps_per_chunk: int):
+    """Median, 10th and 90th percentile of the time per step (ms) over the
+    chunks between consecutive recorded events (None for fewer than two
+    chunks). The machine's GPUs are shared, so the spread is part of the
+    record."""
+    if len(marks) < 3:
+        return None
+    per = sorted(a.elapsed_time(b) / steps_per_chunk for a, b in zip(marks, marks[1:]))
+    return {"median_ms": round(percentile(per, 50), 5), "p10_ms": round(percentile(per, 10), 5),
+            "p90_ms": round(percentile(per, 90), 5), "chunks": len(per),
+            "steps_per_chunk": steps_per_chunk}
+
+
+def percentile(sorted_vals, q: float) -> float:
+    """Linear-interpolated percentile q (0..100) of an ascending list."""
+    if not sorted_vals:
+        raise ValueError("no values")
+    x = (len(sorted_vals) - 1) * q / 100.0
+    lo = int(x)
+    hi = min(lo + 1, len(sorted_vals) - 1)
+    return sorted_vals[lo] + (sorted_vals[hi] - sorted_vals[lo]) * (x - lo)
+
+
 def pipelined_steps(steps: int, stream, up, down, h2d, compute, d2h):
     """Enqueue `steps` end-to-end steps on two buffer sets: step i's
     host-to-device copy (h2d(i, b) on stream `up`) overlaps step i - 1's
@@ -465,17 +488,22 @@ def run_ours(args, rank: int, world: int):
     clocks.start()
     time.sleep(0.3)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # an event after every chunk (between graph replays, which do not overlap
+    # anyway): the spread of the time per step across the chunks
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(n_chunks)]
     barrier()
     torch.cuda.synchronize()
     t0.record(stream)
-    for _ in range(n_chunks):
+    for c in range(n_chunks):
         chunk_graph.replay()
+        marks[c].record(stream)
     for i in range(rem):
         single[(n_chunks * S + i) % copies].replay()
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
     total_ms = t0.elapsed_time(t1)
+    spread = step_spread([t0] + marks, S)
 
     # The split between quantiser and GEMV launches (non-stack workloads):
     # graphs of S steps' quantiser calls alone and GEMV calls alone.
@@ -586,6 +614,7 @@ def run_ours(args, rank: int, world: int):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5),
+        "step_spread": spread,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

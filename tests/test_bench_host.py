@@ -6,6 +6,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 import bench
@@ -117,3 +118,28 @@ def test_prefill_kernel_name(monkeypatch):
     monkeypatch.setenv("TQ_PREFILL_PAIR", "0")
     assert bench.prefill_kernel_name(512) == "prefill_tc_kernel"
 
+
+
+def test_percentile_matches_numpy():
+    rng = np.random.default_rng(3)
+    for n in (1, 2, 7, 125):
+        v = sorted(rng.random(n).tolist())
+        for q in (0, 10, 50, 90, 100):
+            assert abs(bench.percentile(v, q) - np.percentile(v, q)) < 1e-12
+
+
+def test_step_spread_from_chunk_events():
+    class Mark:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, later):
+            return later.t - self.t
+
+    # four chunks of 16 steps: 1.6, 1.6, 1.8, 1.6 ms
+    marks = [Mark(t) for t in (0.0, 1.6, 3.2, 5.0, 6.6)]
+    sp = bench.step_spread(marks, 16)
+    assert sp["chunks"] == 4 and sp["steps_per_chunk"] == 16
+    assert sp["median_ms"] == 0.1 and sp["p10_ms"] == 0.1
+    assert abs(sp["p90_ms"] - 0.10875) < 1e-9
+    assert bench.step_spread(marks[:2], 16) is None
