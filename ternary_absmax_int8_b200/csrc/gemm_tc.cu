@@ -129,18 +129,18 @@ __device__ __forceinline__ void store_out(const PrefillProj &e, int N, int m, in
 
 // 4 x 4 transpose within each quad of lanes: lane 4a + i holds m[k] = the
 // value of feature 4a + i at token k (k = 0..3); on return f[j] = the value
-// of feature 4a + j at token i (two rounds of exchanges, lanes i ^ 2 then i ^ 1).
+// of feature 4a + j at token i (two exchanges, lanes i ^ 2 then i ^ 1).
 __device__ __forceinline__ void quad_transpose(const int32_t (&m)[4], int32_t (&f)[4], int i)
 {
     const bool b1 = i & 2, b0 = i & 1;
-    // round 1: keep the tokens whose bit 1 equals ours, trade the others
+    // first exchange: keep the tokens whose bit 1 equals ours, trade the others
     const int32_t r0 = __shfl_xor_sync(0xffffffffu, b1 ? m[0] : m[2], 2);
     const int32_t r1 = __shfl_xor_sync(0xffffffffu, b1 ? m[1] : m[3], 2);
     const int32_t k0 = b1 ? m[2] : m[0], k1 = b1 ? m[3] : m[1];
     // w[rb][kb]: rb = bit 1 of the feature, kb = bit 0 of the token
     const int32_t w00 = b1 ? r0 : k0, w01 = b1 ? r1 : k1;
     const int32_t w10 = b1 ? k0 : r0, w11 = b1 ? k1 : r1;
-    // round 2: keep kb == bit 0 of ours, trade the other
+    // second exchange: keep kb == bit 0 of ours, trade the other
     const int32_t u0 = __shfl_xor_sync(0xffffffffu, b0 ? w00 : w01, 1);
     const int32_t u1 = __shfl_xor_sync(0xffffffffu, b0 ? w10 : w11, 1);
     const int32_t c0 = b0 ? w01 : w00, c1 = b0 ? w11 : w10;
