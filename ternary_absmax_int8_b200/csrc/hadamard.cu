@@ -18,12 +18,13 @@
 // is exact, so the butterfly's order gives the same value as the plain
 // matrix-vector sum; fl64(sum * fl64(1/sqrt(n))) is then rounded once to fp32.
 //
-// One CTA of 256 threads per token row (one launch per call, or per table of
-// projections in the stack form). Warp w rotates blocks w, w + 8, ...:
-// lane l holds entries l*E .. l*E + E - 1 of a block (E = n / 32) in fp64
-// registers; butterfly stages with a stride below E stay in the lane, the
-// others pair lane l with lane l ^ (stride / E) through shuffles. The fp32
-// results wait in shared memory for the row's amax, then become codes.
+// One CTA of 128 threads per token row (one launch per call, or per table of
+// projections in the stack form). A block of n entries is held by E = n / 32
+// lanes, 32 consecutive entries each in fp64 registers, so a warp rotates
+// 32 / E blocks at a time: the five butterfly stages with a stride below 32
+// stay in the lane, the log2(E) others pair lane l with lane l ^ (stride /
+// 32) through shuffles. The fp32 results wait in shared memory for the
+// row's amax, then become codes.
 #include <atomic>
 #include <cmath>
 
@@ -33,7 +34,7 @@ namespace tq {
 
 namespace {
 
-constexpr int kHadThreads = 256;
+constexpr int kHadThreads = 128;
 constexpr int kHadWarps = kHadThreads / 32;
 
 template <typename T, typename Op>
@@ -67,43 +68,51 @@ __device__ __forceinline__ int code4(float h, float s)
     return min(max(r, -7), 7);
 }
 
-// One token row (the whole CTA): E entries per lane (block size n = 32 E).
+// The rotated row waits in shared memory as fp32, each lane's run of 32
+// values followed by 4 floats of padding, so that the lanes' 16-byte stores
+// fall in distinct banks: value k sits at k + 4 (k / 32).
+__host__ __device__ constexpr size_t had_smem_floats(int K) { return size_t(K) + size_t(K / 32) * 4; }
+
+// One token row (the whole CTA), block size n = 32 E: a block is held by E
+// lanes of 32 consecutive entries each, so a warp takes 32 / E blocks at a
+// time; the five butterfly stages with a stride below 32 stay in the lane,
+// the log2(E) others pair lanes through shuffles.
 template <int E>
 __device__ __forceinline__ void hadamard_row(const uint16_t *__restrict__ row,
                                              int8_t *__restrict__ qrow, float *__restrict__ x_scale,
                                              int32_t *__restrict__ x_sum, int K, double c)
 {
-    extern __shared__ __align__(16) float hs[];  // [K] rotated row, fp32
+    extern __shared__ __align__(16) float hs[];  // rotated row, fp32, padded
     __shared__ float red_f[kHadWarps];
     __shared__ int red_i[kHadWarps];
     constexpr int n = 32 * E;
+    constexpr int kEL = 32;       // entries per lane
+    constexpr int kBPW = 32 / E;  // blocks per warp pass
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int slot = lane / E, sl = lane % E;  // block slot of the pass, lane within the block
+    const int nblk = K / n;
 
     float amax = 0.0f;
-    for (int b = warp; b < K / n; b += kHadWarps) {
-        const uint16_t *src = row + size_t(b) * n + lane * E;
-        double v[E];
-        if constexpr (E >= 8) {
+    for (int b0 = warp * kBPW; b0 < nblk; b0 += kHadWarps * kBPW) {
+        const int b = b0 + slot;
+        const bool ok = b < nblk;  // lanes past the last block run on zeros
+        const uint16_t *src = row + size_t(ok ? b : 0) * n + sl * kEL;
+        double v[kEL];
 #pragma unroll
-            for (int i = 0; i < E; i += 8) {
-                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + i));
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int i = 0; i < kEL; i += 8) {
+            const uint4 u = ok ? __ldg(reinterpret_cast<const uint4 *>(src + i)) : make_uint4(0, 0, 0, 0);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    v[i + 2 * j] = double(__uint_as_float(w[j] << 16));
-                    v[i + 2 * j + 1] = double(__uint_as_float(w[j] & 0xFFFF0000u));
-                }
+            for (int j = 0; j < 4; ++j) {
+                v[i + 2 * j] = double(__uint_as_float(w[j] << 16));
+                v[i + 2 * j + 1] = double(__uint_as_float(w[j] & 0xFFFF0000u));
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < E; ++i)
-                v[i] = double(__uint_as_float(uint32_t(__ldg(src + i)) << 16));
         }
-        // in-lane stages: stride h < E
+        // in-lane stages: stride h < 32
 #pragma unroll
-        for (int h = 1; h < E; h <<= 1) {
+        for (int h = 1; h < kEL; h <<= 1) {
 #pragma unroll
-            for (int i = 0; i < E; ++i) {
+            for (int i = 0; i < kEL; ++i) {
                 if ((i & h) == 0) {
                     const double a = v[i], d = v[i + h];
                     v[i] = __dadd_rn(a, d);
@@ -111,23 +120,32 @@ __device__ __forceinline__ void hadamard_row(const uint16_t *__restrict__ row,
                 }
             }
         }
-        // cross-lane stages: stride E t pairs lane l with lane l ^ t; the
-        // lower lane keeps a + b, the upper b' = a - b
+        // cross-lane stages: stride 32 t pairs lane sl with lane sl ^ t of
+        // the same block; the lower lane keeps a + b, the upper a - b, as
+        // (+-own) + other (a negation is exact, the add commutes)
 #pragma unroll
-        for (int t = 1; t < 32; t <<= 1) {
-            const bool upper = lane & t;
+        for (int t = 1; t < E; t <<= 1) {
+            const uint32_t flip = (sl & t) ? 0x80000000u : 0u;
 #pragma unroll
-            for (int i = 0; i < E; ++i) {
+            for (int i = 0; i < kEL; ++i) {
                 const double o = __shfl_xor_sync(0xffffffffu, v[i], t);
-                v[i] = upper ? __dsub_rn(o, v[i]) : __dadd_rn(v[i], o);
+                const double own = __hiloint2double(int(uint32_t(__double2hiint(v[i])) ^ flip),
+                                                    __double2loint(v[i]));
+                v[i] = __dadd_rn(own, o);
             }
         }
-        float *dst = hs + b * n + lane * E;
+        if (ok) {
+            float4 *dst = reinterpret_cast<float4 *>(hs + had_smem_floats(b * n + sl * kEL));
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const float h = __double2float_rn(__dmul_rn(v[i], c));
-            dst[i] = h;
-            amax = fmaxf(amax, fabsf(h));
+            for (int i = 0; i < kEL; i += 4) {
+                float4 f;
+                f.x = __double2float_rn(__dmul_rn(v[i], c));
+                f.y = __double2float_rn(__dmul_rn(v[i + 1], c));
+                f.z = __double2float_rn(__dmul_rn(v[i + 2], c));
+                f.w = __double2float_rn(__dmul_rn(v[i + 3], c));
+                dst[i / 4] = f;
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+            }
         }
     }
     amax = block_reduce_had(amax, HMax(), red_f);  // also orders the hs stores
@@ -136,7 +154,7 @@ __device__ __forceinline__ void hadamard_row(const uint16_t *__restrict__ row,
     int sum = 0;
     uint32_t *qw = reinterpret_cast<uint32_t *>(qrow);
     for (int k4 = threadIdx.x; k4 < K / 4; k4 += kHadThreads) {
-        const float4 h = reinterpret_cast<const float4 *>(hs)[k4];
+        const float4 h = *reinterpret_cast<const float4 *>(hs + had_smem_floats(4 * k4));
         const int a = code4(h.x, s), b = code4(h.y, s), cc = code4(h.z, s), d = code4(h.w, s);
         sum += a + b + cc + d;
         qw[k4] = (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) |
@@ -185,18 +203,18 @@ template <int E>
 cudaError_t launch_e(const uint16_t *x, int8_t *xq, float *x_scale, int32_t *x_sum, int M, int K,
                      cudaStream_t stream)
 {
-    const size_t smem = size_t(K) * sizeof(float);
+    const size_t smem = had_smem_floats(K) * sizeof(float);
     static std::atomic<int> configured_dev{-1};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (configured_dev != dev) {
-        // the rotated row of the longest K (32768 fp32), next to 64 bytes of
-        // static reduction slots
+        // the rotated row of the longest K (32768 fp32 and its padding), next
+        // to 64 bytes of static reduction slots
         e = cudaFuncSetAttribute(hadamard_quant4_kernel<E>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(kStreamMaxK * sizeof(float)));
+                                 int(had_smem_floats(kStreamMaxK) * sizeof(float)));
         if (e != cudaSuccess)
             return e;
         configured_dev = dev;
@@ -218,13 +236,14 @@ cudaError_t launch_stack_e(const QuantStackParams &p, int max_k, cudaStream_t st
     if (configured_dev != dev) {
         e = cudaFuncSetAttribute(hadamard_quant4_stack_kernel<E>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(kStreamMaxK * sizeof(float)));
+                                 int(had_smem_floats(kStreamMaxK) * sizeof(float)));
         if (e != cudaSuccess)
             return e;
         configured_dev = dev;
     }
     const double c = 1.0 / sqrt(double(32 * E));  // IEEE sqrt and divide: the oracle's constant
-    hadamard_quant4_stack_kernel<E><<<p.rows, kHadThreads, size_t(max_k) * sizeof(float), stream>>>(p, c);
+    hadamard_quant4_stack_kernel<E>
+        <<<p.rows, kHadThreads, had_smem_floats(max_k) * sizeof(float), stream>>>(p, c);
     return cudaGetLastError();
 }
 
